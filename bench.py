@@ -1,0 +1,369 @@
+"""Batch-1 decode benchmark of the hybrid Gated-DeltaNet + attention megakernel.
+
+Workload: the 0.8B-shaped hybrid (24 layers, [D,D,D,A] x 6, hidden 1024, vocab
+151936, bf16 weights from N(0, 0.02), seed 1), a 128-token uniform random prompt,
+then tg128: 128 greedy decode steps at batch 1. One bench step = restore the
+post-prompt state, then 128 decode launches (one kernel launch per token).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {mk,reference}]
+
+Prints one JSON line (rank 0). With --gpus N > 1 (launched by torchrun) every rank
+runs an independent replica on its own GPU; there is no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "batch-1 decode tok/s (hybrid DeltaNet, tg128) and % of B200 HBM roofline"
+PROMPT = 128
+TG = 128
+MAX_CTX = PROMPT + TG + 16
+WORKLOAD = ("0.8B-shaped hybrid Gated-DeltaNet + attention (24 layers [D,D,D,A]x6, hidden 1024, "
+            "vocab 151936 tied, DeltaNet 16 heads dk=dv=128, attention 8q/2kv heads D=256, SwiGLU 3584), "
+            "bf16 weights N(0,0.02) seed 1, 128-token random prompt, tg128 greedy decode, batch 1")
+KERNEL_SOURCES = ["hybrid_deltanet_attention_b200/csrc/decode.cu", "hybrid_deltanet_attention_b200/csrc/dev.cuh",
+                  "hybrid_deltanet_attention_b200/csrc/mk_internal.h"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def bytes_per_token(cfg, pos: int) -> dict:
+    """Algorithmic bytes one decode step at position `pos` reads (and writes)."""
+    H, V, F = cfg.hidden, cfg.vocab, cfg.ffn
+    w = V * H * 2 + H * 2                                  # tied LM head + final gain
+    for kind in cfg.pattern:
+        w += 2 * H * 2 + 3 * F * H * 2                     # gains, gate, up, down
+        if kind == "D":
+            w += cfg.dn_in_rows * H * 2 + cfg.dn_conv_channels * cfg.conv_width * 2
+            w += H * cfg.dn_heads * cfg.dn_dv * 2
+        else:
+            w += cfg.at_in_rows * H * 2 + H * cfg.at_q_heads * cfg.at_head_dim * 2
+    s = cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
+    conv = cfg.n_dn * cfg.conv_width * cfg.dn_conv_channels * 4
+    kv = cfg.n_at * cfg.at_kv_heads * (pos + 1) * cfg.at_head_dim * 2 * 2
+    return {"weights": w, "state": s, "conv": conv, "kv": kv, "read": w + s + conv + kv,
+            "write": s + cfg.n_dn * cfg.dn_conv_channels * 4 + cfg.n_at * cfg.at_kv_heads * cfg.at_head_dim * 4}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def recorded_traffic(khash: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on this kernel."""
+    p = os.path.join(ROOT, "profiles", "decode_0.8b_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as fh:
+        for line in fh:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_hash") != khash:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 6:
+                    continue
+                try:
+                    sms.append(float(parts[0]))
+                    mx = float(parts[1])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[2:6]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    if n_gpus > 1 or int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import datetime
+        import torch.distributed as dist
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return dist.get_rank(), dist.get_world_size(), local
+    torch.cuda.set_device(0)
+    return 0, 1, 0
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+def oracle_sample(seconds_budget: float = 15.0, n_prompt: int = 16, n_decode: int = 64):
+    """Time the CPU oracle on a bounded sample of the same workload: weights prepared
+    untimed, a short prompt fed untimed, then n_decode greedy steps timed."""
+    import oracle
+    import synth
+    cfg = synth.QWEN_08B
+    W = oracle.prepare_weights(cfg, synth.make_weights(cfg))
+    st = oracle.new_state(cfg, n_prompt + n_decode + 1)
+    z = oracle.prefill(cfg, W, st, synth.make_prompt(cfg, n_prompt))
+    tok = int(np.argmax(z))
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(n_decode):
+        z = oracle.decode_step(cfg, W, st, tok)
+        tok = int(np.argmax(z))
+        done += 1
+        if time.perf_counter() - t0 > seconds_budget:
+            break
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    sample = (f"oracle (numpy float64) on the 0.8B-shaped model: {done} greedy decode steps at positions "
+              f"{n_prompt}..{n_prompt + done - 1} after a {n_prompt}-token prompt (prompt and weight preparation untimed)")
+    return done / dt, cores, sample
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    vals = []
+    cores, sample = 1, ""
+    for _ in range(args.warmup + args.steps):
+        v, cores, sample = oracle_sample(seconds_budget=6.0, n_prompt=8, n_decode=16)
+        vals.append(v)
+    timed = vals[args.warmup:]
+    value = float(np.mean(timed))
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 16 * 1000.0 / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "reference": "the CPU oracle (numpy float64), bounded sample per step"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ the CUDA path
+def run_mk(args):
+    import torch
+    import hybrid_deltanet_attention_b200 as hda
+    import synth
+
+    rank, world, local = dist_setup(args.gpus)
+    cfg = synth.QWEN_08B
+    dev = torch.device("cuda", local)
+    raw = synth.make_weights(cfg)
+    m = hda.Model(cfg, hda.weights_to_device(raw, dev), max_ctx=MAX_CTX)
+    del raw
+    prompt_np = synth.make_prompt(cfg, PROMPT)
+    prompt = torch.from_numpy(prompt_np).to(dev)
+
+    # context after the prompt, snapshotted once; every step restores it
+    first = torch.empty(1, dtype=torch.int32, device=dev)
+    m.reset()
+    m.prefill(prompt, next_token=first)
+    assert m.sync() == 0
+    snap = m.state.clone()
+    first_tok = first.clone()
+    toks = torch.empty(TG + 1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_step(ev=None):
+        m.state.copy_(snap)
+        m.set_position(PROMPT)          # same value as the snapshot; keeps the handle's position in step
+        toks[0:1].copy_(first_tok)
+        if ev is not None:
+            ev[0].record(stream)
+        for i in range(TG):
+            m.decode(toks[i:i + 1], toks[i + 1:i + 2])
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    assert m.sync() == 0
+    launches0 = m.launches
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for k in range(args.steps):
+            one_step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    dev_err = m.sync()
+    if dev_err:
+        raise RuntimeError(f"device error word 0x{dev_err:x}")
+    launches = m.launches - launches0
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    decode_ms = sum(a.elapsed_time(b) for a, b in evs)
+    decode_ms = max_over_ranks(decode_ms, world)
+    value = world * args.steps * TG / (total_ms / 1000.0)
+
+    # roofline of the decode kernel: algorithmic bytes per launch / average launch duration
+    P0 = PROMPT
+    per = [bytes_per_token(cfg, P0 + i) for i in range(TG)]
+    read_avg = float(np.mean([b["read"] for b in per]))
+    write_avg = float(np.mean([b["write"] for b in per]))
+    t_launch = decode_ms / 1000.0 / (args.steps * TG)
+    peak, peak_kind = measured_peaks()
+    achieved = read_avg / t_launch / 1e9
+    khash = kernel_hash()
+    traffic = recorded_traffic(khash)
+
+    # end to end through the public C call with host buffers: prompt in, tokens out
+    pinned_in = torch.from_numpy(prompt_np).pin_memory()
+    pinned_out = torch.empty(TG, dtype=torch.int32).pin_memory()
+    for _ in range(max(1, args.warmup // 2)):
+        m.reset()
+        m.generate(pinned_in.numpy(), TG, out=pinned_out.numpy())
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        m.reset()
+        m.generate(pinned_in.numpy(), TG, out=pinned_out.numpy())
+    dt = max_over_ranks(time.perf_counter() - t0, world)
+    e2e = world * e2e_steps * TG / dt
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_sample()
+        cpu = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_step": TG, "prompt": PROMPT,
+                   "l2": "inputs larger than L2: every step streams 1.23 GB of weights (L2 is 126 MB)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "peak_kind": peak_kind,
+                     "bytes_per_launch_read": read_avg, "bytes_per_launch_write": write_avg,
+                     "kernel": "mk_decode_kernel", "avg_launch_us": t_launch * 1e6, "kernel_hash": khash},
+        "e2e": {"value": e2e, "unit": "tok/s", "h2d_bytes_per_step": PROMPT * 4, "d2h_bytes_per_step": TG * 4,
+                "what": "mk_generate: pinned host prompt (128) -> prefill -> 128 greedy tokens -> pinned host"},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mk(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

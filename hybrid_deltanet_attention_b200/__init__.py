@@ -1,0 +1,7 @@
+"""Batch-1 hybrid Gated-DeltaNet + attention inference on B200 (sm_100a).
+
+The compute path is libmk.so (C ABI, include/mk.h); this package is its thin
+Python binding. There is no CPU fallback.
+"""
+from ._abi import MkError, load_library  # noqa: F401
+from .model import Model, make_config, weights_to_device  # noqa: F401

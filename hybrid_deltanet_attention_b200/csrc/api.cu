@@ -1,0 +1,623 @@
+// C ABI of libmk.so: validation, weight repacking, state/workspace layout and launches.
+// Every step of the forward pass runs in this library's kernels; the caller only
+// provides device memory and a stream.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  g_err = std::string(what) + ": " + cudaGetErrorString(e);
+  return MK_ERR_CUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct Expect {
+  int dtype;
+  int ndim;
+  int64_t shape[2];
+  uint64_t bytes;
+};
+
+int n_kind(const mk_config& c, char k) {
+  int n = 0;
+  for (int i = 0; i < c.n_layers; ++i) n += (c.pattern[i] == k);
+  return n;
+}
+
+}  // namespace
+
+struct mk_model {
+  mk_config cfg;
+  mk_sizes sz;
+  uint8_t* packed;
+  uint8_t* state;
+  uint8_t* ws;
+  int grid;
+  int device;
+  mk::DecodeParams base;
+  std::vector<mk::LayerW> layers_host;
+  int64_t launches;
+  int64_t pos_hint;      // host shadow of the device position (calls through this handle)
+  // workspace sub-buffers used by the host-side drivers
+  int32_t* ws_tok;       // [max_ctx + 8] token staging for prefill / generate
+  int32_t* ws_g;         // [max_draft + 1] greedy tokens of a verify pass
+  int32_t* ws_n;         // accepted-draft count of the last verify pass
+  uint8_t* ws_snap;      // DeltaNet S + conv history + pos snapshot for verify
+  size_t snap_S_bytes, snap_conv_bytes;
+};
+
+namespace mk {
+
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ src, uint16_t* __restrict__ dst, int rows,
+                                      int cols) {
+  __shared__ uint16_t tile[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = src[static_cast<size_t>(r) * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) dst[static_cast<size_t>(c) * rows + r] = tile[threadIdx.x][i];
+  }
+}
+
+cudaError_t launch_transpose_bf16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t s) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
+  transpose_bf16_kernel<<<grid, block, 0, s>>>(src, dst, rows, cols);
+  return cudaGetLastError();
+}
+
+__global__ void set_int_kernel(int* p, int v) { *p = v; }
+
+// Longest-prefix greedy acceptance of one verify pass.
+// tokens = [last, d_1..d_K], g[i] = greedy token after input i (i = 0..K).
+__global__ void accept_kernel(const int* tokens, const int* g, int K, int* n_out, int* n_acc, int* out) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int n = 0;
+  while (n < K && tokens[1 + n] == g[n]) ++n;
+  for (int i = 0; i < n; ++i) out[i] = tokens[1 + i];
+  out[n] = g[n];
+  *n_out = n;
+  *n_acc = n;
+}
+
+}  // namespace mk
+
+namespace {
+
+int check_config(const mk_config* c) {
+  if (!c) return fail(MK_ERR_ARG, "config is NULL");
+  if (c->n_layers < 1 || c->n_layers > MK_MAX_LAYERS) return fail(MK_ERR_ARG, "n_layers out of range");
+  if (static_cast<int>(strnlen(c->pattern, MK_MAX_LAYERS + 1)) != c->n_layers)
+    return fail(MK_ERR_ARG, "pattern length differs from n_layers");
+  for (int i = 0; i < c->n_layers; ++i)
+    if (c->pattern[i] != 'D' && c->pattern[i] != 'A') return fail(MK_ERR_ARG, "pattern must hold only 'D' and 'A'");
+  if (c->hidden <= 0 || c->hidden % 8 || c->hidden > 8192) return fail(MK_ERR_ARG, "hidden must be a multiple of 8, <= 8192");
+  if (c->vocab <= 0) return fail(MK_ERR_ARG, "vocab must be positive");
+  if (!(c->rms_eps > 0.f)) return fail(MK_ERR_ARG, "rms_eps must be positive");
+  if (c->ffn <= 0) return fail(MK_ERR_ARG, "ffn must be positive");
+  if (c->max_ctx <= 0) return fail(MK_ERR_ARG, "max_ctx must be positive");
+  if (c->max_draft < 0 || c->max_draft > 16) return fail(MK_ERR_ARG, "max_draft must be in [0, 16]");
+  if (c->weight_format != MK_W_BF16 && c->weight_format != MK_W_Q4K) return fail(MK_ERR_ARG, "unknown weight_format");
+  if (c->weight_format == MK_W_Q4K)
+    return fail(MK_ERR_ARG, "weight_format MK_W_Q4K is not supported by this build's decode kernel");
+  const int nd = n_kind(*c, 'D'), na = n_kind(*c, 'A');
+  if (nd) {
+    if (c->dn_heads <= 0 || c->dn_dk <= 0 || c->dn_dk % 32 || c->dn_dk > 256 || c->dn_dv <= 0 || c->dn_dv > 256)
+      return fail(MK_ERR_ARG, "DeltaNet dims: dk must be a multiple of 32 and <= 256, 0 < dv <= 256");
+    if (c->conv_width < 2 || c->conv_width > 8) return fail(MK_ERR_ARG, "conv_width must be in [2, 8]");
+  }
+  if (na) {
+    if (c->at_q_heads <= 0 || c->at_kv_heads <= 0 || c->at_q_heads % c->at_kv_heads)
+      return fail(MK_ERR_ARG, "attention heads: Hq must be a positive multiple of Hkv");
+    if (c->at_q_heads / c->at_kv_heads > 8) return fail(MK_ERR_ARG, "at most 8 query heads per KV head");
+    if (c->at_head_dim <= 0 || c->at_head_dim % 64 || c->at_head_dim > 256)
+      return fail(MK_ERR_ARG, "at_head_dim must be a multiple of 64, <= 256");
+    if (!(c->rope_theta > 0.f)) return fail(MK_ERR_ARG, "rope_theta must be positive");
+  }
+  return MK_OK;
+}
+
+int device_grid(int* grid, int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  int coop = 0;
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, *dev);
+  if (!coop) return fail(MK_ERR_RESIDENCY, "device does not support cooperative launches");
+  *grid = sms;
+  return MK_OK;
+}
+
+// Scratch and shared-memory budget checks that depend on the grid size.
+int check_budget(const mk_config& c, int grid) {
+  if (mk::decode_smem_bytes(c.hidden) > 232448) return fail(MK_ERR_ARG, "shared-memory budget exceeded");
+  auto ceil_div = [](long a, long b) { return (a + b - 1) / b; };
+  const long S = mk::kScratchFloats;
+  if (n_kind(c, 'D')) {
+    const long rows = ceil_div(static_cast<long>(c.dn_heads) * c.dn_dv, grid);
+    const long nh = ceil_div(rows, c.dn_dv) + 1;
+    if (nh * (2 * c.dn_dk + 2) + 2 * rows > S) return fail(MK_ERR_ARG, "DeltaNet rows per CTA exceed the scratch budget");
+  }
+  if (n_kind(c, 'A')) {
+    const long grp = c.at_q_heads / c.at_kv_heads;
+    if (grp * c.at_head_dim + grp * mk::kAttnSub + 3 * grp > S) return fail(MK_ERR_ARG, "attention scratch budget exceeded");
+    if (ceil_div(static_cast<long>(c.at_q_heads) * c.at_head_dim, grid) > S)
+      return fail(MK_ERR_ARG, "attention columns per CTA exceed the scratch budget");
+  }
+  if (2 * ceil_div(c.ffn, grid) > S) return fail(MK_ERR_ARG, "MLP rows per CTA exceed the scratch budget");
+  return MK_OK;
+}
+
+struct Layout {
+  mk_sizes sz;
+  // packed
+  size_t p_table, p_freq, p_embed, p_normf;
+  std::vector<size_t> p_layer;   // start of each layer block
+  // workspace
+  size_t w_sync, w_h, w_z, w_part, w_tok, w_g, w_n, w_snap;
+  size_t snap_S, snap_conv;
+  int max_splits;
+};
+
+size_t layer_block_bytes(const mk_config& c, char kind) {
+  const size_t H = c.hidden, rb = H * 2;
+  size_t b = align256(H * 2) * 2;                        // norm1, norm2
+  if (kind == 'D') {
+    const size_t C = static_cast<size_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
+    b += align256((C + 2 * c.dn_heads) * rb);              // w_in
+    b += align256(C * c.conv_width * 2);                    // conv
+    b += align256(static_cast<size_t>(c.dn_heads) * c.dn_dv * rb);   // w_outT
+  } else {
+    const size_t qd = static_cast<size_t>(c.at_q_heads) * c.at_head_dim;
+    const size_t rows = qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim;
+    b += align256(rows * rb);
+    b += align256(qd * rb);
+  }
+  b += 3 * align256(static_cast<size_t>(c.ffn) * rb);     // gate, up, downT
+  return b;
+}
+
+Layout make_layout(const mk_config& c, int grid) {
+  Layout L{};
+  const size_t H = c.hidden;
+  const int nd = n_kind(c, 'D'), na = n_kind(c, 'A');
+  size_t off = 0;
+  L.p_table = off; off = align256(off + sizeof(mk::LayerW) * c.n_layers);
+  L.p_freq = off; off = align256(off + sizeof(double) * (c.at_head_dim > 0 ? c.at_head_dim / 2 : 1));
+  L.p_embed = off; off = align256(off + static_cast<size_t>(c.vocab) * H * 2);
+  L.p_normf = off; off = align256(off + H * 2);
+  for (int l = 0; l < c.n_layers; ++l) {
+    L.p_layer.push_back(off);
+    off += layer_block_bytes(c, c.pattern[l]);
+  }
+  L.sz.packed_bytes = off;
+
+  const size_t C = static_cast<size_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
+  off = 0;
+  L.sz.off_S = off; off = align256(off + static_cast<size_t>(nd) * c.dn_heads * c.dn_dv * c.dn_dk * 4);
+  L.sz.off_conv = off; off = align256(off + static_cast<size_t>(nd) * c.conv_width * C * 4);
+  const size_t kv = static_cast<size_t>(na) * c.at_kv_heads * c.max_ctx * c.at_head_dim * 2;
+  L.sz.off_k = off; off = align256(off + kv);
+  L.sz.off_v = off; off = align256(off + kv);
+  L.sz.off_pos = off; off = align256(off + 4);
+  L.sz.off_err = off; off = align256(off + 4);
+  L.sz.state_bytes = off;
+
+  L.max_splits = (na ? mk::decode_max_splits(grid, c.at_kv_heads) : 1);
+  off = 0;
+  L.w_sync = off; off = align256(off + 1024);
+  L.w_h = off; off = align256(off + 3 * H * 4);
+  const size_t zf = std::max<size_t>(2 * c.dn_heads,
+                                     na ? static_cast<size_t>(c.at_q_heads) * c.at_head_dim * (c.at_out_gate ? 2 : 1) +
+                                              2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim
+                                        : 0);
+  L.w_z = off; off = align256(off + zf * 4);
+  L.w_part = off;
+  off = align256(off + (na ? static_cast<size_t>(c.at_q_heads) * L.max_splits * (c.at_head_dim + 2) * 4 : 4));
+  L.w_tok = off; off = align256(off + (static_cast<size_t>(c.max_ctx) + 8) * 4);
+  L.w_g = off; off = align256(off + (static_cast<size_t>(c.max_draft) + 2) * 4);
+  L.w_n = off; off = align256(off + 4);
+  L.snap_S = static_cast<size_t>(nd) * c.dn_heads * c.dn_dv * c.dn_dk * 4;
+  L.snap_conv = static_cast<size_t>(nd) * c.conv_width * C * 4;
+  L.w_snap = off;
+  if (c.max_draft > 0) off = align256(off + align256(L.snap_S) + align256(L.snap_conv) + 256);
+  L.sz.workspace_bytes = off;
+  L.sz.grid_ctas = grid;
+  return L;
+}
+
+void expected_tensors(const mk_config& c, std::map<std::string, Expect>& ex) {
+  const int64_t H = c.hidden;
+  auto mat = [&](const std::string& n, int64_t r, int64_t k) {
+    ex[n] = Expect{MK_DT_BF16, 2, {r, k}, static_cast<uint64_t>(r * k * 2)};
+  };
+  auto vec = [&](const std::string& n, int64_t r) { ex[n] = Expect{MK_DT_BF16, 1, {r, 0}, static_cast<uint64_t>(r * 2)}; };
+  mat("embed", c.vocab, H);
+  vec("norm_f", H);
+  const int64_t C = static_cast<int64_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
+  for (int l = 0; l < c.n_layers; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    vec(p + "norm1", H);
+    vec(p + "norm2", H);
+    if (c.pattern[l] == 'D') {
+      mat(p + "dn.w_in", C + 2 * c.dn_heads, H);
+      mat(p + "dn.conv", C, c.conv_width);
+      mat(p + "dn.w_out", H, static_cast<int64_t>(c.dn_heads) * c.dn_dv);
+    } else {
+      const int64_t qd = static_cast<int64_t>(c.at_q_heads) * c.at_head_dim;
+      mat(p + "attn.w_in", qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<int64_t>(c.at_kv_heads) * c.at_head_dim, H);
+      mat(p + "attn.w_out", H, qd);
+    }
+    mat(p + "mlp.w_gate", c.ffn, H);
+    mat(p + "mlp.w_up", c.ffn, H);
+    mat(p + "mlp.w_down", H, c.ffn);
+  }
+}
+
+std::string shape_str(int ndim, const int64_t* s) {
+  std::string r = "[";
+  for (int i = 0; i < ndim; ++i) r += (i ? ", " : "") + std::to_string(s[i]);
+  return r + "]";
+}
+
+int launch_step(mk_model* m, const int32_t* in_tok, int32_t* out_tok, float* logits, cudaStream_t s) {
+  mk::DecodeParams p = m->base;
+  p.in_token = in_tok;
+  p.out_token = out_tok;
+  p.logits = logits;
+  cudaError_t e = mk::launch_decode(p, m->grid, s);
+  if (e == cudaErrorCooperativeLaunchTooLarge)
+    return fail(MK_ERR_RESIDENCY, "persistent grid cannot be co-resident: " + std::string(cudaGetErrorString(e)));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  ++m->launches;
+  ++m->pos_hint;
+  return MK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mk_query_sizes(const mk_config* cfg, mk_sizes* out) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!out) return fail(MK_ERR_ARG, "out is NULL");
+  int grid = 0, dev = 0;
+  rc = device_grid(&grid, &dev);
+  if (rc) return rc;
+  rc = check_budget(*cfg, grid);
+  if (rc) return rc;
+  *out = make_layout(*cfg, grid).sz;
+  return MK_OK;
+}
+
+int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_tensors, void* d_packed, void* d_state,
+                    void* d_workspace, void* stream, mk_model** out) {
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!out) return fail(MK_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (!tensors || n_tensors <= 0) return fail(MK_ERR_ARG, "no tensors given");
+  if (!d_packed || !d_state || !d_workspace) return fail(MK_ERR_ARG, "device buffer pointer is NULL");
+  int grid = 0, dev = 0;
+  rc = device_grid(&grid, &dev);
+  if (rc) return rc;
+  rc = check_budget(*cfg, grid);
+  if (rc) return rc;
+  const mk_config& c = *cfg;
+
+  // ---- type-check every tensor ----
+  std::map<std::string, Expect> ex;
+  expected_tensors(c, ex);
+  std::map<std::string, const mk_tensor*> got;
+  for (int i = 0; i < n_tensors; ++i) {
+    const mk_tensor& t = tensors[i];
+    if (!t.name) return fail(MK_ERR_TENSOR, "tensor " + std::to_string(i) + " has no name");
+    const std::string nm(t.name);
+    auto it = ex.find(nm);
+    if (it == ex.end()) return fail(MK_ERR_TENSOR, "unknown tensor '" + nm + "'");
+    if (got.count(nm)) return fail(MK_ERR_TENSOR, "tensor '" + nm + "' given twice");
+    const Expect& e = it->second;
+    if (t.dtype != e.dtype) return fail(MK_ERR_TENSOR, "tensor '" + nm + "': wrong dtype " + std::to_string(t.dtype));
+    if (t.ndim != e.ndim) return fail(MK_ERR_TENSOR, "tensor '" + nm + "': wrong rank " + std::to_string(t.ndim));
+    for (int d = 0; d < e.ndim; ++d)
+      if (t.shape[d] != e.shape[d])
+        return fail(MK_ERR_TENSOR, "tensor '" + nm + "': shape " + shape_str(t.ndim, t.shape) + ", expected " +
+                                       shape_str(e.ndim, e.shape));
+    if (t.bytes != e.bytes) return fail(MK_ERR_TENSOR, "tensor '" + nm + "': wrong byte size");
+    if (!t.data) return fail(MK_ERR_TENSOR, "tensor '" + nm + "': data is NULL");
+    if (reinterpret_cast<uintptr_t>(t.data) % 16) return fail(MK_ERR_TENSOR, "tensor '" + nm + "': data not 16-byte aligned");
+    got[nm] = &t;
+  }
+  for (auto& kv : ex)
+    if (!got.count(kv.first)) return fail(MK_ERR_TENSOR, "missing tensor '" + kv.first + "'");
+
+  // ---- layout, repack ----
+  Layout L = make_layout(c, grid);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* P = static_cast<uint8_t*>(d_packed);
+  uint8_t* St = static_cast<uint8_t*>(d_state);
+  uint8_t* W = static_cast<uint8_t*>(d_workspace);
+  if (reinterpret_cast<uintptr_t>(P) % 256 || reinterpret_cast<uintptr_t>(St) % 256 ||
+      reinterpret_cast<uintptr_t>(W) % 256)
+    return fail(MK_ERR_ARG, "device buffers must be 256-byte aligned");
+
+  mk_model* m = new mk_model();
+  m->cfg = c;
+  m->sz = L.sz;
+  m->packed = P;
+  m->state = St;
+  m->ws = W;
+  m->grid = grid;
+  m->device = dev;
+  m->launches = 0;
+  m->pos_hint = 0;
+
+  auto copy = [&](const std::string& nm, size_t dst_off) -> cudaError_t {
+    const mk_tensor* t = got[nm];
+    return cudaMemcpyAsync(P + dst_off, t->data, t->bytes, cudaMemcpyDeviceToDevice, s);
+  };
+  auto transpose = [&](const std::string& nm, size_t dst_off) -> cudaError_t {
+    const mk_tensor* t = got[nm];
+    ++m->launches;
+    return mk::launch_transpose_bf16(static_cast<const uint16_t*>(t->data), reinterpret_cast<uint16_t*>(P + dst_off),
+                                     static_cast<int>(t->shape[0]), static_cast<int>(t->shape[1]), s);
+  };
+  const size_t H = c.hidden, rb = H * 2;
+  const size_t C = static_cast<size_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
+  cudaError_t e = copy("embed", L.p_embed);
+  if (e == cudaSuccess) e = copy("norm_f", L.p_normf);
+  int di = 0, ai = 0;
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+    const std::string p = "layers." + std::to_string(l) + ".";
+    size_t off = L.p_layer[l];
+    mk::LayerW lw{};
+    lw.kind = c.pattern[l] == 'D' ? mk::kDeltaNet : mk::kAttention;
+    lw.idx = c.pattern[l] == 'D' ? di++ : ai++;
+    lw.norm1 = reinterpret_cast<const uint16_t*>(P + off);
+    e = copy(p + "norm1", off); off += align256(H * 2);
+    lw.norm2 = reinterpret_cast<const uint16_t*>(P + off);
+    if (e == cudaSuccess) e = copy(p + "norm2", off);
+    off += align256(H * 2);
+    if (lw.kind == mk::kDeltaNet) {
+      lw.w_in = P + off;
+      if (e == cudaSuccess) e = copy(p + "dn.w_in", off);
+      off += align256((C + 2 * c.dn_heads) * rb);
+      lw.conv = reinterpret_cast<const uint16_t*>(P + off);
+      if (e == cudaSuccess) e = copy(p + "dn.conv", off);
+      off += align256(C * c.conv_width * 2);
+      lw.w_outT = P + off;
+      if (e == cudaSuccess) e = transpose(p + "dn.w_out", off);
+      off += align256(static_cast<size_t>(c.dn_heads) * c.dn_dv * rb);
+    } else {
+      const size_t qd = static_cast<size_t>(c.at_q_heads) * c.at_head_dim;
+      const size_t rows = qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim;
+      lw.w_in = P + off;
+      if (e == cudaSuccess) e = copy(p + "attn.w_in", off);
+      off += align256(rows * rb);
+      lw.w_outT = P + off;
+      if (e == cudaSuccess) e = transpose(p + "attn.w_out", off);
+      off += align256(qd * rb);
+    }
+    lw.w_gate = P + off;
+    if (e == cudaSuccess) e = copy(p + "mlp.w_gate", off);
+    off += align256(static_cast<size_t>(c.ffn) * rb);
+    lw.w_up = P + off;
+    if (e == cudaSuccess) e = copy(p + "mlp.w_up", off);
+    off += align256(static_cast<size_t>(c.ffn) * rb);
+    lw.w_downT = P + off;
+    if (e == cudaSuccess) e = transpose(p + "mlp.w_down", off);
+    m->layers_host.push_back(lw);
+  }
+  std::vector<double> freq(c.at_head_dim > 0 ? c.at_head_dim / 2 : 1, 0.0);
+  for (int i = 0; i < c.at_head_dim / 2; ++i)
+    freq[i] = std::pow(static_cast<double>(c.rope_theta), -2.0 * i / static_cast<double>(c.at_head_dim));
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(P + L.p_table, m->layers_host.data(), sizeof(mk::LayerW) * c.n_layers, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(P + L.p_freq, freq.data(), sizeof(double) * freq.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(St, 0, L.sz.state_bytes, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(W, 0, L.sz.workspace_bytes, s);
+  // the two host vectors above are pageable: make sure the copies have read them
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    delete m;
+    return cuda_fail(e, "weight repack");
+  }
+
+  mk::DecodeParams& b = m->base;
+  b = mk::DecodeParams{};
+  b.layers = reinterpret_cast<const mk::LayerW*>(P + L.p_table);
+  b.n_layers = c.n_layers;
+  b.embed = P + L.p_embed;
+  b.norm_f = reinterpret_cast<const uint16_t*>(P + L.p_normf);
+  b.inv_freq = reinterpret_cast<const double*>(P + L.p_freq);
+  b.H = c.hidden; b.V = c.vocab; b.F = c.ffn;
+  b.Hd = c.dn_heads; b.dk = c.dn_dk; b.dv = c.dn_dv; b.convw = c.conv_width; b.C = static_cast<int>(C);
+  b.Hq = c.at_q_heads; b.Hkv = c.at_kv_heads; b.D = c.at_head_dim; b.gated = c.at_out_gate;
+  b.at_in_rows = static_cast<int>(static_cast<size_t>(c.at_q_heads) * c.at_head_dim * (c.at_out_gate ? 2 : 1) +
+                                  2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim);
+  b.max_ctx = c.max_ctx;
+  b.row_bytes = static_cast<int>(rb);
+  b.eps = c.rms_eps;
+  b.S = reinterpret_cast<float*>(St + L.sz.off_S);
+  b.conv_ring = reinterpret_cast<float*>(St + L.sz.off_conv);
+  b.kc = reinterpret_cast<uint16_t*>(St + L.sz.off_k);
+  b.vc = reinterpret_cast<uint16_t*>(St + L.sz.off_v);
+  b.pos = reinterpret_cast<int*>(St + L.sz.off_pos);
+  b.err = reinterpret_cast<int*>(St + L.sz.off_err);
+  b.hbuf = reinterpret_cast<float*>(W + L.w_h);
+  b.z = reinterpret_cast<float*>(W + L.w_z);
+  b.part = reinterpret_cast<float*>(W + L.w_part);
+  b.bar = reinterpret_cast<unsigned*>(W + L.w_sync);
+  b.done = reinterpret_cast<unsigned*>(W + L.w_sync + 128);
+  b.amax = reinterpret_cast<unsigned long long*>(W + L.w_sync + 256);
+  b.max_splits = L.max_splits;
+  m->ws_tok = reinterpret_cast<int32_t*>(W + L.w_tok);
+  m->ws_g = reinterpret_cast<int32_t*>(W + L.w_g);
+  m->ws_n = reinterpret_cast<int32_t*>(W + L.w_n);
+  m->ws_snap = c.max_draft > 0 ? W + L.w_snap : nullptr;
+  m->snap_S_bytes = L.snap_S;
+  m->snap_conv_bytes = L.snap_conv;
+  *out = m;
+  return MK_OK;
+}
+
+int mk_reset_state(mk_model* m, void* stream) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(m->state, 0, m->sz.state_bytes, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(m->ws, 0, 1024, s);   // barrier, arrival and argmax words
+  if (e != cudaSuccess) return cuda_fail(e, "reset");
+  m->pos_hint = 0;
+  return MK_OK;
+}
+
+int mk_set_position(mk_model* m, int32_t pos, void* stream) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  if (pos < 0 || pos > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "position outside [0, max_ctx]");
+  mk::set_int_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(m->base.pos, pos);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "set position");
+  ++m->launches;
+  m->pos_hint = pos;
+  return MK_OK;
+}
+
+int mk_decode_step(mk_model* m, const int32_t* d_in_token, int32_t* d_out_token, float* d_logits, void* stream) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  if (!d_in_token || !d_out_token) return fail(MK_ERR_ARG, "token pointer is NULL");
+  if (m->pos_hint + 1 > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "context capacity reached");
+  return launch_step(m, d_in_token, d_out_token, d_logits, static_cast<cudaStream_t>(stream));
+}
+
+int mk_prefill(mk_model* m, const int32_t* d_tokens, int32_t n, float* d_last_logits, int32_t* d_next_token,
+               void* stream) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  if (!d_tokens || n <= 0) return fail(MK_ERR_ARG, "no prompt tokens");
+  if (m->pos_hint + n > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "prompt exceeds the context capacity");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* sink = m->ws_tok + m->cfg.max_ctx + 4;
+  for (int i = 0; i < n; ++i) {
+    const bool last = (i == n - 1);
+    int rc = launch_step(m, d_tokens + i, last && d_next_token ? d_next_token : sink, last ? d_last_logits : nullptr, s);
+    if (rc) return rc;
+  }
+  return MK_OK;
+}
+
+int mk_verify_drafts(mk_model* m, const int32_t* d_tokens, int32_t K, int32_t* d_n_accepted, int32_t* d_out_tokens,
+                     float* d_logits, void* stream) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  if (!d_tokens || !d_n_accepted || !d_out_tokens) return fail(MK_ERR_ARG, "pointer is NULL");
+  if (K < 1 || K > m->cfg.max_draft) return fail(MK_ERR_ARG, "K outside [1, max_draft]");
+  if (m->pos_hint + K + 1 > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "drafts exceed the context capacity");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const mk::DecodeParams& b = m->base;
+  uint8_t* snapS = m->ws_snap;
+  uint8_t* snapC = snapS + align256(m->snap_S_bytes);
+  uint8_t* snapP = snapC + align256(m->snap_conv_bytes);
+  // 1. snapshot the recurrent state (S, conv history, position)
+  cudaError_t e = cudaMemcpyAsync(snapS, b.S, m->snap_S_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(snapC, b.conv_ring, m->snap_conv_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(snapP, b.pos, 4, cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "verify snapshot");
+  const int64_t pos0 = m->pos_hint;
+  // 2. score the K + 1 positions
+  for (int i = 0; i <= K; ++i) {
+    int rc = launch_step(m, d_tokens + i, m->ws_g + i,
+                         d_logits ? d_logits + static_cast<size_t>(i) * m->cfg.vocab : nullptr, s);
+    if (rc) return rc;
+  }
+  // 3. longest matching prefix + bonus token
+  mk::accept_kernel<<<1, 32, 0, s>>>(d_tokens, m->ws_g, K, m->ws_n, d_n_accepted, d_out_tokens);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "accept");
+  ++m->launches;
+  // 4. roll back and 5. replay the accepted prefix (steps past n return at once)
+  e = cudaMemcpyAsync(b.S, snapS, m->snap_S_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(b.conv_ring, snapC, m->snap_conv_bytes, cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(b.pos, snapP, 4, cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "verify rollback");
+  m->pos_hint = pos0;
+  for (int i = 0; i <= K; ++i) {
+    mk::DecodeParams p = m->base;
+    p.in_token = d_tokens + i;
+    p.out_token = m->ws_tok + m->cfg.max_ctx + 4;
+    p.logits = nullptr;
+    p.gate_n = m->ws_n;
+    p.gate_i = i;
+    e = mk::launch_decode(p, m->grid, s);
+    if (e != cudaSuccess) return cuda_fail(e, "verify replay");
+    ++m->launches;
+  }
+  m->pos_hint = pos0 + 1;   // at least one position is always committed; the exact count is on the device
+  return MK_OK;
+}
+
+int mk_generate(mk_model* m, const int32_t* h_prompt, int32_t n_prompt, int32_t* h_out, int32_t n_new, void* stream) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  if (!h_prompt || n_prompt <= 0 || !h_out || n_new <= 0) return fail(MK_ERR_ARG, "bad prompt or output buffer");
+  if (m->pos_hint + n_prompt + n_new - 1 > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "generation exceeds max_ctx");
+  if (n_prompt + n_new > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "generation exceeds max_ctx");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* d_prompt = m->ws_tok;
+  int32_t* d_gen = m->ws_tok + n_prompt;
+  cudaError_t e = cudaMemcpyAsync(d_prompt, h_prompt, sizeof(int32_t) * n_prompt, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prompt upload");
+  int rc = mk_prefill(m, d_prompt, n_prompt, nullptr, d_gen, stream);
+  if (rc) return rc;
+  for (int i = 1; i < n_new; ++i) {
+    rc = launch_step(m, d_gen + i - 1, d_gen + i, nullptr, s);
+    if (rc) return rc;
+  }
+  e = cudaMemcpyAsync(h_out, d_gen, sizeof(int32_t) * n_new, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "generate");
+  return MK_OK;
+}
+
+int mk_sync_status(mk_model* m, void* stream, int32_t* dev_err) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&word, m->base.err, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "sync");
+  if (dev_err) *dev_err = word;
+  if (word) {
+    char buf[96];
+    snprintf(buf, sizeof buf, "device error word 0x%x", word);
+    return fail(MK_ERR_DEVICE, buf);
+  }
+  return MK_OK;
+}
+
+int64_t mk_launch_count(const mk_model* m) { return m ? m->launches : 0; }
+
+const char* mk_last_error(void) { return g_err.c_str(); }
+
+void mk_free(mk_model* m) { delete m; }
+
+}  // extern "C"

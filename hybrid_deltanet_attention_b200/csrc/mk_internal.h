@@ -1,0 +1,77 @@
+// Internal definitions shared by the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mk {
+
+// Persistent decode kernel geometry: 8 consumer warps do the math, one producer
+// warp streams this CTA's weights through a ring of shared-memory slots with bulk
+// asynchronous copies (cp.async.bulk, no multicast).
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kSlotBytes = 32768;
+constexpr int kSlots = 6;
+constexpr int kScratchFloats = 4096;
+constexpr int kAttnSub = 64;          // positions per online-softmax sub-block
+constexpr int kAttnMinChunk = 32;     // smallest split-K chunk of the KV cache
+
+enum LayerKind : int { kDeltaNet = 0, kAttention = 1 };
+
+// Per-layer device pointers into the packed weight buffer.
+struct LayerW {
+  int kind;
+  int idx;                  // index among layers of the same kind
+  const uint16_t* norm1;    // [H] bf16
+  const uint16_t* norm2;    // [H] bf16
+  const uint8_t* w_in;      // [in_rows][row_bytes]      (row-major [out, in])
+  const uint16_t* conv;     // [C][W] bf16 (DeltaNet)
+  const uint8_t* w_outT;    // [K_mix][row_bytes]       transposed: row j = column j of W_out
+  const uint8_t* w_gate;    // [F][row_bytes]
+  const uint8_t* w_up;      // [F][row_bytes]
+  const uint8_t* w_downT;   // [F][row_bytes]           transposed: row j = column j of W_down
+};
+
+struct DecodeParams {
+  const LayerW* layers;     // device array [n_layers]
+  int n_layers;
+  const uint8_t* embed;     // [V][row_bytes]
+  const uint16_t* norm_f;   // [H]
+  const double* inv_freq;   // [D/2] RoPE frequencies theta^(-2i/D)
+  // shape
+  int H, V, F, Hd, dk, dv, convw, C, Hq, Hkv, D, gated, at_in_rows, max_ctx, row_bytes;
+  float eps;
+  // state (caller-owned)
+  float* S;                 // [n_dn][Hd][dv][dk]
+  float* conv_ring;         // [n_dn][W][C]
+  uint16_t* kc;             // [n_at][Hkv][max_ctx][D]
+  uint16_t* vc;
+  int* pos;
+  int* err;
+  // workspace (caller-owned)
+  float* hbuf;              // [3][H] rotating residual buffers
+  float* z;                 // projection outputs not kept in the conv history
+  float* part;              // attention split-K partials [Hq][max_splits][D + 2]
+  unsigned* bar;            // grid barrier counter
+  unsigned* done;           // end-of-step arrival counter
+  unsigned long long* amax; // packed (logit, index) maximum
+  int max_splits;
+  // per-call io
+  const int* in_token;
+  int* out_token;
+  float* logits;            // may be null
+  // optional gate: when gate_n != null and gate_i > *gate_n the launch does nothing
+  // (used to replay only the accepted prefix of a verify pass without a host round trip)
+  const int* gate_n;
+  int gate_i;
+};
+
+size_t decode_smem_bytes(int H);
+cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s);
+int decode_max_splits(int grid, int hkv);
+
+// repack helpers (api.cu launches them)
+cudaError_t launch_transpose_bf16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t s);
+
+}  // namespace mk
