@@ -228,9 +228,9 @@ __device__ __forceinline__ float cons_sum(float v, Shared* sh, int warp, int lan
   return warp_sum(t);
 }
 
-// xs = bf16( h / sqrt(mean(h^2) + eps) * gamma )
+// xs = h / sqrt(mean(h^2) + eps) * gamma   (fp32, kept on chip)
 __device__ void rmsnorm_to_smem(const DecodeParams& p, const float* h, bool h_is_bf16_row, const uint8_t* bf_row,
-                                const uint16_t* gamma, uint16_t* xs, Shared* sh, int tid, int warp, int lane) {
+                                const uint16_t* gamma, float* xs, Shared* sh, int tid, int warp, int lane) {
   float ss = 0.f;
   for (int c = tid; c < p.H; c += kConsumerThreads) {
     const float v = h_is_bf16_row ? bf16_to_f(reinterpret_cast<const uint16_t*>(bf_row)[c]) : __ldcg(h + c);
@@ -240,14 +240,15 @@ __device__ void rmsnorm_to_smem(const DecodeParams& p, const float* h, bool h_is
   const float inv = 1.0f / sqrtf(ss / static_cast<float>(p.H) + p.eps);
   for (int c = tid; c < p.H; c += kConsumerThreads) {
     const float v = h_is_bf16_row ? bf16_to_f(reinterpret_cast<const uint16_t*>(bf_row)[c]) : __ldcg(h + c);
-    xs[c] = f_to_bf16(v * inv * bf16_to_f(gamma[c]));
+    xs[c] = v * inv * bf16_to_f(gamma[c]);
   }
   cons_sync(kConsumerThreads);
 }
 
-// Warp-per-row dot products of a chunk of bf16 rows with xs; f(row, value) runs on lane 0.
+// Warp-per-row dot products of a chunk of bf16 rows with the fp32 vector xs;
+// f(row, value) runs on lane 0.
 template <class F>
-__device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int nrows, int rb, const uint16_t* xs, int H,
+__device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int nrows, int rb, const float* xs, int H,
                                            int warp, int lane, F&& f) {
   int r = warp;
   for (; r + kConsumerWarps < nrows; r += 2 * kConsumerWarps) {
@@ -255,9 +256,10 @@ __device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int nrows, int 
     const uint8_t* r1 = r0 + static_cast<size_t>(kConsumerWarps) * rb;
     float a0 = 0.f, a1 = 0.f;
     for (int c = lane * 8; c < H; c += 256) {
-      const uint4 x = *reinterpret_cast<const uint4*>(xs + c);
-      a0 = dot8_bf16(*reinterpret_cast<const uint4*>(r0 + 2 * c), x, a0);
-      a1 = dot8_bf16(*reinterpret_cast<const uint4*>(r1 + 2 * c), x, a1);
+      const float4 xa = *reinterpret_cast<const float4*>(xs + c);
+      const float4 xb = *reinterpret_cast<const float4*>(xs + c + 4);
+      a0 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(r0 + 2 * c), xa, xb, a0);
+      a1 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(r1 + 2 * c), xa, xb, a1);
     }
     a0 = warp_sum(a0);
     a1 = warp_sum(a1);
@@ -267,7 +269,8 @@ __device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int nrows, int 
     const uint8_t* r0 = chunk + static_cast<size_t>(r) * rb;
     float a0 = 0.f;
     for (int c = lane * 8; c < H; c += 256)
-      a0 = dot8_bf16(*reinterpret_cast<const uint4*>(r0 + 2 * c), *reinterpret_cast<const uint4*>(xs + c), a0);
+      a0 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(r0 + 2 * c), *reinterpret_cast<const float4*>(xs + c),
+                         *reinterpret_cast<const float4*>(xs + c + 4), a0);
     a0 = warp_sum(a0);
     if (lane == 0) f(r, a0);
   }
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   uint8_t* ring = smem;
   Shared* sh = reinterpret_cast<Shared*>(smem + static_cast<size_t>(kSlots) * kSlotBytes);
   float* fs = reinterpret_cast<float*>(sh + 1);                          // scratch [kScratchFloats]
-  uint16_t* xs = reinterpret_cast<uint16_t*>(fs + kScratchFloats);       // normed input [H] bf16
+  float* xs = fs + kScratchFloats;                                       // normed input [H] fp32
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x, G = gridDim.x;
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
                   }
                 }
                 o = warp_sum(o);
-                if (lane == 0) oc[lr] = round_bf16(o);
+                if (lane == 0) oc[lr] = o;
               }
               release(cs);
             }
@@ -698,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
           }
           float o = O / Ls;
           if (p.gated) o *= sigmoidf_(__ldcg(p.z + p.Hq * p.D + col));
-          oc[cc] = round_bf16(o);
+          oc[cc] = o;
         }
         cons_sync(kConsumerThreads);
         if (ns) {
@@ -736,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
                 gemv_chunk(ch, nr, rb, xs, p.H, warp, lane, [&](int r, float v) { gs[r0 + r] = v; });
               } else {
                 gemv_chunk(ch, nr, rb, xs, p.H, warp, lane,
-                           [&](int r, float v) { act[r0 + r] = round_bf16(siluf_(gs[r0 + r]) * v); });
+                           [&](int r, float v) { act[r0 + r] = siluf_(gs[r0 + r]) * v; });
               }
               release(cs);
             }
@@ -815,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
 
 size_t decode_smem_bytes(int H) {
   return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + kScratchFloats * sizeof(float) +
-         static_cast<size_t>(H) * 2;
+         static_cast<size_t>(H) * 4;
 }
 
 int decode_max_splits(int grid, int hkv) {

@@ -126,6 +126,19 @@ __device__ __forceinline__ float dot8_bf16(const uint4 w, const uint4 x, float a
   return acc;
 }
 
+// 8 bf16 weights (one uint4) dotted with 8 fp32 activations.
+__device__ __forceinline__ float dot8_bf16_f32(const uint4 w, const float4 a, const float4 b, float acc) {
+  acc = fmaf(bf16lo(w.x), a.x, acc);
+  acc = fmaf(bf16hi(w.x), a.y, acc);
+  acc = fmaf(bf16lo(w.y), a.z, acc);
+  acc = fmaf(bf16hi(w.y), a.w, acc);
+  acc = fmaf(bf16lo(w.z), b.x, acc);
+  acc = fmaf(bf16hi(w.z), b.y, acc);
+  acc = fmaf(bf16lo(w.w), b.z, acc);
+  acc = fmaf(bf16hi(w.w), b.w, acc);
+  return acc;
+}
+
 // Ordered key for a float so that unsigned comparison follows float order.
 __device__ __forceinline__ uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f);

@@ -13,7 +13,7 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kSlotBytes = 32768;
 constexpr int kSlots = 6;
-constexpr int kScratchFloats = 4096;
+constexpr int kScratchFloats = 3072;
 constexpr int kAttnSub = 64;          // positions per online-softmax sub-block
 constexpr int kAttnMinChunk = 32;     // smallest split-K chunk of the KV cache
 

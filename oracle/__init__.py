@@ -9,12 +9,12 @@ with float64 arithmetic, token by token (the recurrent form), with one
 library primitive per step (matrix-vector products, a triangular solve).
 It shares no code with the CUDA path; both read their inputs from ``synth``.
 
-Rounding contract (the megakernel post's "BF16 weights and activations, FP32
-accumulation"): weights are bf16; the vectors that feed a projection (the
-normalised hidden state, the mixer output, the SwiGLU activation) and the KV
-cache entries are rounded to bf16; everything else stays in full precision
-(float64 here, float32 on the GPU). ``round_inputs=False`` drops the bf16
-rounding of activations for diagnostics.
+Rounding contract: weights are bf16 and the KV cache entries are stored in bf16;
+every other quantity stays in full precision (float64 here, float32 on the GPU,
+where activations live in registers and shared memory and never leave the chip).
+``act_bf16=True`` additionally rounds every projection input (normalised hidden
+state, mixer output, SwiGLU activation) to bf16 -- the megakernel post's "BF16
+weights and activations" taken literally -- for diagnostics.
 """
 from .model import *          # noqa: F401,F403
 from .chunked import *        # noqa: F401,F403

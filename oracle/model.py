@@ -198,7 +198,7 @@ def _deltanet_mixer(cfg, W, p, st: OracleState, li: int, x: np.ndarray) -> np.nd
     return o.reshape(-1)
 
 
-def _attention_mixer(cfg, W, p, st: OracleState, li: int, x: np.ndarray, rnd) -> np.ndarray:
+def _attention_mixer(cfg, W, p, st: OracleState, li: int, x: np.ndarray) -> np.ndarray:
     Hq, Hkv, D = cfg.at_q_heads, cfg.at_kv_heads, cfg.at_head_dim
     z = W[p + "attn.w_in"] @ x                                 # [q; gate; k; v]
     off = 0
@@ -210,17 +210,22 @@ def _attention_mixer(cfg, W, p, st: OracleState, li: int, x: np.ndarray, rnd) ->
     pos = st.pos
     q = rope(q, pos, cfg.rope_theta)
     k = rope(k, pos, cfg.rope_theta)
-    st.K[li][:, pos] = rnd(k)
-    st.V[li][:, pos] = rnd(v)
+    st.K[li][:, pos] = round_bf16(k)          # the KV cache is stored in bf16
+    st.V[li][:, pos] = round_bf16(v)
     o = attention_decode(q, st.K[li][:, :pos + 1], st.V[li][:, :pos + 1]).reshape(-1)
     if cfg.at_out_gate:
         o = o * sigmoid(g)
     return o
 
 
-def decode_step(cfg, W, st: OracleState, tok: int, round_inputs: bool = True) -> np.ndarray:
-    """Feed one token at position st.pos; returns the logits [vocab] and advances pos."""
-    rnd = round_bf16 if round_inputs else (lambda a: a)
+def decode_step(cfg, W, st: OracleState, tok: int, act_bf16: bool = False) -> np.ndarray:
+    """Feed one token at position st.pos; returns the logits [vocab] and advances pos.
+
+    The KV cache entries are always bf16 (stored state). act_bf16=True also rounds
+    every projection input (normed hidden state, mixer output, SwiGLU activation)
+    to bf16; by default they stay in full precision, as on the GPU, where they never
+    leave the chip."""
+    rnd = round_bf16 if act_bf16 else (lambda a: a)
     eps = cfg.rms_eps
     if st.K and st.pos >= st.K[0].shape[1]:
         raise ValueError("context capacity exceeded")
@@ -233,7 +238,7 @@ def decode_step(cfg, W, st: OracleState, tok: int, round_inputs: bool = True) ->
             o = _deltanet_mixer(cfg, W, p, st, di, x); di += 1
             h = h + W[p + "dn.w_out"] @ rnd(o)
         else:
-            o = _attention_mixer(cfg, W, p, st, ai, x, rnd); ai += 1
+            o = _attention_mixer(cfg, W, p, st, ai, x); ai += 1
             h = h + W[p + "attn.w_out"] @ rnd(o)
         x = rnd(rmsnorm(h, W[p + "norm2"], eps))
         h = h + W[p + "mlp.w_down"] @ rnd(swiglu(x, W[p + "mlp.w_gate"], W[p + "mlp.w_up"]))
@@ -242,15 +247,15 @@ def decode_step(cfg, W, st: OracleState, tok: int, round_inputs: bool = True) ->
     return W["embed"] @ x
 
 
-def prefill(cfg, W, st: OracleState, tokens, round_inputs: bool = True) -> np.ndarray:
+def prefill(cfg, W, st: OracleState, tokens, act_bf16: bool = False) -> np.ndarray:
     """Feed a prompt token by token; returns the logits after the last one."""
     logits = None
     for t in tokens:
-        logits = decode_step(cfg, W, st, int(t), round_inputs)
+        logits = decode_step(cfg, W, st, int(t), act_bf16)
     return logits
 
 
-def greedy_generate(cfg, W, st: OracleState, first_tok: int, n: int, round_inputs: bool = True,
+def greedy_generate(cfg, W, st: OracleState, first_tok: int, n: int, act_bf16: bool = False,
                     keep_logits: bool = False):
     """Greedy decode of n tokens starting from first_tok (fed at st.pos).
 
@@ -260,7 +265,7 @@ def greedy_generate(cfg, W, st: OracleState, first_tok: int, n: int, round_input
     out, lg = [], []
     tok = int(first_tok)
     for _ in range(n):
-        z = decode_step(cfg, W, st, tok, round_inputs)
+        z = decode_step(cfg, W, st, tok, act_bf16)
         tok = int(np.argmax(z))          # first maximal index = lowest index on ties
         out.append(tok)
         if keep_logits:
@@ -268,7 +273,7 @@ def greedy_generate(cfg, W, st: OracleState, first_tok: int, n: int, round_input
     return np.array(out, dtype=np.int32), (lg if keep_logits else None)
 
 
-def verify_drafts(cfg, W, st: OracleState, last_tok: int, drafts, round_inputs: bool = True):
+def verify_drafts(cfg, W, st: OracleState, last_tok: int, drafts, act_bf16: bool = False):
     """Speculative verify by its plain definition (exact greedy acceptance).
 
     Feeds [last_tok, d_1..d_K] one at a time on a copy of the state, recording
@@ -283,7 +288,7 @@ def verify_drafts(cfg, W, st: OracleState, last_tok: int, drafts, round_inputs: 
     feed = [int(last_tok)] + drafts
     g, logits = [], []
     for t in feed:
-        z = decode_step(cfg, W, trial, t, round_inputs)
+        z = decode_step(cfg, W, trial, t, act_bf16)
         logits.append(z)
         g.append(int(np.argmax(z)))
     n = 0
@@ -291,5 +296,5 @@ def verify_drafts(cfg, W, st: OracleState, last_tok: int, drafts, round_inputs: 
         n += 1
     committed = drafts[:n] + [g[n]]
     for t in feed[:n + 1]:
-        decode_step(cfg, W, st, t, round_inputs)
+        decode_step(cfg, W, st, t, act_bf16)
     return n, np.array(committed, dtype=np.int32), np.stack(logits)

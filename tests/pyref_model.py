@@ -57,9 +57,10 @@ class PyModel:
         self.V = [[] for _ in range(c.n_at)]
         self.pos = 0
 
-    def step(self, tok, rnd=True):
+    def step(self, tok, act=False):
+        """act=True also rounds every projection input to bf16; the KV cache is always bf16."""
         c, W = self.c, self.W
-        r = bf16 if rnd else (lambda v: v)
+        r = bf16 if act else (lambda v: v)
         h = list(W["embed"][tok])
         di = ai = 0
         for l, kind in enumerate(c.pattern):
@@ -70,7 +71,7 @@ class PyModel:
                 di += 1
                 h = [a + b for a, b in zip(h, matvec(W[p + "dn.w_out"], [r(v) for v in o]))]
             else:
-                o = self._at(p, ai, x, r)
+                o = self._at(p, ai, x)
                 ai += 1
                 h = [a + b for a, b in zip(h, matvec(W[p + "attn.w_out"], [r(v) for v in o]))]
             x = [r(v) for v in rms(h, W[p + "norm2"], c.rms_eps)]
@@ -117,7 +118,7 @@ class PyModel:
             out += [math.fsum(S[i][j] * q[j] for j in range(dk)) for i in range(dv)]
         return out
 
-    def _at(self, p, li, x, r):
+    def _at(self, p, li, x):
         c, W = self.c, self.W
         Hq, Hkv, D = c.at_q_heads, c.at_kv_heads, c.at_head_dim
         z = matvec(W[p + "attn.w_in"], x)
@@ -141,8 +142,8 @@ class PyModel:
             return o
 
         qs = [rot(q[h * D:(h + 1) * D], self.pos) for h in range(Hq)]
-        ks = [[r(t) for t in rot(k[h * D:(h + 1) * D], self.pos)] for h in range(Hkv)]
-        vs = [[r(t) for t in v[h * D:(h + 1) * D]] for h in range(Hkv)]
+        ks = [[bf16(t) for t in rot(k[h * D:(h + 1) * D], self.pos)] for h in range(Hkv)]
+        vs = [[bf16(t) for t in v[h * D:(h + 1) * D]] for h in range(Hkv)]
         self.K[li].append(ks)
         self.V[li].append(vs)
         out = []

@@ -18,15 +18,15 @@ def mini():
     return raw, oracle.prepare_weights(MINI, raw)
 
 
-@pytest.mark.parametrize("rnd", [True, False])
-def test_oracle_matches_independent_python_model(mini, rnd):
+@pytest.mark.parametrize("act", [False, True])
+def test_oracle_matches_independent_python_model(mini, act):
     raw, W = mini
     py = PyModel(MINI, raw)
     st = oracle.new_state(MINI, 32)
     toks = [3, 17, 60, 0, 41, 41, 9]
     for t in toks:
-        z_or = oracle.decode_step(MINI, W, st, t, round_inputs=rnd)
-        z_py = np.array(py.step(t, rnd))
+        z_or = oracle.decode_step(MINI, W, st, t, act_bf16=act)
+        z_py = np.array(py.step(t, act))
         np.testing.assert_allclose(z_or, z_py, rtol=1e-9, atol=1e-12)
     # states too
     for li in range(MINI.n_dn):
