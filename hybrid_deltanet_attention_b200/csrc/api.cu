@@ -3,6 +3,7 @@
 // provides device memory and a stream.
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <string>
@@ -123,7 +124,7 @@ int check_config(const mk_config* c) {
   if (nd) {
     if (c->dn_heads <= 0 || c->dn_dk <= 0 || c->dn_dk % 32 || c->dn_dk > 256 || c->dn_dv <= 0 || c->dn_dv > 256)
       return fail(MK_ERR_ARG, "DeltaNet dims: dk must be a multiple of 32 and <= 256, 0 < dv <= 256");
-    if (c->conv_width < 2 || c->conv_width > 8) return fail(MK_ERR_ARG, "conv_width must be in [2, 8]");
+    if (c->conv_width < 2 || c->conv_width > 4) return fail(MK_ERR_ARG, "conv_width must be in [2, 4]");
   }
   if (na) {
     if (c->at_q_heads <= 0 || c->at_kv_heads <= 0 || c->at_q_heads % c->at_kv_heads)
@@ -151,18 +152,23 @@ int device_grid(int* grid, int* dev) {
 
 // Scratch and shared-memory budget checks that depend on the grid size.
 int check_budget(const mk_config& c, int grid) {
-  if (mk::decode_smem_bytes(c.hidden) > 232448) return fail(MK_ERR_ARG, "shared-memory budget exceeded");
+  const long S = static_cast<long>(mk::decode_scratch_floats(c.hidden));
+  if (S < 256) return fail(MK_ERR_ARG, "shared-memory budget exceeded (hidden too large)");
   auto ceil_div = [](long a, long b) { return (a + b - 1) / b; };
-  const long S = mk::kScratchFloats;
   if (n_kind(c, 'D')) {
     const long rows = ceil_div(static_cast<long>(c.dn_heads) * c.dn_dv, grid);
     const long nh = ceil_div(rows, c.dn_dv) + 1;
     if (nh * (2 * c.dn_dk + 2) + 2 * rows > S) return fail(MK_ERR_ARG, "DeltaNet rows per CTA exceed the scratch budget");
+    if (2 * nh * c.dn_dk + rows + nh > 3L * mk::kConsumerThreads)
+      return fail(MK_ERR_ARG, "DeltaNet conv channels per CTA exceed the prologue budget");
   }
   if (n_kind(c, 'A')) {
     const long grp = c.at_q_heads / c.at_kv_heads;
-    if (grp * c.at_head_dim + grp * mk::kAttnSub + 3 * grp > S) return fail(MK_ERR_ARG, "attention scratch budget exceeded");
-    if (ceil_div(static_cast<long>(c.at_q_heads) * c.at_head_dim, grid) > S)
+    if (2 * grp * c.at_head_dim + grp * mk::kAttnSub + 3 * grp + 2 * c.at_head_dim > S)
+      return fail(MK_ERR_ARG, "attention scratch budget exceeded");
+    const long cols = ceil_div(static_cast<long>(c.at_q_heads) * c.at_head_dim, grid);
+    const long nhd = ceil_div(cols, c.at_head_dim) + 1;
+    if (nhd * mk::decode_max_splits(grid, c.at_kv_heads) + 2 * cols > S)
       return fail(MK_ERR_ARG, "attention columns per CTA exceed the scratch budget");
   }
   if (2 * ceil_div(c.ffn, grid) > S) return fail(MK_ERR_ARG, "MLP rows per CTA exceed the scratch budget");
@@ -227,7 +233,7 @@ Layout make_layout(const mk_config& c, int grid) {
   L.max_splits = (na ? mk::decode_max_splits(grid, c.at_kv_heads) : 1);
   off = 0;
   L.w_sync = off; off = align256(off + 1024);
-  L.w_h = off; off = align256(off + 3 * H * 4);
+  L.w_h = off; off = align256(off + 5 * H * 4);   // residual: 2 bases + 3 deltas
   const size_t zf = std::max<size_t>(2 * c.dn_heads,
                                      na ? static_cast<size_t>(c.at_q_heads) * c.at_head_dim * (c.at_out_gate ? 2 : 1) +
                                               2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim
@@ -474,6 +480,8 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   b.done = reinterpret_cast<unsigned*>(W + L.w_sync + 128);
   b.amax = reinterpret_cast<unsigned long long*>(W + L.w_sync + 256);
   b.max_splits = L.max_splits;
+  b.prefetch_bytes = 384 * 1024;
+  if (const char* env = getenv("MK_PREFETCH_KB")) b.prefetch_bytes = atoi(env) * 1024;
   m->ws_tok = reinterpret_cast<int32_t*>(W + L.w_tok);
   m->ws_g = reinterpret_cast<int32_t*>(W + L.w_g);
   m->ws_n = reinterpret_cast<int32_t*>(W + L.w_n);
@@ -611,6 +619,14 @@ int mk_sync_status(mk_model* m, void* stream, int32_t* dev_err) {
     snprintf(buf, sizeof buf, "device error word 0x%x", word);
     return fail(MK_ERR_DEVICE, buf);
   }
+  return MK_OK;
+}
+
+int mk_phase_trace(mk_model* m, uint64_t* d_trace, int32_t capacity) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  if (d_trace && capacity <= 0) return fail(MK_ERR_ARG, "capacity must be positive");
+  m->base.trace = reinterpret_cast<unsigned long long*>(d_trace);
+  m->base.trace_cap = d_trace ? capacity : 0;
   return MK_OK;
 }
 

@@ -1,17 +1,20 @@
 // Persistent decode megakernel: one launch runs every layer of one batch-1 forward step.
 //
-// Design (the Hacker News post on the fused Qwen3.5-0.8B kernel, design bullets,
-// is the prior art: one launch per token, persistent blocks on every SM, a grid-wide
+// Design (the Hacker News post on the fused Qwen3.5-0.8B kernel, design bullets, is
+// the prior art: one launch per token, persistent blocks on every SM, a grid-wide
 // barrier instead of kernel boundaries; re-done here for sm_100a):
 //  * grid = one CTA per SM (cooperative launch, so all CTAs are co-resident);
-//  * each CTA owns a fixed contiguous slice of every weight matrix; a producer warp
-//    streams the CTA's whole per-step weight sequence through a 6 x 32 KB shared-memory
-//    ring with cp.async.bulk, independent of the grid barriers, so HBM stays busy while
-//    the consumer warps wait at a barrier;
-//  * 8 consumer warps do the arithmetic in fp32 from shared memory;
+//  * each CTA owns a fixed contiguous slice of every weight matrix, of the DeltaNet
+//    state rows, and of the KV cache positions of its attention split. Its slice
+//    bounds are computed once per launch into shared memory. A producer lane streams
+//    that whole per-step sequence through a 6 x 32 KB shared-memory ring with
+//    cp.async.bulk (no multicast), independent of the grid barriers; its per-chunk
+//    work is a handful of instructions so it never limits the stream;
+//  * 8 consumer warps do the arithmetic in fp32 from shared memory; activations never
+//    leave the chip except the small vectors exchanged between phases (L2);
 //  * out-projections and the MLP down-projection are split over their input dim
-//    (split-K) and accumulated into the residual with vector atomics, so a DeltaNet
-//    layer needs 3 grid barriers and an attention layer 4;
+//    (split-K) and added to the residual with vector reductions, so a DeltaNet layer
+//    needs 3 grid barriers and an attention layer 4;
 //  * every wait (grid barrier, pipeline slot) has a time limit; on expiry the kernel
 //    latches a bit in the device error word and every CTA returns.
 #include "dev.cuh"
@@ -22,14 +25,20 @@ namespace mk {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s: a healthy wait takes microseconds
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 200 ms for in-flight copies to land
-constexpr int kMaxGroups = 8;                      // float4 groups per thread: H <= 8192
+constexpr int kMaxConv = 4;          // causal conv width limit (the configs use 4)
+constexpr int kConvItems = 3;        // conv items per consumer thread in the DeltaNet prologue
+constexpr int kNoSplit = 0x7FFFFFFF;
 
-enum Phase : int { kPhIn = 0, kPhMix = 1, kPhAttOut = 2, kPhMlp = 3, kPhFinal = 4 };
-
-struct Seg {
-  const uint8_t* src;
-  int rows;
-  int row_bytes;
+// Per-CTA slice bounds, computed once per launch by thread 0.
+struct Ranges {
+  int in_dn_b, in_dn_e;   // DeltaNet in-projection rows
+  int in_at_b, in_at_e;   // attention in-projection rows
+  int dn_b, dn_e;         // DeltaNet state rows (head*dv + i) and out-projection columns
+  int col_b, col_e;       // attention output columns (out-projection split-K)
+  int f_b, f_e;           // MLP intermediate rows
+  int v_b, v_e;           // LM-head rows
+  int au_valid, au_g, au_j, au_p0, au_p1, au_q1;   // attention split unit
+  int nsplit;
 };
 
 struct __align__(16) Shared {
@@ -43,6 +52,7 @@ struct __align__(16) Shared {
   float red[kConsumerWarps];
   float best_v[kConsumerWarps];
   int best_i[kConsumerWarps];
+  Ranges rg;
 };
 
 __device__ __forceinline__ void split_range(int n, int c, int G, int& b, int& e) {
@@ -50,6 +60,8 @@ __device__ __forceinline__ void split_range(int n, int c, int G, int& b, int& e)
   e = static_cast<int>((static_cast<long long>(n) * (c + 1)) / G);
 }
 
+// Split of the n = pos + 1 cached positions into chunks of CH positions so that
+// Hkv * nsplit <= grid (every CTA owns at most one (kv head, chunk) unit).
 __device__ __forceinline__ void attn_split(int n, int G, int Hkv, int max_splits, int& CH, int& nsplit) {
   int per = G / Hkv;
   if (per < 1) per = 1;
@@ -61,139 +73,179 @@ __device__ __forceinline__ void attn_split(int n, int G, int Hkv, int max_splits
   nsplit = (n + ch - 1) / ch;
 }
 
-// The weight (and DeltaNet-state) rows a CTA streams in one phase. Producer and
-// consumers both call this, so they agree on the chunk sequence.
-__device__ int phase_segments(const DecodeParams& p, const LayerW& L, int phase, int cta, int G, Seg* s) {
-  const int rb = p.row_bytes;
-  int b, e, n = 0;
-  switch (phase) {
-    case kPhIn: {
-      const int rows = (L.kind == kDeltaNet) ? (p.C + 2 * p.Hd) : p.at_in_rows;
-      split_range(rows, cta, G, b, e);
-      if (e > b) s[n++] = {L.w_in + static_cast<size_t>(b) * rb, e - b, rb};
-      break;
-    }
-    case kPhMix: {
-      if (L.kind != kDeltaNet) break;
-      split_range(p.Hd * p.dv, cta, G, b, e);
-      if (e > b) {
-        const float* S = p.S + (static_cast<size_t>(L.idx) * p.Hd * p.dv + b) * p.dk;
-        s[n++] = {reinterpret_cast<const uint8_t*>(S), e - b, p.dk * 4};
-        s[n++] = {L.w_outT + static_cast<size_t>(b) * rb, e - b, rb};
-      }
-      break;
-    }
-    case kPhAttOut: {
-      split_range(p.Hq * p.D, cta, G, b, e);
-      if (e > b) s[n++] = {L.w_outT + static_cast<size_t>(b) * rb, e - b, rb};
-      break;
-    }
-    case kPhMlp: {
-      split_range(p.F, cta, G, b, e);
-      if (e > b) {
-        s[n++] = {L.w_gate + static_cast<size_t>(b) * rb, e - b, rb};
-        s[n++] = {L.w_up + static_cast<size_t>(b) * rb, e - b, rb};
-        s[n++] = {L.w_downT + static_cast<size_t>(b) * rb, e - b, rb};
-      }
-      break;
-    }
-    default: {   // final: LM head rows (tied embedding)
-      split_range(p.V, cta, G, b, e);
-      if (e > b) s[n++] = {p.embed + static_cast<size_t>(b) * rb, e - b, rb};
-      break;
-    }
+__device__ void compute_ranges(const DecodeParams& p, int cta, int G, int pos, Ranges& r) {
+  split_range(p.C + 2 * p.Hd, cta, G, r.in_dn_b, r.in_dn_e);
+  split_range(p.at_in_rows, cta, G, r.in_at_b, r.in_at_e);
+  split_range(p.Hd * p.dv, cta, G, r.dn_b, r.dn_e);
+  split_range(p.Hq * p.D, cta, G, r.col_b, r.col_e);
+  split_range(p.F, cta, G, r.f_b, r.f_e);
+  split_range(p.V, cta, G, r.v_b, r.v_e);
+  const int n = pos + 1;
+  int CH = 1, nsplit = 1;
+  if (p.Hkv > 0) attn_split(n, G, p.Hkv, p.max_splits, CH, nsplit);
+  r.nsplit = nsplit;
+  r.au_valid = (p.Hkv > 0 && cta < p.Hkv * nsplit) ? 1 : 0;
+  if (r.au_valid) {
+    r.au_g = cta % p.Hkv;
+    r.au_j = cta / p.Hkv;
+    r.au_p0 = r.au_j * CH;
+    r.au_p1 = min(n, r.au_p0 + CH);
+    r.au_q1 = min(r.au_p1, pos);
+  } else {
+    r.au_g = r.au_j = r.au_p0 = r.au_p1 = r.au_q1 = 0;
   }
-  return n;
 }
 
-__device__ __forceinline__ int n_phases(const LayerW& L) { return L.kind == kDeltaNet ? 3 : 4; }
-__device__ __forceinline__ int phase_id(const LayerW& L, int k) {
-  if (L.kind == kDeltaNet) return k == 0 ? kPhIn : (k == 1 ? kPhMix : kPhMlp);
-  return k == 0 ? kPhIn : (k == 1 ? kPhMix : (k == 2 ? kPhAttOut : kPhMlp));
+// Diagnostics (off unless p.trace is set): CTA 0 stamps its SM cycle counter. Entries
+// below kTraceChunks: phase boundaries; from kTraceChunks: chunk n issued (4n), warp 0
+// starts waiting for it (4n+1), has it (4n+2), is done with it (4n+3).
+constexpr int kTraceChunks = 512;
+__device__ __forceinline__ void trace_at(const DecodeParams& p, int idx) {
+  if (p.trace && blockIdx.x == 0 && idx < p.trace_cap) p.trace[idx] = clock64();
 }
 
 // ------------------------------------------------------------------ producer
-__device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring, int cta, int G) {
+// Segment s of layer l in stream order (weights, DeltaNet state rows, KV sub-blocks);
+// returns false past the end of the layer. The final "layer" p.n_layers is the LM head.
+__device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Ranges& r, const LayerW& L, int l, int s,
+                                              const uint8_t*& src, int& rows, int& rb) {
+  const int wrb = p.row_bytes;
+  if (l == p.n_layers) {
+    if (s > 0) return false;
+    src = p.embed + static_cast<size_t>(r.v_b) * wrb;
+    rows = r.v_e - r.v_b;
+    rb = wrb;
+    return true;
+  }
+  const int nkv = (L.kind == kAttention && r.au_valid && r.au_q1 > r.au_p0)
+                      ? 2 * ((r.au_q1 - r.au_p0 + kAttnSub - 1) / kAttnSub) : 0;
+  // order: in-proj | (S rows, out^T rows) or (KV sub-blocks..., out^T rows) | gate | up | down^T
+  if (s == 0) {
+    const int b = L.kind == kDeltaNet ? r.in_dn_b : r.in_at_b;
+    const int e = L.kind == kDeltaNet ? r.in_dn_e : r.in_at_e;
+    src = L.w_in + static_cast<size_t>(b) * wrb;
+    rows = e - b;
+    rb = wrb;
+    return true;
+  }
+  s -= 1;
+  if (L.kind == kDeltaNet) {
+    if (s == 0) {
+      src = reinterpret_cast<const uint8_t*>(p.S + (static_cast<size_t>(L.idx) * p.Hd * p.dv + r.dn_b) * p.dk);
+      rows = r.dn_e - r.dn_b;
+      rb = p.dk * 4;
+      return true;
+    }
+    if (s == 1) {
+      src = L.w_outT + static_cast<size_t>(r.dn_b) * wrb;
+      rows = r.dn_e - r.dn_b;
+      rb = wrb;
+      return true;
+    }
+    s -= 2;
+  } else {
+    if (s < nkv) {
+      const int sb = r.au_p0 + (s >> 1) * kAttnSub;
+      const uint16_t* base = ((s & 1) ? p.vc : p.kc) +
+                             (static_cast<size_t>(L.idx) * p.Hkv + r.au_g) * p.max_ctx * p.D +
+                             static_cast<size_t>(sb) * p.D;
+      src = reinterpret_cast<const uint8_t*>(base);
+      rows = min(kAttnSub, r.au_q1 - sb);
+      rb = p.D * 2;
+      return true;
+    }
+    s -= nkv;
+    if (s == 0) {
+      src = L.w_outT + static_cast<size_t>(r.col_b) * wrb;
+      rows = r.col_e - r.col_b;
+      rb = wrb;
+      return true;
+    }
+    s -= 1;
+  }
+  if (s < 3) {
+    const uint8_t* m = s == 0 ? L.w_gate : (s == 1 ? L.w_up : L.w_downT);
+    src = m + static_cast<size_t>(r.f_b) * wrb;
+    rows = r.f_e - r.f_b;
+    rb = wrb;
+    return true;
+  }
+  return false;
+}
+
+// One lane streams the CTA's chunks into the shared-memory ring.
+__device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) {
   const uint64_t pol = policy_evict_first();
-  uint32_t n = 0;
-  int last_in_slot[kSlots];
-#pragma unroll
-  for (int i = 0; i < kSlots; ++i) last_in_slot[i] = -1;
+  const Ranges r = sh->rg;
   volatile int* abort = &sh->abort_flag;
+  uint32_t n = 0;
   bool ok = true;
-  Seg segs[3];
+  LayerW L = p.layers[0];
   for (int l = 0; l <= p.n_layers && ok; ++l) {
-    const bool final = (l == p.n_layers);
-    const LayerW L = final ? LayerW{} : p.layers[l];
-    const int nph = final ? 1 : n_phases(L);
-    for (int k = 0; k < nph && ok; ++k) {
-      const int ph = final ? static_cast<int>(kPhFinal) : phase_id(L, k);
-      const int ns = phase_segments(p, L, ph, cta, G, segs);
-      for (int si = 0; si < ns && ok; ++si) {
-        const Seg sg = segs[si];
-        const int rpc = kSlotBytes / sg.row_bytes;
-        for (int r = 0; r < sg.rows; r += rpc) {
-          const int nr = min(rpc, sg.rows - r);
-          const uint32_t bytes = static_cast<uint32_t>(nr) * sg.row_bytes;
-          const int slot = n % kSlots;
-          if (n >= static_cast<uint32_t>(kSlots)) {
-            if (!mbar_wait(&sh->empty[slot], ((n / kSlots) - 1) & 1, abort, kWaitLimitNs)) {
-              if (!*abort) atomicOr(p.err, MK_DEVERR_PIPE_TIMEOUT);
-              *abort = 1;
-              ok = false;
-              break;
-            }
+    const LayerW Lnext = (l + 1 < p.n_layers) ? p.layers[l + 1] : L;   // load ahead of use
+    const uint8_t* src;
+    int rows, rb;
+    for (int s = 0; ok && layer_segment(p, r, L, l, s, src, rows, rb); ++s) {
+      const int rpc = kSlotBytes / rb;
+      for (int r0 = 0; r0 < rows; r0 += rpc) {
+        const uint32_t bytes = static_cast<uint32_t>(min(rpc, rows - r0)) * rb;
+        const int slot = n % kSlots;
+        if (n >= static_cast<uint32_t>(kSlots)) {
+          if (!mbar_wait(&sh->empty[slot], ((n / kSlots) - 1) & 1, abort, kWaitLimitNs)) {
+            if (!*abort) atomicOr(p.err, MK_DEVERR_PIPE_TIMEOUT);
+            *abort = 1;
+            ok = false;
+            break;
           }
-          mbar_arrive_expect_tx(&sh->full[slot], bytes);
-          bulk_g2s(ring + static_cast<size_t>(slot) * kSlotBytes, sg.src + static_cast<size_t>(r) * sg.row_bytes,
-                   bytes, &sh->full[slot], pol);
-          last_in_slot[slot] = static_cast<int>(n);
-          ++n;
         }
+        mbar_arrive_expect_tx(&sh->full[slot], bytes);
+        bulk_g2s(ring + static_cast<size_t>(slot) * kSlotBytes, src + static_cast<size_t>(r0) * rb, bytes,
+                 &sh->full[slot], pol);
+        trace_at(p, kTraceChunks + 4 * static_cast<int>(n));
+        ++n;
       }
     }
+    L = Lnext;
   }
-  // Let every issued copy land before this warp leaves (bounded).
+  // Let every issued copy land before this lane leaves (bounded): the last chunk
+  // issued to each slot is one of the last kSlots chunks.
   int never = 0;
-  for (int s = 0; s < kSlots; ++s) {
-    if (last_in_slot[s] >= 0)
-      mbar_wait(&sh->full[s], (static_cast<uint32_t>(last_in_slot[s]) / kSlots) & 1, &never, kDrainLimitNs);
-  }
+  for (uint32_t m = (n > static_cast<uint32_t>(kSlots) ? n - kSlots : 0); m < n; ++m)
+    mbar_wait(&sh->full[m % kSlots], (m / kSlots) & 1, &never, kDrainLimitNs);
 }
 
 // ------------------------------------------------------------------ consumer helpers
-struct Cons {
-  uint8_t* ring;
-  Shared* sh;
-  uint32_t n;      // next chunk index (same in all consumer threads)
-  int tid, warp, lane;
-};
-
-__device__ __forceinline__ const uint8_t* acquire(Cons& c, int* err) {
-  const int slot = c.n % kSlots;
-  if (!mbar_wait(&c.sh->full[slot], (c.n / kSlots) & 1, &c.sh->abort_flag, kWaitLimitNs)) {
-    if (c.lane == 0) {
-      if (!c.sh->abort_flag) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
-      c.sh->abort_flag = 1;
+__device__ __forceinline__ const uint8_t* acquire(const DecodeParams& p, Shared* sh, uint8_t* ring, uint32_t n,
+                                                  int tid, int lane) {
+  const int slot = n % kSlots;
+  if (tid == 0) trace_at(p, kTraceChunks + 4 * static_cast<int>(n) + 1);
+  if (!mbar_wait(&sh->full[slot], (n / kSlots) & 1, &sh->abort_flag, kWaitLimitNs)) {
+    if (lane == 0) {
+      if (!sh->abort_flag) atomicOr(p.err, MK_DEVERR_PIPE_TIMEOUT);
+      sh->abort_flag = 1;
     }
   }
-  return c.ring + static_cast<size_t>(slot) * kSlotBytes;
+  if (tid == 0) trace_at(p, kTraceChunks + 4 * static_cast<int>(n) + 2);
+  return ring + static_cast<size_t>(slot) * kSlotBytes;
 }
-__device__ __forceinline__ void release(Cons& c) {
+__device__ __forceinline__ void release(const DecodeParams& p, Shared* sh, uint32_t& n, int lane) {
+  if (threadIdx.x == 0) trace_at(p, kTraceChunks + 4 * static_cast<int>(n) + 3);
   __syncwarp();
-  if (c.lane == 0) mbar_arrive(&c.sh->empty[c.n % kSlots]);
-  ++c.n;
+  if (lane == 0) mbar_arrive(&sh->empty[n % kSlots]);
+  ++n;
 }
 
-// Grid-wide barrier among consumer thread groups of all CTAs. Returns false if this
-// CTA must stop (own or remote failure); the result is the same in every consumer thread.
-__device__ bool grid_barrier(const DecodeParams& p, Shared* sh, unsigned target) {
+// Grid-wide barrier among the consumer threads of all CTAs (release reduction on one
+// counter, acquire polling). Returns false if this CTA must stop (own or remote
+// failure); the result is the same in every consumer thread.
+__device__ bool grid_barrier(const DecodeParams& p, Shared* sh, unsigned k, int tid) {
+  const unsigned target = k * gridDim.x;
   cons_sync(kConsumerThreads);
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
+    trace_at(p, 2 * static_cast<int>(k) - 1);
     int stop = sh->abort_flag;
     if (!stop) {
-      __threadfence();
-      atomicAdd(p.bar, 1u);
+      red_release_add(p.bar, 1u);
       uint64_t t0 = 0;
       for (uint32_t it = 1;; ++it) {
         const unsigned v = ld_acquire(p.bar);
@@ -209,8 +261,8 @@ __device__ bool grid_barrier(const DecodeParams& p, Shared* sh, unsigned target)
           }
         }
       }
-      __threadfence();
     }
+    trace_at(p, 2 * static_cast<int>(k));
     if (stop) sh->abort_flag = 1;
     sh->decision = stop;
   }
@@ -224,68 +276,202 @@ __device__ __forceinline__ float cons_sum(float v, Shared* sh, int warp, int lan
   cons_sync(kConsumerThreads);
   if (lane == 0) sh->red[warp] = v;
   cons_sync(kConsumerThreads);
-  float t = (lane < kConsumerWarps) ? sh->red[lane] : 0.0f;
+  const float t = (lane < kConsumerWarps) ? sh->red[lane] : 0.0f;
   return warp_sum(t);
 }
 
-// xs = h / sqrt(mean(h^2) + eps) * gamma   (fp32, kept on chip)
-__device__ void rmsnorm_to_smem(const DecodeParams& p, const float* h, bool h_is_bf16_row, const uint8_t* bf_row,
-                                const uint16_t* gamma, float* xs, Shared* sh, int tid, int warp, int lane) {
+// Residual stream between norm phases j and j+1 (j counts every RMSNorm of the step):
+// h_j = base[j % 2] + delta[j % 3]. The update between norms j and j+1 reduces its
+// partial sums into delta[(j+1) % 3]; the RMSNorm of phase j+1 adds the two, and CTA 0
+// writes the sum to base[(j+1) % 2]. CTA G-1 zeroes delta[(j+2) % 3] during phase j.
+// No CTA reads the old residual on its own critical path.
+__device__ __forceinline__ float* res_base(const DecodeParams& p, int H, int j) {
+  return p.hbuf + static_cast<size_t>(j % 2) * H;
+}
+__device__ __forceinline__ float* res_delta(const DecodeParams& p, int H, int j) {
+  return p.hbuf + static_cast<size_t>(2 + j % 3) * H;
+}
+
+// Norm phase j: xs = h_j / sqrt(mean(h_j^2) + eps) * gamma (fp32, kept on chip), with
+// h_j = base + delta (or, for j = 0, the bf16 embedding row). All loads are issued together.
+template <int MG>
+__device__ __forceinline__ void rmsnorm(const DecodeParams& p, int H, int j, const uint16_t* bf_row,
+                                       const uint16_t* gamma, float* xs, Shared* sh, int tid, int warp, int lane) {
+  const int ng = H / 4;
+  const int cta = blockIdx.x, G = gridDim.x;
+  float4 v[MG];
+  if (bf_row) {
+#pragma unroll
+    for (int k = 0; k < MG; ++k) {
+      const int g = tid + k * kConsumerThreads;
+      if (g < ng) {
+        const uint2 w = *reinterpret_cast<const uint2*>(bf_row + 4 * g);
+        v[k] = make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
+      }
+    }
+  } else {
+    const float4* hb = reinterpret_cast<const float4*>(res_base(p, H, j));
+    const float4* hd = reinterpret_cast<const float4*>(res_delta(p, H, j));
+    float4 d[MG];
+#pragma unroll
+    for (int k = 0; k < MG; ++k) {
+      const int g = tid + k * kConsumerThreads;
+      if (g < ng) {
+        v[k] = __ldcg(hb + g);
+        d[k] = __ldcg(hd + g);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < MG; ++k) {
+      v[k].x += d[k].x; v[k].y += d[k].y; v[k].z += d[k].z; v[k].w += d[k].w;
+    }
+  }
+  if (cta == 0) {    // materialise h_j as the next base
+    float4* nb = reinterpret_cast<float4*>(res_base(p, H, j + 1));
+#pragma unroll
+    for (int k = 0; k < MG; ++k) {
+      const int g = tid + k * kConsumerThreads;
+      if (g < ng) __stcg(nb + g, v[k]);
+    }
+  }
+  if (cta == G - 1) {  // the delta that the update after norm j+1 accumulates into
+    float4* z = reinterpret_cast<float4*>(res_delta(p, H, j + 2));
+    for (int g = tid; g < ng; g += kConsumerThreads) __stcg(z + g, make_float4(0.f, 0.f, 0.f, 0.f));
+    if (j == 0) {
+      float4* z1 = reinterpret_cast<float4*>(res_delta(p, H, 1));
+      for (int g = tid; g < ng; g += kConsumerThreads) __stcg(z1 + g, make_float4(0.f, 0.f, 0.f, 0.f));
+    }
+  }
   float ss = 0.f;
-  for (int c = tid; c < p.H; c += kConsumerThreads) {
-    const float v = h_is_bf16_row ? bf16_to_f(reinterpret_cast<const uint16_t*>(bf_row)[c]) : __ldcg(h + c);
-    ss = fmaf(v, v, ss);
+#pragma unroll
+  for (int k = 0; k < MG; ++k) {
+    const int g = tid + k * kConsumerThreads;
+    if (g < ng) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
   }
   ss = cons_sum(ss, sh, warp, lane);
-  const float inv = 1.0f / sqrtf(ss / static_cast<float>(p.H) + p.eps);
-  for (int c = tid; c < p.H; c += kConsumerThreads) {
-    const float v = h_is_bf16_row ? bf16_to_f(reinterpret_cast<const uint16_t*>(bf_row)[c]) : __ldcg(h + c);
-    xs[c] = v * inv * bf16_to_f(gamma[c]);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(H) + p.eps);
+#pragma unroll
+  for (int k = 0; k < MG; ++k) {
+    const int g = tid + k * kConsumerThreads;
+    if (g < ng) {
+      const uint2 gw = *reinterpret_cast<const uint2*>(gamma + 4 * g);
+      reinterpret_cast<float4*>(xs)[g] = make_float4(v[k].x * inv * bf16lo(gw.x), v[k].y * inv * bf16hi(gw.x),
+                                                     v[k].z * inv * bf16lo(gw.y), v[k].w * inv * bf16hi(gw.y));
+    }
   }
   cons_sync(kConsumerThreads);
 }
 
-// Warp-per-row dot products of a chunk of bf16 rows with the fp32 vector xs;
-// f(row, value) runs on lane 0.
-template <class F>
-__device__ __forceinline__ void gemv_chunk(const uint8_t* chunk, int nrows, int rb, const float* xs, int H,
-                                           int warp, int lane, F&& f) {
-  int r = warp;
-  for (; r + kConsumerWarps < nrows; r += 2 * kConsumerWarps) {
-    const uint8_t* r0 = chunk + static_cast<size_t>(r) * rb;
-    const uint8_t* r1 = r0 + static_cast<size_t>(kConsumerWarps) * rb;
-    float a0 = 0.f, a1 = 0.f;
-    for (int c = lane * 8; c < H; c += 256) {
-      const float4 xa = *reinterpret_cast<const float4*>(xs + c);
-      const float4 xb = *reinterpret_cast<const float4*>(xs + c + 4);
-      a0 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(r0 + 2 * c), xa, xb, a0);
-      a1 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(r1 + 2 * c), xa, xb, a1);
-    }
-    a0 = warp_sum(a0);
-    a1 = warp_sum(a1);
-    if (lane == 0) { f(r, a0); f(r + kConsumerWarps, a1); }
-  }
-  for (; r < nrows; r += kConsumerWarps) {
-    const uint8_t* r0 = chunk + static_cast<size_t>(r) * rb;
-    float a0 = 0.f;
-    for (int c = lane * 8; c < H; c += 256)
-      a0 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(r0 + 2 * c), *reinterpret_cast<const float4*>(xs + c),
-                         *reinterpret_cast<const float4*>(xs + c + 4), a0);
-    a0 = warp_sum(a0);
-    if (lane == 0) f(r, a0);
+// The normed input, as each lane needs it for a warp-per-row dot product: lane l holds
+// x[l*8 + 256*k .. +8) for k < XK. Used (kept in registers for a whole phase) when the
+// hidden size is exactly XK * 256; XK = 0 reads x from shared memory instead.
+template <int XK>
+struct XReg {
+  float4 a[XK > 0 ? XK : 1], b[XK > 0 ? XK : 1];
+};
+
+template <int XK>
+__device__ __forceinline__ void load_xreg(XReg<XK>& x, const float* xs, int H, int lane) {
+#pragma unroll
+  for (int k = 0; k < XK; ++k) {
+    const int c = lane * 8 + 256 * k;
+    x.a[k] = *reinterpret_cast<const float4*>(xs + c);
+    x.b[k] = *reinterpret_cast<const float4*>(xs + c + 4);
   }
 }
 
-// Split-K accumulate: acc[out] += sum_r row_r[out] * coef[r] over a chunk of rows of
-// length H (bf16). Thread tid owns float4 groups tid, tid + 256, ...
-__device__ __forceinline__ void splitk_chunk(const uint8_t* chunk, int nrows, int rb, const float* coef, int H,
-                                             int tid, float4* acc) {
+// Dot products of two bf16 rows with x (register or shared-memory copy).
+template <int XK>
+__device__ __forceinline__ void dot2_rows(const uint8_t* p0, const uint8_t* p1, const XReg<XK>& x, const float* xs,
+                                          int H, int lane, float& a0, float& a1) {
+  a0 = 0.f;
+  a1 = 0.f;
+  if (XK > 0) {
+    uint4 w0[XK > 0 ? XK : 1], w1[XK > 0 ? XK : 1];
+#pragma unroll
+    for (int k = 0; k < XK; ++k) {     // all shared-memory loads first, then the arithmetic
+      const int c = lane * 8 + 256 * k;
+      w0[k] = *reinterpret_cast<const uint4*>(p0 + 2 * c);
+      w1[k] = *reinterpret_cast<const uint4*>(p1 + 2 * c);
+    }
+#pragma unroll
+    for (int k = 0; k < XK; ++k) {
+      a0 = dot8_bf16_f32(w0[k], x.a[k], x.b[k], a0);
+      a1 = dot8_bf16_f32(w1[k], x.a[k], x.b[k], a1);
+    }
+  } else {
+    for (int c = lane * 8; c < H; c += 256) {
+      const float4 xa = *reinterpret_cast<const float4*>(xs + c);
+      const float4 xb = *reinterpret_cast<const float4*>(xs + c + 4);
+      a0 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p0 + 2 * c), xa, xb, a0);
+      a1 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p1 + 2 * c), xa, xb, a1);
+    }
+  }
+}
+
+// Warp-per-row dot products of nrows bf16 rows (stride rb bytes) with x. Row r's value
+// goes to lo[row_base + r] if row_base + r < split, else to hi[row_base + r - split];
+// lane 0 writes it.
+template <int XK>
+__device__ __forceinline__ void gemv_rows(const uint8_t* chunk, int nrows, int rb, const XReg<XK>& x, const float* xs,
+                                          int H, int warp, int lane, int row_base, int split, float* lo, float* hi) {
+  for (int r = warp; r < nrows; r += 2 * kConsumerWarps) {
+    const int r1 = r + kConsumerWarps;
+    const bool two = r1 < nrows;
+    float a0, a1;
+    dot2_rows<XK>(chunk + static_cast<size_t>(r) * rb, chunk + static_cast<size_t>(two ? r1 : r) * rb, x, xs, H,
+                  lane, a0, a1);
+    a0 = warp_sum(a0);
+    a1 = warp_sum(a1);
+    if (lane == 0) {
+      const int g0 = row_base + r;
+      if (g0 < split) lo[g0] = a0; else hi[g0 - split] = a0;
+      if (two) {
+        const int g1 = row_base + r1;
+        if (g1 < split) lo[g1] = a1; else hi[g1 - split] = a1;
+      }
+    }
+  }
+}
+
+// Split-K accumulate into registers: acc[out] += sum_r row_r[out] * coef[r]. Thread tid
+// owns float4 groups tid, tid + 256, ... Rows are taken four at a time, loads first.
+template <int MG>
+__device__ __forceinline__ void splitk_rows(const uint8_t* chunk, int nrows, int rb, const float* coef, int H,
+                                            float4* acc, int tid) {
   const int ng = H / 4;
-  for (int r = 0; r < nrows; ++r) {
+  int r = 0;
+  for (; r + 4 <= nrows; r += 4) {
+    uint2 w[4][MG];
+    float cf[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      cf[q] = coef[r + q];
+#pragma unroll
+      for (int k = 0; k < MG; ++k) {
+        const int g = tid + k * kConsumerThreads;
+        if (g < ng) w[q][k] = *reinterpret_cast<const uint2*>(chunk + static_cast<size_t>(r + q) * rb + 8 * g);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int k = 0; k < MG; ++k) {
+        const int g = tid + k * kConsumerThreads;
+        if (g < ng) {
+          acc[k].x = fmaf(bf16lo(w[q][k].x), cf[q], acc[k].x);
+          acc[k].y = fmaf(bf16hi(w[q][k].x), cf[q], acc[k].y);
+          acc[k].z = fmaf(bf16lo(w[q][k].y), cf[q], acc[k].z);
+          acc[k].w = fmaf(bf16hi(w[q][k].y), cf[q], acc[k].w);
+        }
+      }
+    }
+  }
+  for (; r < nrows; ++r) {
     const uint8_t* row = chunk + static_cast<size_t>(r) * rb;
     const float cf = coef[r];
 #pragma unroll
-    for (int k = 0; k < kMaxGroups; ++k) {
+    for (int k = 0; k < MG; ++k) {
       const int g = tid + k * kConsumerThreads;
       if (g < ng) {
         const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * g);
@@ -298,41 +484,85 @@ __device__ __forceinline__ void splitk_chunk(const uint8_t* chunk, int nrows, in
   }
 }
 
-// Residual update u: nxt += acc (+ cur from CTA 0); CTA G-1 zeroes the buffer that update u+1 adds into.
-__device__ __forceinline__ void residual_epilogue(const DecodeParams& p, int u, bool has_rows, const float4* acc,
-                                                  int cta, int G, int tid) {
-  const int H = p.H;
-  float* cur = p.hbuf + static_cast<size_t>(u % 3) * H;
-  float* nxt = p.hbuf + static_cast<size_t>((u + 1) % 3) * H;
-  float* third = p.hbuf + static_cast<size_t>((u + 2) % 3) * H;
+// The update that follows norm j: delta[(j+1) % 3] += this CTA's partial sums.
+template <int MG>
+__device__ __forceinline__ void residual_add(const DecodeParams& p, int H, int j, bool has_rows, const float4* acc,
+                                             int tid) {
+  if (!has_rows) return;
   const int ng = H / 4;
-  if (has_rows || cta == 0) {
+  float4* nd = reinterpret_cast<float4*>(res_delta(p, H, j + 1));
 #pragma unroll
-    for (int k = 0; k < kMaxGroups; ++k) {
-      const int g = tid + k * kConsumerThreads;
-      if (g < ng) {
-        float4 a = acc[k];
-        if (cta == 0) {
-          const float4 c = __ldcg(reinterpret_cast<const float4*>(cur) + g);
-          a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
-        }
-        atomicAdd(reinterpret_cast<float4*>(nxt) + g, a);
-      }
+  for (int k = 0; k < MG; ++k) {
+    const int g = tid + k * kConsumerThreads;
+    if (g < ng) atomicAdd(nd + g, acc[k]);
+  }
+}
+
+// Causal depthwise conv at channel ch over the W-slot history, then SiLU. All loads
+// are issued before the arithmetic.
+__device__ __forceinline__ float conv_silu_at(const DecodeParams& p, const float* ringl, const uint16_t* taps, int ch,
+                                              int pos) {
+  float w[kMaxConv], x[kMaxConv];
+#pragma unroll
+  for (int j = 0; j < kMaxConv; ++j) {
+    if (j < p.convw) {
+      const int src = pos - (p.convw - 1) + j;
+      const int slot = ((src % p.convw) + p.convw) % p.convw;
+      w[j] = bf16_to_f(taps[static_cast<size_t>(ch) * p.convw + j]);
+      x[j] = __ldcg(ringl + static_cast<size_t>(slot) * p.C + ch);
     }
   }
-  if (cta == G - 1) {
-    for (int g = tid; g < ng; g += kConsumerThreads)
-      __stcg(reinterpret_cast<float4*>(third) + g, make_float4(0.f, 0.f, 0.f, 0.f));
+  float y = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxConv; ++j)
+    if (j < p.convw) y = fmaf(w[j], x[j], y);
+  return siluf_(y);
+}
+
+// RoPE angle pos * inv_freq reduced to [-pi, pi] in double, then sin/cos in fp32.
+__device__ __forceinline__ void rope_cs(double ang, float& c, float& s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double r = ang - two_pi * rint(ang / two_pi);
+  sincosf(static_cast<float>(r), &s, &c);
+}
+
+// Online-softmax update of one block of np scores in sc (one warp per head).
+__device__ __forceinline__ void softmax_block(float* sc, float* mlc, int grp, int np, int warp, int lane) {
+  if (warp >= grp) return;
+  const int t = warp;
+  float mx = -INFINITY;
+  for (int pp = lane; pp < np; pp += 32) mx = fmaxf(mx, sc[t * kAttnSub + pp]);
+  mx = warp_max(mx);
+  const float m_old = mlc[3 * t];
+  const float m_new = fmaxf(m_old, mx);
+  float ls = 0.f;
+  for (int pp = lane; pp < np; pp += 32) {
+    const float e = expf(sc[t * kAttnSub + pp] - m_new);
+    sc[t * kAttnSub + pp] = e;
+    ls += e;
+  }
+  ls = warp_sum(ls);
+  __syncwarp();
+  if (lane == 0) {
+    const float corr = expf(m_old - m_new);
+    mlc[3 * t] = m_new;
+    mlc[3 * t + 1] = mlc[3 * t + 1] * corr + ls;
+    mlc[3 * t + 2] = corr;
   }
 }
 
 // ------------------------------------------------------------------ the kernel
+// HK > 0: the hidden size is exactly HK * 256 (compile-time, so the hot loops carry no
+// bound checks and x lives in registers); HK = 0: any hidden size up to 8192.
+template <int HK>
 __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int XK = HK;                                // x register groups (0: shared memory)
+  constexpr int MG = HK > 0 ? (HK + 3) / 4 : 8;         // float4 groups of the hidden vector per thread
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   Shared* sh = reinterpret_cast<Shared*>(smem + static_cast<size_t>(kSlots) * kSlotBytes);
-  float* fs = reinterpret_cast<float*>(sh + 1);                          // scratch [kScratchFloats]
-  float* xs = fs + kScratchFloats;                                       // normed input [H] fp32
+  float* xs = reinterpret_cast<float*>(sh + 1);      // [H] normed input
+  float* fs = xs + p.H;                               // scratch
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x, G = gridDim.x;
@@ -361,252 +591,238 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     }
     if (!bad && p.gate_n && p.gate_i > ld_volatile(p.gate_n)) bad = 1;   // skipped replay step
     sh->bad = bad;
+    if (!bad) compute_ranges(p, cta, G, pos, sh->rg);
   }
   __syncthreads();
   if (sh->bad) return;
 
   if (warp == kConsumerWarps) {
-    if (lane == 0) producer_loop(p, sh, ring, cta, G);
+    if (lane == 0) producer_loop(p, sh, ring);
     return;
   }
 
   // ---------------- consumers ----------------
-  Cons cs{ring, sh, 0u, tid, warp, lane};
+  if (tid == 0) trace_at(p, 0);
   const int pos = sh->pos;
-  const int tok = sh->tok;
-  const uint8_t* emb_row = p.embed + static_cast<size_t>(tok) * p.row_bytes;
+  const Ranges& rg = sh->rg;
   const int rb = p.row_bytes;
+  const int H = HK > 0 ? HK * 256 : p.H;
+  const int ng = H / 4;
+  uint32_t n = 0;               // next chunk index
   unsigned nbar = 0;
-  int u = 0;                    // residual update counter
-  Seg segs[3];
 
   for (int l = 0; l < p.n_layers; ++l) {
     const LayerW L = p.layers[l];
-    const int nph = n_phases(L);
-    for (int k = 0; k < nph; ++k) {
-      const int ph = phase_id(L, k);
-      if (l > 0 || k > 0) {
-        if (!grid_barrier(p, sh, ++nbar * static_cast<unsigned>(G))) return;
+    // ---- phase 1: pre-mixer RMSNorm + input projection ----
+    if (l > 0 && !grid_barrier(p, sh, ++nbar, tid)) return;
+    if (l == 0) {
+      const uint16_t* emb_row = reinterpret_cast<const uint16_t*>(p.embed + static_cast<size_t>(sh->tok) * rb);
+      rmsnorm<MG>(p, H, 0, emb_row, L.norm1, xs, sh, tid, warp, lane);   // the residual starts as the embedding
+    } else {
+      rmsnorm<MG>(p, H, 2 * l, nullptr, L.norm1, xs, sh, tid, warp, lane);
+    }
+    {
+      const bool dn = (L.kind == kDeltaNet);
+      const int b = dn ? rg.in_dn_b : rg.in_at_b, e = dn ? rg.in_dn_e : rg.in_at_e;
+      float* ringc = p.conv_ring + static_cast<size_t>(L.idx) * p.convw * p.C + static_cast<size_t>(pos % p.convw) * p.C;
+      const int split = dn ? p.C : kNoSplit;
+      float* lo = dn ? ringc : p.z;
+      const int rpc = kSlotBytes / rb;
+      XReg<XK> xr;
+      load_xreg<XK>(xr, xs, H, lane);
+      for (int r0 = 0; r0 < e - b; r0 += rpc) {
+        const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
+        gemv_rows<XK>(ch, min(rpc, e - b - r0), rb, xr, xs, H, warp, lane, b + r0, split, lo, p.z);
+        release(p, sh, n, lane);
       }
-      const int ns = phase_segments(p, L, ph, cta, G, segs);
+    }
+    if (!grid_barrier(p, sh, ++nbar, tid)) return;
 
-      if (ph == kPhIn) {
-        // ---- pre-mixer RMSNorm + input projection ----
-        if (l == 0) {
-          rmsnorm_to_smem(p, nullptr, true, emb_row, L.norm1, xs, sh, tid, warp, lane);
-          if (cta == 0) {     // residual stream starts as the embedding row
-            for (int c = tid; c < p.H; c += kConsumerThreads) {
-              __stcg(p.hbuf + c, bf16_to_f(reinterpret_cast<const uint16_t*>(emb_row)[c]));
-              __stcg(p.hbuf + p.H + c, 0.f);
-            }
-          }
-        } else {
-          rmsnorm_to_smem(p, p.hbuf + static_cast<size_t>(u % 3) * p.H, false, nullptr, L.norm1, xs, sh, tid,
-                          warp, lane);
-        }
-        int b = 0, e = 0;
-        const int rows = (L.kind == kDeltaNet) ? (p.C + 2 * p.Hd) : p.at_in_rows;
-        split_range(rows, cta, G, b, e);
-        if (ns) {
-          const Seg sg = segs[0];
-          const int rpc = kSlotBytes / sg.row_bytes;
-          float* ringc = p.conv_ring + static_cast<size_t>(L.idx) * p.convw * p.C +
-                         static_cast<size_t>(pos % p.convw) * p.C;
-          for (int r0 = 0; r0 < sg.rows; r0 += rpc) {
-            const int nr = min(rpc, sg.rows - r0);
-            const uint8_t* ch = acquire(cs, p.err);
-            const int base = b + r0;
-            if (L.kind == kDeltaNet) {
-              gemv_chunk(ch, nr, rb, xs, p.H, warp, lane, [&](int r, float v) {
-                const int row = base + r;
-                if (row < p.C) __stcg(ringc + row, v);
-                else __stcg(p.z + (row - p.C), v);
-              });
+    if (L.kind == kDeltaNet) {
+      // ---- phase 2 (DeltaNet): conv + SiLU + L2 norm + gates, delta rule on this CTA's rows of S, out-proj split-K ----
+      const int g0 = rg.dn_b, g1 = rg.dn_e, nrows = g1 - g0;
+      float4 acc[MG];
+#pragma unroll
+      for (int k = 0; k < MG; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (nrows > 0) {
+        const int h0 = g0 / p.dv, h1 = (g1 - 1) / p.dv;
+        const int nh = h1 - h0 + 1;
+        // scratch: qk[2 nh][dk] (q_h0, k_h0, q_h1, k_h1, ...) | ab[nh][2] | vv[nrows] | oc[nrows]
+        float* qk = fs;
+        float* ab = qk + nh * 2 * p.dk;
+        float* vv = ab + 2 * nh;
+        float* oc = vv + nrows;
+        const float* ringl = p.conv_ring + static_cast<size_t>(L.idx) * p.convw * p.C;
+        const int nqk = 2 * nh * p.dk;
+        const int nitems = nqk + nrows + nh;
+        // Items (up to kConvItems per thread): q/k channels of the heads, v channels of
+        // the rows, then the (alpha, beta) gate pairs. Every load is issued first.
+        float wv[kConvItems][kMaxConv], xv[kConvItems][kMaxConv];
+#pragma unroll
+        for (int it = 0; it < kConvItems; ++it) {
+          const int i = tid + it * kConsumerThreads;
+          if (i < nqk + nrows) {
+            int ch;
+            if (i < nqk) {
+              const int vec = i / p.dk, d = i % p.dk;
+              ch = ((vec & 1) ? p.Hd * p.dk : 0) + (h0 + (vec >> 1)) * p.dk + d;
             } else {
-              gemv_chunk(ch, nr, rb, xs, p.H, warp, lane, [&](int r, float v) { __stcg(p.z + base + r, v); });
+              ch = 2 * p.Hd * p.dk + g0 + (i - nqk);   // v channel of (head g/dv, row g%dv)
             }
-            release(cs);
-          }
-        }
-      } else if (ph == kPhMix && L.kind == kDeltaNet) {
-        // ---- conv + SiLU + L2 norm + gates, gated delta rule on this CTA's rows of S, out-proj split-K ----
-        int g0 = 0, g1 = 0;
-        split_range(p.Hd * p.dv, cta, G, g0, g1);
-        const int nrows = g1 - g0;
-        float4 acc[kMaxGroups];
 #pragma unroll
-        for (int q = 0; q < kMaxGroups; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (nrows > 0) {
-          const int h0 = g0 / p.dv, h1 = (g1 - 1) / p.dv;
-          const int nh = h1 - h0 + 1;
-          // scratch layout: qk[nh][2][dk] | ab[nh][2] | vv[nrows] | oc[nrows]
-          float* qk = fs;
-          float* ab = qk + nh * 2 * p.dk;
-          float* vv = ab + 2 * nh;
-          float* oc = vv + nrows;
-          const float* ringl = p.conv_ring + static_cast<size_t>(L.idx) * p.convw * p.C;
-          const uint16_t* taps = L.conv;
-          auto conv_at = [&](int ch) -> float {
-            float y = 0.f;
-            for (int j = 0; j < p.convw; ++j) {
-              int src = pos - (p.convw - 1) + j;
-              int slot = ((src % p.convw) + p.convw) % p.convw;
-              y = fmaf(bf16_to_f(taps[static_cast<size_t>(ch) * p.convw + j]),
-                       __ldcg(ringl + static_cast<size_t>(slot) * p.C + ch), y);
-            }
-            return siluf_(y);
-          };
-          // q and k vectors: one warp per (head, q|k) vector, with its L2 norm
-          for (int vec = warp; vec < 2 * nh; vec += kConsumerWarps) {
-            const int hh = h0 + (vec >> 1);
-            const int isk = vec & 1;
-            const int chb = isk ? (p.Hd * p.dk + hh * p.dk) : (hh * p.dk);
-            float* dst = qk + vec * p.dk;
-            float ss = 0.f;
-            for (int i = lane; i < p.dk; i += 32) {
-              const float y = conv_at(chb + i);
-              dst[i] = y;
-              ss = fmaf(y, y, ss);
-            }
-            ss = warp_sum(ss);
-            const float inv = 1.0f / sqrtf(ss + 1e-6f);
-            __syncwarp();
-            for (int i = lane; i < p.dk; i += 32) dst[i] *= inv;
-          }
-          for (int i = tid; i < nh; i += kConsumerThreads) {
-            const float al = __ldcg(p.z + h0 + i);
-            const float be = __ldcg(p.z + p.Hd + h0 + i);
-            ab[2 * i] = sigmoidf_(-al);        // exp(-softplus(alpha))
-            ab[2 * i + 1] = sigmoidf_(be);
-          }
-          for (int r = tid; r < nrows; r += kConsumerThreads) {
-            const int g = g0 + r;
-            vv[r] = conv_at(2 * p.Hd * p.dk + g);   // v channel of (head g/dv, row g%dv)
-          }
-          cons_sync(kConsumerThreads);
-          // S rows (fp32) through the ring
-          {
-            const Seg sg = segs[0];
-            const int rpc = kSlotBytes / sg.row_bytes;
-            const int vpl = p.dk / 32;
-            for (int r0 = 0; r0 < sg.rows; r0 += rpc) {
-              const int nr = min(rpc, sg.rows - r0);
-              const float* ch = reinterpret_cast<const float*>(acquire(cs, p.err));
-              for (int r = warp; r < nr; r += kConsumerWarps) {
-                const int lr = r0 + r;
-                const int g = g0 + lr;
-                const int hl = g / p.dv - h0;
-                const float a = ab[2 * hl], bb = ab[2 * hl + 1];
-                const float* qv = qk + (2 * hl) * p.dk;
-                const float* kv = qk + (2 * hl + 1) * p.dk;
-                const float* srow = ch + static_cast<size_t>(r) * p.dk;
-                float s[8];
-                float ukk = 0.f;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  if (q < vpl) {
-                    s[q] = a * srow[lane + 32 * q];
-                    ukk = fmaf(s[q], kv[lane + 32 * q], ukk);
-                  }
-                }
-                ukk = warp_sum(ukk);
-                const float coef = bb * (vv[lr] - ukk);
-                float o = 0.f;
-                float* sg_out = p.S + (static_cast<size_t>(L.idx) * p.Hd * p.dv + g) * p.dk;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  if (q < vpl) {
-                    s[q] = fmaf(coef, kv[lane + 32 * q], s[q]);
-                    o = fmaf(s[q], qv[lane + 32 * q], o);
-                    __stcg(sg_out + lane + 32 * q, s[q]);
-                  }
-                }
-                o = warp_sum(o);
-                if (lane == 0) oc[lr] = o;
+            for (int j = 0; j < kMaxConv; ++j) {
+              if (j < p.convw) {
+                const int slot = (pos + 1 + j) % p.convw;   // holds position pos - (W-1) + j
+                wv[it][j] = bf16_to_f(L.conv[static_cast<size_t>(ch) * p.convw + j]);
+                xv[it][j] = __ldcg(ringl + static_cast<size_t>(slot) * p.C + ch);
               }
-              release(cs);
             }
-          }
-          cons_sync(kConsumerThreads);
-          // out-projection, split over this CTA's value rows
-          {
-            const Seg sg = segs[1];
-            const int rpc = kSlotBytes / sg.row_bytes;
-            for (int r0 = 0; r0 < sg.rows; r0 += rpc) {
-              const int nr = min(rpc, sg.rows - r0);
-              const uint8_t* ch = acquire(cs, p.err);
-              splitk_chunk(ch, nr, rb, oc + r0, p.H, tid, acc);
-              release(cs);
-            }
+          } else if (i < nitems) {
+            const int hh = i - nqk - nrows;
+            xv[it][0] = __ldcg(p.z + h0 + hh);
+            xv[it][1] = __ldcg(p.z + p.Hd + h0 + hh);
           }
         }
-        residual_epilogue(p, u, nrows > 0, acc, cta, G, tid);
-        ++u;
-      } else if (ph == kPhMix) {
-        // ---- attention: RoPE, KV append, split-K partial softmax over the cache ----
-        const int n = pos + 1;
-        int CH, nsplit;
-        attn_split(n, G, p.Hkv, p.max_splits, CH, nsplit);
+#pragma unroll
+        for (int it = 0; it < kConvItems; ++it) {
+          const int i = tid + it * kConsumerThreads;
+          if (i < nqk + nrows) {
+            float y = 0.f;
+#pragma unroll
+            for (int j = 0; j < kMaxConv; ++j)
+              if (j < p.convw) y = fmaf(wv[it][j], xv[it][j], y);
+            y = siluf_(y);
+            if (i < nqk) qk[i] = y;
+            else vv[i - nqk] = y;
+          } else if (i < nitems) {
+            const int hh = i - nqk - nrows;
+            ab[2 * hh] = sigmoidf_(-xv[it][0]);      // exp(-softplus(alpha))
+            ab[2 * hh + 1] = sigmoidf_(xv[it][1]);
+          }
+        }
+        cons_sync(kConsumerThreads);
+        for (int vec = warp; vec < 2 * nh; vec += kConsumerWarps) {   // L2-normalise q and k per head
+          float* dst = qk + vec * p.dk;
+          float ss = 0.f;
+          for (int i = lane; i < p.dk; i += 32) ss = fmaf(dst[i], dst[i], ss);
+          ss = warp_sum(ss);
+          const float inv = 1.0f / sqrtf(ss + 1e-6f);
+          for (int i = lane; i < p.dk; i += 32) dst[i] *= inv;
+        }
+        cons_sync(kConsumerThreads);
+        // S rows: S = a S; u = S k; S += b (v - u) k^T; o = S q
+        const int srb = p.dk * 4, srpc = kSlotBytes / srb, vpl = p.dk / 32;
+        for (int r0 = 0; r0 < nrows; r0 += srpc) {
+          const float* ch = reinterpret_cast<const float*>(acquire(p, sh, ring, n, tid, lane));
+          const int nr = min(srpc, nrows - r0);
+          for (int r = warp; r < nr; r += kConsumerWarps) {
+            const int lr = r0 + r;
+            const int g = g0 + lr;
+            const int hl = g / p.dv - h0;
+            const float a = ab[2 * hl], bb = ab[2 * hl + 1];
+            const float* qv = qk + (2 * hl) * p.dk;
+            const float* kv = qk + (2 * hl + 1) * p.dk;
+            const float* srow = ch + static_cast<size_t>(r) * p.dk;
+            float s[8];
+            float ukk = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              if (q < vpl) {
+                s[q] = a * srow[lane + 32 * q];
+                ukk = fmaf(s[q], kv[lane + 32 * q], ukk);
+              }
+            }
+            ukk = warp_sum(ukk);
+            const float coef = bb * (vv[lr] - ukk);
+            float o = 0.f;
+            float* sg_out = p.S + (static_cast<size_t>(L.idx) * p.Hd * p.dv + g) * p.dk;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              if (q < vpl) {
+                s[q] = fmaf(coef, kv[lane + 32 * q], s[q]);
+                o = fmaf(s[q], qv[lane + 32 * q], o);
+                __stcg(sg_out + lane + 32 * q, s[q]);
+              }
+            }
+            o = warp_sum(o);
+            if (lane == 0) oc[lr] = o;
+          }
+          release(p, sh, n, lane);
+        }
+        cons_sync(kConsumerThreads);
+        const int rpc = kSlotBytes / rb;
+        for (int r0 = 0; r0 < nrows; r0 += rpc) {
+          const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
+          splitk_rows<MG>(ch, min(rpc, nrows - r0), rb, oc + r0, H, acc, tid);
+          release(p, sh, n, lane);
+        }
+      }
+      residual_add<MG>(p, H, 2 * l, nrows > 0, acc, tid);
+    } else {
+      // ---- phase 2 (attention): RoPE, KV append, split-K partial softmax over this CTA's positions ----
+      if (rg.au_valid) {
         const int grp = p.Hq / p.Hkv;
         const int D = p.D, half = D / 2;
         const float scale = 1.0f / sqrtf(static_cast<float>(D));
-        const int qoff = 0;
         const int koff = p.Hq * D * (p.gated ? 2 : 1);
         const int voff = koff + p.Hkv * D;
-        float* qs = fs;                       // [grp][D]
+        const int ug = rg.au_g, uj = rg.au_j, p0 = rg.au_p0, q1 = rg.au_q1;
+        float* qs = fs;                       // [grp][D]  roped, pre-scaled queries
         float* sc = qs + grp * D;             // [grp][kAttnSub]
         float* mlc = sc + grp * kAttnSub;     // [grp][3]: m, l, corr
-        const size_t cache_base = static_cast<size_t>(L.idx) * p.Hkv * p.max_ctx * D;
-        const int units = p.Hkv * nsplit;
-        for (int un = cta; un < units; un += G) {
-          const int g = un % p.Hkv, j = un / p.Hkv;
-          const int p0 = j * CH, p1 = min(n, p0 + CH);
-          uint16_t* Kg = p.kc + cache_base + static_cast<size_t>(g) * p.max_ctx * D;
-          uint16_t* Vg = p.vc + cache_base + static_cast<size_t>(g) * p.max_ctx * D;
-          for (int idx = tid; idx < grp * half; idx += kConsumerThreads) {
-            const int t = idx / half, i = idx % half;
-            const int hq = g * grp + t;
-            double sn, cn;
-            sincos(static_cast<double>(pos) * p.inv_freq[i], &sn, &cn);
-            const float c = static_cast<float>(cn), s = static_cast<float>(sn);
-            const float x1 = __ldcg(p.z + qoff + hq * D + i), x2 = __ldcg(p.z + qoff + hq * D + i + half);
-            qs[t * D + i] = (x1 * c - x2 * s) * scale;
-            qs[t * D + i + half] = (x1 * s + x2 * c) * scale;
+        float* kcur = mlc + 3 * grp;          // [D] current key (bf16-rounded)
+        float* vcur = kcur + D;               // [D] current value (bf16-rounded)
+        const bool has_cur = (rg.au_p1 == pos + 1);
+        const size_t cache_g = (static_cast<size_t>(L.idx) * p.Hkv + ug) * p.max_ctx * D;
+        for (int idx = tid; idx < (grp + (has_cur ? 1 : 0)) * half; idx += kConsumerThreads) {
+          const int t = idx / half, i = idx % half;
+          float cs, sn;
+          rope_cs(static_cast<double>(pos) * p.inv_freq[i], cs, sn);
+          if (t < grp) {
+            const int hq = ug * grp + t;
+            const float x1 = __ldcg(p.z + hq * D + i), x2 = __ldcg(p.z + hq * D + i + half);
+            qs[t * D + i] = (x1 * cs - x2 * sn) * scale;
+            qs[t * D + i + half] = (x1 * sn + x2 * cs) * scale;
+          } else {   // current key: rotate, round to bf16, append to the cache
+            const float x1 = __ldcg(p.z + koff + ug * D + i), x2 = __ldcg(p.z + koff + ug * D + i + half);
+            const uint16_t k1 = f_to_bf16(x1 * cs - x2 * sn), k2 = f_to_bf16(x1 * sn + x2 * cs);
+            p.kc[cache_g + static_cast<size_t>(pos) * D + i] = k1;
+            p.kc[cache_g + static_cast<size_t>(pos) * D + i + half] = k2;
+            kcur[i] = bf16_to_f(k1);
+            kcur[i + half] = bf16_to_f(k2);
           }
-          if (p1 == n) {   // this unit holds the current position: append k, v (bf16)
-            for (int i = tid; i < half; i += kConsumerThreads) {
-              double sn, cn;
-              sincos(static_cast<double>(pos) * p.inv_freq[i], &sn, &cn);
-              const float c = static_cast<float>(cn), s = static_cast<float>(sn);
-              const float x1 = __ldcg(p.z + koff + g * D + i), x2 = __ldcg(p.z + koff + g * D + i + half);
-              Kg[static_cast<size_t>(pos) * D + i] = f_to_bf16(x1 * c - x2 * s);
-              Kg[static_cast<size_t>(pos) * D + i + half] = f_to_bf16(x1 * s + x2 * c);
-            }
-            for (int d = tid; d < D; d += kConsumerThreads)
-              Vg[static_cast<size_t>(pos) * D + d] = f_to_bf16(__ldcg(p.z + voff + g * D + d));
+        }
+        if (has_cur) {
+          for (int d = tid; d < D; d += kConsumerThreads) {
+            const uint16_t vb = f_to_bf16(__ldcg(p.z + voff + ug * D + d));
+            p.vc[cache_g + static_cast<size_t>(pos) * D + d] = vb;
+            vcur[d] = bf16_to_f(vb);
           }
-          if (tid < grp) {
-            mlc[3 * tid] = -INFINITY;
-            mlc[3 * tid + 1] = 0.f;
-            mlc[3 * tid + 2] = 0.f;
-          }
-          float oacc[8];
+        }
+        if (tid < grp) {
+          mlc[3 * tid] = -INFINITY;
+          mlc[3 * tid + 1] = 0.f;
+          mlc[3 * tid + 2] = 0.f;
+        }
+        float oacc[8];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) oacc[t] = 0.f;
-          cons_sync(kConsumerThreads);
-          const int dpl = D / 32;      // dims per lane (2..8)
-          for (int sb = p0; sb < p1; sb += kAttnSub) {
-            const int np = min(kAttnSub, p1 - sb);
+        for (int t = 0; t < 8; ++t) oacc[t] = 0.f;
+        cons_sync(kConsumerThreads);
+        const int dpl = D / 32;
+        for (int sb = p0; sb < q1; sb += kAttnSub) {
+          const int np = min(kAttnSub, q1 - sb);
+          {   // scores q_t . K[pp] from the K rows in shared memory, one warp per row
+            const uint16_t* kch = reinterpret_cast<const uint16_t*>(acquire(p, sh, ring, n, tid, lane));
             for (int pp = warp; pp < np; pp += kConsumerWarps) {
-              const uint16_t* krow = Kg + static_cast<size_t>(sb + pp) * D + lane * dpl;
+              const uint16_t* krow = kch + static_cast<size_t>(pp) * D + lane * dpl;
               float kf[8];
               if (dpl == 8) {
-                const uint4 kw = __ldcg(reinterpret_cast<const uint4*>(krow));
+                const uint4 kw = *reinterpret_cast<const uint4*>(krow);
                 kf[0] = bf16lo(kw.x); kf[1] = bf16hi(kw.x); kf[2] = bf16lo(kw.y); kf[3] = bf16hi(kw.y);
                 kf[4] = bf16lo(kw.z); kf[5] = bf16hi(kw.z); kf[6] = bf16lo(kw.w); kf[7] = bf16hi(kw.w);
               } else {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) kf[q] = (q < dpl) ? bf16_to_f(__ldcg(krow + q)) : 0.f;
+                for (int q = 0; q < 8; ++q) kf[q] = (q < dpl) ? bf16_to_f(krow[q]) : 0.f;
               }
               for (int t = 0; t < grp; ++t) {
                 const float* qv = qs + t * D + lane * dpl;
@@ -618,171 +834,188 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
                 if (lane == 0) sc[t * kAttnSub + pp] = d0;
               }
             }
-            cons_sync(kConsumerThreads);
-            if (warp < grp) {
-              const int t = warp;
-              float mx = -INFINITY;
-              for (int pp = lane; pp < np; pp += 32) mx = fmaxf(mx, sc[t * kAttnSub + pp]);
-              mx = warp_max(mx);
-              const float m_old = mlc[3 * t];
-              const float m_new = fmaxf(m_old, mx);
-              float ls = 0.f;
-              for (int pp = lane; pp < np; pp += 32) {
-                const float e = expf(sc[t * kAttnSub + pp] - m_new);
-                sc[t * kAttnSub + pp] = e;
-                ls += e;
-              }
-              ls = warp_sum(ls);
-              __syncwarp();
-              if (lane == 0) {
-                const float corr = expf(m_old - m_new);
-                mlc[3 * t] = m_new;
-                mlc[3 * t + 1] = mlc[3 * t + 1] * corr + ls;
-                mlc[3 * t + 2] = corr;
-              }
-            }
-            cons_sync(kConsumerThreads);
+            release(p, sh, n, lane);
+          }
+          cons_sync(kConsumerThreads);
+          softmax_block(sc, mlc, grp, np, warp, lane);
+          cons_sync(kConsumerThreads);
+          {   // values: thread d accumulates sum_pp p[pp] V[pp][d]
+            const uint16_t* vch = reinterpret_cast<const uint16_t*>(acquire(p, sh, ring, n, tid, lane));
             if (tid < D) {
               float vsum[8];
 #pragma unroll
               for (int t = 0; t < 8; ++t) vsum[t] = 0.f;
               for (int pp = 0; pp < np; ++pp) {
-                const float vv = bf16_to_f(__ldcg(Vg + static_cast<size_t>(sb + pp) * D + tid));
+                const float vvv = bf16_to_f(vch[static_cast<size_t>(pp) * D + tid]);
 #pragma unroll
                 for (int t = 0; t < 8; ++t)
-                  if (t < grp) vsum[t] = fmaf(sc[t * kAttnSub + pp], vv, vsum[t]);
+                  if (t < grp) vsum[t] = fmaf(sc[t * kAttnSub + pp], vvv, vsum[t]);
               }
 #pragma unroll
               for (int t = 0; t < 8; ++t)
                 if (t < grp) oacc[t] = oacc[t] * mlc[3 * t + 2] + vsum[t];
             }
-            cons_sync(kConsumerThreads);
-          }
-          // partials: [hq][split][D + 2] = acc..., m, l
-          if (tid < D) {
-            for (int t = 0; t < grp; ++t) {
-              const int hq = g * grp + t;
-              float* dst = p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (D + 2);
-              __stcg(dst + tid, oacc[t]);
-            }
-          }
-          if (tid < grp) {
-            const int hq = g * grp + tid;
-            float* dst = p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (D + 2);
-            __stcg(dst + D, mlc[3 * tid]);
-            __stcg(dst + D + 1, mlc[3 * tid + 1]);
+            release(p, sh, n, lane);
           }
           cons_sync(kConsumerThreads);
         }
-      } else if (ph == kPhAttOut) {
-        // ---- combine split-K partials for this CTA's output columns, gate, out-proj split-K ----
-        const int n = pos + 1;
-        int CH, nsplit;
-        attn_split(n, G, p.Hkv, p.max_splits, CH, nsplit);
-        int c0 = 0, c1 = 0;
-        split_range(p.Hq * p.D, cta, G, c0, c1);
-        const int ncol = c1 - c0;
-        float4 acc[kMaxGroups];
-#pragma unroll
-        for (int q = 0; q < kMaxGroups; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        float* oc = fs;
-        for (int cc = tid; cc < ncol; cc += kConsumerThreads) {
-          const int col = c0 + cc;
-          const int hq = col / p.D, d = col % p.D;
-          const float* base = p.part + static_cast<size_t>(hq) * p.max_splits * (p.D + 2);
-          float M = -INFINITY;
-          for (int j = 0; j < nsplit; ++j) M = fmaxf(M, __ldcg(base + static_cast<size_t>(j) * (p.D + 2) + p.D));
-          float Ls = 0.f, O = 0.f;
-          for (int j = 0; j < nsplit; ++j) {
-            const float* pj = base + static_cast<size_t>(j) * (p.D + 2);
-            const float w = expf(__ldcg(pj + p.D) - M);
-            Ls = fmaf(__ldcg(pj + p.D + 1), w, Ls);
-            O = fmaf(__ldcg(pj + d), w, O);
+        if (has_cur) {   // the current position, from the freshly computed k, v
+          if (warp < grp) {
+            float d0 = 0.f;
+            for (int i = lane; i < D; i += 32) d0 = fmaf(qs[warp * D + i], kcur[i], d0);
+            d0 = warp_sum(d0);
+            if (lane == 0) sc[warp * kAttnSub] = d0;
           }
-          float o = O / Ls;
-          if (p.gated) o *= sigmoidf_(__ldcg(p.z + p.Hq * p.D + col));
-          oc[cc] = o;
+          cons_sync(kConsumerThreads);
+          softmax_block(sc, mlc, grp, 1, warp, lane);
+          cons_sync(kConsumerThreads);
+          if (tid < D) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              if (t < grp) oacc[t] = oacc[t] * mlc[3 * t + 2] + sc[t * kAttnSub] * vcur[tid];
+          }
+        }
+        // partials: [hq][split][D + 2] = acc..., m, l
+        if (tid < D) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (t < grp) {
+              float* dst = p.part + (static_cast<size_t>(ug * grp + t) * p.max_splits + uj) * (D + 2);
+              __stcg(dst + tid, oacc[t]);
+            }
+          }
+        }
+        if (tid < grp) {
+          float* dst = p.part + (static_cast<size_t>(ug * grp + tid) * p.max_splits + uj) * (D + 2);
+          __stcg(dst + D, mlc[3 * tid]);
+          __stcg(dst + D + 1, mlc[3 * tid + 1]);
+        }
+      }
+      if (!grid_barrier(p, sh, ++nbar, tid)) return;
+
+      // ---- phase 3 (attention): combine partials for this CTA's columns, gate, out-proj split-K ----
+      const int nsplit = rg.nsplit;
+      const int c0 = rg.col_b, c1 = rg.col_e, ncol = c1 - c0;
+      float4 acc[MG];
+#pragma unroll
+      for (int k = 0; k < MG; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ncol > 0) {
+        const int hA = c0 / p.D, hB = (c1 - 1) / p.D;
+        const int nhd = hB - hA + 1;
+        // scratch: wts[nhd][nsplit] (m_j, then e^{m_j - M} / L) | gte[ncol] | oc[ncol]
+        float* wts = fs;
+        float* gte = wts + nhd * nsplit;
+        float* oc = gte + ncol;
+        for (int i = tid; i < nhd * nsplit + ncol; i += kConsumerThreads) {
+          if (i < nhd * nsplit) {
+            const int hq = hA + i / nsplit, j = i % nsplit;
+            wts[i] = __ldcg(p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (p.D + 2) + p.D);
+          } else {
+            const int cc = i - nhd * nsplit;
+            gte[cc] = p.gated ? sigmoidf_(__ldcg(p.z + p.Hq * p.D + c0 + cc)) : 1.0f;
+          }
         }
         cons_sync(kConsumerThreads);
-        if (ns) {
-          const Seg sg = segs[0];
-          const int rpc = kSlotBytes / sg.row_bytes;
-          for (int r0 = 0; r0 < sg.rows; r0 += rpc) {
-            const int nr = min(rpc, sg.rows - r0);
-            const uint8_t* ch = acquire(cs, p.err);
-            splitk_chunk(ch, nr, rb, oc + r0, p.H, tid, acc);
-            release(cs);
-          }
+        for (int hh = warp; hh < nhd; hh += kConsumerWarps) {
+          const int hq = hA + hh;
+          float M = -INFINITY;
+          for (int j = lane; j < nsplit; j += 32) M = fmaxf(M, wts[hh * nsplit + j]);
+          M = warp_max(M);
+          float Ls = 0.f;
+          for (int j = lane; j < nsplit; j += 32)
+            Ls = fmaf(__ldcg(p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (p.D + 2) + p.D + 1),
+                      expf(wts[hh * nsplit + j] - M), Ls);
+          Ls = warp_sum(Ls);
+          __syncwarp();
+          for (int j = lane; j < nsplit; j += 32) wts[hh * nsplit + j] = expf(wts[hh * nsplit + j] - M) / Ls;
         }
-        residual_epilogue(p, u, ncol > 0, acc, cta, G, tid);
-        ++u;
-      } else {
-        // ---- pre-MLP RMSNorm, SwiGLU gate/up for this CTA's intermediate rows, down split-K ----
-        rmsnorm_to_smem(p, p.hbuf + static_cast<size_t>(u % 3) * p.H, false, nullptr, L.norm2, xs, sh, tid, warp,
-                        lane);
-        int j0 = 0, j1 = 0;
-        split_range(p.F, cta, G, j0, j1);
-        const int nj = j1 - j0;
-        float4 acc[kMaxGroups];
-#pragma unroll
-        for (int q = 0; q < kMaxGroups; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        float* gs = fs;
-        float* act = fs + nj;
-        if (ns) {
-          for (int si = 0; si < 2; ++si) {
-            const Seg sg = segs[si];
-            const int rpc = kSlotBytes / sg.row_bytes;
-            for (int r0 = 0; r0 < sg.rows; r0 += rpc) {
-              const int nr = min(rpc, sg.rows - r0);
-              const uint8_t* ch = acquire(cs, p.err);
-              if (si == 0) {
-                gemv_chunk(ch, nr, rb, xs, p.H, warp, lane, [&](int r, float v) { gs[r0 + r] = v; });
-              } else {
-                gemv_chunk(ch, nr, rb, xs, p.H, warp, lane,
-                           [&](int r, float v) { act[r0 + r] = siluf_(gs[r0 + r]) * v; });
-              }
-              release(cs);
-            }
-            cons_sync(kConsumerThreads);
-          }
-          const Seg sg = segs[2];
-          const int rpc = kSlotBytes / sg.row_bytes;
-          for (int r0 = 0; r0 < sg.rows; r0 += rpc) {
-            const int nr = min(rpc, sg.rows - r0);
-            const uint8_t* ch = acquire(cs, p.err);
-            splitk_chunk(ch, nr, rb, act + r0, p.H, tid, acc);
-            release(cs);
-          }
+        cons_sync(kConsumerThreads);
+        for (int cc = warp; cc < ncol; cc += kConsumerWarps) {   // warp per column, lanes over splits
+          const int col = c0 + cc;
+          const int hq = col / p.D, d = col % p.D;
+          const float* wrow = wts + (hq - hA) * nsplit;
+          float o = 0.f;
+          for (int j = lane; j < nsplit; j += 32)
+            o = fmaf(__ldcg(p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (p.D + 2) + d), wrow[j], o);
+          o = warp_sum(o);
+          if (lane == 0) oc[cc] = o * gte[cc];
         }
-        residual_epilogue(p, u, nj > 0, acc, cta, G, tid);
-        ++u;
+        cons_sync(kConsumerThreads);
+        const int rpc = kSlotBytes / rb;
+        for (int r0 = 0; r0 < ncol; r0 += rpc) {
+          const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
+          splitk_rows<MG>(ch, min(rpc, ncol - r0), rb, oc + r0, H, acc, tid);
+          release(p, sh, n, lane);
+        }
       }
+      residual_add<MG>(p, H, 2 * l, ncol > 0, acc, tid);
+    }
+
+    // ---- last phase: pre-MLP RMSNorm, SwiGLU gate/up, down-projection split-K ----
+    if (!grid_barrier(p, sh, ++nbar, tid)) return;
+    rmsnorm<MG>(p, H, 2 * l + 1, nullptr, L.norm2, xs, sh, tid, warp, lane);
+    {
+      const int nj = rg.f_e - rg.f_b;
+      float4 acc[MG];
+#pragma unroll
+      for (int k = 0; k < MG; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (nj > 0) {
+        float* gs = fs;
+        float* us = fs + nj;
+        const int rpc = kSlotBytes / rb;
+        XReg<XK> xr;
+        load_xreg<XK>(xr, xs, H, lane);
+        for (int half = 0; half < 2; ++half) {
+          float* out = half ? us : gs;
+          for (int r0 = 0; r0 < nj; r0 += rpc) {
+            const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
+            gemv_rows<XK>(ch, min(rpc, nj - r0), rb, xr, xs, H, warp, lane, r0, kNoSplit, out, out);
+            release(p, sh, n, lane);
+          }
+        }
+        cons_sync(kConsumerThreads);
+        for (int j = tid; j < nj; j += kConsumerThreads) us[j] = siluf_(gs[j]) * us[j];
+        cons_sync(kConsumerThreads);
+        for (int r0 = 0; r0 < nj; r0 += rpc) {
+          const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
+          splitk_rows<MG>(ch, min(rpc, nj - r0), rb, us + r0, H, acc, tid);
+          release(p, sh, n, lane);
+        }
+      }
+      residual_add<MG>(p, H, 2 * l + 1, nj > 0, acc, tid);
     }
   }
 
   // ---------------- final norm, tied LM head, argmax ----------------
-  if (!grid_barrier(p, sh, ++nbar * static_cast<unsigned>(G))) return;
-  rmsnorm_to_smem(p, p.hbuf + static_cast<size_t>(u % 3) * p.H, false, nullptr, p.norm_f, xs, sh, tid, warp, lane);
+  if (!grid_barrier(p, sh, ++nbar, tid)) return;
+  rmsnorm<MG>(p, H, 2 * p.n_layers, nullptr, p.norm_f, xs, sh, tid, warp, lane);
   {
-    const LayerW dummy{};
-    const int ns = phase_segments(p, dummy, kPhFinal, cta, G, segs);
-    int v0 = 0, v1 = 0;
-    split_range(p.V, cta, G, v0, v1);
     float bv = -INFINITY;
     int bi = 0x7FFFFFFF;
-    if (ns) {
-      const Seg sg = segs[0];
-      const int rpc = kSlotBytes / sg.row_bytes;
-      for (int r0 = 0; r0 < sg.rows; r0 += rpc) {
-        const int nr = min(rpc, sg.rows - r0);
-        const uint8_t* ch = acquire(cs, p.err);
-        gemv_chunk(ch, nr, rb, xs, p.H, warp, lane, [&](int r, float v) {
-          const int idx = v0 + r0 + r;
-          if (p.logits) __stcg(p.logits + idx, v);
-          if (v > bv || (v == bv && idx < bi)) { bv = v; bi = idx; }
-        });
-        release(cs);
+    const int v0 = rg.v_b, nv = rg.v_e - rg.v_b;
+    const int rpc = kSlotBytes / rb;
+    XReg<XK> xr;
+    load_xreg<XK>(xr, xs, H, lane);
+    for (int r0 = 0; r0 < nv; r0 += rpc) {
+      const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
+      const int nr = min(rpc, nv - r0);
+      for (int r = warp; r < nr; r += 2 * kConsumerWarps) {
+        const int r1 = r + kConsumerWarps;
+        const bool two = r1 < nr;
+        float a0, a1;
+        dot2_rows<XK>(ch + static_cast<size_t>(r) * rb, ch + static_cast<size_t>(two ? r1 : r) * rb, xr, xs, H, lane,
+                      a0, a1);
+        a0 = warp_sum(a0);
+        a1 = warp_sum(a1);
+        const int i0 = v0 + r0 + r, i1 = v0 + r0 + r1;
+        if (lane == 0 && p.logits) {
+          __stcg(p.logits + i0, a0);
+          if (two) __stcg(p.logits + i1, a1);
+        }
+        if (a0 > bv || (a0 == bv && i0 < bi)) { bv = a0; bi = i0; }
+        if (two && (a1 > bv || (a1 == bv && i1 < bi))) { bv = a1; bi = i1; }
       }
+      release(p, sh, n, lane);
     }
     if (lane == 0) {
       sh->best_v[warp] = bv;
@@ -800,6 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
         }
       }
       if (ci != 0x7FFFFFFF) atomicMax(p.amax, pack_argmax(cv, ci));
+      trace_at(p, 2 * static_cast<int>(nbar) + 1);
       __threadfence();
       const unsigned prev = atomicAdd(p.done, 1u);
       if (prev == static_cast<unsigned>(G - 1)) {
@@ -816,9 +1050,19 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   }
 }
 
+constexpr size_t kSmemLimit = 232448;
+
+size_t decode_scratch_floats(int H) {
+  const size_t fixed = static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + static_cast<size_t>(H) * 4;
+  if (fixed >= kSmemLimit) return 0;
+  size_t f = (kSmemLimit - fixed) / 4;
+  f &= ~static_cast<size_t>(3);
+  return f > 8192 ? 8192 : f;
+}
+
 size_t decode_smem_bytes(int H) {
-  return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + kScratchFloats * sizeof(float) +
-         static_cast<size_t>(H) * 4;
+  return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + static_cast<size_t>(H) * 4 +
+         decode_scratch_floats(H) * 4;
 }
 
 int decode_max_splits(int grid, int hkv) {
@@ -826,34 +1070,33 @@ int decode_max_splits(int grid, int hkv) {
   return per < 1 ? 1 : per;
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s) {
-  const size_t smem = decode_smem_bytes(p.H);
+template <int HK>
+cudaError_t launch_hk(const DecodeParams& p, int grid, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(mk_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem > 232448 ? 232448 : 232448));
+    cudaError_t e = cudaFuncSetAttribute(mk_decode_kernel<HK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemLimit));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.H);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mk_decode_kernel, p);
+  return cudaLaunchKernelEx(&cfg, mk_decode_kernel<HK>, p);
 }
 
-int decode_grid_for_device(int device, int* grid_out) {
-  int sms = 0;
-  cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
-  if (e != cudaSuccess) return -1;
-  *grid_out = sms;
-  return 0;
+cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s) {
+  if (p.H == 1024) return launch_hk<4>(p, grid, s);
+  if (p.H == 256) return launch_hk<1>(p, grid, s);
+  if (p.H == 2048) return launch_hk<8>(p, grid, s);
+  return launch_hk<0>(p, grid, s);
 }
 
 }  // namespace mk

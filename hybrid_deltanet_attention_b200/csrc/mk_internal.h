@@ -13,7 +13,6 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kSlotBytes = 32768;
 constexpr int kSlots = 6;
-constexpr int kScratchFloats = 3072;
 constexpr int kAttnSub = 64;          // positions per online-softmax sub-block
 constexpr int kAttnMinChunk = 32;     // smallest split-K chunk of the KV cache
 
@@ -50,7 +49,7 @@ struct DecodeParams {
   int* pos;
   int* err;
   // workspace (caller-owned)
-  float* hbuf;              // [3][H] rotating residual buffers
+  float* hbuf;              // [5][H] residual stream: 2 bases + 3 deltas (see decode.cu)
   float* z;                 // projection outputs not kept in the conv history
   float* part;              // attention split-K partials [Hq][max_splits][D + 2]
   unsigned* bar;            // grid barrier counter
@@ -65,9 +64,16 @@ struct DecodeParams {
   // (used to replay only the accepted prefix of a verify pass without a host round trip)
   const int* gate_n;
   int gate_i;
+  // optional diagnostics: CTA 0 records %globaltimer (ns) at kernel start, at each grid
+  // barrier arrival and exit, and at the end: trace[0], trace[2k-1], trace[2k], ...
+  unsigned long long* trace;
+  int trace_cap;
+  // how far (bytes per CTA) the L2 prefetch cursor runs ahead of the shared-memory fill
+  int prefetch_bytes;
 };
 
 size_t decode_smem_bytes(int H);
+size_t decode_scratch_floats(int H);   // fp32 scratch per CTA left after the ring and xs
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s);
 int decode_max_splits(int grid, int hkv);
 

@@ -179,6 +179,13 @@ class Model:
         self.lib.mk_sync_status(self.h, _stream_ptr(None), C.byref(err))
         return err.value
 
+    def phase_trace(self, buf: Optional[torch.Tensor]):
+        """Diagnostics: record per-barrier timestamps of CTA 0 into buf (int64 CUDA tensor), or stop (None)."""
+        if buf is None:
+            check(self.lib.mk_phase_trace(self.h, None, 0))
+        else:
+            check(self.lib.mk_phase_trace(self.h, buf.data_ptr(), buf.numel()))
+
     @property
     def launches(self) -> int:
         return int(self.lib.mk_launch_count(self.h))

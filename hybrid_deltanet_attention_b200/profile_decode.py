@@ -1,0 +1,78 @@
+"""Small decode driver for profilers and the per-barrier phase trace.
+
+    python -m hybrid_deltanet_attention_b200.profile_decode [--model 0.8b|tiny] [--prompt 8] [--steps 4] [--trace]
+
+Loads the seeded synthetic model, feeds a short prompt (one decode launch per
+token) and runs `--steps` decode launches. With --trace it prints, for the last
+launch, CTA 0's time between consecutive grid-barrier exits (the phase times) and
+its wait inside each barrier, in microseconds.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--model", default="0.8b")
+    ap.add_argument("--prompt", type=int, default=8)
+    ap.add_argument("--steps", type=int, default=4)
+    ap.add_argument("--trace", action="store_true")
+    ap.add_argument("--mhz", type=float, default=1965.0, help="SM clock used to convert trace cycles to us")
+    args = ap.parse_args()
+
+    import torch
+    import synth
+    import hybrid_deltanet_attention_b200 as hda
+
+    cfg = synth.CONFIGS[args.model]
+    dev = torch.device("cuda", 0)
+    m = hda.Model(cfg, hda.weights_to_device(synth.make_weights(cfg), dev), max_ctx=args.prompt + args.steps + 8)
+    tok = torch.empty(args.steps + 1, dtype=torch.int32, device=dev)
+    m.prefill(torch.from_numpy(synth.make_prompt(cfg, args.prompt)).to(dev), next_token=tok[0:1])
+    buf = torch.zeros(4096, dtype=torch.int64, device=dev) if args.trace else None
+    for i in range(args.steps):
+        if buf is not None and i == args.steps - 1:
+            m.phase_trace(buf)
+        m.decode(tok[i:i + 1], tok[i + 1:i + 2])
+    m.phase_trace(None)
+    err = m.sync()
+    if err:
+        raise SystemExit(f"device error word 0x{err:x}")
+    if buf is not None:
+        t = buf.cpu().numpy()
+        nbar = sum(3 if k == "D" else 4 for k in cfg.pattern)
+        t = t.astype("float64") * (1000.0 / args.mhz)      # cycles -> ns
+        exits = [t[0]] + [t[2 * k] for k in range(1, nbar + 1)]
+        arrivals = [t[2 * k - 1] for k in range(1, nbar + 1)]
+        end = t[2 * nbar + 1]
+        phases = [(exits[k + 1] - exits[k]) / 1e3 for k in range(nbar)] + [(end - exits[nbar]) / 1e3]
+        waits = [(exits[k] - arrivals[k - 1]) / 1e3 for k in range(1, nbar + 1)]
+        names = []
+        for li, kind in enumerate(cfg.pattern):
+            names += [f"L{li}.in", f"L{li}.dn+out", f"L{li}.mlp"] if kind == "D" else \
+                     [f"L{li}.in", f"L{li}.attn", f"L{li}.attn_out", f"L{li}.mlp"]
+        names.append("lm_head")
+        rows = [{"phase": n, "us": round(p, 2), "barrier_wait_us": round(w, 2) if i < len(waits) else None}
+                for i, (n, p, w) in enumerate(zip(names, phases, waits + [0.0]))]
+        total = (end - t[0]) / 1e3
+        chunks = []
+        for n in range((len(t) - 512) // 4):
+            iss, arr, acq, done = t[512 + 4 * n], t[513 + 4 * n], t[514 + 4 * n], t[515 + 4 * n]
+            if iss == 0 and acq == 0:
+                break
+            chunks.append([round((x - t[0]) / 1e3, 3) for x in (iss, arr, acq, done)])
+        print(json.dumps({"total_us": round(total, 1), "phases": rows, "exits_us": [round((e - t[0]) / 1e3, 2) for e in exits],
+                          "chunks_issue_wait_have_done_us": chunks}))
+    print(f"ok: {m.launches} launches")
+
+
+if __name__ == "__main__":
+    main()

@@ -83,7 +83,7 @@ typedef struct mk_config {
   int32_t dn_heads;        /* DeltaNet heads Hd */
   int32_t dn_dk;           /* key dim per head (multiple of 32, <= 256) */
   int32_t dn_dv;           /* value dim per head (<= 256) */
-  int32_t conv_width;      /* causal depthwise conv width W (2..8) */
+  int32_t conv_width;      /* causal depthwise conv width W (2..4) */
   int32_t at_q_heads;      /* attention query heads Hq */
   int32_t at_kv_heads;     /* attention key/value heads Hkv (Hq % Hkv == 0) */
   int32_t at_head_dim;     /* D (multiple of 64, <= 256) */
@@ -200,6 +200,15 @@ int mk_generate(mk_model* m, const int32_t* h_prompt, int32_t n_prompt,
 /* Synchronise `stream`, then return MK_OK, MK_ERR_DEVICE (device error word set; the
  * word itself is stored to *dev_err if non-NULL) or MK_ERR_CUDA. */
 int mk_sync_status(mk_model* m, void* stream, int32_t* dev_err);
+
+/* Diagnostics: while d_trace (device uint64[capacity]) is non-NULL, every decode launch
+ * has CTA 0 record its SM cycle counter at its start (entry 0), at the arrival at and
+ * exit from grid barrier k (entries 2k-1, 2k) and when its LM-head slice is done
+ * (entry 2*n_barriers+1); from entry 512 on, chunk n of its weight stream was issued
+ * (512+4n), consumer warp 0 started waiting for it (513+4n), had it (514+4n) and was
+ * done with it (515+4n). Pass NULL to stop. The buffer
+ * stays the caller's. */
+int mk_phase_trace(mk_model* m, uint64_t* d_trace, int32_t capacity);
 
 /* Number of kernel launches issued by this handle so far (decode, prefill, verify,
  * repack); used to report launch counts. */
