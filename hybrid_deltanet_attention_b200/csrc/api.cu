@@ -28,6 +28,8 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+constexpr size_t kResetBytes = 4096;   // workspace head: barrier/arrival/argmax words, per-head sums of squares
+
 struct Expect {
   int dtype;
   int ndim;
@@ -78,6 +80,26 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ src, uint16_t
     const int c = c0 + i, r = r0 + threadIdx.x;
     if (r < rows && c < cols) dst[static_cast<size_t>(c) * rows + r] = tile[threadIdx.x][i];
   }
+}
+
+// Row r of dst = row r of w (cols bf16) followed by a 16-byte tail: the W conv taps of
+// channel r (bf16) when r < nconv, zeros otherwise.
+__global__ void pack_rows_tail_kernel(const uint16_t* __restrict__ w, const uint16_t* __restrict__ taps,
+                                      uint16_t* __restrict__ dst, int rows, int cols, int nconv, int W) {
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  const int stride = cols + 8;
+  for (int c = threadIdx.x; c < cols; c += blockDim.x) dst[static_cast<size_t>(r) * stride + c] = w[static_cast<size_t>(r) * cols + c];
+  if (threadIdx.x < 8) {
+    const int j = threadIdx.x;
+    dst[static_cast<size_t>(r) * stride + cols + j] = (r < nconv && j < W) ? taps[static_cast<size_t>(r) * W + j] : 0;
+  }
+}
+
+cudaError_t launch_pack_rows_tail(const uint16_t* w, const uint16_t* taps, void* dst, int rows, int cols, int nconv,
+                                  int W, cudaStream_t s) {
+  pack_rows_tail_kernel<<<rows, 256, 0, s>>>(w, taps, static_cast<uint16_t*>(dst), rows, cols, nconv, W);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_transpose_bf16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t s) {
@@ -160,7 +182,11 @@ int check_budget(const mk_config& c, int grid) {
     const long nh = ceil_div(rows, c.dn_dv) + 1;
     if (nh * (2 * c.dn_dk + 2) + 2 * rows > S) return fail(MK_ERR_ARG, "DeltaNet rows per CTA exceed the scratch budget");
     if (2 * nh * c.dn_dk + rows + nh > 3L * mk::kConsumerThreads)
-      return fail(MK_ERR_ARG, "DeltaNet conv channels per CTA exceed the prologue budget");
+      return fail(MK_ERR_ARG, "DeltaNet channels per CTA exceed the prologue budget");
+    const long inrows = ceil_div(static_cast<long>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv) + 2 * c.dn_heads, grid);
+    if (inrows > mk::kConsumerThreads || 7 * inrows > S)
+      return fail(MK_ERR_ARG, "DeltaNet in-projection rows per CTA exceed the conv budget");
+    if (4L * c.dn_heads * 4 + 512 > 4096) return fail(MK_ERR_ARG, "too many DeltaNet heads for the norm buffer");
   }
   if (n_kind(c, 'A')) {
     const long grp = c.at_q_heads / c.at_kv_heads;
@@ -181,7 +207,7 @@ struct Layout {
   size_t p_table, p_freq, p_embed, p_normf;
   std::vector<size_t> p_layer;   // start of each layer block
   // workspace
-  size_t w_sync, w_h, w_z, w_part, w_tok, w_g, w_n, w_snap;
+  size_t w_sync, w_h, w_z, w_y, w_part, w_tok, w_g, w_n, w_snap;
   size_t snap_S, snap_conv;
   int max_splits;
 };
@@ -191,7 +217,7 @@ size_t layer_block_bytes(const mk_config& c, char kind) {
   size_t b = align256(H * 2) * 2;                        // norm1, norm2
   if (kind == 'D') {
     const size_t C = static_cast<size_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
-    b += align256((C + 2 * c.dn_heads) * rb);              // w_in
+    b += align256((C + 2 * c.dn_heads) * (rb + 16));       // w_in, each row + its conv taps
     b += align256(C * c.conv_width * 2);                    // conv
     b += align256(static_cast<size_t>(c.dn_heads) * c.dn_dv * rb);   // w_outT
   } else {
@@ -232,13 +258,14 @@ Layout make_layout(const mk_config& c, int grid) {
 
   L.max_splits = (na ? mk::decode_max_splits(grid, c.at_kv_heads) : 1);
   off = 0;
-  L.w_sync = off; off = align256(off + 1024);
+  L.w_sync = off; off = align256(off + kResetBytes);   // sync words + per-head norms (zeroed on reset)
   L.w_h = off; off = align256(off + 5 * H * 4);   // residual: 2 bases + 3 deltas
   const size_t zf = std::max<size_t>(2 * c.dn_heads,
                                      na ? static_cast<size_t>(c.at_q_heads) * c.at_head_dim * (c.at_out_gate ? 2 : 1) +
                                               2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim
                                         : 0);
   L.w_z = off; off = align256(off + zf * 4);
+  L.w_y = off; off = align256(off + C * 4);
   L.w_part = off;
   off = align256(off + (na ? static_cast<size_t>(c.at_q_heads) * L.max_splits * (c.at_head_dim + 2) * 4 : 4));
   L.w_tok = off; off = align256(off + (static_cast<size_t>(c.max_ctx) + 8) * 4);
@@ -408,8 +435,14 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     off += align256(H * 2);
     if (lw.kind == mk::kDeltaNet) {
       lw.w_in = P + off;
-      if (e == cudaSuccess) e = copy(p + "dn.w_in", off);
-      off += align256((C + 2 * c.dn_heads) * rb);
+      if (e == cudaSuccess) {
+        ++m->launches;
+        e = mk::launch_pack_rows_tail(static_cast<const uint16_t*>(got[p + "dn.w_in"]->data),
+                                      static_cast<const uint16_t*>(got[p + "dn.conv"]->data), P + off,
+                                      static_cast<int>(C + 2 * c.dn_heads), static_cast<int>(H), static_cast<int>(C),
+                                      c.conv_width, s);
+      }
+      off += align256((C + 2 * c.dn_heads) * (rb + 16));
       lw.conv = reinterpret_cast<const uint16_t*>(P + off);
       if (e == cudaSuccess) e = copy(p + "dn.conv", off);
       off += align256(C * c.conv_width * 2);
@@ -479,6 +512,8 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   b.bar = reinterpret_cast<unsigned*>(W + L.w_sync);
   b.done = reinterpret_cast<unsigned*>(W + L.w_sync + 128);
   b.amax = reinterpret_cast<unsigned long long*>(W + L.w_sync + 256);
+  b.ssq = reinterpret_cast<float*>(W + L.w_sync + 512);
+  b.ybuf = reinterpret_cast<float*>(W + L.w_y);
   b.max_splits = L.max_splits;
   b.prefetch_bytes = 384 * 1024;
   if (const char* env = getenv("MK_PREFETCH_KB")) b.prefetch_bytes = atoi(env) * 1024;
@@ -496,7 +531,7 @@ int mk_reset_state(mk_model* m, void* stream) {
   if (!m) return fail(MK_ERR_ARG, "model is NULL");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(m->state, 0, m->sz.state_bytes, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(m->ws, 0, 1024, s);   // barrier, arrival and argmax words
+  if (e == cudaSuccess) e = cudaMemsetAsync(m->ws, 0, kResetBytes, s);   // sync words and per-head norms
   if (e != cudaSuccess) return cuda_fail(e, "reset");
   m->pos_hint = 0;
   return MK_OK;

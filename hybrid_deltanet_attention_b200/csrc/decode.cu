@@ -7,7 +7,7 @@
 //  * each CTA owns a fixed contiguous slice of every weight matrix, of the DeltaNet
 //    state rows, and of the KV cache positions of its attention split. Its slice
 //    bounds are computed once per launch into shared memory. A producer lane streams
-//    that whole per-step sequence through a 6 x 32 KB shared-memory ring with
+//    that whole per-step sequence through a 3 x 64 KB shared-memory ring with
 //    cp.async.bulk (no multicast), independent of the grid barriers; its per-chunk
 //    work is a handful of instructions so it never limits the stream;
 //  * 8 consumer warps do the arithmetic in fp32 from shared memory; activations never
@@ -123,9 +123,9 @@ __device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Range
   if (s == 0) {
     const int b = L.kind == kDeltaNet ? r.in_dn_b : r.in_at_b;
     const int e = L.kind == kDeltaNet ? r.in_dn_e : r.in_at_e;
-    src = L.w_in + static_cast<size_t>(b) * wrb;
+    rb = L.kind == kDeltaNet ? wrb + 16 : wrb;     // DeltaNet rows carry their conv taps
+    src = L.w_in + static_cast<size_t>(b) * rb;
     rows = e - b;
-    rb = wrb;
     return true;
   }
   s -= 1;
@@ -409,26 +409,96 @@ __device__ __forceinline__ void dot2_rows(const uint8_t* p0, const uint8_t* p1, 
   }
 }
 
-// Warp-per-row dot products of nrows bf16 rows (stride rb bytes) with x. Row r's value
-// goes to lo[row_base + r] if row_base + r < split, else to hi[row_base + r - split];
-// lane 0 writes it.
+// Dot products of up to four bf16 rows with x, four independent accumulator chains.
+template <int XK>
+__device__ __forceinline__ void dot4_rows(const uint8_t* p0, const uint8_t* p1, const uint8_t* p2, const uint8_t* p3,
+                                          const XReg<XK>& x, const float* xs, int H, int lane, float* a) {
+  a[0] = a[1] = a[2] = a[3] = 0.f;
+  if (XK > 0) {
+#pragma unroll
+    for (int k = 0; k < XK; ++k) {
+      const int c = lane * 8 + 256 * k;
+      const uint4 w0 = *reinterpret_cast<const uint4*>(p0 + 2 * c);
+      const uint4 w1 = *reinterpret_cast<const uint4*>(p1 + 2 * c);
+      const uint4 w2 = *reinterpret_cast<const uint4*>(p2 + 2 * c);
+      const uint4 w3 = *reinterpret_cast<const uint4*>(p3 + 2 * c);
+      a[0] = dot8_bf16_f32(w0, x.a[k], x.b[k], a[0]);
+      a[1] = dot8_bf16_f32(w1, x.a[k], x.b[k], a[1]);
+      a[2] = dot8_bf16_f32(w2, x.a[k], x.b[k], a[2]);
+      a[3] = dot8_bf16_f32(w3, x.a[k], x.b[k], a[3]);
+    }
+  } else {
+    for (int c = lane * 8; c < H; c += 256) {
+      const float4 xa = *reinterpret_cast<const float4*>(xs + c);
+      const float4 xb = *reinterpret_cast<const float4*>(xs + c + 4);
+      a[0] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p0 + 2 * c), xa, xb, a[0]);
+      a[1] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p1 + 2 * c), xa, xb, a[1]);
+      a[2] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p2 + 2 * c), xa, xb, a[2]);
+      a[3] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p3 + 2 * c), xa, xb, a[3]);
+    }
+  }
+}
+
+// DeltaNet conv epilogue of the in-projection: for a q/k/v row g with raw value x_t,
+// store x_t into the conv history slot of this position, y = SiLU(conv) into ybuf, and
+// (q and k rows) add y^2 into the CTA's per-head partial sums of squares. The taps sit
+// in the 16-byte tail of the row in the chunk; the W-1 older inputs of the CTA's rows
+// were staged in shared memory (chist [rows][3]).
+struct ConvEpi {
+  const float* chist;
+  int b;            // first in-projection row of this CTA
+  int W;
+  int H;            // row length (taps start at byte 2H of the row)
+  int qk_rows;      // 2 * Hd * dk
+  int dk;
+  int h_lo;         // first q/k head (index into [q heads | k heads]) this CTA touches
+  float* ybuf;
+  float* ysq;       // shared memory: y^2 of each of the CTA's rows (indexed by row - b)
+};
+
+__device__ __forceinline__ void conv_epilogue(const ConvEpi& ce, int g, float raw, const uint8_t* row, float* ringc) {
+  const int lr = g - ce.b;
+  const uint2 tw = *reinterpret_cast<const uint2*>(row + 2 * ce.H);
+  const float t0 = bf16lo(tw.x), t1 = bf16hi(tw.x), t2 = bf16lo(tw.y), t3 = bf16hi(tw.y);
+  const float tcur = ce.W == 4 ? t3 : (ce.W == 3 ? t2 : t1);    // the tap of the current input
+  float y = tcur * raw;
+  if (ce.W > 1) y = fmaf(t0, ce.chist[lr * 3 + 0], y);
+  if (ce.W > 2) y = fmaf(t1, ce.chist[lr * 3 + 1], y);
+  if (ce.W > 3) y = fmaf(t2, ce.chist[lr * 3 + 2], y);
+  y = siluf_(y);
+  __stcg(ringc + g, raw);
+  __stcg(ce.ybuf + g, y);
+  ce.ysq[lr] = y * y;
+}
+
+// Warp-per-row dot products of nrows bf16 rows (stride rb bytes) with x; each warp takes
+// rows warp, warp+8, warp+16, warp+24 together. Row r's value goes to lo[row_base + r]
+// if row_base + r < split (through the conv epilogue when ce != nullptr), else to
+// hi[row_base + r - split]; lane 0 writes it.
 template <int XK>
 __device__ __forceinline__ void gemv_rows(const uint8_t* chunk, int nrows, int rb, const XReg<XK>& x, const float* xs,
-                                          int H, int warp, int lane, int row_base, int split, float* lo, float* hi) {
-  for (int r = warp; r < nrows; r += 2 * kConsumerWarps) {
-    const int r1 = r + kConsumerWarps;
-    const bool two = r1 < nrows;
-    float a0, a1;
-    dot2_rows<XK>(chunk + static_cast<size_t>(r) * rb, chunk + static_cast<size_t>(two ? r1 : r) * rb, x, xs, H,
-                  lane, a0, a1);
-    a0 = warp_sum(a0);
-    a1 = warp_sum(a1);
-    if (lane == 0) {
-      const int g0 = row_base + r;
-      if (g0 < split) lo[g0] = a0; else hi[g0 - split] = a0;
-      if (two) {
-        const int g1 = row_base + r1;
-        if (g1 < split) lo[g1] = a1; else hi[g1 - split] = a1;
+                                          int H, int warp, int lane, int row_base, int split, float* lo, float* hi,
+                                          bool use_ce = false, ConvEpi ce = ConvEpi{}) {
+  for (int r = warp; r < nrows; r += 4 * kConsumerWarps) {
+    int rr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) rr[q] = (r + q * kConsumerWarps < nrows) ? r + q * kConsumerWarps : r;
+    float a[4];
+    dot4_rows<XK>(chunk + static_cast<size_t>(rr[0]) * rb, chunk + static_cast<size_t>(rr[1]) * rb,
+                  chunk + static_cast<size_t>(rr[2]) * rb, chunk + static_cast<size_t>(rr[3]) * rb, x, xs, H, lane, a);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) a[q] = warp_sum(a[q]);
+    // lanes 0..3 finish the four rows together (one code path, one row per lane)
+    const int q = lane & 3;
+    const float aq = q == 0 ? a[0] : (q == 1 ? a[1] : (q == 2 ? a[2] : a[3]));
+    const int rq = q == 0 ? rr[0] : (q == 1 ? rr[1] : (q == 2 ? rr[2] : rr[3]));
+    if (lane < 4 && (q == 0 || rq != r)) {
+      const int g = row_base + rq;
+      if (g < split) {
+        if (use_ce) conv_epilogue(ce, g, aq, chunk + static_cast<size_t>(rq) * rb, lo);
+        else lo[g] = aq;
+      } else {
+        hi[g - split] = aq;
       }
     }
   }
@@ -613,27 +683,60 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
 
   for (int l = 0; l < p.n_layers; ++l) {
     const LayerW L = p.layers[l];
-    // ---- phase 1: pre-mixer RMSNorm + input projection ----
+    // ---- phase 1: pre-mixer RMSNorm + input projection (+ DeltaNet conv epilogue) ----
     if (l > 0 && !grid_barrier(p, sh, ++nbar, tid)) return;
-    if (l == 0) {
-      const uint16_t* emb_row = reinterpret_cast<const uint16_t*>(p.embed + static_cast<size_t>(sh->tok) * rb);
-      rmsnorm<MG>(p, H, 0, emb_row, L.norm1, xs, sh, tid, warp, lane);   // the residual starts as the embedding
-    } else {
-      rmsnorm<MG>(p, H, 2 * l, nullptr, L.norm1, xs, sh, tid, warp, lane);
-    }
     {
       const bool dn = (L.kind == kDeltaNet);
       const int b = dn ? rg.in_dn_b : rg.in_at_b, e = dn ? rg.in_dn_e : rg.in_at_e;
       float* ringc = p.conv_ring + static_cast<size_t>(L.idx) * p.convw * p.C + static_cast<size_t>(pos % p.convw) * p.C;
-      const int split = dn ? p.C : kNoSplit;
-      float* lo = dn ? ringc : p.z;
-      const int rpc = kSlotBytes / rb;
+      // older conv inputs of this CTA's q/k/v rows: loads issued before the norm
+      const int nconv = dn ? max(0, min(e, p.C) - b) : 0;
+      const int qk_rows = 2 * p.Hd * p.dk;
+      const int h_lo = (b < qk_rows) ? b / p.dk : 0;
+      const int n_ss = (dn && b < qk_rows) ? (min(e, qk_rows) - 1) / p.dk - h_lo + 1 : 0;
+      float th[kMaxConv - 1];
+      if (tid < nconv) {
+        const float* ringl = p.conv_ring + static_cast<size_t>(L.idx) * p.convw * p.C;
+#pragma unroll
+        for (int j = 0; j < kMaxConv - 1; ++j)
+          if (j < p.convw - 1) th[j] = __ldcg(ringl + static_cast<size_t>((pos + 1 + j) % p.convw) * p.C + b + tid);
+      }
+      if (l == 0) {
+        rmsnorm<MG>(p, H, 0, reinterpret_cast<const uint16_t*>(p.embed + static_cast<size_t>(sh->tok) * rb), L.norm1,
+                    xs, sh, tid, warp, lane);   // the residual starts as the embedding row
+      } else {
+        rmsnorm<MG>(p, H, 2 * l, nullptr, L.norm1, xs, sh, tid, warp, lane);
+      }
+      float* ysq = fs + 3 * kConsumerThreads;
+      ConvEpi ce{fs, b, p.convw, H, qk_rows, p.dk, h_lo, p.ybuf, ysq};
+      if (dn) {
+        if (tid < nconv) {
+#pragma unroll
+          for (int j = 0; j < kMaxConv - 1; ++j)
+            if (j < p.convw - 1) fs[tid * 3 + j] = th[j];
+        }
+        cons_sync(kConsumerThreads);
+      }
+      const int rb_in = dn ? rb + 16 : rb;
+      const int rpc = kSlotBytes / rb_in;
       XReg<XK> xr;
       load_xreg<XK>(xr, xs, H, lane);
       for (int r0 = 0; r0 < e - b; r0 += rpc) {
         const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
-        gemv_rows<XK>(ch, min(rpc, e - b - r0), rb, xr, xs, H, warp, lane, b + r0, split, lo, p.z);
+        gemv_rows<XK>(ch, min(rpc, e - b - r0), rb_in, xr, xs, H, warp, lane, b + r0, dn ? p.C : kNoSplit,
+                      dn ? ringc : p.z, p.z, dn, ce);
         release(p, sh, n, lane);
+      }
+      if (n_ss > 0) {   // this CTA's share of the per-head sums of squares of q and k
+        cons_sync(kConsumerThreads);
+        for (int hs = warp; hs < n_ss; hs += kConsumerWarps) {
+          const int hh = h_lo + hs;
+          const int r_lo = max(b, hh * p.dk), r_hi = min(min(e, qk_rows), (hh + 1) * p.dk);
+          float part = 0.f;
+          for (int r = r_lo + lane; r < r_hi; r += 32) part += ysq[r - b];
+          part = warp_sum(part);
+          if (lane == 0) atomicAdd(p.ssq + (L.idx & 1) * 2 * p.Hd + hh, part);
+        }
       }
     }
     if (!grid_barrier(p, sh, ++nbar, tid)) return;
@@ -652,62 +755,45 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
         float* ab = qk + nh * 2 * p.dk;
         float* vv = ab + 2 * nh;
         float* oc = vv + nrows;
-        const float* ringl = p.conv_ring + static_cast<size_t>(L.idx) * p.convw * p.C;
         const int nqk = 2 * nh * p.dk;
         const int nitems = nqk + nrows + nh;
-        // Items (up to kConvItems per thread): q/k channels of the heads, v channels of
-        // the rows, then the (alpha, beta) gate pairs. Every load is issued first.
-        float wv[kConvItems][kMaxConv], xv[kConvItems][kMaxConv];
+        const float* ssq = p.ssq + (L.idx & 1) * 2 * p.Hd;
+        // One batch of loads: conv outputs of the heads' q and k, of the rows' v, the
+        // gates' inputs and the per-head sums of squares; then L2-normalised q, k.
+        float val[kConvItems], nrm[kConvItems];
 #pragma unroll
         for (int it = 0; it < kConvItems; ++it) {
           const int i = tid + it * kConsumerThreads;
-          if (i < nqk + nrows) {
-            int ch;
-            if (i < nqk) {
-              const int vec = i / p.dk, d = i % p.dk;
-              ch = ((vec & 1) ? p.Hd * p.dk : 0) + (h0 + (vec >> 1)) * p.dk + d;
-            } else {
-              ch = 2 * p.Hd * p.dk + g0 + (i - nqk);   // v channel of (head g/dv, row g%dv)
-            }
-#pragma unroll
-            for (int j = 0; j < kMaxConv; ++j) {
-              if (j < p.convw) {
-                const int slot = (pos + 1 + j) % p.convw;   // holds position pos - (W-1) + j
-                wv[it][j] = bf16_to_f(L.conv[static_cast<size_t>(ch) * p.convw + j]);
-                xv[it][j] = __ldcg(ringl + static_cast<size_t>(slot) * p.C + ch);
-              }
-            }
+          if (i < nqk) {
+            const int vec = i / p.dk, d = i % p.dk;
+            const int hh = h0 + (vec >> 1);
+            const int ch = ((vec & 1) ? p.Hd * p.dk : 0) + hh * p.dk + d;
+            val[it] = __ldcg(p.ybuf + ch);
+            nrm[it] = __ldcg(ssq + ((vec & 1) ? p.Hd : 0) + hh);
+          } else if (i < nqk + nrows) {
+            val[it] = __ldcg(p.ybuf + 2 * p.Hd * p.dk + g0 + (i - nqk));
           } else if (i < nitems) {
             const int hh = i - nqk - nrows;
-            xv[it][0] = __ldcg(p.z + h0 + hh);
-            xv[it][1] = __ldcg(p.z + p.Hd + h0 + hh);
+            val[it] = __ldcg(p.z + h0 + hh);
+            nrm[it] = __ldcg(p.z + p.Hd + h0 + hh);
           }
         }
 #pragma unroll
         for (int it = 0; it < kConvItems; ++it) {
           const int i = tid + it * kConsumerThreads;
-          if (i < nqk + nrows) {
-            float y = 0.f;
-#pragma unroll
-            for (int j = 0; j < kMaxConv; ++j)
-              if (j < p.convw) y = fmaf(wv[it][j], xv[it][j], y);
-            y = siluf_(y);
-            if (i < nqk) qk[i] = y;
-            else vv[i - nqk] = y;
+          if (i < nqk) {
+            qk[i] = val[it] / sqrtf(nrm[it] + 1e-6f);
+          } else if (i < nqk + nrows) {
+            vv[i - nqk] = val[it];
           } else if (i < nitems) {
             const int hh = i - nqk - nrows;
-            ab[2 * hh] = sigmoidf_(-xv[it][0]);      // exp(-softplus(alpha))
-            ab[2 * hh + 1] = sigmoidf_(xv[it][1]);
+            ab[2 * hh] = sigmoidf_(-val[it]);      // exp(-softplus(alpha))
+            ab[2 * hh + 1] = sigmoidf_(nrm[it]);
           }
         }
-        cons_sync(kConsumerThreads);
-        for (int vec = warp; vec < 2 * nh; vec += kConsumerWarps) {   // L2-normalise q and k per head
-          float* dst = qk + vec * p.dk;
-          float ss = 0.f;
-          for (int i = lane; i < p.dk; i += 32) ss = fmaf(dst[i], dst[i], ss);
-          ss = warp_sum(ss);
-          const float inv = 1.0f / sqrtf(ss + 1e-6f);
-          for (int i = lane; i < p.dk; i += 32) dst[i] *= inv;
+        if (cta == G - 1) {   // the norm buffer of the next DeltaNet layer starts from zero
+          float* nz = p.ssq + ((L.idx + 1) & 1) * 2 * p.Hd;
+          for (int i = tid; i < 2 * p.Hd; i += kConsumerThreads) nz[i] = 0.f;
         }
         cons_sync(kConsumerThreads);
         // S rows: S = a S; u = S k; S += b (v - u) k^T; o = S q
@@ -824,14 +910,31 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
 #pragma unroll
                 for (int q = 0; q < 8; ++q) kf[q] = (q < dpl) ? bf16_to_f(krow[q]) : 0.f;
               }
-              for (int t = 0; t < grp; ++t) {
-                const float* qv = qs + t * D + lane * dpl;
-                float d0 = 0.f;
+              float dd[8];
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                  if (q < dpl) d0 = fmaf(qv[q], kf[q], d0);
-                d0 = warp_sum(d0);
-                if (lane == 0) sc[t * kAttnSub + pp] = d0;
+              for (int t = 0; t < 8; ++t) {
+                dd[t] = 0.f;
+                if (t < grp) {
+                  const float* qv = qs + t * D + lane * dpl;
+                  if (dpl == 8) {
+                    const float4 qa = *reinterpret_cast<const float4*>(qv);
+                    const float4 qb = *reinterpret_cast<const float4*>(qv + 4);
+                    dd[t] = qa.x * kf[0] + qa.y * kf[1] + qa.z * kf[2] + qa.w * kf[3] +
+                            qb.x * kf[4] + qb.y * kf[5] + qb.z * kf[6] + qb.w * kf[7];
+                  } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                      if (q < dpl) dd[t] = fmaf(qv[q], kf[q], dd[t]);
+                  }
+                }
+              }
+#pragma unroll
+              for (int t = 0; t < 8; ++t)
+                if (t < grp) dd[t] = warp_sum(dd[t]);
+              if (lane == 0) {
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                  if (t < grp) sc[t * kAttnSub + pp] = dd[t];
               }
             }
             release(p, sh, n, lane);
@@ -845,7 +948,23 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
               float vsum[8];
 #pragma unroll
               for (int t = 0; t < 8; ++t) vsum[t] = 0.f;
-              for (int pp = 0; pp < np; ++pp) {
+              int pp = 0;
+              for (; pp + 4 <= np; pp += 4) {
+                float v4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) v4[q] = bf16_to_f(vch[static_cast<size_t>(pp + q) * D + tid]);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                  if (t < grp) {
+                    const float4 s4 = *reinterpret_cast<const float4*>(sc + t * kAttnSub + pp);
+                    vsum[t] = fmaf(s4.x, v4[0], vsum[t]);
+                    vsum[t] = fmaf(s4.y, v4[1], vsum[t]);
+                    vsum[t] = fmaf(s4.z, v4[2], vsum[t]);
+                    vsum[t] = fmaf(s4.w, v4[3], vsum[t]);
+                  }
+                }
+              }
+              for (; pp < np; ++pp) {
                 const float vvv = bf16_to_f(vch[static_cast<size_t>(pp) * D + tid]);
 #pragma unroll
                 for (int t = 0; t < 8; ++t)
@@ -989,6 +1108,9 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   // ---------------- final norm, tied LM head, argmax ----------------
   if (!grid_barrier(p, sh, ++nbar, tid)) return;
   rmsnorm<MG>(p, H, 2 * p.n_layers, nullptr, p.norm_f, xs, sh, tid, warp, lane);
+  if (cta == G - 1 && p.Hd > 0) {   // the first DeltaNet layer of the next step starts from zero norms
+    for (int i = tid; i < 2 * p.Hd; i += kConsumerThreads) p.ssq[i] = 0.f;
+  }
   {
     float bv = -INFINITY;
     int bi = 0x7FFFFFFF;
@@ -999,21 +1121,26 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     for (int r0 = 0; r0 < nv; r0 += rpc) {
       const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
       const int nr = min(rpc, nv - r0);
-      for (int r = warp; r < nr; r += 2 * kConsumerWarps) {
-        const int r1 = r + kConsumerWarps;
-        const bool two = r1 < nr;
-        float a0, a1;
-        dot2_rows<XK>(ch + static_cast<size_t>(r) * rb, ch + static_cast<size_t>(two ? r1 : r) * rb, xr, xs, H, lane,
-                      a0, a1);
-        a0 = warp_sum(a0);
-        a1 = warp_sum(a1);
-        const int i0 = v0 + r0 + r, i1 = v0 + r0 + r1;
-        if (lane == 0 && p.logits) {
-          __stcg(p.logits + i0, a0);
-          if (two) __stcg(p.logits + i1, a1);
+      for (int r = warp; r < nr; r += 4 * kConsumerWarps) {
+        int rr[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) rr[q] = (r + q * kConsumerWarps < nr) ? r + q * kConsumerWarps : r;
+        float a[4];
+        dot4_rows<XK>(ch + static_cast<size_t>(rr[0]) * rb, ch + static_cast<size_t>(rr[1]) * rb,
+                      ch + static_cast<size_t>(rr[2]) * rb, ch + static_cast<size_t>(rr[3]) * rb, xr, xs, H, lane, a);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a[q] = warp_sum(a[q]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (q == 0 || rr[q] != r) {
+            const int idx = v0 + r0 + rr[q];
+            if (lane == 0 && p.logits) __stcg(p.logits + idx, a[q]);
+            if (a[q] > bv || (a[q] == bv && idx < bi)) {
+              bv = a[q];
+              bi = idx;
+            }
+          }
         }
-        if (a0 > bv || (a0 == bv && i0 < bi)) { bv = a0; bi = i0; }
-        if (two && (a1 > bv || (a1 == bv && i1 < bi))) { bv = a1; bi = i1; }
       }
       release(p, sh, n, lane);
     }

@@ -11,8 +11,8 @@ namespace mk {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
-constexpr int kSlotBytes = 32768;
-constexpr int kSlots = 6;
+constexpr int kSlotBytes = 65536;
+constexpr int kSlots = 3;
 constexpr int kAttnSub = 64;          // positions per online-softmax sub-block
 constexpr int kAttnMinChunk = 32;     // smallest split-K chunk of the KV cache
 
@@ -24,7 +24,8 @@ struct LayerW {
   int idx;                  // index among layers of the same kind
   const uint16_t* norm1;    // [H] bf16
   const uint16_t* norm2;    // [H] bf16
-  const uint8_t* w_in;      // [in_rows][row_bytes]      (row-major [out, in])
+  const uint8_t* w_in;      // [in_rows][row_bytes]      (row-major [out, in]); DeltaNet rows carry a
+                            // 16-byte tail with the row's conv taps (row stride row_bytes + 16)
   const uint16_t* conv;     // [C][W] bf16 (DeltaNet)
   const uint8_t* w_outT;    // [K_mix][row_bytes]       transposed: row j = column j of W_out
   const uint8_t* w_gate;    // [F][row_bytes]
@@ -55,6 +56,8 @@ struct DecodeParams {
   unsigned* bar;            // grid barrier counter
   unsigned* done;           // end-of-step arrival counter
   unsigned long long* amax; // packed (logit, index) maximum
+  float* ybuf;              // [C] conv + SiLU output of the current DeltaNet layer
+  float* ssq;               // [2][2*Hd] per-head sum of squares of q and k (by DeltaNet layer parity)
   int max_splits;
   // per-call io
   const int* in_token;
@@ -79,5 +82,7 @@ int decode_max_splits(int grid, int hkv);
 
 // repack helpers (api.cu launches them)
 cudaError_t launch_transpose_bf16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t s);
+cudaError_t launch_pack_rows_tail(const uint16_t* w, const uint16_t* taps, void* dst, int rows, int cols, int nconv,
+                                  int W, cudaStream_t s);
 
 }  // namespace mk
