@@ -21,6 +21,12 @@ int fail(int code, const std::string& msg) {
   return code;
 }
 
+}  // namespace
+
+void mk_set_last_error(const std::string& msg) { g_err = msg; }
+
+namespace {
+
 int cuda_fail(cudaError_t e, const char* what) {
   g_err = std::string(what) + ": " + cudaGetErrorString(e);
   return MK_ERR_CUDA;
@@ -45,25 +51,7 @@ int n_kind(const mk_config& c, char k) {
 
 }  // namespace
 
-struct mk_model {
-  mk_config cfg;
-  mk_sizes sz;
-  uint8_t* packed;
-  uint8_t* state;
-  uint8_t* ws;
-  int grid;
-  int device;
-  mk::DecodeParams base;
-  std::vector<mk::LayerW> layers_host;
-  int64_t launches;
-  int64_t pos_hint;      // host shadow of the device position (calls through this handle)
-  // workspace sub-buffers used by the host-side drivers
-  int32_t* ws_tok;       // [max_ctx + 8] token staging for prefill / generate
-  int32_t* ws_g;         // [max_draft + 1] greedy tokens of a verify pass
-  int32_t* ws_n;         // accepted-draft count of the last verify pass
-  uint8_t* ws_snap;      // DeltaNet S + conv history + pos snapshot for verify
-  size_t snap_S_bytes, snap_conv_bytes;
-};
+#include "mk_model.h"
 
 namespace mk {
 
@@ -522,6 +510,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   m->ws_n = reinterpret_cast<int32_t*>(W + L.w_n);
   m->ws_snap = c.max_draft > 0 ? W + L.w_snap : nullptr;
   m->snap_S_bytes = L.snap_S;
+  m->step_scratch_bytes = L.w_tok;   // sync words, residual, projections, attention partials
   m->snap_conv_bytes = L.snap_conv;
   *out = m;
   return MK_OK;

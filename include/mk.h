@@ -180,6 +180,26 @@ int mk_set_position(mk_model* m, int32_t pos, void* stream);
 int mk_decode_step(mk_model* m, const int32_t* d_in_token, int32_t* d_out_token,
                    float* d_logits, void* stream);
 
+/* The same decode step as mk_decode_step, but its scratch memory (the barrier words,
+ * residual stream, projection outputs and attention partials that the step uses
+ * internally) lives in a fixed 4 MiB device array inside this library instead of the
+ * workspace given to mk_load_weights. It is for callers that cannot allocate device
+ * memory at the point where they step the model: code running in a CUDA host callback
+ * or stream-ordered host function (where allocating CUDA calls are not allowed), hard
+ * real-time loops that must not stall on cudaMalloc's implicit synchronisation, or hosts
+ * that keep a fixed device-memory budget. It calls no cudaMalloc, cudaFree or other
+ * allocating routine. The paper has no counterpart to it.
+ * - The array is reserved on every GPU that loads libmk.so until the process exits.
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ * - Every call shares the array and it keeps the last call's contents: each call clears,
+ *   on `stream`, the part that must start at zero. Calls whose kernels overlap on the
+ *   GPU (other streams, other threads, other models) race on the array.
+ * - Returns MK_ERR_CAPACITY if the model's per-step scratch exceeds 4 MiB; otherwise the
+ *   same arguments, results and errors as mk_decode_step. */
+int mk_decode_step_noalloc(mk_model* m, const int32_t* d_in_token, int32_t* d_out_token,
+                           float* d_logits, void* stream);
+
 /* Speculative verify (exact greedy acceptance, the open-jet follow-up's speed section):
  * d_tokens = [last committed token, d_1 .. d_K] (device int32[K+1]), 1 <= K <= max_draft.
  * Scores all K+1 positions; n = the longest prefix with d_j equal to the greedy token
