@@ -5,7 +5,11 @@ Workload: the 0.8B-shaped hybrid (24 layers, [D,D,D,A] x 6, hidden 1024, vocab
 then tg128: 128 greedy decode steps at batch 1. One bench step = restore the
 post-prompt state, then 128 decode launches (one kernel launch per token).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {mk,reference}]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {mk,reference}] [--workload {tg128,long}]
+
+--workload long times the long-context variant instead: the same model with a seeded
+32768-position bf16 KV cache in every attention layer (N(0, 1), RoPE applied) and
+DeltaNet states from N(0, 0.1), then 128 greedy decode steps from position 32768.
 
 Prints one JSON line (rank 0). With --gpus N > 1 (launched by torchrun) every rank
 runs an independent replica on its own GPU; there is no data-path collective.
@@ -32,9 +36,13 @@ METRIC = "batch-1 decode tok/s (hybrid DeltaNet, tg128) and % of B200 HBM roofli
 PROMPT = 128
 TG = 128
 MAX_CTX = PROMPT + TG + 16
+LONG_POS = 32768
 WORKLOAD = ("0.8B-shaped hybrid Gated-DeltaNet + attention (24 layers [D,D,D,A]x6, hidden 1024, "
             "vocab 151936 tied, DeltaNet 16 heads dk=dv=128, attention 8q/2kv heads D=256, SwiGLU 3584), "
             "bf16 weights N(0,0.02) seed 1, 128-token random prompt, tg128 greedy decode, batch 1")
+LONG_WORKLOAD = ("0.8B-shaped hybrid (as tg128), long context: seeded bf16 KV cache of 32768 positions per "
+                 "attention layer (N(0,1), RoPE applied, seed 3), DeltaNet states N(0,0.1), then 128 greedy "
+                 "decode steps at batch 1 from position 32768")
 KERNEL_SOURCES = ["hybrid_deltanet_attention_b200/csrc/decode.cu", "hybrid_deltanet_attention_b200/csrc/dev.cuh",
                   "hybrid_deltanet_attention_b200/csrc/mk_internal.h"]
 
@@ -234,6 +242,22 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ the CUDA path
+def seed_long_context(m, cfg, n_pos, dev):
+    """Write the seeded long-context state into the model's state buffer."""
+    import torch
+    import synth
+    ks, vs, ss = synth.long_context_state(cfg, n_pos)
+    m.reset()
+    kc, vc, S = m.k_cache, m.v_cache, m.S
+    for ai in range(cfg.n_at):
+        kc[ai, :, :n_pos] = torch.from_numpy(ks[ai].view(np.int16)).to(dev).view(torch.bfloat16)
+        vc[ai, :, :n_pos] = torch.from_numpy(vs[ai].view(np.int16)).to(dev).view(torch.bfloat16)
+    for li in range(cfg.n_dn):
+        S[li] = torch.from_numpy(ss[li]).to(dev)
+    m.set_position(n_pos)
+    return int(synth.stream(3, "long.first_token").integers(0, cfg.vocab))
+
+
 def run_mk(args):
     import torch
     import hybrid_deltanet_attention_b200 as hda
@@ -242,16 +266,21 @@ def run_mk(args):
     rank, world, local = dist_setup(args.gpus)
     cfg = synth.QWEN_08B
     dev = torch.device("cuda", local)
+    long_ctx = args.workload == "long"
+    P0 = LONG_POS if long_ctx else PROMPT
     raw = synth.make_weights(cfg)
-    m = hda.Model(cfg, hda.weights_to_device(raw, dev), max_ctx=MAX_CTX)
+    m = hda.Model(cfg, hda.weights_to_device(raw, dev), max_ctx=(LONG_POS + TG + 16) if long_ctx else MAX_CTX)
     del raw
     prompt_np = synth.make_prompt(cfg, PROMPT)
     prompt = torch.from_numpy(prompt_np).to(dev)
 
-    # context after the prompt, snapshotted once; every step restores it
+    # context after the prompt (or the seeded long context), snapshotted once; every step restores it
     first = torch.empty(1, dtype=torch.int32, device=dev)
-    m.reset()
-    m.prefill(prompt, next_token=first)
+    if long_ctx:
+        first.fill_(seed_long_context(m, cfg, LONG_POS, dev))
+    else:
+        m.reset()
+        m.prefill(prompt, next_token=first)
     assert m.sync() == 0
     snap = m.state.clone()
     first_tok = first.clone()
@@ -260,7 +289,7 @@ def run_mk(args):
 
     def one_step(ev=None):
         m.state.copy_(snap)
-        m.set_position(PROMPT)          # same value as the snapshot; keeps the handle's position in step
+        m.set_position(P0)              # same value as the snapshot; keeps the handle's position in step
         toks[0:1].copy_(first_tok)
         if ev is not None:
             ev[0].record(stream)
@@ -294,7 +323,6 @@ def run_mk(args):
     value = world * args.steps * TG / (total_ms / 1000.0)
 
     # roofline of the decode kernel: algorithmic bytes per launch / average launch duration
-    P0 = PROMPT
     per = [bytes_per_token(cfg, P0 + i) for i in range(TG)]
     read_avg = float(np.mean([b["read"] for b in per]))
     write_avg = float(np.mean([b["write"] for b in per]))
@@ -302,28 +330,55 @@ def run_mk(args):
     peak, peak_kind = measured_peaks()
     achieved = read_avg / t_launch / 1e9
     khash = kernel_hash()
-    traffic = recorded_traffic(khash)
+    traffic = None if long_ctx else recorded_traffic(khash)
 
-    # end to end through the public C call with host buffers: prompt in, tokens out
-    pinned_in = torch.from_numpy(prompt_np).pin_memory()
-    pinned_out = torch.empty(TG, dtype=torch.int32).pin_memory()
-    for _ in range(max(1, args.warmup // 2)):
-        m.reset()
-        m.generate(pinned_in.numpy(), TG, out=pinned_out.numpy())
-    e2e_steps = max(1, min(args.steps, 5))
-    barrier(world)
-    torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        m.reset()
-        m.generate(pinned_in.numpy(), TG, out=pinned_out.numpy())
-    dt = max_over_ranks(time.perf_counter() - t0, world)
-    e2e = world * e2e_steps * TG / dt
+    if long_ctx:
+        # end to end: the first token from pinned host memory in, 128 decode launches,
+        # the generated tokens back to pinned host memory (the seeded context stays resident)
+        h_in = torch.tensor([int(first_tok.item())], dtype=torch.int32).pin_memory()
+        h_out = torch.empty(TG + 1, dtype=torch.int32).pin_memory()
+
+        def e2e_step():
+            m.state.copy_(snap)
+            m.set_position(P0)
+            toks[0:1].copy_(h_in, non_blocking=True)
+            for i in range(TG):
+                m.decode(toks[i:i + 1], toks[i + 1:i + 2])
+            h_out.copy_(toks, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+        e2e_step()
+        e2e_steps = max(1, min(args.steps, 5))
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            e2e_step()
+        dt = max_over_ranks(time.perf_counter() - t0, world)
+        e2e = world * e2e_steps * TG / dt
+        e2e_io = (4, (TG + 1) * 4, "first token pinned host -> device, 128 decode launches over the seeded "
+                                   "32K context, tokens device -> pinned host")
+    else:
+        # end to end through the public C call with host buffers: prompt in, tokens out
+        pinned_in = torch.from_numpy(prompt_np).pin_memory()
+        pinned_out = torch.empty(TG, dtype=torch.int32).pin_memory()
+        for _ in range(max(1, args.warmup // 2)):
+            m.reset()
+            m.generate(pinned_in.numpy(), TG, out=pinned_out.numpy())
+        e2e_steps = max(1, min(args.steps, 5))
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            m.reset()
+            m.generate(pinned_in.numpy(), TG, out=pinned_out.numpy())
+        dt = max_over_ranks(time.perf_counter() - t0, world)
+        e2e = world * e2e_steps * TG / dt
+        e2e_io = (PROMPT * 4, TG * 4, "mk_generate: pinned host prompt (128) -> prefill -> 128 greedy tokens -> pinned host")
     if rank != 0:
         return 0
 
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not long_ctx:
         v, cores, sample = oracle_sample()
         cpu = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample}
 
@@ -332,15 +387,16 @@ def run_mk(args):
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens_per_step": TG, "prompt": PROMPT,
+        "config": {"workload": LONG_WORKLOAD if long_ctx else WORKLOAD, "tokens_per_step": TG,
+                   "context_at_start": P0,
                    "l2": "inputs larger than L2: every step streams 1.23 GB of weights (L2 is 126 MB)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_kind": peak_kind,
                      "bytes_per_launch_read": read_avg, "bytes_per_launch_write": write_avg,
                      "kernel": "mk_decode_kernel", "avg_launch_us": t_launch * 1e6, "kernel_hash": khash},
-        "e2e": {"value": e2e, "unit": "tok/s", "h2d_bytes_per_step": PROMPT * 4, "d2h_bytes_per_step": TG * 4,
-                "what": "mk_generate: pinned host prompt (128) -> prefill -> 128 greedy tokens -> pinned host"},
+        "e2e": {"value": e2e, "unit": "tok/s", "h2d_bytes_per_step": e2e_io[0], "d2h_bytes_per_step": e2e_io[1],
+                "what": e2e_io[2]},
         "gpu_launches": launches,
         "clocks": clocks,
         "cpu_baseline": cpu,
@@ -359,6 +415,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="tg128", choices=["tg128", "long"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

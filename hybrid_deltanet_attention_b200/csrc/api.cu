@@ -247,7 +247,7 @@ Layout make_layout(const mk_config& c, int grid) {
   L.max_splits = (na ? mk::decode_max_splits(grid, c.at_kv_heads) : 1);
   off = 0;
   L.w_sync = off; off = align256(off + kResetBytes);   // sync words + per-head norms (zeroed on reset)
-  L.w_h = off; off = align256(off + 5 * H * 4);   // residual: 2 bases + 3 deltas
+  L.w_h = off; off = align256(off + (2 + 3 * mk::kResCopies) * H * 4);   // residual: 2 bases + 3 spread deltas
   const size_t zf = std::max<size_t>(2 * c.dn_heads,
                                      na ? static_cast<size_t>(c.at_q_heads) * c.at_head_dim * (c.at_out_gate ? 2 : 1) +
                                               2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim
@@ -503,7 +503,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   b.ssq = reinterpret_cast<float*>(W + L.w_sync + 512);
   b.ybuf = reinterpret_cast<float*>(W + L.w_y);
   b.max_splits = L.max_splits;
-  b.prefetch_bytes = 384 * 1024;
+  b.prefetch_bytes = 0;   // L2 prefetch ahead of the ring: measured slower on B200, off by default
   if (const char* env = getenv("MK_PREFETCH_KB")) b.prefetch_bytes = atoi(env) * 1024;
   m->ws_tok = reinterpret_cast<int32_t*>(W + L.w_tok);
   m->ws_g = reinterpret_cast<int32_t*>(W + L.w_g);

@@ -173,13 +173,50 @@ __device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Range
   return false;
 }
 
-// One lane streams the CTA's chunks into the shared-memory ring.
+// A second walk over the same chunk sequence, used to issue L2 prefetches ahead of the
+// shared-memory fill. next() yields the chunks in stream order; false at the end.
+struct PrefetchCursor {
+  int l = 0, s = -1, r0 = 0, rows = 0, rb = 1;
+  const uint8_t* src = nullptr;
+  LayerW L;
+
+  __device__ bool next(const DecodeParams& p, const Ranges& r, const uint8_t*& ptr, uint32_t& bytes) {
+    for (;;) {
+      if (l > p.n_layers) return false;
+      if (r0 < rows) {
+        const int rpc = kSlotBytes / rb;
+        ptr = src + static_cast<size_t>(r0) * rb;
+        bytes = static_cast<uint32_t>(min(rpc, rows - r0)) * rb;
+        r0 += rpc;
+        return true;
+      }
+      if (s < 0) L = p.layers[l < p.n_layers ? l : p.n_layers - 1];
+      ++s;
+      r0 = 0;
+      rows = 0;
+      if (!layer_segment(p, r, L, l, s, src, rows, rb)) {
+        ++l;
+        s = -1;
+        rows = 0;
+      }
+    }
+  }
+};
+
+// One lane streams the CTA's chunks into the shared-memory ring. With a nonzero
+// p.prefetch_bytes it also keeps L2 prefetches of the chunks that follow running that
+// many bytes ahead, so HBM keeps streaming while the ring is full and the consumers
+// wait at a grid barrier.
 __device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) {
   const uint64_t pol = policy_evict_first();
   const Ranges r = sh->rg;
   volatile int* abort = &sh->abort_flag;
   uint32_t n = 0;
   bool ok = true;
+  PrefetchCursor pf;
+  const uint64_t pf_dist = p.prefetch_bytes > 0 ? static_cast<uint64_t>(p.prefetch_bytes) : 0;
+  uint64_t filled = 0, prefetched = 0;
+  bool pf_live = pf_dist > 0;
   LayerW L = p.layers[0];
   for (int l = 0; l <= p.n_layers && ok; ++l) {
     const LayerW Lnext = (l + 1 < p.n_layers) ? p.layers[l + 1] : L;   // load ahead of use
@@ -203,6 +240,17 @@ __device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) 
                  &sh->full[slot], pol);
         trace_at(p, kTraceChunks + 4 * static_cast<int>(n));
         ++n;
+        filled += bytes;
+        while (pf_live && prefetched < filled + pf_dist) {
+          const uint8_t* pp;
+          uint32_t pb;
+          if (!pf.next(p, r, pp, pb)) {
+            pf_live = false;
+            break;
+          }
+          if (prefetched + pb > filled) prefetch_l2(pp, pb);   // chunks already in the ring need none
+          prefetched += pb;
+        }
       }
     }
     L = Lnext;
@@ -281,15 +329,17 @@ __device__ __forceinline__ float cons_sum(float v, Shared* sh, int warp, int lan
 }
 
 // Residual stream between norm phases j and j+1 (j counts every RMSNorm of the step):
-// h_j = base[j % 2] + delta[j % 3]. The update between norms j and j+1 reduces its
-// partial sums into delta[(j+1) % 3]; the RMSNorm of phase j+1 adds the two, and CTA 0
-// writes the sum to base[(j+1) % 2]. CTA G-1 zeroes delta[(j+2) % 3] during phase j.
-// No CTA reads the old residual on its own critical path.
+// h_j = base[j % 2] + sum_c delta[j % 3][c]. The update between norms j and j+1 reduces
+// its partial sums into delta[(j+1) % 3]; CTA i adds into copy i % kResCopies, so each
+// address takes G / kResCopies additions instead of G (the additions of all CTAs to one
+// address serialise in L2). The RMSNorm of phase j+1 adds base and the copies, and CTA 0
+// writes the sum to base[(j+1) % 2]. During phase j the last kResCopies CTAs zero one
+// copy each of delta[(j+2) % 3]. No CTA reads the old residual on its own critical path.
 __device__ __forceinline__ float* res_base(const DecodeParams& p, int H, int j) {
   return p.hbuf + static_cast<size_t>(j % 2) * H;
 }
-__device__ __forceinline__ float* res_delta(const DecodeParams& p, int H, int j) {
-  return p.hbuf + static_cast<size_t>(2 + j % 3) * H;
+__device__ __forceinline__ float* res_delta(const DecodeParams& p, int H, int j, int copy) {
+  return p.hbuf + static_cast<size_t>(2 + (j % 3) * kResCopies + copy) * H;
 }
 
 // Norm phase j: xs = h_j / sqrt(mean(h_j^2) + eps) * gamma (fp32, kept on chip), with
@@ -311,19 +361,22 @@ __device__ __forceinline__ void rmsnorm(const DecodeParams& p, int H, int j, con
     }
   } else {
     const float4* hb = reinterpret_cast<const float4*>(res_base(p, H, j));
-    const float4* hd = reinterpret_cast<const float4*>(res_delta(p, H, j));
-    float4 d[MG];
 #pragma unroll
     for (int k = 0; k < MG; ++k) {
       const int g = tid + k * kConsumerThreads;
-      if (g < ng) {
-        v[k] = __ldcg(hb + g);
-        d[k] = __ldcg(hd + g);
-      }
+      if (g < ng) v[k] = __ldcg(hb + g);
     }
 #pragma unroll
-    for (int k = 0; k < MG; ++k) {
-      v[k].x += d[k].x; v[k].y += d[k].y; v[k].z += d[k].z; v[k].w += d[k].w;
+    for (int c = 0; c < kResCopies; ++c) {
+      const float4* hd = reinterpret_cast<const float4*>(res_delta(p, H, j, c));
+#pragma unroll
+      for (int k = 0; k < MG; ++k) {
+        const int g = tid + k * kConsumerThreads;
+        if (g < ng) {
+          const float4 d = __ldcg(hd + g);
+          v[k].x += d.x; v[k].y += d.y; v[k].z += d.z; v[k].w += d.w;
+        }
+      }
     }
   }
   if (cta == 0) {    // materialise h_j as the next base
@@ -334,11 +387,13 @@ __device__ __forceinline__ void rmsnorm(const DecodeParams& p, int H, int j, con
       if (g < ng) __stcg(nb + g, v[k]);
     }
   }
-  if (cta == G - 1) {  // the delta that the update after norm j+1 accumulates into
-    float4* z = reinterpret_cast<float4*>(res_delta(p, H, j + 2));
+  // the delta that the update after norm j+1 accumulates into: copy c is zeroed by CTA
+  // G-1-c (by CTA G-1-(c mod G) on a grid smaller than kResCopies)
+  for (int c = G - 1 - cta; c < kResCopies; c += G) {
+    float4* z = reinterpret_cast<float4*>(res_delta(p, H, j + 2, c));
     for (int g = tid; g < ng; g += kConsumerThreads) __stcg(z + g, make_float4(0.f, 0.f, 0.f, 0.f));
     if (j == 0) {
-      float4* z1 = reinterpret_cast<float4*>(res_delta(p, H, 1));
+      float4* z1 = reinterpret_cast<float4*>(res_delta(p, H, 1, c));
       for (int g = tid; g < ng; g += kConsumerThreads) __stcg(z1 + g, make_float4(0.f, 0.f, 0.f, 0.f));
     }
   }
@@ -554,17 +609,18 @@ __device__ __forceinline__ void splitk_rows(const uint8_t* chunk, int nrows, int
   }
 }
 
-// The update that follows norm j: delta[(j+1) % 3] += this CTA's partial sums.
+// The update that follows norm j: delta[(j+1) % 3][cta % kResCopies] += this CTA's
+// partial sums (fire-and-forget vector reductions).
 template <int MG>
 __device__ __forceinline__ void residual_add(const DecodeParams& p, int H, int j, bool has_rows, const float4* acc,
                                              int tid) {
   if (!has_rows) return;
   const int ng = H / 4;
-  float4* nd = reinterpret_cast<float4*>(res_delta(p, H, j + 1));
+  float4* nd = reinterpret_cast<float4*>(res_delta(p, H, j + 1, static_cast<int>(blockIdx.x) % kResCopies));
 #pragma unroll
   for (int k = 0; k < MG; ++k) {
     const int g = tid + k * kConsumerThreads;
-    if (g < ng) atomicAdd(nd + g, acc[k]);
+    if (g < ng) red_add_v4(nd + g, acc[k]);
   }
 }
 

@@ -106,6 +106,13 @@ __device__ __forceinline__ int ld_volatile(const int* p) {
   return *reinterpret_cast<const volatile int*>(p);
 }
 
+// Vector reduction without a return value: *p += v (four fp32 adds, relaxed, gpu scope).
+__device__ __forceinline__ void red_add_v4(float4* p, float4 v) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+
 // Named barrier over the consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void cons_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");

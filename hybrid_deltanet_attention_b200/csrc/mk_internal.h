@@ -14,6 +14,7 @@ constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kSlotBytes = 65536;
 constexpr int kSlots = 3;
 constexpr int kAttnSub = 64;          // positions per online-softmax sub-block
+constexpr int kResCopies = 8;          // copies of each residual delta (CTA c adds into copy c % 8)
 constexpr int kAttnMinChunk = 32;     // smallest split-K chunk of the KV cache
 
 enum LayerKind : int { kDeltaNet = 0, kAttention = 1 };
@@ -50,7 +51,7 @@ struct DecodeParams {
   int* pos;
   int* err;
   // workspace (caller-owned)
-  float* hbuf;              // [5][H] residual stream: 2 bases + 3 deltas (see decode.cu)
+  float* hbuf;              // [2 + 3 * kResCopies][H] residual stream: 2 bases + 3 deltas (see decode.cu)
   float* z;                 // projection outputs not kept in the conv history
   float* part;              // attention split-K partials [Hq][max_splits][D + 2]
   unsigned* bar;            // grid barrier counter
