@@ -28,6 +28,7 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;   // 200 ms for in-flight copie
 constexpr int kMaxConv = 4;          // causal conv width limit (the configs use 4)
 constexpr int kConvItems = 3;        // conv items per consumer thread in the DeltaNet prologue
 constexpr int kNoSplit = 0x7FFFFFFF;
+constexpr int kMaxHead = 256;        // largest attention head dim
 
 // Per-CTA slice bounds, computed once per launch by thread 0.
 struct Ranges {
@@ -50,6 +51,8 @@ struct __align__(16) Shared {
   int pos;
   int bad;
   float red[kConsumerWarps];
+  float rope_c[kMaxHead / 2];   // cos / sin of pos * inv_freq_i for this launch's position
+  float rope_s[kMaxHead / 2];
   float best_v[kConsumerWarps];
   int best_i[kConsumerWarps];
   Ranges rg;
@@ -102,6 +105,14 @@ __device__ void compute_ranges(const DecodeParams& p, int cta, int G, int pos, R
 constexpr int kTraceChunks = 512;
 __device__ __forceinline__ void trace_at(const DecodeParams& p, int idx) {
   if (p.trace && blockIdx.x == 0 && idx < p.trace_cap) p.trace[idx] = clock64();
+}
+// From kTraceGrid: every CTA stamps %globaltimer (ns) when it arrives at grid barrier k
+// (entry kTraceGrid + 2 (k G + cta)) and when it leaves it (the next entry).
+constexpr int kTraceGrid = 8192;
+__device__ __forceinline__ void trace_grid(const DecodeParams& p, unsigned k, int leave) {
+  if (!p.trace) return;
+  const long long ix = kTraceGrid + 2ll * (static_cast<long long>(k) * gridDim.x + blockIdx.x) + leave;
+  if (ix < p.trace_cap) p.trace[ix] = global_ns();
 }
 
 // ------------------------------------------------------------------ producer
@@ -291,6 +302,7 @@ __device__ bool grid_barrier(const DecodeParams& p, Shared* sh, unsigned k, int 
   cons_sync(kConsumerThreads);
   if (tid == 0) {
     trace_at(p, 2 * static_cast<int>(k) - 1);
+    trace_grid(p, k, 0);
     int stop = sh->abort_flag;
     if (!stop) {
       red_release_add(p.bar, 1u);
@@ -311,6 +323,7 @@ __device__ bool grid_barrier(const DecodeParams& p, Shared* sh, unsigned k, int 
       }
     }
     trace_at(p, 2 * static_cast<int>(k));
+    trace_grid(p, k, 1);
     if (stop) sh->abort_flag = 1;
     sh->decision = stop;
   }
@@ -730,6 +743,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   // ---------------- consumers ----------------
   if (tid == 0) trace_at(p, 0);
   const int pos = sh->pos;
+  if (p.Hkv > 0) {   // RoPE table of this position, shared by every attention layer
+    for (int i = tid; i < p.D / 2; i += kConsumerThreads)
+      rope_cs(static_cast<double>(pos) * p.inv_freq[i], sh->rope_c[i], sh->rope_s[i]);
+  }   // published to the other consumer warps by the named barriers inside the first RMSNorm
   const Ranges& rg = sh->rg;
   const int rb = p.row_bytes;
   const int H = HK > 0 ? HK * 256 : p.H;
@@ -918,8 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
         const size_t cache_g = (static_cast<size_t>(L.idx) * p.Hkv + ug) * p.max_ctx * D;
         for (int idx = tid; idx < (grp + (has_cur ? 1 : 0)) * half; idx += kConsumerThreads) {
           const int t = idx / half, i = idx % half;
-          float cs, sn;
-          rope_cs(static_cast<double>(pos) * p.inv_freq[i], cs, sn);
+          const float cs = sh->rope_c[i], sn = sh->rope_s[i];
           if (t < grp) {
             const int hq = ug * grp + t;
             const float x1 = __ldcg(p.z + hq * D + i), x2 = __ldcg(p.z + hq * D + i + half);

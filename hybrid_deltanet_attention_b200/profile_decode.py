@@ -28,6 +28,7 @@ def main():
     ap.add_argument("--mhz", type=float, default=1965.0, help="SM clock used to convert trace cycles to us")
     args = ap.parse_args()
 
+    import numpy as np
     import torch
     import synth
     import hybrid_deltanet_attention_b200 as hda
@@ -37,7 +38,9 @@ def main():
     m = hda.Model(cfg, hda.weights_to_device(synth.make_weights(cfg), dev), max_ctx=args.prompt + args.steps + 8)
     tok = torch.empty(args.steps + 1, dtype=torch.int32, device=dev)
     m.prefill(torch.from_numpy(synth.make_prompt(cfg, args.prompt)).to(dev), next_token=tok[0:1])
-    buf = torch.zeros(4096, dtype=torch.int64, device=dev) if args.trace else None
+    nbar = sum(3 if k == "D" else 4 for k in cfg.pattern)
+    G = int(m.sizes.grid_ctas)
+    buf = torch.zeros(8192 + 2 * (nbar + 1) * G, dtype=torch.int64, device=dev) if args.trace else None
     for i in range(args.steps):
         if buf is not None and i == args.steps - 1:
             m.phase_trace(buf)
@@ -47,9 +50,8 @@ def main():
     if err:
         raise SystemExit(f"device error word 0x{err:x}")
     if buf is not None:
-        t = buf.cpu().numpy()
-        nbar = sum(3 if k == "D" else 4 for k in cfg.pattern)
-        t = t.astype("float64") * (1000.0 / args.mhz)      # cycles -> ns
+        raw = buf.cpu().numpy()
+        t = raw[:8192].astype("float64") * (1000.0 / args.mhz)      # cycles -> ns
         exits = [t[0]] + [t[2 * k] for k in range(1, nbar + 1)]
         arrivals = [t[2 * k - 1] for k in range(1, nbar + 1)]
         end = t[2 * nbar + 1]
@@ -69,8 +71,25 @@ def main():
             if iss == 0 and acq == 0:
                 break
             chunks.append([round((x - t[0]) / 1e3, 3) for x in (iss, arr, acq, done)])
+        # all CTAs (global timer, ns): per phase kind, the work (median arrival - median
+        # exit of the previous barrier), the skew (last arrival - median arrival) and the
+        # propagation (median exit - last arrival)
+        grid = raw[8192:8192 + 2 * (nbar + 1) * G].astype("float64").reshape(nbar + 1, G, 2)
+        kinds = {}
+        for k in range(1, nbar + 1):
+            a, e = grid[k, :, 0], grid[k, :, 1]
+            work = (np.median(a) - np.median(grid[k - 1, :, 1])) / 1e3 if k > 1 else None
+            kind = names[k - 1].split(".")[-1]
+            d = kinds.setdefault(kind, {"n": 0, "work_us": 0.0, "skew_us": 0.0, "prop_us": 0.0})
+            d["n"] += 1
+            d["work_us"] += (work or 0.0)
+            d["skew_us"] += (a.max() - np.median(a)) / 1e3
+            d["prop_us"] += (np.median(e) - a.max()) / 1e3
+        for d in kinds.values():
+            for key in ("work_us", "skew_us", "prop_us"):
+                d[key] = round(d[key] / d["n"], 3)
         print(json.dumps({"total_us": round(total, 1), "phases": rows, "exits_us": [round((e - t[0]) / 1e3, 2) for e in exits],
-                          "chunks_issue_wait_have_done_us": chunks}))
+                          "chunks_issue_wait_have_done_us": chunks, "grid_barriers": kinds}))
     print(f"ok: {m.launches} launches")
 
 
