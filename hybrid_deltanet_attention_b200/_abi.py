@@ -35,7 +35,7 @@ MK_MAX_LAYERS = 128
 EXPORTS = [
     "mk_query_sizes", "mk_load_weights", "mk_reset_state", "mk_set_position", "mk_prefill",
     "mk_decode_step", "mk_decode_step_noalloc", "mk_verify_drafts", "mk_generate", "mk_sync_status", "mk_phase_trace", "mk_launch_count",
-    "mk_last_error", "mk_free",
+    "mk_linear", "mk_last_error", "mk_free",
 ]
 
 
@@ -118,6 +118,7 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "mk_sync_status": (C.c_int, [vp, vp, p_i32]),
         "mk_phase_trace": (C.c_int, [vp, vp, i32]),
         "mk_launch_count": (i64, [vp]),
+        "mk_linear": (C.c_int, [vp, i64, i32, i32, vp, i64, i32, vp, i64, i32, vp, C.c_size_t, vp, vp]),
         "mk_last_error": (C.c_char_p, []),
         "mk_free": (None, [vp]),
     }

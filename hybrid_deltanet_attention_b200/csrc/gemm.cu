@@ -1,0 +1,296 @@
+// Linear layers of the prefill on the sm_100a tensor cores.
+//
+//   C[m][n] (+)= sum_k X[m][k] * W[n][k]      (m < M tokens, n < N features, k < K)
+//
+// X arrives as fp32 and is split into bf16 high and low parts (X = Xhi + Xlo up to the
+// rounding of Xlo, about 16 bits of X's mantissa kept); W is bf16. Both parts multiply
+// the same W tile into one fp32 accumulator in tensor memory, so the product carries
+// the activations at about fp32 precision, the same precision the decode megakernel
+// keeps its activations at.
+//
+// One CTA computes one 128 x BN tile of C:
+//   warp 0   allocates BN TMEM columns; its lane 0 is the TMA producer: per 64-wide K
+//            block it loads Xhi, Xlo [128 x 64] and W [BN x 64] (128-byte swizzled) into a
+//            4-stage shared-memory ring;
+//   warp 1   lane 0 issues tcgen05.mma (M = 128, N = BN, K = 16; 8 per K block) and
+//            commits each stage back to the producer, then the accumulator;
+//   warps 2-5 read the accumulator rows from TMEM (warp w owns lanes 32 (w % 4) ..) and
+//            store (or add into) C.
+// Every wait has a time limit; on expiry the CTA latches an error bit and winds down.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+#include "mk_model.h"
+#include "tc.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace mk {
+
+namespace {
+
+constexpr uint64_t kGemmWaitNs = 1000000000ull;
+constexpr int kBM = 128, kBK = 64;
+
+template <int BN>
+struct GemmShape {
+  static constexpr int kStages = BN >= 256 ? 3 : 4;
+  static constexpr int kABytes = kBM * kBK * 2;        // 16 KB
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = 2 * kABytes + kBBytes;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kRingBytes + 256 + 1024;   // + barriers, + alignment slack
+};
+
+struct GemmBars {
+  uint64_t full[4];
+  uint64_t empty[4];
+  uint64_t acc;
+  uint32_t tmem;
+  int abort;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    linear_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
+                  const __grid_constant__ CUtensorMap tb, float* __restrict__ C, long long ldc, int M, int N, int K,
+                  int accumulate, int* err) {
+  using S = GemmShape<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  GemmBars* gb = reinterpret_cast<GemmBars*>(smem + S::kRingBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+  const int nk = K / kBK;
+  auto a_hi = [&](int s) { return smem + s * S::kStageBytes; };
+  auto a_lo = [&](int s) { return smem + s * S::kStageBytes + S::kABytes; };
+  auto b_t = [&](int s) { return smem + s * S::kStageBytes + 2 * S::kABytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::kStages; ++s) {
+      mbar_init(&gb->full[s], 1);
+      mbar_init(&gb->empty[s], 1);
+    }
+    mbar_init(&gb->acc, 1);
+    gb->abort = 0;
+    fence_barrier_init();
+    tc::prefetch_tensormap(&ta_hi);
+    tc::prefetch_tensormap(&ta_lo);
+    tc::prefetch_tensormap(&tb);
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&gb->tmem, BN);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = gb->tmem;
+  volatile int* abort = &gb->abort;
+
+  if (warp == 0) {
+    if (lane == 0) {   // ---- TMA producer
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % S::kStages;
+        if (kb >= S::kStages && !mbar_wait(&gb->empty[s], ((kb / S::kStages) - 1) & 1, abort, kGemmWaitNs)) {
+          if (!*abort) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&gb->full[s], S::kStageBytes);
+        tc::tma_load_2d(a_hi(s), &ta_hi, kb * kBK, m0, &gb->full[s]);
+        tc::tma_load_2d(a_lo(s), &ta_lo, kb * kBK, m0, &gb->full[s]);
+        tc::tma_load_2d(b_t(s), &tb, kb * kBK, n0, &gb->full[s]);
+        ++issued;
+      }
+      int never = 0;   // let the copies this lane issued land before the CTA ends (bounded)
+      for (int kb = issued > S::kStages ? issued - S::kStages : 0; kb < issued; ++kb)
+        mbar_wait(&gb->full[kb % S::kStages], (kb / S::kStages) & 1, &never, kGemmWaitNs / 5);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {   // ---- MMA issuer
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % S::kStages;
+        if (!mbar_wait(&gb->full[s], (kb / S::kStages) & 1, abort, kGemmWaitNs)) {
+          if (!*abort) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t bd = tc::desc_kmajor_sw128(b_t(s) + kk * 32);
+          tc::mma_bf16(tmem, tc::desc_kmajor_sw128(a_hi(s) + kk * 32), bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          tc::mma_bf16(tmem, tc::desc_kmajor_sw128(a_lo(s) + kk * 32), bd, idesc, 1u);
+        }
+        tc::mma_commit(&gb->empty[s]);
+      }
+      tc::mma_commit(&gb->acc);   // arrives once every MMA issued above has completed
+    }
+  } else {   // ---- epilogue: warps 2..5
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const bool ok = mbar_wait(&gb->acc, 0, abort, kGemmWaitNs);
+    tc::fence_after_sync();
+    if (!ok && lane == 0) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
+    if (__all_sync(0xffffffffu, ok) && !*abort) {
+      const int m = m0 + row;
+      float* crow = C + static_cast<long long>(m) * ldc + n0;
+      const bool vec = (ldc % 4 == 0) && ((reinterpret_cast<uintptr_t>(C) & 15) == 0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+        if (m < M) {
+          if (vec && n0 + c0 + 16 <= N) {
+            float4* d4 = reinterpret_cast<float4*>(crow + c0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+              if (accumulate) {
+                const float4 c = d4[j];
+                o.x += c.x; o.y += c.y; o.z += c.z; o.w += c.w;
+              }
+              d4[j] = o;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (n0 + c0 + j < N) crow[c0 + j] = accumulate ? crow[c0 + j] + v[j] : v[j];
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, BN);
+  }
+}
+
+__global__ void split_bf16_kernel(const float* __restrict__ x, long long ldx, uint16_t* __restrict__ hi,
+                                  uint16_t* __restrict__ lo, int M, int K) {
+  const long long total = static_cast<long long>(M) * K;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long m = i / K, k = i % K;
+    const float v = x[m * ldx + k];
+    const uint16_t h = f_to_bf16(v);
+    hi[i] = h;
+    lo[i] = f_to_bf16(v - bf16_to_f(h));
+  }
+}
+
+// ---- host: tensor maps through the driver entry point (no link-time libcuda dependency)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 row-major [rows][cols] with a row stride of `stride_bytes`; box = 64 columns x box_rows.
+bool make_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long stride_bytes,
+              int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
+  using S = GemmShape<BN>;
+  CUtensorMap ma_hi, ma_lo, mb;
+  if (!make_map(&ma_hi, a.x_hi, a.M, a.K, static_cast<long long>(a.K) * 2, kBM) ||
+      !make_map(&ma_lo, a.x_lo, a.M, a.K, static_cast<long long>(a.K) * 2, kBM) ||
+      !make_map(&mb, a.w, a.N, a.K, a.ldw_bytes, BN))
+    return cudaErrorInvalidValue;
+  const cudaError_t attr =
+      cudaFuncSetAttribute(linear_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  dim3 grid((a.N + BN - 1) / BN, (a.M + kBM - 1) / kBM);
+  linear_kernel<BN><<<grid, 192, S::kSmemBytes, s>>>(ma_hi, ma_lo, mb, a.c, a.ldc, a.M, a.N, a.K, a.accumulate,
+                                                     a.err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_split_bf16(const float* x, long long ldx, uint16_t* hi, uint16_t* lo, int M, int K,
+                              cudaStream_t s) {
+  const long long total = static_cast<long long>(M) * K;
+  if (total == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 16));
+  split_bf16_kernel<<<blocks, 256, 0, s>>>(x, ldx, hi, lo, M, K);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s) {
+  if (a.M <= 0 || a.N <= 0) return cudaSuccess;
+  if (a.K <= 0 || a.K % kBK != 0 || a.ldw_bytes % 16 != 0 || a.ldw_bytes < 2LL * a.K ||
+      (reinterpret_cast<uintptr_t>(a.x_hi) & 15) || (reinterpret_cast<uintptr_t>(a.x_lo) & 15) ||
+      (reinterpret_cast<uintptr_t>(a.w) & 15))
+    return cudaErrorInvalidValue;
+  return a.N >= 2048 ? launch_bn<256>(a, s) : launch_bn<128>(a, s);
+}
+
+}  // namespace mk
+
+// ---------------------------------------------------------------- C ABI
+extern "C" int mk_linear(const float* d_x, int64_t ldx, int32_t M, int32_t K, const void* d_w, int64_t ldw_bytes,
+                         int32_t N, float* d_c, int64_t ldc, int32_t accumulate, void* d_scratch, size_t scratch_bytes,
+                         int32_t* d_err, void* stream) {
+  if (!d_x || !d_w || !d_c || !d_err || !d_scratch) {
+    mk_set_last_error("mk_linear: NULL pointer");
+    return MK_ERR_ARG;
+  }
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || ldx < K || ldc < N || ldw_bytes < 2LL * K || ldw_bytes % 16 != 0) {
+    mk_set_last_error("mk_linear: bad sizes (K must be a positive multiple of 64, ldw_bytes a multiple of 16 "
+                      "and >= 2K, ldx >= K, ldc >= N)");
+    return MK_ERR_ARG;
+  }
+  if (scratch_bytes < 4ull * static_cast<unsigned long long>(M) * K) {
+    mk_set_last_error("mk_linear: scratch must hold 4*M*K bytes");
+    return MK_ERR_ARG;
+  }
+  if ((reinterpret_cast<uintptr_t>(d_w) & 15) || (reinterpret_cast<uintptr_t>(d_scratch) & 15)) {
+    mk_set_last_error("mk_linear: d_w and d_scratch must be 16-byte aligned");
+    return MK_ERR_ARG;
+  }
+  if (M == 0 || N == 0) return MK_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* hi = static_cast<uint16_t*>(d_scratch);
+  uint16_t* lo = hi + static_cast<size_t>(M) * K;
+  cudaError_t e = mk::launch_split_bf16(d_x, ldx, hi, lo, M, K, s);
+  if (e == cudaSuccess) {
+    mk::LinearArgs a{hi, lo, d_w, ldw_bytes, d_c, ldc, M, N, K, accumulate ? 1 : 0, d_err};
+    e = mk::launch_linear(a, s);
+  }
+  if (e != cudaSuccess) {
+    mk_set_last_error(std::string("mk_linear: ") + cudaGetErrorString(e));
+    return MK_ERR_CUDA;
+  }
+  return MK_OK;
+}

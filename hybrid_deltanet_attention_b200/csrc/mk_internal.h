@@ -81,6 +81,22 @@ size_t decode_scratch_floats(int H);   // fp32 scratch per CTA left after the ri
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s);
 int decode_max_splits(int grid, int hkv);
 
+// prefill linear layers on the tensor cores (gemm.cu): C[m][n] (+)= sum_k X[m][k] W[n][k]
+// with X given as its bf16 high and low parts.
+struct LinearArgs {
+  const uint16_t* x_hi;     // bf16 [M][K], row stride K
+  const uint16_t* x_lo;
+  const void* w;            // bf16 rows of K, row stride ldw_bytes (multiple of 16)
+  long long ldw_bytes;
+  float* c;                 // fp32 [M][ldc]
+  long long ldc;
+  int M, N, K;              // K a multiple of 64
+  int accumulate;
+  int* err;
+};
+cudaError_t launch_split_bf16(const float* x, long long ldx, uint16_t* hi, uint16_t* lo, int M, int K, cudaStream_t s);
+cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s);
+
 // repack helpers (api.cu launches them)
 cudaError_t launch_transpose_bf16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t s);
 cudaError_t launch_pack_rows_tail(const uint16_t* w, const uint16_t* taps, void* dst, int rows, int cols, int nconv,

@@ -236,6 +236,26 @@ int mk_phase_trace(mk_model* m, uint64_t* d_trace, int32_t capacity);
  * repack); used to report launch counts. */
 int64_t mk_launch_count(const mk_model* m);
 
+/* Tensor-core linear layer, the building block of the prefill's projections (also
+ * usable on its own): for m < M, n < N
+ *     C[m][n] = sum_k X[m][k] * W[n][k]         (accumulate == 0)
+ *     C[m][n] += sum_k X[m][k] * W[n][k]        (accumulate != 0)
+ * d_x      device fp32, row-major [M][ldx] (ldx >= K). Split on the device into bf16
+ *          high and low parts (X = hi + lo to about 16 bits of X's mantissa), each
+ *          multiplied by W on the tensor cores into one fp32 accumulator.
+ * d_w      device bf16, N rows of K weights, row stride ldw_bytes (a multiple of 16,
+ *          >= 2K); 16-byte aligned.
+ * d_c      device fp32, row-major [M][ldc] (ldc >= N).
+ * K        a positive multiple of 64; M, N >= 0 (0 does nothing).
+ * d_scratch, scratch_bytes: device buffer of at least 4*M*K bytes, 16-byte aligned,
+ *          used for the bf16 parts of X; the caller owns it.
+ * d_err    device int32 error word; a timed-out wait ORs MK_DEVERR_PIPE_TIMEOUT into it.
+ * Asynchronous on `stream`. Returns MK_OK, MK_ERR_ARG (sizes, NULL or misaligned
+ * pointers; nothing is launched) or MK_ERR_CUDA. */
+int mk_linear(const float* d_x, int64_t ldx, int32_t M, int32_t K, const void* d_w, int64_t ldw_bytes, int32_t N,
+              float* d_c, int64_t ldc, int32_t accumulate, void* d_scratch, size_t scratch_bytes, int32_t* d_err,
+              void* stream);
+
 /* Thread-local description of the last nonzero return on this thread. */
 const char* mk_last_error(void);
 
