@@ -1,6 +1,7 @@
 // C ABI of libmk.so: validation, weight repacking, state/workspace layout and launches.
 // Every step of the forward pass runs in this library's kernels; the caller only
 // provides device memory and a stream.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -189,6 +190,8 @@ int check_budget(const mk_config& c, int grid) {
   return MK_OK;
 }
 
+constexpr int kBatchedPrefillMin = 16;   // shorter prompts run as decode launches
+
 struct Layout {
   mk_sizes sz;
   // packed
@@ -198,7 +201,21 @@ struct Layout {
   size_t w_sync, w_h, w_z, w_y, w_part, w_tok, w_g, w_n, w_snap;
   size_t snap_S, snap_conv;
   int max_splits;
+  // batched prefill workspace
+  int pf_rows;
+  size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec;
 };
+
+// Tokens per batched prefill pass: the whole context up to 4096, 0 when a shape is outside
+// what the prefill kernels take (then the prompt runs through decode launches).
+int prefill_rows(const mk_config& c) {
+  const long qd = static_cast<long>(c.at_q_heads) * c.at_head_dim;
+  const long kdn = static_cast<long>(c.dn_heads) * c.dn_dv;
+  if (c.hidden % 64 || c.ffn % 64 || kdn % 64 || qd % 64) return 0;
+  if (c.dn_heads > 64 || c.dn_dk > 128 || c.dn_dv > 128 || c.dn_dv % 16) return 0;
+  if (c.at_kv_heads > 0 && c.at_q_heads / c.at_kv_heads > 8) return 0;
+  return std::min(c.max_ctx, 4096);
+}
 
 size_t layer_block_bytes(const mk_config& c, char kind) {
   const size_t H = c.hidden, rb = H * 2;
@@ -207,14 +224,14 @@ size_t layer_block_bytes(const mk_config& c, char kind) {
     const size_t C = static_cast<size_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
     b += align256((C + 2 * c.dn_heads) * (rb + 16));       // w_in, each row + its conv taps
     b += align256(C * c.conv_width * 2);                    // conv
-    b += align256(static_cast<size_t>(c.dn_heads) * c.dn_dv * rb);   // w_outT
+    b += 2 * align256(static_cast<size_t>(c.dn_heads) * c.dn_dv * rb);   // w_outT, w_out (K-major, prefill)
   } else {
     const size_t qd = static_cast<size_t>(c.at_q_heads) * c.at_head_dim;
     const size_t rows = qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim;
     b += align256(rows * rb);
-    b += align256(qd * rb);
+    b += 2 * align256(qd * rb);                               // w_outT, w_out (K-major, prefill)
   }
-  b += 3 * align256(static_cast<size_t>(c.ffn) * rb);     // gate, up, downT
+  b += 4 * align256(static_cast<size_t>(c.ffn) * rb);     // gate, up, downT, down (K-major, prefill)
   return b;
 }
 
@@ -263,6 +280,29 @@ Layout make_layout(const mk_config& c, int grid) {
   L.snap_conv = static_cast<size_t>(nd) * c.conv_width * C * 4;
   L.w_snap = off;
   if (c.max_draft > 0) off = align256(off + align256(L.snap_S) + align256(L.snap_conv) + 256);
+  L.pf_rows = prefill_rows(c);
+  if (L.pf_rows > 0) {
+    const size_t T = L.pf_rows;
+    const size_t qd = static_cast<size_t>(c.at_q_heads) * c.at_head_dim;
+    const size_t kdn = static_cast<size_t>(c.dn_heads) * c.dn_dv;
+    const size_t at_rows = na ? qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim : 0;
+    const size_t kmax = std::max({H, static_cast<size_t>(c.ffn), kdn, qd});
+    const size_t zmax = std::max({C + 2 * static_cast<size_t>(c.dn_heads), at_rows, 2 * static_cast<size_t>(c.ffn)});
+    const size_t ymax = std::max(C + 2 * static_cast<size_t>(c.dn_heads), qd);
+    const size_t omax = std::max(kdn, qd);
+    const size_t nch = (T + 63) / 64;
+    L.pf_h = off; off = align256(off + T * H * 4);
+    L.pf_xhi = off; off = align256(off + T * kmax * 2);
+    L.pf_xlo = off; off = align256(off + T * kmax * 2);
+    L.pf_z = off; off = align256(off + T * zmax * 4);
+    L.pf_y = off; off = align256(off + T * ymax * 4);
+    L.pf_o = off; off = align256(off + T * omax * 4);
+    L.pf_u = off; off = align256(off + T * kdn * 4);
+    L.pf_w = off; off = align256(off + T * static_cast<size_t>(c.dn_heads) * c.dn_dk * 4);
+    L.pf_p = off; off = align256(off + nch * c.dn_heads * 64 * 64 * 4);
+    L.pf_gam = off; off = align256(off + T * c.dn_heads * 4);
+    L.pf_dec = off; off = align256(off + T * c.dn_heads * 4);
+  }
   L.sz.workspace_bytes = off;
   L.sz.grid_ctas = grid;
   return L;
@@ -414,6 +454,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     const std::string p = "layers." + std::to_string(l) + ".";
     size_t off = L.p_layer[l];
     mk::LayerW lw{};
+    mk_prefill_layer pl{};
     lw.kind = c.pattern[l] == 'D' ? mk::kDeltaNet : mk::kAttention;
     lw.idx = c.pattern[l] == 'D' ? di++ : ai++;
     lw.norm1 = reinterpret_cast<const uint16_t*>(P + off);
@@ -437,6 +478,9 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
       lw.w_outT = P + off;
       if (e == cudaSuccess) e = transpose(p + "dn.w_out", off);
       off += align256(static_cast<size_t>(c.dn_heads) * c.dn_dv * rb);
+      pl.w_out = P + off;
+      if (e == cudaSuccess) e = copy(p + "dn.w_out", off);
+      off += align256(static_cast<size_t>(c.dn_heads) * c.dn_dv * rb);
     } else {
       const size_t qd = static_cast<size_t>(c.at_q_heads) * c.at_head_dim;
       const size_t rows = qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim;
@@ -445,6 +489,9 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
       off += align256(rows * rb);
       lw.w_outT = P + off;
       if (e == cudaSuccess) e = transpose(p + "attn.w_out", off);
+      off += align256(qd * rb);
+      pl.w_out = P + off;
+      if (e == cudaSuccess) e = copy(p + "attn.w_out", off);
       off += align256(qd * rb);
     }
     lw.w_gate = P + off;
@@ -455,7 +502,11 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     off += align256(static_cast<size_t>(c.ffn) * rb);
     lw.w_downT = P + off;
     if (e == cudaSuccess) e = transpose(p + "mlp.w_down", off);
+    off += align256(static_cast<size_t>(c.ffn) * rb);
+    pl.w_down = P + off;
+    if (e == cudaSuccess) e = copy(p + "mlp.w_down", off);
     m->layers_host.push_back(lw);
+    m->pf_layers.push_back(pl);
   }
   std::vector<double> freq(c.at_head_dim > 0 ? c.at_head_dim / 2 : 1, 0.0);
   for (int i = 0; i < c.at_head_dim / 2; ++i)
@@ -512,6 +563,20 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   m->snap_S_bytes = L.snap_S;
   m->step_scratch_bytes = L.w_tok;   // sync words, residual, projections, attention partials
   m->snap_conv_bytes = L.snap_conv;
+  m->pf.rows = L.pf_rows;
+  if (L.pf_rows > 0) {
+    m->pf.h = reinterpret_cast<float*>(W + L.pf_h);
+    m->pf.xhi = reinterpret_cast<uint16_t*>(W + L.pf_xhi);
+    m->pf.xlo = reinterpret_cast<uint16_t*>(W + L.pf_xlo);
+    m->pf.z = reinterpret_cast<float*>(W + L.pf_z);
+    m->pf.y = reinterpret_cast<float*>(W + L.pf_y);
+    m->pf.o = reinterpret_cast<float*>(W + L.pf_o);
+    m->pf.u = reinterpret_cast<float*>(W + L.pf_u);
+    m->pf.w = reinterpret_cast<float*>(W + L.pf_w);
+    m->pf.p = reinterpret_cast<float*>(W + L.pf_p);
+    m->pf.gam = reinterpret_cast<float*>(W + L.pf_gam);
+    m->pf.dec = reinterpret_cast<float*>(W + L.pf_dec);
+  }
   *out = m;
   return MK_OK;
 }
@@ -551,6 +616,13 @@ int mk_prefill(mk_model* m, const int32_t* d_tokens, int32_t n, float* d_last_lo
   if (m->pos_hint + n > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "prompt exceeds the context capacity");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* sink = m->ws_tok + m->cfg.max_ctx + 4;
+  if (m->pf.rows > 0 && n > kBatchedPrefillMin && !getenv("MK_PREFILL_BY_DECODE")) {
+    // all but the last token through the batched layers, the last one through the
+    // decode kernel (its logits and the next token)
+    int rc = mk_prefill_batched(m, d_tokens, n - 1, s);
+    if (rc) return rc;
+    return launch_step(m, d_tokens + n - 1, d_next_token ? d_next_token : sink, d_last_logits, s);
+  }
   for (int i = 0; i < n; ++i) {
     const bool last = (i == n - 1);
     int rc = launch_step(m, d_tokens + i, last && d_next_token ? d_next_token : sink, last ? d_last_logits : nullptr, s);

@@ -658,13 +658,6 @@ __device__ __forceinline__ float conv_silu_at(const DecodeParams& p, const float
   return siluf_(y);
 }
 
-// RoPE angle pos * inv_freq reduced to [-pi, pi] in double, then sin/cos in fp32.
-__device__ __forceinline__ void rope_cs(double ang, float& c, float& s) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double r = ang - two_pi * rint(ang / two_pi);
-  sincosf(static_cast<float>(r), &s, &c);
-}
-
 // Online-softmax update of one block of np scores in sc (one warp per head).
 __device__ __forceinline__ void softmax_block(float* sc, float* mlc, int grp, int np, int warp, int lane) {
   if (warp >= grp) return;

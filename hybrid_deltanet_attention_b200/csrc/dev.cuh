@@ -113,6 +113,13 @@ __device__ __forceinline__ void red_add_v4(float4* p, float4 v) {
                : "memory");
 }
 
+// RoPE angle pos * inv_freq reduced to [-pi, pi] in double, then sin/cos in fp32.
+__device__ __forceinline__ void rope_cs(double ang, float& c, float& s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double r = ang - two_pi * rint(ang / two_pi);
+  sincosf(static_cast<float>(r), &s, &c);
+}
+
 // Named barrier over the consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void cons_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");

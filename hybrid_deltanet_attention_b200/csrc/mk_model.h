@@ -11,6 +11,30 @@
 // Sets the thread-local message returned by mk_last_error().
 void mk_set_last_error(const std::string& msg);
 
+// Workspace of the batched prefill (rows = tokens per pass; 0 when the model has none).
+struct mk_prefill_ws {
+  int rows = 0;
+  float* h = nullptr;        // [rows][H] residual stream
+  uint16_t* xhi = nullptr;   // [rows][Kmax] bf16 high part of the current GEMM input
+  uint16_t* xlo = nullptr;   // [rows][Kmax] bf16 low part
+  float* z = nullptr;        // [rows][Zmax] projection outputs
+  float* y = nullptr;        // [rows][Ymax] DeltaNet q k v log-a b / roped attention queries
+  float* o = nullptr;        // [rows][Omax] mixer outputs
+  float* u = nullptr;        // [rows][Hd dv] chunked delta rule: U
+  float* w = nullptr;        // [rows][Hd dk] chunked delta rule: W
+  float* p = nullptr;        // [chunks][Hd][64][64] chunked delta rule: masked decayed Q K^T
+  float* gam = nullptr;      // [rows][Hd]
+  float* dec = nullptr;      // [rows][Hd]
+};
+
+struct mk_prefill_layer {   // K-major copies of the projections the decode kernel keeps transposed
+  const uint8_t* w_out;      // [H][K_mix] bf16
+  const uint8_t* w_down;     // [H][F] bf16
+};
+
+// Batched prefill of n tokens at the device position (+ off): every layer, no logits.
+int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t s);
+
 struct mk_model {
   mk_config cfg;
   mk_sizes sz;
@@ -30,4 +54,6 @@ struct mk_model {
   uint8_t* ws_snap;      // DeltaNet S + conv history + pos snapshot for verify
   size_t snap_S_bytes, snap_conv_bytes;
   size_t step_scratch_bytes;   // leading part of the workspace one decode step uses
+  mk_prefill_ws pf;
+  std::vector<mk_prefill_layer> pf_layers;
 };

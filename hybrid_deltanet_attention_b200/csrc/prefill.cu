@@ -1,0 +1,605 @@
+// Batched prefill: a prompt's tokens go through every layer together, the projections
+// as tensor-core GEMMs (gemm.cu), the DeltaNet mixer in its chunked (WY) form, the
+// attention mixer causally over the KV cache. The last prompt token then runs through
+// the decode megakernel, which produces its logits and the next token.
+//
+// Per layer, for T tokens at positions pos0 .. pos0+T-1 (activations fp32 in HBM; every
+// GEMM input is written as bf16 high/low parts):
+//   x = RMSNorm(h)                          rms_split
+//   DeltaNet: z = x W_in^T                  linear
+//             conv + SiLU, q/k L2 norms,    dn_prep, conv_history_update
+//             log a = -softplus(alpha), b = sigmoid(beta)
+//             chunked delta rule            wy_prep (per chunk and head), wy_state (per head and row group)
+//   attention: z = x W_in^T                 linear
+//             RoPE, K/V into the cache      at_prep
+//             causal softmax attention      attn_prefill
+//   h += o W_out^T                          split (with the output gate), linear (accumulate)
+//   x = RMSNorm(h); g|u = x [W_gate|W_up]^T; h += (SiLU(g) u) W_down^T
+#include <algorithm>
+#include <cmath>
+#include <string>
+
+#include "../../include/mk.h"
+#include "dev.cuh"
+#include "mk_internal.h"
+#include "mk_model.h"
+
+namespace mk {
+namespace {
+
+constexpr int kPT = 256;    // threads of the row kernels
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = (l < static_cast<int>(blockDim.x >> 5)) ? red[l] : 0.f;
+  return warp_sum(t);
+}
+
+__device__ __forceinline__ void put_split(uint16_t* hi, uint16_t* lo, long long i, float v) {
+  const uint16_t h = f_to_bf16(v);
+  hi[i] = h;
+  lo[i] = f_to_bf16(v - bf16_to_f(h));
+}
+
+// h[t] = E[tok[t]] (bf16 -> fp32). An out-of-range id latches MK_DEVERR_BAD_TOKEN and
+// gives a zero row.
+__global__ void embed_rows(const int32_t* __restrict__ tok, int T, const uint16_t* __restrict__ embed, int H, int V,
+                           float* __restrict__ h, int* err) {
+  const int t = blockIdx.x;
+  const int id = tok[t];
+  const bool ok = id >= 0 && id < V;
+  if (!ok && threadIdx.x == 0) atomicOr(err, MK_DEVERR_BAD_TOKEN);
+  for (int i = threadIdx.x; i < H; i += blockDim.x)
+    h[static_cast<long long>(t) * H + i] = ok ? bf16_to_f(embed[static_cast<long long>(id) * H + i]) : 0.f;
+}
+
+// x[t] = h[t] / sqrt(mean(h[t]^2) + eps) * gamma, written as bf16 high/low parts.
+__global__ void rms_split(const float* __restrict__ h, int H, const uint16_t* __restrict__ gamma, float eps,
+                          uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  const float* row = h + static_cast<long long>(t) * H;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) ss += row[i] * row[i];
+  ss = block_sum(ss, red);
+  const float inv = 1.0f / sqrtf(ss / static_cast<float>(H) + eps);
+  for (int i = threadIdx.x; i < H; i += blockDim.x)
+    put_split(xhi, xlo, static_cast<long long>(t) * H + i, row[i] * inv * bf16_to_f(gamma[i]));
+}
+
+// DeltaNet token prep. z[t] = [q~ k~ v~ (C channels) | alpha (Hd) | beta (Hd)].
+// y[t] = [q/|q| (Hd dk) | k/|k| (Hd dk) | v (Hd dv) | log a (Hd) | b (Hd)] with the causal
+// conv + SiLU over the C channels (inputs before pos0 come from the conv history ring,
+// slot p mod W holding position p), log a = -softplus(alpha), b = sigmoid(beta).
+__global__ void dn_prep(const float* __restrict__ z, int ldz, const int* __restrict__ posp, int off,
+                        const float* __restrict__ ring, int W, int C, int Hd, int dk, const uint16_t* __restrict__ taps,
+                        float* __restrict__ y, int ldy) {
+  extern __shared__ float ys[];   // [C]
+  __shared__ float nrm[2 * 64];
+  const int t = blockIdx.x;
+  const int pos0 = *posp + off;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float acc = 0.f;
+    for (int j = 0; j < W; ++j) {
+      const int s = t - (W - 1) + j;        // token index inside this batch
+      float x;
+      if (s >= 0) x = z[static_cast<long long>(s) * ldz + c];
+      else {
+        const int p = pos0 + s;             // absolute position
+        x = p >= 0 ? ring[static_cast<long long>(p % W) * C + c] : 0.f;
+      }
+      acc = fmaf(bf16_to_f(taps[static_cast<long long>(c) * W + j]), x, acc);
+    }
+    ys[c] = siluf_(acc);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int vec = warp; vec < 2 * Hd; vec += nw) {     // q heads then k heads
+    float ss = 0.f;
+    for (int d = lane; d < dk; d += 32) ss += ys[vec * dk + d] * ys[vec * dk + d];
+    ss = warp_sum(ss);
+    if (lane == 0) nrm[vec] = 1.0f / sqrtf(ss + 1e-6f);
+  }
+  __syncthreads();
+  float* yr = y + static_cast<long long>(t) * ldy;
+  const int qk = 2 * Hd * dk;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) yr[c] = c < qk ? ys[c] * nrm[c / dk] : ys[c];
+  for (int hh = threadIdx.x; hh < Hd; hh += blockDim.x) {
+    const float al = z[static_cast<long long>(t) * ldz + C + hh];
+    const float be = z[static_cast<long long>(t) * ldz + C + Hd + hh];
+    yr[C + hh] = -(fmaxf(al, 0.f) + log1pf(expf(-fabsf(al))));
+    yr[C + Hd + hh] = sigmoidf_(be);
+  }
+}
+
+// Conv history after the batch: the raw inputs of the last W-1 positions go to their ring slots.
+__global__ void conv_history_update(const float* __restrict__ z, int ldz, int T, const int* __restrict__ posp, int off,
+                                    float* __restrict__ ring, int W, int C) {
+  const int m = blockIdx.y;                 // 0 .. W-2: position pos0 + T - 1 - m
+  const int s = T - 1 - m;
+  if (s < 0) return;
+  const int p = *posp + off + s;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < C; c += gridDim.x * blockDim.x)
+    ring[static_cast<long long>(p % W) * C + c] = z[static_cast<long long>(s) * ldz + c];
+}
+
+// Attention token prep: RoPE (half-split pairs (i, i + D/2), angle (pos0+t) * inv_freq_i)
+// on the Hq query heads (then scaled by 1/sqrt(D)) and the Hkv key heads; keys and values
+// appended to the bf16 cache at position pos0 + t.
+__global__ void at_prep(const float* __restrict__ z, int ldz, const int* __restrict__ posp, int off,
+                        const double* __restrict__ inv_freq, int Hq, int Hkv, int D, int gated, uint16_t* __restrict__ kc,
+                        uint16_t* __restrict__ vc, int max_ctx, float* __restrict__ q, int ldq) {
+  const int t = blockIdx.x, pos = *posp + off + t, half = D / 2;
+  if (pos < 0 || pos >= max_ctx) return;    // capacity: latched by check_capacity
+  const float scale = 1.0f / sqrtf(static_cast<float>(D));
+  const float* zr = z + static_cast<long long>(t) * ldz;
+  const int koff = Hq * D * (gated ? 2 : 1), voff = koff + Hkv * D;
+  for (int idx = threadIdx.x; idx < (Hq + Hkv) * half; idx += blockDim.x) {
+    const int hv = idx / half, i = idx % half;
+    float cs, sn;
+    rope_cs(static_cast<double>(pos) * inv_freq[i], cs, sn);
+    if (hv < Hq) {
+      const float x1 = zr[hv * D + i], x2 = zr[hv * D + i + half];
+      q[static_cast<long long>(t) * ldq + hv * D + i] = (x1 * cs - x2 * sn) * scale;
+      q[static_cast<long long>(t) * ldq + hv * D + i + half] = (x1 * sn + x2 * cs) * scale;
+    } else {
+      const int g = hv - Hq;
+      const float x1 = zr[koff + g * D + i], x2 = zr[koff + g * D + i + half];
+      const long long base = (static_cast<long long>(g) * max_ctx + pos) * D;
+      kc[base + i] = f_to_bf16(x1 * cs - x2 * sn);
+      kc[base + i + half] = f_to_bf16(x1 * sn + x2 * cs);
+    }
+  }
+  for (int idx = threadIdx.x; idx < Hkv * D; idx += blockDim.x) {
+    const int g = idx / D, d = idx % D;
+    vc[(static_cast<long long>(g) * max_ctx + pos) * D + d] = f_to_bf16(zr[voff + idx]);
+  }
+}
+
+// x = o (* sigmoid(gate) when gate != null), as bf16 high/low parts [T][n].
+__global__ void gate_split(const float* __restrict__ o, int ldo, const float* __restrict__ gate, int ldg, int n,
+                           uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
+  const int t = blockIdx.x;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    float v = o[static_cast<long long>(t) * ldo + i];
+    if (gate) v *= sigmoidf_(gate[static_cast<long long>(t) * ldg + i]);
+    put_split(xhi, xlo, static_cast<long long>(t) * n + i, v);
+  }
+}
+
+// act = SiLU(g) * u from gu[t] = [g (F) | u (F)], as bf16 high/low parts [T][F].
+__global__ void act_split(const float* __restrict__ gu, int F, uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
+  const int t = blockIdx.x;
+  const float* r = gu + static_cast<long long>(t) * 2 * F;
+  for (int i = threadIdx.x; i < F; i += blockDim.x)
+    put_split(xhi, xlo, static_cast<long long>(t) * F + i, siluf_(r[i]) * r[F + i]);
+}
+
+// ------------------------------------------------------------------ chunked delta rule
+// One head, one chunk of n <= 64 tokens (r = 0..n-1) with incoming state S0 [dv][dk]:
+//   g_r = sum_{s<=r} log a_s,  gamma_r = e^{g_r},  dec_r = e^{g_{n-1} - g_r}
+//   A[r][s] = b_r e^{g_r - g_s} (k_r . k_s)  (s < r, strictly lower triangular)
+//   U = (I + A)^-1 diag(b) V,   W = (I + A)^-1 diag(b gamma) K
+//   P[r][s] = e^{g_r - g_s} (q_r . k_s)  (s <= r)
+// and then, with Delta = U - W S0^T (row r = the delta-rule update of token r),
+//   o_r = gamma_r S0 q_r + sum_{s<=r} P[r][s] Delta_s,
+//   S_n = gamma_{n-1} S0 + sum_r dec_r Delta_r k_r^T.
+// Only differences g_r - g_s with s <= r are exponentiated, so every factor is <= 1.
+constexpr int kChunk = 64;
+constexpr int kRowGroup = 16;   // rows of S per CTA in the state pass
+
+struct WyBufs {
+  const float* y;   // dn_prep output, row stride ldy
+  int ldy;
+  float* u;         // [T][Hd dv]
+  float* w;         // [T][Hd dk]
+  float* p;         // [n_chunks][Hd][64][64]
+  float* gam;       // [T][Hd]
+  float* dec;       // [T][Hd]
+  float* o;         // [T][Hd dv]
+  int T, Hd, dk, dv;
+};
+
+__global__ void __launch_bounds__(256) wy_prep(WyBufs b) {
+  extern __shared__ float sm[];
+  const int dk = b.dk, dv = b.dv, Hd = b.Hd;
+  const int ch = blockIdx.x, h = blockIdx.y;
+  const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
+  const int kp = dk + 1, xw = dv + dk;
+  float* K = sm;                       // [64][dk+1]
+  float* Q = K + kChunk * kp;          // [64][dk+1]
+  float* X = Q + kChunk * kp;          // [64][dv+dk]: right-hand sides, then U | W
+  float* A = X + kChunk * xw;          // [64][65]
+  float* g = A + kChunk * 65;          // [64]
+  float* bb = g + kChunk;              // [64]
+  const int qo = h * dk, ko = Hd * dk + h * dk, vo = 2 * Hd * dk + h * dv;
+  const int C = 2 * Hd * dk + Hd * dv;
+  for (int idx = threadIdx.x; idx < kChunk * dk; idx += blockDim.x) {
+    const int r = idx / dk, j = idx % dk;
+    const float* yr = b.y + static_cast<long long>(t0 + r) * b.ldy;
+    K[r * kp + j] = r < n ? yr[ko + j] : 0.f;
+    Q[r * kp + j] = r < n ? yr[qo + j] : 0.f;
+  }
+  if (threadIdx.x < kChunk) {
+    const int r = threadIdx.x;
+    const float* yr = b.y + static_cast<long long>(t0 + r) * b.ldy;
+    g[r] = r < n ? yr[C + h] : 0.f;     // log a, summed below
+    bb[r] = r < n ? yr[C + Hd + h] : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float acc = 0.f;
+    for (int r = 0; r < kChunk; ++r) {
+      acc += g[r];
+      g[r] = acc;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < kChunk * xw; idx += blockDim.x) {
+    const int r = idx / xw, j = idx % xw;
+    float v = 0.f;
+    if (r < n) {
+      if (j < dv) v = bb[r] * b.y[static_cast<long long>(t0 + r) * b.ldy + vo + j];
+      else v = bb[r] * expf(g[r]) * K[r * kp + (j - dv)];
+    }
+    X[r * xw + j] = v;
+  }
+  // A (strictly lower) and P (lower with the diagonal); P goes straight to global memory
+  float* P = b.p + (static_cast<long long>(ch) * Hd + h) * kChunk * kChunk;
+  for (int idx = threadIdx.x; idx < kChunk * kChunk; idx += blockDim.x) {
+    const int r = idx / kChunk, s = idx % kChunk;
+    float a = 0.f, pq = 0.f;
+    if (s <= r && r < n) {
+      float dkk = 0.f, dqk = 0.f;
+      for (int j = 0; j < dk; ++j) {
+        const float ks = K[s * kp + j];
+        dkk = fmaf(K[r * kp + j], ks, dkk);
+        dqk = fmaf(Q[r * kp + j], ks, dqk);
+      }
+      const float e = expf(g[r] - g[s]);
+      if (s < r) a = bb[r] * e * dkk;
+      pq = e * dqk;
+    }
+    A[r * 65 + s] = a;
+    P[idx] = pq;
+  }
+  __syncthreads();
+  // forward substitution (I + A) X = RHS; column j is owned by one thread
+  for (int j = threadIdx.x; j < xw; j += blockDim.x) {
+    for (int r = 1; r < n; ++r) {
+      float acc = X[r * xw + j];
+      for (int s = 0; s < r; ++s) acc = fmaf(-A[r * 65 + s], X[s * xw + j], acc);
+      X[r * xw + j] = acc;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < n * xw; idx += blockDim.x) {
+    const int r = idx / xw, j = idx % xw;
+    if (j < dv) b.u[static_cast<long long>(t0 + r) * Hd * dv + h * dv + j] = X[r * xw + j];
+    else b.w[static_cast<long long>(t0 + r) * Hd * dk + h * dk + (j - dv)] = X[r * xw + j];
+  }
+  if (threadIdx.x < n) {
+    const int r = threadIdx.x;
+    b.gam[static_cast<long long>(t0 + r) * Hd + h] = expf(g[r]);
+    b.dec[static_cast<long long>(t0 + r) * Hd + h] = expf(g[n - 1] - g[r]);
+  }
+}
+
+// State pass over the chunks of one head for kRowGroup rows of S (rows are independent).
+__global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S /* this layer [Hd][dv][dk] */) {
+  extern __shared__ float sm[];
+  const int dk = b.dk, dv = b.dv, Hd = b.Hd;
+  const int h = blockIdx.x, i0 = blockIdx.y * kRowGroup;
+  const int kp = dk + 1;
+  float* S0 = sm;                          // [16][dk+1]
+  float* Wc = S0 + kRowGroup * kp;         // [64][dk+1]
+  float* Qc = Wc + kChunk * kp;            // [64][dk+1]
+  float* Kc = Qc + kChunk * kp;            // [64][dk]
+  float* Pc = Kc + kChunk * dk;            // [64][65]
+  float* Uc = Pc + kChunk * 65;            // [64][16]
+  float* Dl = Uc + kChunk * kRowGroup;     // [64][17]
+  float* gm = Dl + kChunk * 17;            // [64]
+  float* dc = gm + kChunk;                 // [64]
+  float* Sg = S + (static_cast<long long>(h) * dv + i0) * dk;
+  for (int idx = threadIdx.x; idx < kRowGroup * dk; idx += blockDim.x)
+    S0[(idx / dk) * kp + idx % dk] = Sg[idx];
+  const int qo = h * dk, ko = Hd * dk + h * dk;
+  const int nch = (b.T + kChunk - 1) / kChunk;
+  const int ti = threadIdx.x % kRowGroup, tr = threadIdx.x / kRowGroup;   // (row of S, token group)
+  for (int ch = 0; ch < nch; ++ch) {
+    const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < kChunk * dk; idx += blockDim.x) {
+      const int r = idx / dk, j = idx % dk;
+      const bool in = r < n;
+      const long long t = t0 + r;
+      Wc[r * kp + j] = in ? b.w[t * Hd * dk + h * dk + j] : 0.f;
+      Qc[r * kp + j] = in ? b.y[t * b.ldy + qo + j] : 0.f;
+      Kc[r * dk + j] = in ? b.y[t * b.ldy + ko + j] : 0.f;
+    }
+    const float* P = b.p + (static_cast<long long>(ch) * Hd + h) * kChunk * kChunk;
+    for (int idx = threadIdx.x; idx < kChunk * kChunk; idx += blockDim.x) Pc[(idx / kChunk) * 65 + idx % kChunk] = P[idx];
+    for (int idx = threadIdx.x; idx < kChunk * kRowGroup; idx += blockDim.x) {
+      const int r = idx / kRowGroup, i = idx % kRowGroup;
+      Uc[idx] = r < n ? b.u[static_cast<long long>(t0 + r) * Hd * dv + h * dv + i0 + i] : 0.f;
+    }
+    if (threadIdx.x < kChunk) {
+      const int r = threadIdx.x;
+      gm[r] = r < n ? b.gam[static_cast<long long>(t0 + r) * Hd + h] : 0.f;
+      dc[r] = r < n ? b.dec[static_cast<long long>(t0 + r) * Hd + h] : 0.f;
+    }
+    __syncthreads();
+    // Delta = U - W S0^T
+    for (int r = tr; r < kChunk; r += 256 / kRowGroup) {
+      float acc = 0.f;
+      for (int j = 0; j < dk; ++j) acc = fmaf(Wc[r * kp + j], S0[ti * kp + j], acc);
+      Dl[r * 17 + ti] = Uc[r * kRowGroup + ti] - acc;
+    }
+    __syncthreads();
+    // o_r = gamma_r S0 q_r + sum_{s<=r} P[r][s] Delta_s
+    for (int r = tr; r < n; r += 256 / kRowGroup) {
+      float sq = 0.f;
+      for (int j = 0; j < dk; ++j) sq = fmaf(Qc[r * kp + j], S0[ti * kp + j], sq);
+      float acc = gm[r] * sq;
+      for (int s = 0; s <= r; ++s) acc = fmaf(Pc[r * 65 + s], Dl[s * 17 + ti], acc);
+      b.o[static_cast<long long>(t0 + r) * Hd * dv + h * dv + i0 + ti] = acc;
+    }
+    __syncthreads();
+    // S0 <- gamma_{n-1} S0 + sum_r dec_r Delta_r k_r^T
+    const float gl = gm[n - 1];
+    for (int idx = threadIdx.x; idx < kRowGroup * dk; idx += blockDim.x) {
+      const int i = idx / dk, j = idx % dk;
+      float acc = gl * S0[i * kp + j];
+      for (int r = 0; r < n; ++r) acc = fmaf(dc[r] * Dl[r * 17 + i], Kc[r * dk + j], acc);
+      S0[i * kp + j] = acc;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < kRowGroup * dk; idx += blockDim.x) Sg[idx] = S0[(idx / dk) * kp + idx % dk];
+}
+
+size_t wy_prep_smem(int dk, int dv) {
+  return sizeof(float) * (2 * kChunk * (dk + 1) + kChunk * (dv + dk) + kChunk * 65 + 2 * kChunk);
+}
+size_t wy_state_smem(int dk) {
+  return sizeof(float) * (kRowGroup * (dk + 1) + 2 * kChunk * (dk + 1) + kChunk * dk + kChunk * 65 +
+                          kChunk * kRowGroup + kChunk * 17 + 2 * kChunk);
+}
+
+// ------------------------------------------------------------------ causal attention
+// One CTA per (query token t, kv head g): the Hq/Hkv query heads of group g attend to the
+// cached positions 0 .. pos0+t in blocks of 64 keys with an online softmax.
+constexpr int kKeyBlock = 64;
+
+__global__ void __launch_bounds__(256) attn_prefill(const float* __restrict__ q, int ldq, const uint16_t* __restrict__ kc,
+                                                    const uint16_t* __restrict__ vc, const int* __restrict__ posp,
+                                                    int off, int Hq, int Hkv, int D, int max_ctx, float* __restrict__ o,
+                                                    int ldo) {
+  extern __shared__ float sm[];
+  const int t = blockIdx.x, g = blockIdx.y, grp = Hq / Hkv;
+  const int nkeys = min(*posp + off + t + 1, max_ctx);
+  float* qs = sm;                                   // [grp][D]
+  float* sc = qs + grp * D;                         // [grp][64]
+  float* ml = sc + grp * kKeyBlock;                 // [grp][3]: m, l, corr
+  uint16_t* kb = reinterpret_cast<uint16_t*>(ml + 3 * 8);   // [64][D]
+  uint16_t* vb = kb + kKeyBlock * D;                // [64][D]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int idx = threadIdx.x; idx < grp * D; idx += blockDim.x)
+    qs[idx] = q[static_cast<long long>(t) * ldq + (g * grp) * D + idx];
+  if (threadIdx.x < grp) {
+    ml[3 * threadIdx.x] = -INFINITY;
+    ml[3 * threadIdx.x + 1] = 0.f;
+    ml[3 * threadIdx.x + 2] = 0.f;
+  }
+  float acc[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+  const uint16_t* kg = kc + static_cast<long long>(g) * max_ctx * D;
+  const uint16_t* vg = vc + static_cast<long long>(g) * max_ctx * D;
+  for (int p0 = 0; p0 < nkeys; p0 += kKeyBlock) {
+    const int np = min(kKeyBlock, nkeys - p0);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < np * D / 8; idx += blockDim.x) {
+      reinterpret_cast<uint4*>(kb)[idx] = reinterpret_cast<const uint4*>(kg + static_cast<long long>(p0) * D)[idx];
+      reinterpret_cast<uint4*>(vb)[idx] = reinterpret_cast<const uint4*>(vg + static_cast<long long>(p0) * D)[idx];
+    }
+    __syncthreads();
+    for (int pp = warp; pp < np; pp += 8) {        // scores: warp per key, lanes over D
+      float d[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) d[u] = 0.f;
+      for (int i = lane; i < D; i += 32) {
+        const float kv = bf16_to_f(kb[pp * D + i]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (u < grp) d[u] = fmaf(qs[u * D + i], kv, d[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u < grp) {
+          d[u] = warp_sum(d[u]);
+          if (lane == 0) sc[u * kKeyBlock + pp] = d[u];
+        }
+    }
+    __syncthreads();
+    if (warp < grp) {                               // online softmax, warp per query head
+      float mx = -INFINITY;
+      for (int pp = lane; pp < np; pp += 32) mx = fmaxf(mx, sc[warp * kKeyBlock + pp]);
+      mx = warp_max(mx);
+      const float m_old = ml[3 * warp], m_new = fmaxf(m_old, mx);
+      float ls = 0.f;
+      for (int pp = lane; pp < np; pp += 32) {
+        const float e = expf(sc[warp * kKeyBlock + pp] - m_new);
+        sc[warp * kKeyBlock + pp] = e;
+        ls += e;
+      }
+      ls = warp_sum(ls);
+      __syncwarp();
+      if (lane == 0) {
+        const float corr = expf(m_old - m_new);
+        ml[3 * warp] = m_new;
+        ml[3 * warp + 1] = ml[3 * warp + 1] * corr + ls;
+        ml[3 * warp + 2] = corr;
+      }
+    }
+    __syncthreads();
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {   // values: thread per dim (D <= 256)
+      float vs[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) vs[u] = 0.f;
+      for (int pp = 0; pp < np; ++pp) {
+        const float vv = bf16_to_f(vb[pp * D + d]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (u < grp) vs[u] = fmaf(sc[u * kKeyBlock + pp], vv, vs[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u < grp) acc[u] = acc[u] * ml[3 * u + 2] + vs[u];
+    }
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (u < grp) o[static_cast<long long>(t) * ldo + (g * grp + u) * D + d] = acc[u] / ml[3 * u + 1];
+  }
+}
+
+size_t attn_prefill_smem(int grp, int D) {
+  return sizeof(float) * (grp * D + grp * kKeyBlock + 3 * 8) + 2 * sizeof(uint16_t) * kKeyBlock * D;
+}
+
+}  // namespace
+}  // namespace mk
+
+namespace mk {
+namespace {
+
+__global__ void check_capacity(const int* pos, int n, int max_ctx, int* err) {
+  if (*pos + n > max_ctx) atomicOr(err, MK_DEVERR_CAPACITY);
+}
+__global__ void advance_pos(int* pos, int n, int max_ctx) {
+  *pos = min(*pos + n, max_ctx);
+}
+
+// One pass of every layer over T tokens at device position *pos + off.
+cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaStream_t s) {
+  const mk_config& c = m->cfg;
+  const DecodeParams& b = m->base;
+  const mk_prefill_ws& pf = m->pf;
+  const int H = c.hidden, F = c.ffn, C = b.C, Hd = c.dn_heads, dk = c.dn_dk, dv = c.dn_dv, Wc = c.conv_width;
+  const int Hq = c.at_q_heads, Hkv = c.at_kv_heads, D = c.at_head_dim;
+  const int qd = Hq * D;
+  cudaError_t e = cudaSuccess;
+  auto chk = [&]() {
+    if (e == cudaSuccess) e = cudaGetLastError();
+    ++m->launches;
+  };
+  auto linear = [&](const void* w, long long ldw, int N, int K, float* out, long long ldc, int acc) {
+    if (e != cudaSuccess) return;
+    LinearArgs a{pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, b.err};
+    e = launch_linear(a, s);
+    ++m->launches;
+  };
+  embed_rows<<<T, kPT, 0, s>>>(tok, T, reinterpret_cast<const uint16_t*>(b.embed), H, c.vocab, pf.h, b.err);
+  chk();
+  int di = 0, ai = 0;
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+    const LayerW& L = m->layers_host[l];
+    const mk_prefill_layer& PL = m->pf_layers[l];
+    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm1, b.eps, pf.xhi, pf.xlo);
+    chk();
+    if (L.kind == kDeltaNet) {
+      const int rows = C + 2 * Hd;
+      float* S = b.S + static_cast<size_t>(di) * Hd * dv * dk;
+      float* ring = b.conv_ring + static_cast<size_t>(di) * Wc * C;
+      ++di;
+      linear(L.w_in, 2LL * H + 16, rows, H, pf.z, rows, 0);
+      dn_prep<<<T, kPT, C * sizeof(float), s>>>(pf.z, rows, b.pos, off, ring, Wc, C, Hd, dk, L.conv, pf.y, rows);
+      chk();
+      conv_history_update<<<dim3((C + kPT - 1) / kPT, Wc - 1), kPT, 0, s>>>(pf.z, rows, T, b.pos, off, ring, Wc, C);
+      chk();
+      WyBufs wy{pf.y, rows, pf.u, pf.w, pf.p, pf.gam, pf.dec, pf.o, T, Hd, dk, dv};
+      const int nch = (T + kChunk - 1) / kChunk;
+      wy_prep<<<dim3(nch, Hd), 256, wy_prep_smem(dk, dv), s>>>(wy);
+      chk();
+      wy_state<<<dim3(Hd, dv / kRowGroup), 256, wy_state_smem(dk), s>>>(wy, S);
+      chk();
+      gate_split<<<T, kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo);
+      chk();
+      linear(PL.w_out, 2LL * Hd * dv, H, Hd * dv, pf.h, H, 1);
+    } else {
+      const int rows = b.at_in_rows;
+      uint16_t* kc = b.kc + static_cast<size_t>(ai) * Hkv * c.max_ctx * D;
+      uint16_t* vc = b.vc + static_cast<size_t>(ai) * Hkv * c.max_ctx * D;
+      ++ai;
+      linear(L.w_in, 2LL * H, rows, H, pf.z, rows, 0);
+      at_prep<<<T, kPT, 0, s>>>(pf.z, rows, b.pos, off, b.inv_freq, Hq, Hkv, D, c.at_out_gate, kc, vc, c.max_ctx,
+                                 pf.y, qd);
+      chk();
+      attn_prefill<<<dim3(T, Hkv), 256, attn_prefill_smem(Hq / Hkv, D), s>>>(pf.y, qd, kc, vc, b.pos, off, Hq, Hkv,
+                                                                              D, c.max_ctx, pf.o, qd);
+      chk();
+      gate_split<<<T, kPT, 0, s>>>(pf.o, qd, c.at_out_gate ? pf.z + qd : nullptr, rows, qd, pf.xhi, pf.xlo);
+      chk();
+      linear(PL.w_out, 2LL * qd, H, qd, pf.h, H, 1);
+    }
+    if (e != cudaSuccess) break;
+    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm2, b.eps, pf.xhi, pf.xlo);
+    chk();
+    linear(L.w_gate, 2LL * H, F, H, pf.z, 2LL * F, 0);
+    linear(L.w_up, 2LL * H, F, H, pf.z + F, 2LL * F, 0);
+    act_split<<<T, kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
+    chk();
+    linear(PL.w_down, 2LL * F, H, F, pf.h, H, 1);
+  }
+  return e;
+}
+
+}  // namespace
+
+cudaError_t set_prefill_smem_limits() {
+  cudaError_t e = cudaFuncSetAttribute(wy_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(dn_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  return e;
+}
+
+size_t prefill_smem_need(int dk, int dv, int grp, int D, int C) {
+  size_t n = std::max(wy_prep_smem(dk, dv), wy_state_smem(dk));
+  n = std::max(n, attn_prefill_smem(grp, D));
+  return std::max(n, static_cast<size_t>(C) * sizeof(float));
+}
+
+}  // namespace mk
+
+int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t s) {
+  const mk::DecodeParams& b = m->base;
+  cudaError_t e = mk::set_prefill_smem_limits();
+  if (e == cudaSuccess) {
+    mk::check_capacity<<<1, 1, 0, s>>>(b.pos, n, m->cfg.max_ctx, b.err);
+    e = cudaGetLastError();
+    ++m->launches;
+  }
+  for (int off = 0; off < n && e == cudaSuccess; off += m->pf.rows) {
+    const int T = std::min(m->pf.rows, n - off);
+    e = mk::prefill_pass(m, d_tokens + off, T, off, s);
+  }
+  if (e == cudaSuccess) {
+    mk::advance_pos<<<1, 1, 0, s>>>(b.pos, n, m->cfg.max_ctx);
+    e = cudaGetLastError();
+    ++m->launches;
+  }
+  if (e != cudaSuccess) {
+    mk_set_last_error(std::string("batched prefill: ") + cudaGetErrorString(e));
+    return MK_ERR_CUDA;
+  }
+  m->pos_hint += n;
+  return MK_OK;
+}

@@ -1,0 +1,108 @@
+"""Batched prefill (tensor-core projections, chunked WY delta rule, causal attention)
+through mk_prefill, against the oracle's token-by-token prefill.
+
+Prompts longer than 16 tokens take the batched path for all but the last token; the
+last token runs through the decode kernel. The lengths below cover one partial chunk,
+exact chunks of 64, ragged tails, several chunks, and a second prefill that continues
+from a non-empty state (conv history and KV cache carried over).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity_util import LOGIT_MAX_ABS, STATE_REL_FROB, conv_history_as_window, near_tie, rel_frob
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _model(cfg, max_ctx):
+    import hybrid_deltanet_attention_b200 as hda
+    raw = synth.make_weights(cfg)
+    m = hda.Model(cfg, hda.weights_to_device(raw), max_ctx=max_ctx)
+    return m, oracle.prepare_weights(cfg, raw)
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = synth.TINY
+    m, W = _model(cfg, 512)
+    return cfg, m, W
+
+
+def _check(cfg, m, st, zo, zg, tok_g):
+    err = np.abs(zo - zg).max()
+    assert err <= LOGIT_MAX_ABS, err
+    if not near_tie(zo):
+        assert tok_g == int(np.argmax(zo))
+    S = m.S.cpu().numpy()
+    worst = max([rel_frob(S[li], st.S[li]) for li in range(cfg.n_dn)] + [0.0])
+    assert worst <= STATE_REL_FROB, worst
+    ring = m.conv_history.cpu().numpy()
+    for li in range(cfg.n_dn):
+        assert rel_frob(conv_history_as_window(ring[li], st.pos, cfg.conv_width), st.conv[li]) <= STATE_REL_FROB
+    K = m.k_cache.float().cpu().numpy()
+    V = m.v_cache.float().cpu().numpy()
+    for ai in range(cfg.n_at):
+        np.testing.assert_allclose(K[ai][:, :st.pos], st.K[ai][:, :st.pos], atol=2e-2, rtol=2e-2)
+        np.testing.assert_allclose(V[ai][:, :st.pos], st.V[ai][:, :st.pos], atol=2e-2, rtol=2e-2)
+    assert int(m.pos_tensor.item()) == st.pos
+
+
+def _prefill_both(cfg, m, st, W, prompt):
+    dev = torch.device("cuda")
+    zo = oracle.prefill(cfg, W, st, prompt)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device=dev)
+    nxt = torch.empty(1, dtype=torch.int32, device=dev)
+    m.prefill(torch.from_numpy(prompt).to(dev), logits=logits, next_token=nxt)
+    assert m.sync() == 0
+    return zo, logits.double().cpu().numpy(), int(nxt.item())
+
+
+@pytest.mark.parametrize("n", [17, 64, 65, 66, 130, 200])
+def test_tiny_batched_prefill(tiny, n):
+    cfg, m, W = tiny
+    m.reset()
+    st = oracle.new_state(cfg, 512)
+    prompt = synth.make_prompt(cfg, n, tag=f"pf{n}")
+    zo, zg, tg = _prefill_both(cfg, m, st, W, prompt)
+    _check(cfg, m, st, zo, zg, tg)
+
+
+def test_tiny_prefill_continues_from_state(tiny):
+    cfg, m, W = tiny
+    m.reset()
+    st = oracle.new_state(cfg, 512)
+    _prefill_both(cfg, m, st, W, synth.make_prompt(cfg, 40, tag="cont-a"))
+    zo, zg, tg = _prefill_both(cfg, m, st, W, synth.make_prompt(cfg, 90, tag="cont-b"))
+    _check(cfg, m, st, zo, zg, tg)
+
+
+def test_tiny_prefill_then_decode(tiny):
+    cfg, m, W = tiny
+    dev = torch.device("cuda")
+    m.reset()
+    st = oracle.new_state(cfg, 512)
+    zo, zg, tg = _prefill_both(cfg, m, st, W, synth.make_prompt(cfg, 100, tag="pd"))
+    tok = int(np.argmax(zo))
+    tin = torch.tensor([tok], dtype=torch.int32, device=dev)
+    tout = torch.empty(1, dtype=torch.int32, device=dev)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device=dev)
+    for _ in range(4):
+        m.decode(tin, tout, logits)
+        z = oracle.decode_step(cfg, W, st, tok)
+        assert np.abs(z - logits.double().cpu().numpy()).max() <= LOGIT_MAX_ABS
+        tok = int(np.argmax(z))
+        tin.fill_(tok)
+    assert m.sync() == 0
+    _check(cfg, m, st, z, logits.double().cpu().numpy(), int(tout.item()))
+
+
+def test_08b_batched_prefill_130():
+    cfg = synth.QWEN_08B
+    m, W = _model(cfg, 256)
+    m.reset()
+    st = oracle.new_state(cfg, 256)
+    zo, zg, tg = _prefill_both(cfg, m, st, W, synth.make_prompt(cfg, 130, tag="pf08"))
+    _check(cfg, m, st, zo, zg, tg)
