@@ -408,6 +408,101 @@ def run_mk(args):
     return 0
 
 
+def linear_macs_per_token(cfg) -> int:
+    """Multiply-accumulates of the prefill's linear layers per token (the LM head excluded)."""
+    H, F = cfg.hidden, cfg.ffn
+    tot = 0
+    for kind in cfg.pattern:
+        tot += 3 * F * H
+        if kind == "D":
+            tot += cfg.dn_in_rows * H + H * cfg.dn_heads * cfg.dn_dv
+        else:
+            tot += cfg.at_in_rows * H + H * cfg.at_q_heads * cfg.at_head_dim
+    return tot
+
+
+def run_prefill(args):
+    """Prefill throughput: one step = reset + mk_prefill of a uniform random prompt."""
+    import torch
+    import hybrid_deltanet_attention_b200 as hda
+    import synth
+
+    rank, world, local = dist_setup(args.gpus)
+    cfg = synth.QWEN_08B
+    T = int(args.workload[2:])
+    dev = torch.device("cuda", local)
+    raw = synth.make_weights(cfg)
+    m = hda.Model(cfg, hda.weights_to_device(raw, dev), max_ctx=T + 16)
+    del raw
+    prompt_np = synth.make_prompt(cfg, T, tag=f"pp{T}")
+    prompt = torch.from_numpy(prompt_np).to(dev)
+    nxt = torch.empty(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_step():
+        m.reset()
+        m.prefill(prompt, next_token=nxt)
+
+    for _ in range(args.warmup):
+        one_step()
+    assert m.sync() == 0
+    launches0 = m.launches
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.steps):
+            one_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    assert m.sync() == 0
+    ms = max_over_ranks(a.elapsed_time(b), world) / args.steps
+    value = world * T / (ms / 1000.0)
+    # end to end: pinned host prompt -> prefill -> next token to pinned host
+    h_in = torch.from_numpy(prompt_np).pin_memory()
+    h_out = torch.empty(1, dtype=torch.int32).pin_memory()
+
+    def e2e_step():
+        m.reset()
+        prompt.copy_(h_in, non_blocking=True)
+        m.prefill(prompt, next_token=nxt)
+        h_out.copy_(nxt, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    e2e_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    e2e = world * args.steps * T / max_over_ranks(time.perf_counter() - t0, world)
+    if rank != 0:
+        return 0
+    macs = linear_macs_per_token(cfg) * (T - 1)          # the last token runs through the decode kernel
+    useful_tflops = 2.0 * macs / (ms / 1000.0) / 1e12
+    peak = None
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            peak = float(json.load(fh).get("bf16_tflops") or 0) or None
+    line = {
+        "metric": f"prefill tok/s (pp{T}) and tensor-core FLOP/s of the linear layers", "value": value,
+        "unit": "tok/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (fp32 activations as bf16 hi+lo)",
+        "data": "synthetic",
+        "config": {"workload": f"0.8B-shaped hybrid, bf16 weights N(0,0.02) seed 1, {T}-token uniform random prompt, "
+                               "batch 1, reset + prefill per step", "prompt": T},
+        "roofline": {"bound": "tensor", "achieved": useful_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (useful_tflops / peak) if peak else None, "traffic": None,
+                     "what": "whole-prefill time against the linear-layer FLOPs (2 x MACs x tokens); the bf16 hi/lo "
+                             "split issues twice these tensor-core FLOPs", "peak_kind": "measured, burst (the prefill is timed alone)"},
+        "e2e": {"value": e2e, "unit": "tok/s", "h2d_bytes_per_step": T * 4, "d2h_bytes_per_step": 4},
+        "gpu_launches": (m.launches - launches0) // max(1, args.steps),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,10 +510,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="tg128", choices=["tg128", "long"])
+    ap.add_argument("--workload", default="tg128", choices=["tg128", "long", "pp520", "pp4096"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload.startswith("pp"):
+        return run_prefill(args)
     return run_mk(args)
 
 

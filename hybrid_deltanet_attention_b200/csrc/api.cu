@@ -204,6 +204,9 @@ struct Layout {
   // batched prefill workspace
   int pf_rows;
   size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec;
+  // batched verify saves
+  int vf_rows;
+  size_t vf_delta, vf_k, vf_g, vf_raw, vf_logits, vf_greedy;
 };
 
 // Tokens per batched prefill pass: the whole context up to 4096, 0 when a shape is outside
@@ -302,6 +305,16 @@ Layout make_layout(const mk_config& c, int grid) {
     L.pf_p = off; off = align256(off + nch * c.dn_heads * 64 * 64 * 4);
     L.pf_gam = off; off = align256(off + T * c.dn_heads * 4);
     L.pf_dec = off; off = align256(off + T * c.dn_heads * 4);
+  }
+  L.vf_rows = (L.pf_rows > 0 && c.max_draft > 0 && c.max_draft + 1 <= std::min(64, L.pf_rows)) ? c.max_draft + 1 : 0;
+  if (L.vf_rows > 0) {
+    const size_t R = static_cast<size_t>(L.vf_rows) * nd;
+    L.vf_delta = off; off = align256(off + R * c.dn_heads * c.dn_dv * 4);
+    L.vf_k = off; off = align256(off + R * c.dn_heads * c.dn_dk * 4);
+    L.vf_g = off; off = align256(off + R * c.dn_heads * 4);
+    L.vf_raw = off; off = align256(off + R * C * 4);
+    L.vf_logits = off; off = align256(off + static_cast<size_t>(L.vf_rows) * c.vocab * 4);
+    L.vf_greedy = off; off = align256(off + static_cast<size_t>(L.vf_rows) * 4);
   }
   L.sz.workspace_bytes = off;
   L.sz.grid_ctas = grid;
@@ -577,6 +590,15 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     m->pf.gam = reinterpret_cast<float*>(W + L.pf_gam);
     m->pf.dec = reinterpret_cast<float*>(W + L.pf_dec);
   }
+  m->vf.rows = L.vf_rows;
+  if (L.vf_rows > 0) {
+    m->vf.delta = reinterpret_cast<float*>(W + L.vf_delta);
+    m->vf.k = reinterpret_cast<float*>(W + L.vf_k);
+    m->vf.g = reinterpret_cast<float*>(W + L.vf_g);
+    m->vf.raw = reinterpret_cast<float*>(W + L.vf_raw);
+    m->vf.logits = reinterpret_cast<float*>(W + L.vf_logits);
+    m->vf.greedy = reinterpret_cast<int32_t*>(W + L.vf_greedy);
+  }
   *out = m;
   return MK_OK;
 }
@@ -638,6 +660,8 @@ int mk_verify_drafts(mk_model* m, const int32_t* d_tokens, int32_t K, int32_t* d
   if (K < 1 || K > m->cfg.max_draft) return fail(MK_ERR_ARG, "K outside [1, max_draft]");
   if (m->pos_hint + K + 1 > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "drafts exceed the context capacity");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (m->vf.rows >= K + 1 && !getenv("MK_VERIFY_BY_DECODE"))
+    return mk_verify_batched(m, d_tokens, K, d_n_accepted, d_out_tokens, d_logits, s);
   const mk::DecodeParams& b = m->base;
   uint8_t* snapS = m->ws_snap;
   uint8_t* snapC = snapS + align256(m->snap_S_bytes);

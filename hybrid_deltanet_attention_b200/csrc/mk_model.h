@@ -32,8 +32,24 @@ struct mk_prefill_layer {   // K-major copies of the projections the decode kern
   const uint8_t* w_down;     // [H][F] bf16
 };
 
-// Batched prefill of n tokens at the device position (+ off): every layer, no logits.
+// What a verify pass keeps so that the recurrent state can be committed to any accepted
+// prefix afterwards (per DeltaNet layer, per token of the pass).
+struct mk_verify_ws {
+  int rows = 0;              // tokens per pass it holds (max_draft + 1); 0: no batched verify
+  float* delta = nullptr;    // [n_dn][rows][Hd dv] delta-rule updates
+  float* k = nullptr;        // [n_dn][rows][Hd dk] normalised keys
+  float* g = nullptr;        // [n_dn][rows][Hd] cumulative log decay inside the pass
+  float* raw = nullptr;      // [n_dn][rows][C] conv inputs
+  float* logits = nullptr;   // [rows][V]
+  int32_t* greedy = nullptr; // [rows]
+};
+
+// Batched prefill of n tokens at the device position: every layer, no logits.
 int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t s);
+// Verify pass of K+1 tokens in one pass over the weights, acceptance, and commit of the
+// accepted prefix (DeltaNet state and conv history rebuilt from the saved updates).
+int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
+                      float* d_logits, cudaStream_t s);
 
 struct mk_model {
   mk_config cfg;
@@ -56,4 +72,5 @@ struct mk_model {
   size_t step_scratch_bytes;   // leading part of the workspace one decode step uses
   mk_prefill_ws pf;
   std::vector<mk_prefill_layer> pf_layers;
+  mk_verify_ws vf;
 };

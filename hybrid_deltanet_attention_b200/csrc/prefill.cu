@@ -202,6 +202,11 @@ struct WyBufs {
   float* dec;       // [T][Hd]
   float* o;         // [T][Hd dv]
   int T, Hd, dk, dv;
+  // verify passes (one chunk): keep g, k and the updates Delta, leave S untouched
+  float* save_g;     // [T][Hd] or null
+  float* save_k;     // [T][Hd dk] or null
+  float* save_delta; // [T][Hd dv] or null
+  int keep_state;
 };
 
 __global__ void __launch_bounds__(256) wy_prep(WyBufs b) {
@@ -286,6 +291,13 @@ __global__ void __launch_bounds__(256) wy_prep(WyBufs b) {
     const int r = threadIdx.x;
     b.gam[static_cast<long long>(t0 + r) * Hd + h] = expf(g[r]);
     b.dec[static_cast<long long>(t0 + r) * Hd + h] = expf(g[n - 1] - g[r]);
+    if (b.save_g) b.save_g[static_cast<long long>(t0 + r) * Hd + h] = g[r];
+  }
+  if (b.save_k) {
+    for (int idx = threadIdx.x; idx < n * dk; idx += blockDim.x) {
+      const int r = idx / dk, j = idx % dk;
+      b.save_k[static_cast<long long>(t0 + r) * Hd * dk + h * dk + j] = K[r * kp + j];
+    }
   }
 }
 
@@ -338,6 +350,7 @@ __global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S 
       float acc = 0.f;
       for (int j = 0; j < dk; ++j) acc = fmaf(Wc[r * kp + j], S0[ti * kp + j], acc);
       Dl[r * 17 + ti] = Uc[r * kRowGroup + ti] - acc;
+      if (b.save_delta && r < n) b.save_delta[static_cast<long long>(t0 + r) * Hd * dv + h * dv + i0 + ti] = Dl[r * 17 + ti];
     }
     __syncthreads();
     // o_r = gamma_r S0 q_r + sum_{s<=r} P[r][s] Delta_s
@@ -349,6 +362,7 @@ __global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S 
       b.o[static_cast<long long>(t0 + r) * Hd * dv + h * dv + i0 + ti] = acc;
     }
     __syncthreads();
+    if (b.keep_state) continue;
     // S0 <- gamma_{n-1} S0 + sum_r dec_r Delta_r k_r^T
     const float gl = gm[n - 1];
     for (int idx = threadIdx.x; idx < kRowGroup * dk; idx += blockDim.x) {
@@ -359,6 +373,7 @@ __global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S 
     }
   }
   __syncthreads();
+  if (b.keep_state) return;
   for (int idx = threadIdx.x; idx < kRowGroup * dk; idx += blockDim.x) Sg[idx] = S0[(idx / dk) * kp + idx % dk];
 }
 
@@ -487,8 +502,77 @@ __global__ void advance_pos(int* pos, int n, int max_ctx) {
   *pos = min(*pos + n, max_ctx);
 }
 
-// One pass of every layer over T tokens at device position *pos + off.
-cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaStream_t s) {
+// Greedy token of each logits row (lowest index among equal maxima).
+__global__ void row_argmax(const float* __restrict__ logits, int V, int32_t* __restrict__ out) {
+  __shared__ unsigned long long best[32];
+  const float* r = logits + static_cast<long long>(blockIdx.x) * V;
+  unsigned long long b = 0;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) {
+    const unsigned long long k = pack_argmax(r[i], i);
+    b = k > b ? k : b;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long x = __shfl_xor_sync(0xffffffffu, b, o);
+    b = x > b ? x : b;
+  }
+  if ((threadIdx.x & 31) == 0) best[threadIdx.x >> 5] = b;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) b = best[w] > b ? best[w] : b;
+    b = best[0] > b ? best[0] : b;
+    out[blockIdx.x] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(b & 0xFFFFFFFFull));
+  }
+}
+
+// Commit of a verify pass to its accepted prefix: tokens 0 .. n of the pass (n = *n_acc)
+// enter the state, S = e^{g_n} S0 + sum_{r<=n} e^{g_n - g_r} Delta_r k_r^T, for one row
+// group of one head.
+__global__ void __launch_bounds__(256) commit_state(float* __restrict__ S, const float* __restrict__ delta,
+                                                    const float* __restrict__ kk, const float* __restrict__ g,
+                                                    const int* __restrict__ n_acc, int Hd, int dk, int dv) {
+  const int h = blockIdx.x, i0 = blockIdx.y * kRowGroup;
+  const int last = *n_acc;
+  const float gl = g[static_cast<long long>(last) * Hd + h];
+  for (int idx = threadIdx.x; idx < kRowGroup * dk; idx += blockDim.x) {
+    const int i = i0 + idx / dk, j = idx % dk;
+    float* sp = S + (static_cast<long long>(h) * dv + i) * dk + j;
+    float acc = expf(gl) * *sp;
+    for (int r = 0; r <= last; ++r)
+      acc = fmaf(expf(gl - g[static_cast<long long>(r) * Hd + h]) * delta[static_cast<long long>(r) * Hd * dv + h * dv + i],
+                 kk[static_cast<long long>(r) * Hd * dk + h * dk + j], acc);
+    *sp = acc;
+  }
+}
+
+// Conv history of the accepted prefix: the raw inputs of its last W-1 tokens.
+__global__ void commit_conv(const float* __restrict__ raw, float* __restrict__ ring, int W, int C,
+                            const int* __restrict__ posp, const int* __restrict__ n_acc) {
+  const int m = blockIdx.y, r = *n_acc - m;
+  if (r < 0) return;
+  const int p = *posp + r;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < C; c += gridDim.x * blockDim.x)
+    ring[static_cast<long long>(p % W) * C + c] = raw[static_cast<long long>(r) * C + c];
+}
+
+__global__ void advance_pos_accepted(int* pos, const int* n_acc, int max_ctx) {
+  *pos = min(*pos + *n_acc + 1, max_ctx);
+}
+
+__global__ void accept_prefix(const int* tokens, const int* g, int K, int* n_out, int* n_acc, int* out) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int n = 0;
+  while (n < K && tokens[1 + n] == g[n]) ++n;
+  for (int i = 0; i < n; ++i) out[i] = tokens[1 + i];
+  out[n] = g[n];
+  *n_out = n;
+  *n_acc = n;
+}
+
+// One pass of every layer over T tokens at device position *pos + off. With vs (a verify
+// pass, T <= 64) the DeltaNet layers keep their state and conv history untouched and
+// save what the commit of an accepted prefix needs.
+cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaStream_t s,
+                         const mk_verify_ws* vs = nullptr) {
   const mk_config& c = m->cfg;
   const DecodeParams& b = m->base;
   const mk_prefill_ws& pf = m->pf;
@@ -522,9 +606,20 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       linear(L.w_in, 2LL * H + 16, rows, H, pf.z, rows, 0);
       dn_prep<<<T, kPT, C * sizeof(float), s>>>(pf.z, rows, b.pos, off, ring, Wc, C, Hd, dk, L.conv, pf.y, rows);
       chk();
-      conv_history_update<<<dim3((C + kPT - 1) / kPT, Wc - 1), kPT, 0, s>>>(pf.z, rows, T, b.pos, off, ring, Wc, C);
-      chk();
-      WyBufs wy{pf.y, rows, pf.u, pf.w, pf.p, pf.gam, pf.dec, pf.o, T, Hd, dk, dv};
+      WyBufs wy{pf.y, rows, pf.u, pf.w, pf.p, pf.gam, pf.dec, pf.o, T, Hd, dk, dv, nullptr, nullptr, nullptr, 0};
+      if (vs) {
+        const size_t r = static_cast<size_t>(vs->rows) * (di - 1);
+        if (e == cudaSuccess)
+          e = cudaMemcpy2DAsync(vs->raw + r * C, C * sizeof(float), pf.z, rows * sizeof(float), C * sizeof(float), T,
+                                cudaMemcpyDeviceToDevice, s);
+        wy.save_g = vs->g + r * Hd;
+        wy.save_k = vs->k + r * Hd * dk;
+        wy.save_delta = vs->delta + r * Hd * dv;
+        wy.keep_state = 1;
+      } else {
+        conv_history_update<<<dim3((C + kPT - 1) / kPT, Wc - 1), kPT, 0, s>>>(pf.z, rows, T, b.pos, off, ring, Wc, C);
+        chk();
+      }
       const int nch = (T + kChunk - 1) / kChunk;
       wy_prep<<<dim3(nch, Hd), 256, wy_prep_smem(dk, dv), s>>>(wy);
       chk();
@@ -601,5 +696,70 @@ int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t
     return MK_ERR_CUDA;
   }
   m->pos_hint += n;
+  return MK_OK;
+}
+
+int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
+                      float* d_logits, cudaStream_t s) {
+  const mk::DecodeParams& b = m->base;
+  const mk_config& c = m->cfg;
+  const int T = K + 1;
+  const mk_verify_ws& vs = m->vf;
+  cudaError_t e = mk::set_prefill_smem_limits();
+  auto chk = [&]() {
+    if (e == cudaSuccess) e = cudaGetLastError();
+    ++m->launches;
+  };
+  if (e == cudaSuccess) {
+    mk::check_capacity<<<1, 1, 0, s>>>(b.pos, T, c.max_ctx, b.err);
+    chk();
+  }
+  // 1. every layer over the K + 1 tokens, one pass over the weights
+  if (e == cudaSuccess) e = mk::prefill_pass(m, d_tokens, T, 0, s, &vs);
+  // 2. final norm, LM head on the tensor cores for all K + 1 positions, greedy tokens
+  float* logits = d_logits ? d_logits : vs.logits;
+  if (e == cudaSuccess) {
+    mk::rms_split<<<T, mk::kPT, 0, s>>>(m->pf.h, c.hidden, b.norm_f, b.eps, m->pf.xhi, m->pf.xlo);
+    chk();
+  }
+  if (e == cudaSuccess) {
+    mk::LinearArgs a{m->pf.xhi, m->pf.xlo, b.embed, 2LL * c.hidden, logits, c.vocab, T, c.vocab, c.hidden, 0, b.err};
+    e = mk::launch_linear(a, s);
+    ++m->launches;
+  }
+  if (e == cudaSuccess) {
+    mk::row_argmax<<<T, 256, 0, s>>>(logits, c.vocab, vs.greedy);
+    chk();
+  }
+  // 3. longest matching prefix plus the bonus token
+  if (e == cudaSuccess) {
+    mk::accept_prefix<<<1, 32, 0, s>>>(d_tokens, vs.greedy, K, m->ws_n, d_n_accepted, d_out_tokens);
+    chk();
+  }
+  // 4. commit: DeltaNet states and conv histories of the accepted prefix, then the position
+  int di = 0;
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+    if (c.pattern[l] != 'D') continue;
+    const size_t r = static_cast<size_t>(vs.rows) * di;
+    float* S = b.S + static_cast<size_t>(di) * c.dn_heads * c.dn_dv * c.dn_dk;
+    float* ring = b.conv_ring + static_cast<size_t>(di) * c.conv_width * b.C;
+    mk::commit_state<<<dim3(c.dn_heads, c.dn_dv / mk::kRowGroup), 256, 0, s>>>(
+        S, vs.delta + r * c.dn_heads * c.dn_dv, vs.k + r * c.dn_heads * c.dn_dk, vs.g + r * c.dn_heads, m->ws_n,
+        c.dn_heads, c.dn_dk, c.dn_dv);
+    chk();
+    mk::commit_conv<<<dim3((b.C + 255) / 256, c.conv_width - 1), 256, 0, s>>>(vs.raw + r * b.C, ring, c.conv_width,
+                                                                               b.C, b.pos, m->ws_n);
+    chk();
+    ++di;
+  }
+  if (e == cudaSuccess) {
+    mk::advance_pos_accepted<<<1, 1, 0, s>>>(b.pos, m->ws_n, c.max_ctx);
+    chk();
+  }
+  if (e != cudaSuccess) {
+    mk_set_last_error(std::string("verify pass: ") + cudaGetErrorString(e));
+    return MK_ERR_CUDA;
+  }
+  m->pos_hint += 1;   // at least one position is always committed; the exact count is on the device
   return MK_OK;
 }

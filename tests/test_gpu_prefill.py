@@ -106,3 +106,47 @@ def test_08b_batched_prefill_130():
     st = oracle.new_state(cfg, 256)
     zo, zg, tg = _prefill_both(cfg, m, st, W, synth.make_prompt(cfg, 130, tag="pf08"))
     _check(cfg, m, st, zo, zg, tg)
+
+
+def test_08b_verify_one_pass():
+    """Speculative verify on the 0.8B shape: K + 1 tokens in one pass over the weights,
+    acceptance, and the DeltaNet state committed to the accepted prefix."""
+    import hybrid_deltanet_attention_b200 as hda
+    cfg = synth.QWEN_08B
+    raw = synth.make_weights(cfg)
+    m = hda.Model(cfg, hda.weights_to_device(raw), max_ctx=128, max_draft=5)
+    W = oracle.prepare_weights(cfg, raw)
+    del raw
+    dev = torch.device("cuda")
+    K = 5
+    prompt = synth.make_prompt(cfg, 40, tag="vf08")
+    m.reset()
+    st = oracle.new_state(cfg, 128)
+    oracle.prefill(cfg, W, st, prompt[:-1])
+    m.prefill(torch.from_numpy(prompt[:-1]).to(dev))
+    last = int(prompt[-1])
+    for ps in range(3):
+        greedy, _ = oracle.greedy_generate(cfg, W, st.copy(), last, K)
+        use, ids = synth.draft_choices(4, ps, K, cfg.vocab)
+        if ps == 0:
+            use[:] = True
+        if ps == 1:
+            use[:] = False
+        drafts = synth.compose_drafts(greedy, use, ids, cfg.vocab)
+        n_or, committed, z_or = oracle.verify_drafts(cfg, W, st, last, drafts)
+        toks = torch.from_numpy(np.concatenate([[last], drafts]).astype(np.int32)).to(dev)
+        n_acc = torch.zeros(1, dtype=torch.int32, device=dev)
+        out = torch.full((K + 1,), -1, dtype=torch.int32, device=dev)
+        logits = torch.empty((K + 1, cfg.vocab), dtype=torch.float32, device=dev)
+        m.verify(toks, n_acc, out, logits)
+        assert m.sync() == 0
+        assert int(n_acc.item()) == n_or
+        assert list(out.cpu().numpy()[:n_or + 1]) == list(committed)
+        assert np.abs(logits.cpu().numpy() - z_or).max() <= LOGIT_MAX_ABS
+        S = m.S.cpu().numpy()
+        assert max(rel_frob(S[li], st.S[li]) for li in range(cfg.n_dn)) <= STATE_REL_FROB
+        ring = m.conv_history.cpu().numpy()
+        for li in range(cfg.n_dn):
+            assert rel_frob(conv_history_as_window(ring[li], st.pos, cfg.conv_width), st.conv[li]) <= STATE_REL_FROB
+        assert int(m.pos_tensor.item()) == st.pos
+        last = int(committed[-1])
