@@ -377,6 +377,277 @@ __global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S 
   for (int idx = threadIdx.x; idx < kRowGroup * dk; idx += blockDim.x) Sg[idx] = S0[(idx / dk) * kp + idx % dk];
 }
 
+// Register-tiled versions of the two kernels above for dk = dv = 64 or 128: float4
+// shared-memory traffic (rows padded by 4 floats: 16-byte aligned, conflict-free for the
+// access patterns below), 4 x 4 output tiles per thread, and the forward substitution on
+// a right-hand-side column held in registers.
+template <int DK, int DV>
+__global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
+  constexpr int KP = DK + 4, AP = kChunk + 4, XW = DV + DK;
+  static_assert(XW <= 256, "one right-hand-side column per thread");
+  extern __shared__ float4 sm4[];
+  float* K = reinterpret_cast<float*>(sm4);   // [64][KP]
+  float* Q = K + kChunk * KP;                 // [64][KP]
+  float* A = Q + kChunk * KP;                 // [64][AP]
+  float* g = A + kChunk * AP;                 // [64]
+  float* bb = g + kChunk;                     // [64]
+  const int Hd = b.Hd, tid = threadIdx.x;
+  const int ch = blockIdx.x, h = blockIdx.y;
+  const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
+  const int qo = h * DK, ko = Hd * DK + h * DK, vo = 2 * Hd * DK + h * DV;
+  const int C = 2 * Hd * DK + Hd * DV;
+  for (int idx = tid; idx < kChunk * DK / 4; idx += 256) {
+    const int r = idx / (DK / 4), j4 = idx % (DK / 4);
+    float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv;
+    if (r < n) {
+      const float* yr = b.y + static_cast<long long>(t0 + r) * b.ldy;
+      kv = *reinterpret_cast<const float4*>(yr + ko + 4 * j4);
+      qv = *reinterpret_cast<const float4*>(yr + qo + 4 * j4);
+    }
+    *reinterpret_cast<float4*>(K + r * KP + 4 * j4) = kv;
+    *reinterpret_cast<float4*>(Q + r * KP + 4 * j4) = qv;
+  }
+  if (tid < kChunk) {
+    const float* yr = b.y + static_cast<long long>(t0 + tid) * b.ldy;
+    g[tid] = tid < n ? yr[C + h] : 0.f;
+    bb[tid] = tid < n ? yr[C + Hd + h] : 0.f;
+  }
+  __syncthreads();
+  if (tid < 32) {   // inclusive prefix sum of log a over the chunk (two values per lane)
+    float v0 = g[2 * tid], v1 = g[2 * tid + 1];
+    v1 += v0;
+    float run = v1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float x = __shfl_up_sync(0xffffffffu, run, o);
+      if (tid >= o) run += x;
+    }
+    const float before = run - v1;
+    g[2 * tid] = before + v0;
+    g[2 * tid + 1] = run;
+  }
+  __syncthreads();
+  // A[r][s] = b_r e^{g_r - g_s} k_r.k_s (s < r),  P[r][s] = e^{g_r - g_s} q_r.k_s (s <= r)
+  {
+    const int rt = tid >> 4, st = tid & 15;
+    float akk[4][4], aqk[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) akk[a][c] = aqk[a][c] = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < DK; j += 4) {
+      float4 kr[4], qr[4], ks[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        kr[a] = *reinterpret_cast<const float4*>(K + (rt + 16 * a) * KP + j);
+        qr[a] = *reinterpret_cast<const float4*>(Q + (rt + 16 * a) * KP + j);
+        ks[a] = *reinterpret_cast<const float4*>(K + (st + 16 * a) * KP + j);
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          akk[a][c] += kr[a].x * ks[c].x + kr[a].y * ks[c].y + kr[a].z * ks[c].z + kr[a].w * ks[c].w;
+          aqk[a][c] += qr[a].x * ks[c].x + qr[a].y * ks[c].y + qr[a].z * ks[c].z + qr[a].w * ks[c].w;
+        }
+    }
+    float* P = b.p + (static_cast<long long>(ch) * Hd + h) * kChunk * kChunk;
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int r = rt + 16 * a, s2 = st + 16 * c;
+        const bool live = r < n;
+        const float e = (s2 <= r && live) ? expf(g[r] - g[s2]) : 0.f;
+        A[r * AP + s2] = (s2 < r) ? bb[r] * e * akk[a][c] : 0.f;
+        P[r * kChunk + s2] = e * aqk[a][c];
+      }
+  }
+  __syncthreads();
+  // (I + A) X = [diag(b) V | diag(b gamma) K]: column j of X in registers
+  if (tid < XW) {
+    const int j = tid;
+    float x[kChunk];
+#pragma unroll
+    for (int r = 0; r < kChunk; ++r) {
+      float v = 0.f;
+      if (r < n) {
+        v = (j < DV) ? b.y[static_cast<long long>(t0 + r) * b.ldy + vo + j] : expf(g[r]) * K[r * KP + (j - DV)];
+        v *= bb[r];
+      }
+      x[r] = v;
+    }
+#pragma unroll
+    for (int r = 1; r < kChunk; ++r) {
+      float acc = x[r];
+#pragma unroll
+      for (int s4 = 0; s4 < r; s4 += 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(A + r * AP + s4);
+        acc = fmaf(-a4.x, x[s4], acc);
+        if (s4 + 1 < r) acc = fmaf(-a4.y, x[s4 + 1], acc);
+        if (s4 + 2 < r) acc = fmaf(-a4.z, x[s4 + 2], acc);
+        if (s4 + 3 < r) acc = fmaf(-a4.w, x[s4 + 3], acc);
+      }
+      x[r] = acc;
+    }
+#pragma unroll
+    for (int r = 0; r < kChunk; ++r) {
+      if (r < n) {
+        if (j < DV) b.u[static_cast<long long>(t0 + r) * Hd * DV + h * DV + j] = x[r];
+        else b.w[static_cast<long long>(t0 + r) * Hd * DK + h * DK + (j - DV)] = x[r];
+      }
+    }
+  }
+  if (tid < n) {
+    b.gam[static_cast<long long>(t0 + tid) * Hd + h] = expf(g[tid]);
+    b.dec[static_cast<long long>(t0 + tid) * Hd + h] = expf(g[n - 1] - g[tid]);
+    if (b.save_g) b.save_g[static_cast<long long>(t0 + tid) * Hd + h] = g[tid];
+  }
+  if (b.save_k) {
+    for (int idx = tid; idx < n * DK; idx += 256) {
+      const int r = idx / DK, j = idx % DK;
+      b.save_k[static_cast<long long>(t0 + r) * Hd * DK + h * DK + j] = K[r * KP + j];
+    }
+  }
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict__ S) {
+  constexpr int KP = DK + 4, AP = kChunk + 4, RG = kRowGroup;
+  extern __shared__ float4 sm4[];
+  float* S0 = reinterpret_cast<float*>(sm4);  // [16][KP]
+  float* Wc = S0 + RG * KP;                   // [64][KP]
+  float* Qc = Wc + kChunk * KP;               // [64][KP]
+  float* Kc = Qc + kChunk * KP;               // [64][KP]
+  float* Pc = Kc + kChunk * KP;               // [64][AP]
+  float* DT = Pc + kChunk * AP;               // [16][AP]  Delta^T
+  float* Uc = DT + RG * AP;                   // [64][16]
+  float* gm = Uc + kChunk * RG;               // [64]
+  float* dc = gm + kChunk;                    // [64]
+  const int Hd = b.Hd, tid = threadIdx.x;
+  const int h = blockIdx.x, i0 = blockIdx.y * RG;
+  float* Sg = S + (static_cast<long long>(h) * DV + i0) * DK;
+  for (int idx = tid; idx < RG * DK / 4; idx += 256) {
+    const int i = idx / (DK / 4), j4 = idx % (DK / 4);
+    *reinterpret_cast<float4*>(S0 + i * KP + 4 * j4) = *reinterpret_cast<const float4*>(Sg + i * DK + 4 * j4);
+  }
+  const int qo = h * DK, ko = Hd * DK + h * DK;
+  const int nch = (b.T + kChunk - 1) / kChunk;
+  const int rg = tid >> 4, ti = tid & 15;       // rows rg + 16 a of the chunk, column ti of the group
+  for (int ch = 0; ch < nch; ++ch) {
+    const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
+    __syncthreads();
+    for (int idx = tid; idx < kChunk * DK / 4; idx += 256) {
+      const int r = idx / (DK / 4), j4 = idx % (DK / 4);
+      float4 wv = make_float4(0.f, 0.f, 0.f, 0.f), qv = wv, kv = wv;
+      if (r < n) {
+        const long long t = t0 + r;
+        wv = *reinterpret_cast<const float4*>(b.w + t * Hd * DK + h * DK + 4 * j4);
+        qv = *reinterpret_cast<const float4*>(b.y + t * b.ldy + qo + 4 * j4);
+        kv = *reinterpret_cast<const float4*>(b.y + t * b.ldy + ko + 4 * j4);
+      }
+      *reinterpret_cast<float4*>(Wc + r * KP + 4 * j4) = wv;
+      *reinterpret_cast<float4*>(Qc + r * KP + 4 * j4) = qv;
+      *reinterpret_cast<float4*>(Kc + r * KP + 4 * j4) = kv;
+    }
+    const float* P = b.p + (static_cast<long long>(ch) * Hd + h) * kChunk * kChunk;
+    for (int idx = tid; idx < kChunk * kChunk / 4; idx += 256) {
+      const int r = idx / (kChunk / 4), s4 = idx % (kChunk / 4);
+      *reinterpret_cast<float4*>(Pc + r * AP + 4 * s4) = *reinterpret_cast<const float4*>(P + r * kChunk + 4 * s4);
+    }
+    {
+      const int r = tid >> 2, q4 = tid & 3;   // 64 rows x 4 float4 of U
+      float4 uv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < n) uv = *reinterpret_cast<const float4*>(b.u + static_cast<long long>(t0 + r) * Hd * DV + h * DV + i0 + 4 * q4);
+      *reinterpret_cast<float4*>(Uc + r * RG + 4 * q4) = uv;
+    }
+    if (tid < kChunk) {
+      gm[tid] = tid < n ? b.gam[static_cast<long long>(t0 + tid) * Hd + h] : 0.f;
+      dc[tid] = tid < n ? b.dec[static_cast<long long>(t0 + tid) * Hd + h] : 0.f;
+    }
+    __syncthreads();
+    // Delta = U - W S0^T and Q S0^T, rows rg + 16 a, column ti
+    float dw[4] = {0.f, 0.f, 0.f, 0.f}, dq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int j = 0; j < DK; j += 4) {
+      const float4 s4 = *reinterpret_cast<const float4*>(S0 + ti * KP + j);
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float4 w4 = *reinterpret_cast<const float4*>(Wc + (rg + 16 * a) * KP + j);
+        const float4 q4 = *reinterpret_cast<const float4*>(Qc + (rg + 16 * a) * KP + j);
+        dw[a] += w4.x * s4.x + w4.y * s4.y + w4.z * s4.z + w4.w * s4.w;
+        dq[a] += q4.x * s4.x + q4.y * s4.y + q4.z * s4.z + q4.w * s4.w;
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = rg + 16 * a;
+      const float d = Uc[r * RG + ti] - dw[a];
+      DT[ti * AP + r] = d;
+      if (b.save_delta && r < n) b.save_delta[static_cast<long long>(t0 + r) * Hd * DV + h * DV + i0 + ti] = d;
+    }
+    __syncthreads();
+    // o_r = gamma_r (Q S0^T)_r + sum_s P[r][s] Delta_s   (P is zero above the diagonal)
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = rg + 16 * a;
+      float acc = gm[r] * dq[a];
+#pragma unroll 4
+      for (int s = 0; s < kChunk; s += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(Pc + r * AP + s);
+        const float4 d4 = *reinterpret_cast<const float4*>(DT + ti * AP + s);
+        acc += p4.x * d4.x + p4.y * d4.y + p4.z * d4.z + p4.w * d4.w;
+      }
+      if (r < n) b.o[static_cast<long long>(t0 + r) * Hd * DV + h * DV + i0 + ti] = acc;
+    }
+    if (b.keep_state) continue;
+    __syncthreads();
+    for (int idx = tid; idx < RG * kChunk; idx += 256) {   // Delta_r scaled by e^{g_{n-1} - g_r}
+      const int i = idx / kChunk, r = idx % kChunk;
+      DT[i * AP + r] *= dc[r];
+    }
+    __syncthreads();
+    // S0 <- gamma_{n-1} S0 + sum_r (dec_r Delta_r) k_r^T: row ti2, float4 columns jq, jq + 16, ...
+    const float gl = gm[n - 1];
+    const int ti2 = tid >> 4, jq = tid & 15;
+#pragma unroll
+    for (int c = 0; c < DK / 64; ++c) {
+      const int j = 4 * jq + 64 * c;
+      float4 acc = *reinterpret_cast<const float4*>(S0 + ti2 * KP + j);
+      acc.x *= gl; acc.y *= gl; acc.z *= gl; acc.w *= gl;
+#pragma unroll 4
+      for (int r = 0; r < kChunk; r += 4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(DT + ti2 * AP + r);
+        const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 k4 = *reinterpret_cast<const float4*>(Kc + (r + u) * KP + j);
+          acc.x = fmaf(dd[u], k4.x, acc.x);
+          acc.y = fmaf(dd[u], k4.y, acc.y);
+          acc.z = fmaf(dd[u], k4.z, acc.z);
+          acc.w = fmaf(dd[u], k4.w, acc.w);
+        }
+      }
+      *reinterpret_cast<float4*>(S0 + ti2 * KP + j) = acc;   // only this thread touches these elements here
+    }
+  }
+  __syncthreads();
+  if (b.keep_state) return;
+  for (int idx = tid; idx < RG * DK / 4; idx += 256) {
+    const int i = idx / (DK / 4), j4 = idx % (DK / 4);
+    *reinterpret_cast<float4*>(Sg + i * DK + 4 * j4) = *reinterpret_cast<const float4*>(S0 + i * KP + 4 * j4);
+  }
+}
+
+template <int DK, int DV>
+size_t wy_fast_smem() {
+  const size_t prep = sizeof(float) * (2 * kChunk * (DK + 4) + kChunk * (kChunk + 4) + 2 * kChunk);
+  const size_t state = sizeof(float) * (kRowGroup * (DK + 4) + 3 * kChunk * (DK + 4) + kChunk * (kChunk + 4) +
+                                        kRowGroup * (kChunk + 4) + kChunk * kRowGroup + 2 * kChunk);
+  return prep > state ? prep : state;
+}
+
 size_t wy_prep_smem(int dk, int dv) {
   return sizeof(float) * (2 * kChunk * (dk + 1) + kChunk * (dv + dk) + kChunk * 65 + 2 * kChunk);
 }
@@ -621,9 +892,19 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         chk();
       }
       const int nch = (T + kChunk - 1) / kChunk;
-      wy_prep<<<dim3(nch, Hd), 256, wy_prep_smem(dk, dv), s>>>(wy);
-      chk();
-      wy_state<<<dim3(Hd, dv / kRowGroup), 256, wy_state_smem(dk), s>>>(wy, S);
+      if (dk == 128 && dv == 128) {
+        wy_prep_fast<128, 128><<<dim3(nch, Hd), 256, wy_fast_smem<128, 128>(), s>>>(wy);
+        chk();
+        wy_state_fast<128, 128><<<dim3(Hd, dv / kRowGroup), 256, wy_fast_smem<128, 128>(), s>>>(wy, S);
+      } else if (dk == 64 && dv == 64) {
+        wy_prep_fast<64, 64><<<dim3(nch, Hd), 256, wy_fast_smem<64, 64>(), s>>>(wy);
+        chk();
+        wy_state_fast<64, 64><<<dim3(Hd, dv / kRowGroup), 256, wy_fast_smem<64, 64>(), s>>>(wy, S);
+      } else {
+        wy_prep<<<dim3(nch, Hd), 256, wy_prep_smem(dk, dv), s>>>(wy);
+        chk();
+        wy_state<<<dim3(Hd, dv / kRowGroup), 256, wy_state_smem(dk), s>>>(wy, S);
+      }
       chk();
       gate_split<<<T, kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo);
       chk();
@@ -663,6 +944,10 @@ cudaError_t set_prefill_smem_limits() {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(dn_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   return e;
 }
 
