@@ -85,6 +85,27 @@ __global__ void pack_rows_tail_kernel(const uint16_t* __restrict__ w, const uint
   }
 }
 
+// Q4 rows: row r of dst = the rbytes bytes of row r of w followed by the 16-byte taps tail.
+__global__ void pack_q4_rows_tail_kernel(const uint32_t* __restrict__ w, const uint16_t* __restrict__ taps,
+                                         uint32_t* __restrict__ dst, int rows, int rwords, int nconv, int W) {
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  const int stride = rwords + 4;
+  for (int c = threadIdx.x; c < rwords; c += blockDim.x) dst[static_cast<size_t>(r) * stride + c] = w[static_cast<size_t>(r) * rwords + c];
+  if (threadIdx.x < 8) {
+    const int j = threadIdx.x;
+    uint16_t* tail = reinterpret_cast<uint16_t*>(dst + static_cast<size_t>(r) * stride + rwords);
+    tail[j] = (r < nconv && j < W) ? taps[static_cast<size_t>(r) * W + j] : 0;
+  }
+}
+
+cudaError_t launch_pack_q4_rows_tail(const void* w, const uint16_t* taps, void* dst, int rows, int rbytes, int nconv,
+                                     int W, cudaStream_t s) {
+  pack_q4_rows_tail_kernel<<<rows, 256, 0, s>>>(static_cast<const uint32_t*>(w), taps, static_cast<uint32_t*>(dst), rows,
+                                                rbytes / 4, nconv, W);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_pack_rows_tail(const uint16_t* w, const uint16_t* taps, void* dst, int rows, int cols, int nconv,
                                   int W, cudaStream_t s) {
   pack_rows_tail_kernel<<<rows, 256, 0, s>>>(w, taps, static_cast<uint16_t*>(dst), rows, cols, nconv, W);
@@ -129,8 +150,11 @@ int check_config(const mk_config* c) {
   if (c->max_ctx <= 0) return fail(MK_ERR_ARG, "max_ctx must be positive");
   if (c->max_draft < 0 || c->max_draft > 16) return fail(MK_ERR_ARG, "max_draft must be in [0, 16]");
   if (c->weight_format != MK_W_BF16 && c->weight_format != MK_W_Q4K) return fail(MK_ERR_ARG, "unknown weight_format");
-  if (c->weight_format == MK_W_Q4K)
-    return fail(MK_ERR_ARG, "weight_format MK_W_Q4K is not supported by this build's decode kernel");
+  if (c->weight_format == MK_W_Q4K) {
+    const long qd = static_cast<long>(c->at_q_heads) * c->at_head_dim;
+    if (c->hidden % 256 || c->ffn % 256 || (static_cast<long>(c->dn_heads) * c->dn_dv) % 256 || qd % 256)
+      return fail(MK_ERR_ARG, "MK_W_Q4K needs hidden, ffn, dn_heads*dn_dv and at_q_heads*at_head_dim to be multiples of 256");
+  }
   const int nd = n_kind(*c, 'D'), na = n_kind(*c, 'A');
   if (nd) {
     if (c->dn_heads <= 0 || c->dn_dk <= 0 || c->dn_dk % 32 || c->dn_dk > 256 || c->dn_dv <= 0 || c->dn_dv > 256)
@@ -162,8 +186,18 @@ int device_grid(int* grid, int* dev) {
 }
 
 // Scratch and shared-memory budget checks that depend on the grid size.
+bool is_q4(const mk_config& c) { return c.weight_format == MK_W_Q4K; }
+size_t q4_rb(size_t cols) { return cols / 256 * mk::kQ4Block; }
+// Floats of the input vector the decode kernel stages in shared memory: H, or with Q4
+// weights the largest projection input (the out- and down-projections read whole vectors).
+int decode_xcap(const mk_config& c) {
+  if (!is_q4(c)) return c.hidden;
+  const int qd = c.at_q_heads * c.at_head_dim;
+  return std::max({c.hidden, c.dn_heads * c.dn_dv, qd, c.ffn});
+}
+
 int check_budget(const mk_config& c, int grid) {
-  const long S = static_cast<long>(mk::decode_scratch_floats(c.hidden));
+  const long S = static_cast<long>(mk::decode_scratch_floats(c.hidden, is_q4(c), decode_xcap(c)));
   if (S < 256) return fail(MK_ERR_ARG, "shared-memory budget exceeded (hidden too large)");
   auto ceil_div = [](long a, long b) { return (a + b - 1) / b; };
   if (n_kind(c, 'D')) {
@@ -198,7 +232,7 @@ struct Layout {
   size_t p_table, p_freq, p_embed, p_normf;
   std::vector<size_t> p_layer;   // start of each layer block
   // workspace
-  size_t w_sync, w_h, w_z, w_y, w_part, w_tok, w_g, w_n, w_snap;
+  size_t w_sync, w_h, w_z, w_y, w_ob, w_ab, w_part, w_tok, w_g, w_n, w_snap;
   size_t snap_S, snap_conv;
   int max_splits;
   // batched prefill workspace
@@ -212,6 +246,7 @@ struct Layout {
 // Tokens per batched prefill pass: the whole context up to 4096, 0 when a shape is outside
 // what the prefill kernels take (then the prompt runs through decode launches).
 int prefill_rows(const mk_config& c) {
+  if (c.weight_format != MK_W_BF16) return 0;   // the batched path takes bf16 weights
   const long qd = static_cast<long>(c.at_q_heads) * c.at_head_dim;
   const long kdn = static_cast<long>(c.dn_heads) * c.dn_dv;
   if (c.hidden % 64 || c.ffn % 64 || kdn % 64 || qd % 64) return 0;
@@ -223,6 +258,23 @@ int prefill_rows(const mk_config& c) {
 size_t layer_block_bytes(const mk_config& c, char kind) {
   const size_t H = c.hidden, rb = H * 2;
   size_t b = align256(H * 2) * 2;                        // norm1, norm2
+  if (is_q4(c)) {
+    const size_t rq = q4_rb(H);
+    const size_t qd = static_cast<size_t>(c.at_q_heads) * c.at_head_dim;
+    if (kind == 'D') {
+      const size_t C = static_cast<size_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
+      b += align256((C + 2 * c.dn_heads) * (rq + 16));     // w_in rows + conv-taps tail
+      b += align256(C * c.conv_width * 2);                  // conv
+      b += align256(H * q4_rb(static_cast<size_t>(c.dn_heads) * c.dn_dv));   // w_out (row-major Q4)
+    } else {
+      const size_t rows = qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim;
+      b += align256(rows * rq);
+      b += align256(H * q4_rb(qd));
+    }
+    b += 2 * align256(static_cast<size_t>(c.ffn) * rq);   // gate, up
+    b += align256(H * q4_rb(c.ffn));                      // down (row-major Q4)
+    return b;
+  }
   if (kind == 'D') {
     const size_t C = static_cast<size_t>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv);
     b += align256((C + 2 * c.dn_heads) * (rb + 16));       // w_in, each row + its conv taps
@@ -245,7 +297,7 @@ Layout make_layout(const mk_config& c, int grid) {
   size_t off = 0;
   L.p_table = off; off = align256(off + sizeof(mk::LayerW) * c.n_layers);
   L.p_freq = off; off = align256(off + sizeof(double) * (c.at_head_dim > 0 ? c.at_head_dim / 2 : 1));
-  L.p_embed = off; off = align256(off + static_cast<size_t>(c.vocab) * H * 2);
+  L.p_embed = off; off = align256(off + static_cast<size_t>(c.vocab) * (is_q4(c) ? q4_rb(H) : H * 2));
   L.p_normf = off; off = align256(off + H * 2);
   for (int l = 0; l < c.n_layers; ++l) {
     L.p_layer.push_back(off);
@@ -274,6 +326,10 @@ Layout make_layout(const mk_config& c, int grid) {
                                         : 0);
   L.w_z = off; off = align256(off + zf * 4);
   L.w_y = off; off = align256(off + C * 4);
+  L.w_ob = off;
+  off = align256(off + std::max<size_t>(static_cast<size_t>(c.dn_heads) * c.dn_dv,
+                                        static_cast<size_t>(c.at_q_heads) * c.at_head_dim) * 4 + 16);
+  L.w_ab = off; off = align256(off + static_cast<size_t>(c.ffn) * 4);
   L.w_part = off;
   off = align256(off + (na ? static_cast<size_t>(c.at_q_heads) * L.max_splits * (c.at_head_dim + 2) * 4 : 4));
   L.w_tok = off; off = align256(off + (static_cast<size_t>(c.max_ctx) + 8) * 4);
@@ -324,7 +380,10 @@ Layout make_layout(const mk_config& c, int grid) {
 void expected_tensors(const mk_config& c, std::map<std::string, Expect>& ex) {
   const int64_t H = c.hidden;
   auto mat = [&](const std::string& n, int64_t r, int64_t k) {
-    ex[n] = Expect{MK_DT_BF16, 2, {r, k}, static_cast<uint64_t>(r * k * 2)};
+    if (is_q4(c) && n.find("dn.conv") == std::string::npos)
+      ex[n] = Expect{MK_DT_Q4K, 2, {r, k}, static_cast<uint64_t>(r) * static_cast<uint64_t>(q4_rb(static_cast<size_t>(k)))};
+    else
+      ex[n] = Expect{MK_DT_BF16, 2, {r, k}, static_cast<uint64_t>(r * k * 2)};
   };
   auto vec = [&](const std::string& n, int64_t r) { ex[n] = Expect{MK_DT_BF16, 1, {r, 0}, static_cast<uint64_t>(r * 2)}; };
   mat("embed", c.vocab, H);
@@ -463,7 +522,55 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   cudaError_t e = copy("embed", L.p_embed);
   if (e == cudaSuccess) e = copy("norm_f", L.p_normf);
   int di = 0, ai = 0;
-  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+  for (int l = 0; l < c.n_layers && e == cudaSuccess && is_q4(c); ++l) {   // Q4_K-style weights
+    const std::string p = "layers." + std::to_string(l) + ".";
+    size_t off = L.p_layer[l];
+    const size_t rq = q4_rb(H);
+    mk::LayerW lw{};
+    lw.kind = c.pattern[l] == 'D' ? mk::kDeltaNet : mk::kAttention;
+    lw.idx = c.pattern[l] == 'D' ? di++ : ai++;
+    lw.norm1 = reinterpret_cast<const uint16_t*>(P + off);
+    e = copy(p + "norm1", off); off += align256(H * 2);
+    lw.norm2 = reinterpret_cast<const uint16_t*>(P + off);
+    if (e == cudaSuccess) e = copy(p + "norm2", off);
+    off += align256(H * 2);
+    if (lw.kind == mk::kDeltaNet) {
+      lw.w_in = P + off;
+      if (e == cudaSuccess) {
+        ++m->launches;
+        e = mk::launch_pack_q4_rows_tail(got[p + "dn.w_in"]->data, static_cast<const uint16_t*>(got[p + "dn.conv"]->data),
+                                         P + off, static_cast<int>(C + 2 * c.dn_heads), static_cast<int>(rq),
+                                         static_cast<int>(C), c.conv_width, s);
+      }
+      off += align256((C + 2 * c.dn_heads) * (rq + 16));
+      lw.conv = reinterpret_cast<const uint16_t*>(P + off);
+      if (e == cudaSuccess) e = copy(p + "dn.conv", off);
+      off += align256(C * c.conv_width * 2);
+      lw.w_out_q4 = P + off;
+      if (e == cudaSuccess) e = copy(p + "dn.w_out", off);
+      off += align256(H * q4_rb(static_cast<size_t>(c.dn_heads) * c.dn_dv));
+    } else {
+      const size_t qd = static_cast<size_t>(c.at_q_heads) * c.at_head_dim;
+      const size_t rows = qd * (c.at_out_gate ? 2 : 1) + 2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim;
+      lw.w_in = P + off;
+      if (e == cudaSuccess) e = copy(p + "attn.w_in", off);
+      off += align256(rows * rq);
+      lw.w_out_q4 = P + off;
+      if (e == cudaSuccess) e = copy(p + "attn.w_out", off);
+      off += align256(H * q4_rb(qd));
+    }
+    lw.w_gate = P + off;
+    if (e == cudaSuccess) e = copy(p + "mlp.w_gate", off);
+    off += align256(static_cast<size_t>(c.ffn) * rq);
+    lw.w_up = P + off;
+    if (e == cudaSuccess) e = copy(p + "mlp.w_up", off);
+    off += align256(static_cast<size_t>(c.ffn) * rq);
+    lw.w_down_q4 = P + off;
+    if (e == cudaSuccess) e = copy(p + "mlp.w_down", off);
+    m->layers_host.push_back(lw);
+    m->pf_layers.push_back(mk_prefill_layer{});
+  }
+  for (int l = 0; l < c.n_layers && e == cudaSuccess && !is_q4(c); ++l) {
     const std::string p = "layers." + std::to_string(l) + ".";
     size_t off = L.p_layer[l];
     mk::LayerW lw{};
@@ -550,7 +657,14 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   b.at_in_rows = static_cast<int>(static_cast<size_t>(c.at_q_heads) * c.at_head_dim * (c.at_out_gate ? 2 : 1) +
                                   2 * static_cast<size_t>(c.at_kv_heads) * c.at_head_dim);
   b.max_ctx = c.max_ctx;
-  b.row_bytes = static_cast<int>(rb);
+  b.row_bytes = static_cast<int>(is_q4(c) ? q4_rb(H) : rb);
+  b.q4 = is_q4(c) ? 1 : 0;
+  b.rb_dn_out = static_cast<int>(q4_rb(static_cast<size_t>(c.dn_heads) * c.dn_dv));
+  b.rb_at_out = static_cast<int>(q4_rb(static_cast<size_t>(c.at_q_heads) * c.at_head_dim));
+  b.rb_ffn = static_cast<int>(q4_rb(c.ffn));
+  b.xcap = decode_xcap(c);
+  b.obuf = reinterpret_cast<float*>(W + L.w_ob);
+  b.abuf = reinterpret_cast<float*>(W + L.w_ab);
   b.eps = c.rms_eps;
   b.S = reinterpret_cast<float*>(St + L.sz.off_S);
   b.conv_ring = reinterpret_cast<float*>(St + L.sz.off_conv);

@@ -17,6 +17,8 @@
 //    needs 3 grid barriers and an attention layer 4;
 //  * every wait (grid barrier, pipeline slot) has a time limit; on expiry the kernel
 //    latches a bit in the device error word and every CTA returns.
+#include <cuda_fp16.h>
+
 #include "dev.cuh"
 #include "mk_internal.h"
 #include "../../include/mk.h"
@@ -38,6 +40,7 @@ struct Ranges {
   int col_b, col_e;       // attention output columns (out-projection split-K)
   int f_b, f_e;           // MLP intermediate rows
   int v_b, v_e;           // LM-head rows
+  int h_b, h_e;           // output rows of the out- and down-projections (Q4 weights)
   int au_valid, au_g, au_j, au_p0, au_p1, au_q1;   // attention split unit
   int nsplit;
 };
@@ -83,6 +86,7 @@ __device__ void compute_ranges(const DecodeParams& p, int cta, int G, int pos, R
   split_range(p.Hq * p.D, cta, G, r.col_b, r.col_e);
   split_range(p.F, cta, G, r.f_b, r.f_e);
   split_range(p.V, cta, G, r.v_b, r.v_e);
+  split_range(p.H, cta, G, r.h_b, r.h_e);
   const int n = pos + 1;
   int CH = 1, nsplit = 1;
   if (p.Hkv > 0) attn_split(n, G, p.Hkv, p.max_splits, CH, nsplit);
@@ -118,9 +122,66 @@ __device__ __forceinline__ void trace_grid(const DecodeParams& p, unsigned k, in
 // ------------------------------------------------------------------ producer
 // Segment s of layer l in stream order (weights, DeltaNet state rows, KV sub-blocks);
 // returns false past the end of the layer. The final "layer" p.n_layers is the LM head.
+template <bool Q4>
 __device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Ranges& r, const LayerW& L, int l, int s,
                                               const uint8_t*& src, int& rows, int& rb) {
   const int wrb = p.row_bytes;
+  if constexpr (Q4) {
+    // order: in-proj | (S rows or KV sub-blocks...) | W_out rows | gate | up | W_down rows
+    if (l == p.n_layers) {
+      if (s > 0) return false;
+      src = p.embed + static_cast<size_t>(r.v_b) * wrb;
+      rows = r.v_e - r.v_b;
+      rb = wrb;
+      return true;
+    }
+    const bool dn = L.kind == kDeltaNet;
+    const int nkv = (!dn && r.au_valid && r.au_q1 > r.au_p0) ? 2 * ((r.au_q1 - r.au_p0 + kAttnSub - 1) / kAttnSub) : 0;
+    if (s == 0) {
+      const int b = dn ? r.in_dn_b : r.in_at_b, e = dn ? r.in_dn_e : r.in_at_e;
+      rb = dn ? wrb + 16 : wrb;
+      src = L.w_in + static_cast<size_t>(b) * rb;
+      rows = e - b;
+      return true;
+    }
+    s -= 1;
+    const int nmix = dn ? 1 : nkv;
+    if (s < nmix) {
+      if (dn) {
+        src = reinterpret_cast<const uint8_t*>(p.S + (static_cast<size_t>(L.idx) * p.Hd * p.dv + r.dn_b) * p.dk);
+        rows = r.dn_e - r.dn_b;
+        rb = p.dk * 4;
+      } else {
+        const int sb = r.au_p0 + (s >> 1) * kAttnSub;
+        const uint16_t* base = ((s & 1) ? p.vc : p.kc) +
+                               (static_cast<size_t>(L.idx) * p.Hkv + r.au_g) * p.max_ctx * p.D + static_cast<size_t>(sb) * p.D;
+        src = reinterpret_cast<const uint8_t*>(base);
+        rows = min(kAttnSub, r.au_q1 - sb);
+        rb = p.D * 2;
+      }
+      return true;
+    }
+    s -= nmix;
+    if (s == 0) {
+      rb = dn ? p.rb_dn_out : p.rb_at_out;
+      src = L.w_out_q4 + static_cast<size_t>(r.h_b) * rb;
+      rows = r.h_e - r.h_b;
+      return true;
+    }
+    if (s == 1 || s == 2) {
+      src = (s == 1 ? L.w_gate : L.w_up) + static_cast<size_t>(r.f_b) * wrb;
+      rows = r.f_e - r.f_b;
+      rb = wrb;
+      return true;
+    }
+    if (s == 3) {
+      rb = p.rb_ffn;
+      src = L.w_down_q4 + static_cast<size_t>(r.h_b) * rb;
+      rows = r.h_e - r.h_b;
+      return true;
+    }
+    return false;
+  }
   if (l == p.n_layers) {
     if (s > 0) return false;
     src = p.embed + static_cast<size_t>(r.v_b) * wrb;
@@ -186,6 +247,7 @@ __device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Range
 
 // A second walk over the same chunk sequence, used to issue L2 prefetches ahead of the
 // shared-memory fill. next() yields the chunks in stream order; false at the end.
+template <bool Q4>
 struct PrefetchCursor {
   int l = 0, s = -1, r0 = 0, rows = 0, rb = 1;
   const uint8_t* src = nullptr;
@@ -205,7 +267,7 @@ struct PrefetchCursor {
       ++s;
       r0 = 0;
       rows = 0;
-      if (!layer_segment(p, r, L, l, s, src, rows, rb)) {
+      if (!layer_segment<Q4>(p, r, L, l, s, src, rows, rb)) {
         ++l;
         s = -1;
         rows = 0;
@@ -218,13 +280,14 @@ struct PrefetchCursor {
 // p.prefetch_bytes it also keeps L2 prefetches of the chunks that follow running that
 // many bytes ahead, so HBM keeps streaming while the ring is full and the consumers
 // wait at a grid barrier.
+template <int NS, bool Q4>
 __device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) {
   const uint64_t pol = policy_evict_first();
   const Ranges r = sh->rg;
   volatile int* abort = &sh->abort_flag;
   uint32_t n = 0;
   bool ok = true;
-  PrefetchCursor pf;
+  PrefetchCursor<Q4> pf;
   const uint64_t pf_dist = p.prefetch_bytes > 0 ? static_cast<uint64_t>(p.prefetch_bytes) : 0;
   uint64_t filled = 0, prefetched = 0;
   bool pf_live = pf_dist > 0;
@@ -233,13 +296,13 @@ __device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) 
     const LayerW Lnext = (l + 1 < p.n_layers) ? p.layers[l + 1] : L;   // load ahead of use
     const uint8_t* src;
     int rows, rb;
-    for (int s = 0; ok && layer_segment(p, r, L, l, s, src, rows, rb); ++s) {
+    for (int s = 0; ok && layer_segment<Q4>(p, r, L, l, s, src, rows, rb); ++s) {
       const int rpc = kSlotBytes / rb;
       for (int r0 = 0; r0 < rows; r0 += rpc) {
         const uint32_t bytes = static_cast<uint32_t>(min(rpc, rows - r0)) * rb;
-        const int slot = n % kSlots;
-        if (n >= static_cast<uint32_t>(kSlots)) {
-          if (!mbar_wait(&sh->empty[slot], ((n / kSlots) - 1) & 1, abort, kWaitLimitNs)) {
+        const int slot = n % NS;
+        if (n >= static_cast<uint32_t>(NS)) {
+          if (!mbar_wait(&sh->empty[slot], ((n / NS) - 1) & 1, abort, kWaitLimitNs)) {
             if (!*abort) atomicOr(p.err, MK_DEVERR_PIPE_TIMEOUT);
             *abort = 1;
             ok = false;
@@ -267,18 +330,19 @@ __device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) 
     L = Lnext;
   }
   // Let every issued copy land before this lane leaves (bounded): the last chunk
-  // issued to each slot is one of the last kSlots chunks.
+  // issued to each slot is one of the last NS chunks.
   int never = 0;
-  for (uint32_t m = (n > static_cast<uint32_t>(kSlots) ? n - kSlots : 0); m < n; ++m)
-    mbar_wait(&sh->full[m % kSlots], (m / kSlots) & 1, &never, kDrainLimitNs);
+  for (uint32_t m = (n > static_cast<uint32_t>(NS) ? n - NS : 0); m < n; ++m)
+    mbar_wait(&sh->full[m % NS], (m / NS) & 1, &never, kDrainLimitNs);
 }
 
 // ------------------------------------------------------------------ consumer helpers
+template <int NS>
 __device__ __forceinline__ const uint8_t* acquire(const DecodeParams& p, Shared* sh, uint8_t* ring, uint32_t n,
                                                   int tid, int lane) {
-  const int slot = n % kSlots;
+  const int slot = n % NS;
   if (tid == 0) trace_at(p, kTraceChunks + 4 * static_cast<int>(n) + 1);
-  if (!mbar_wait(&sh->full[slot], (n / kSlots) & 1, &sh->abort_flag, kWaitLimitNs)) {
+  if (!mbar_wait(&sh->full[slot], (n / NS) & 1, &sh->abort_flag, kWaitLimitNs)) {
     if (lane == 0) {
       if (!sh->abort_flag) atomicOr(p.err, MK_DEVERR_PIPE_TIMEOUT);
       sh->abort_flag = 1;
@@ -287,10 +351,11 @@ __device__ __forceinline__ const uint8_t* acquire(const DecodeParams& p, Shared*
   if (tid == 0) trace_at(p, kTraceChunks + 4 * static_cast<int>(n) + 2);
   return ring + static_cast<size_t>(slot) * kSlotBytes;
 }
+template <int NS>
 __device__ __forceinline__ void release(const DecodeParams& p, Shared* sh, uint32_t& n, int lane) {
   if (threadIdx.x == 0) trace_at(p, kTraceChunks + 4 * static_cast<int>(n) + 3);
   __syncwarp();
-  if (lane == 0) mbar_arrive(&sh->empty[n % kSlots]);
+  if (lane == 0) mbar_arrive(&sh->empty[n % NS]);
   ++n;
 }
 
@@ -357,13 +422,41 @@ __device__ __forceinline__ float* res_delta(const DecodeParams& p, int H, int j,
 
 // Norm phase j: xs = h_j / sqrt(mean(h_j^2) + eps) * gamma (fp32, kept on chip), with
 // h_j = base + delta (or, for j = 0, the bf16 embedding row). All loads are issued together.
+// Four consecutive weights 4g .. 4g+3 of a Q4_K-style row (144-byte super-blocks): they
+// share a super-block, a sub-block and a nibble half.
+__device__ __forceinline__ float4 q4_dequant4(const uint8_t* row, int g) {
+  const int i = 4 * g, sb = i >> 8, w = i & 255, jb = w >> 5, t = w & 31;
+  const uint8_t* blk = row + static_cast<size_t>(sb) * kQ4Block;
+  const uint32_t dd = *reinterpret_cast<const uint32_t*>(blk);
+  const uint64_t lo = static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 4)) |
+                      (static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 8)) << 32);
+  const uint64_t hi = static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 8)) |
+                      (static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 12)) << 32);
+  const float sc = static_cast<float>(static_cast<uint32_t>(lo >> (6 * jb)) & 63u);
+  const float mm = static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * jb)) & 63u);
+  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) * sc;
+  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) * mm;
+  const uint32_t c = *reinterpret_cast<const uint32_t*>(blk + 16 + 16 * jb + (t & 15));
+  const int sh = (t >= 16) ? 4 : 0;
+  return make_float4(fmaf(s, static_cast<float>((c >> sh) & 15u), -mn), fmaf(s, static_cast<float>((c >> (8 + sh)) & 15u), -mn),
+                     fmaf(s, static_cast<float>((c >> (16 + sh)) & 15u), -mn),
+                     fmaf(s, static_cast<float>((c >> (24 + sh)) & 15u), -mn));
+}
+
 template <int MG>
 __device__ __forceinline__ void rmsnorm(const DecodeParams& p, int H, int j, const uint16_t* bf_row,
-                                       const uint16_t* gamma, float* xs, Shared* sh, int tid, int warp, int lane) {
+                                       const uint16_t* gamma, float* xs, Shared* sh, int tid, int warp, int lane,
+                                       const uint8_t* q4_row = nullptr) {
   const int ng = H / 4;
   const int cta = blockIdx.x, G = gridDim.x;
   float4 v[MG];
-  if (bf_row) {
+  if (q4_row) {
+#pragma unroll
+    for (int k = 0; k < MG; ++k) {
+      const int g = tid + k * kConsumerThreads;
+      if (g < ng) v[k] = q4_dequant4(q4_row, g);
+    }
+  } else if (bf_row) {
 #pragma unroll
     for (int k = 0; k < MG; ++k) {
       const int g = tid + k * kConsumerThreads;
@@ -516,7 +609,7 @@ struct ConvEpi {
   const float* chist;
   int b;            // first in-projection row of this CTA
   int W;
-  int H;            // row length (taps start at byte 2H of the row)
+  int tap_off;      // byte offset of the conv taps in the row (after the weights)
   int qk_rows;      // 2 * Hd * dk
   int dk;
   int h_lo;         // first q/k head (index into [q heads | k heads]) this CTA touches
@@ -526,7 +619,7 @@ struct ConvEpi {
 
 __device__ __forceinline__ void conv_epilogue(const ConvEpi& ce, int g, float raw, const uint8_t* row, float* ringc) {
   const int lr = g - ce.b;
-  const uint2 tw = *reinterpret_cast<const uint2*>(row + 2 * ce.H);
+  const uint2 tw = *reinterpret_cast<const uint2*>(row + ce.tap_off);
   const float t0 = bf16lo(tw.x), t1 = bf16hi(tw.x), t2 = bf16lo(tw.y), t3 = bf16hi(tw.y);
   const float tcur = ce.W == 4 ? t3 : (ce.W == 3 ? t2 : t1);    // the tap of the current input
   float y = tcur * raw;
@@ -683,24 +776,136 @@ __device__ __forceinline__ void softmax_block(float* sc, float* mlc, int grp, in
   }
 }
 
+// ------------------------------------------------------------------ Q4_K-style rows
+// One super-block (144 bytes at blk) against x. Lane l takes sub-block j = l / 4 and code
+// bytes 4 (l % 4) .. +3 of it: weights 32 j + 4 (l % 4) + t (low nibbles) and
+// 32 j + 16 + 4 (l % 4) + t (high nibbles), t = 0..3, whose x values are xl and xh and
+// whose x sum is xsv. With w = (d sc_j) q - (dmin m_j) the lane's share of the product is
+// (d sc_j) sum(q x) - (dmin m_j) sum(x); d sc_j and dmin m_j are exact in fp32.
+__device__ __forceinline__ float q4_part(const uint8_t* blk, int j, int part, const float4& xl, const float4& xh,
+                                         float xsv) {
+  const uint32_t dd = *reinterpret_cast<const uint32_t*>(blk);
+  const uint32_t f0 = *reinterpret_cast<const uint32_t*>(blk + 4);
+  const uint32_t f1 = *reinterpret_cast<const uint32_t*>(blk + 8);
+  const uint32_t f2 = *reinterpret_cast<const uint32_t*>(blk + 12);
+  const uint32_t c = *reinterpret_cast<const uint32_t*>(blk + 16 + 16 * j + 4 * part);
+  const uint64_t lo = static_cast<uint64_t>(f0) | (static_cast<uint64_t>(f1) << 32);
+  const uint64_t hi = static_cast<uint64_t>(f1) | (static_cast<uint64_t>(f2) << 32);
+  const float sc = static_cast<float>(static_cast<uint32_t>(lo >> (6 * j)) & 63u);
+  const float mm = static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * j)) & 63u);
+  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) * sc;
+  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) * mm;
+  float qx = static_cast<float>(c & 15u) * xl.x;
+  qx = fmaf(static_cast<float>((c >> 8) & 15u), xl.y, qx);
+  qx = fmaf(static_cast<float>((c >> 16) & 15u), xl.z, qx);
+  qx = fmaf(static_cast<float>((c >> 24) & 15u), xl.w, qx);
+  qx = fmaf(static_cast<float>((c >> 4) & 15u), xh.x, qx);
+  qx = fmaf(static_cast<float>((c >> 12) & 15u), xh.y, qx);
+  qx = fmaf(static_cast<float>((c >> 20) & 15u), xh.z, qx);
+  qx = fmaf(static_cast<float>((c >> 28) & 15u), xh.w, qx);
+  return fmaf(s, qx, -mn * xsv);
+}
+
+// xsum[sb * 32 + l] = the sum of the 8 x values lane l pairs with in super-block sb.
+__device__ __forceinline__ void q4_xsum(const float* xs, float* xsum, int K, int tid) {
+  const int n = (K >> 8) * 32;
+  for (int i = tid; i < n; i += kConsumerThreads) {
+    const int sb = i >> 5, l = i & 31;
+    const float* xb = xs + sb * 256 + 32 * (l >> 2) + 4 * (l & 3);
+    const float4 a = *reinterpret_cast<const float4*>(xb);
+    const float4 b = *reinterpret_cast<const float4*>(xb + 16);
+    xsum[i] = ((a.x + a.y) + (a.z + a.w)) + ((b.x + b.y) + (b.z + b.w));
+  }
+}
+
+// Row products of one ring chunk of nrows Q4 rows (stride rb) with x (nsb super-blocks).
+// Warp w takes super-blocks ks, ks + WK, ... (ks = w % WK) of rows rs, rs + RS, ...
+// (rs = w / WK), four rows at a time; the warps' partial sums meet in qpart [WK][nrows]
+// (WK * nrows <= 455 for any row length) and out(r, value) runs once per row.
+template <typename Out>
+__device__ __forceinline__ void gemv_rows_q4(const uint8_t* chunk, int nrows, int rb, int nsb, const float* xs,
+                                             const float* xsum, float* qpart, int warp, int lane, int tid, Out&& out) {
+  const int WK = nsb >= 8 ? 8 : (nsb >= 4 ? 4 : (nsb >= 2 ? 2 : 1));
+  const int RS = kConsumerWarps / WK;
+  const int ks = warp % WK, rs = warp / WK;
+  const int j = lane >> 2, part = lane & 3;
+  for (int r0 = rs; r0 < nrows; r0 += 4 * RS) {
+    const uint8_t* rp[4];
+    bool live[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = r0 + q * RS;
+      live[q] = r < nrows;
+      rp[q] = chunk + static_cast<size_t>(live[q] ? r : r0) * rb;
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sb = ks; sb < nsb; sb += WK) {
+      const float* xb = xs + sb * 256 + 32 * j + 4 * part;
+      const float4 xl = *reinterpret_cast<const float4*>(xb);
+      const float4 xh = *reinterpret_cast<const float4*>(xb + 16);
+      const float xsv = xsum[sb * 32 + lane];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] += q4_part(rp[q] + static_cast<size_t>(sb) * kQ4Block, j, part, xl, xh, xsv);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float v = warp_sum(acc[q]);
+      if (lane == 0 && live[q]) qpart[ks * nrows + r0 + q * RS] = v;
+    }
+  }
+  cons_sync(kConsumerThreads);
+  for (int r = tid; r < nrows; r += kConsumerThreads) {
+    float v = 0.f;
+    for (int k = 0; k < WK; ++k) v += qpart[k * nrows + r];
+    out(r, v);
+  }
+  cons_sync(kConsumerThreads);
+}
+
+// Rows [h_b, h_e) of a Q4 projection (row stride rbk) whose K-float input sits in global
+// memory (written by every CTA before the last grid barrier): stage it in xs, then the row
+// products go straight into the residual delta of the update after norm j.
+template <int NS>
+__device__ __forceinline__ void q4_rows_to_residual(const DecodeParams& p, Shared* sh, uint8_t* ring, uint32_t& n,
+                                                    const float* src, int K, int rbk, int j, float* xs, float* xsum,
+                                                    float* qpart, int tid, int warp, int lane) {
+  const Ranges& rg = sh->rg;
+  for (int i = tid; i < K / 4; i += kConsumerThreads)
+    reinterpret_cast<float4*>(xs)[i] = __ldcg(reinterpret_cast<const float4*>(src) + i);
+  cons_sync(kConsumerThreads);
+  q4_xsum(xs, xsum, K, tid);
+  cons_sync(kConsumerThreads);
+  float* dst = res_delta(p, p.H, j + 1, 0);
+  const int nrows = rg.h_e - rg.h_b, rpc = kSlotBytes / rbk;
+  for (int r0 = 0; r0 < nrows; r0 += rpc) {
+    const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+    gemv_rows_q4(ch, min(rpc, nrows - r0), rbk, K >> 8, xs, xsum, qpart, warp, lane, tid,
+                 [&](int r, float v) { __stcg(dst + rg.h_b + r0 + r, v); });
+    release<NS>(p, sh, n, lane);
+  }
+}
+
 // ------------------------------------------------------------------ the kernel
 // HK > 0: the hidden size is exactly HK * 256 (compile-time, so the hot loops carry no
 // bound checks and x lives in registers); HK = 0: any hidden size up to 8192.
-template <int HK>
+template <int HK, bool Q4>
 __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int XK = HK;                                // x register groups (0: shared memory)
   constexpr int MG = HK > 0 ? (HK + 3) / 4 : 8;         // float4 groups of the hidden vector per thread
+  constexpr int NS = Q4 ? 2 : kSlots;                   // ring slots (Q4 stages longer input vectors)
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
-  Shared* sh = reinterpret_cast<Shared*>(smem + static_cast<size_t>(kSlots) * kSlotBytes);
-  float* xs = reinterpret_cast<float*>(sh + 1);      // [H] normed input
-  float* fs = xs + p.H;                               // scratch
+  Shared* sh = reinterpret_cast<Shared*>(smem + static_cast<size_t>(NS) * kSlotBytes);
+  float* xs = reinterpret_cast<float*>(sh + 1);      // [xcap] normed input / staged projection input
+  float* xsum = xs + p.xcap;                          // Q4: [xcap / 8] per-lane x sums
+  float* qpart = xsum + (Q4 ? p.xcap / 8 : 0);        // Q4: [kQ4PartFloats] row partial sums
+  float* fs = Q4 ? qpart + kQ4PartFloats : xs + p.H;  // scratch
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x, G = gridDim.x;
 
   if (tid == 0) {
-    for (int s = 0; s < kSlots; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&sh->full[s], 1);
       mbar_init(&sh->empty[s], kConsumerWarps);
     }
@@ -729,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   if (sh->bad) return;
 
   if (warp == kConsumerWarps) {
-    if (lane == 0) producer_loop(p, sh, ring);
+    if (lane == 0) producer_loop<NS, Q4>(p, sh, ring);
     return;
   }
 
@@ -767,14 +972,17 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
         for (int j = 0; j < kMaxConv - 1; ++j)
           if (j < p.convw - 1) th[j] = __ldcg(ringl + static_cast<size_t>((pos + 1 + j) % p.convw) * p.C + b + tid);
       }
-      if (l == 0) {
-        rmsnorm<MG>(p, H, 0, reinterpret_cast<const uint16_t*>(p.embed + static_cast<size_t>(sh->tok) * rb), L.norm1,
-                    xs, sh, tid, warp, lane);   // the residual starts as the embedding row
+      if (l == 0) {   // the residual starts as the embedding row
+        if constexpr (Q4)
+          rmsnorm<MG>(p, H, 0, nullptr, L.norm1, xs, sh, tid, warp, lane, p.embed + static_cast<size_t>(sh->tok) * rb);
+        else
+          rmsnorm<MG>(p, H, 0, reinterpret_cast<const uint16_t*>(p.embed + static_cast<size_t>(sh->tok) * rb), L.norm1,
+                      xs, sh, tid, warp, lane);
       } else {
         rmsnorm<MG>(p, H, 2 * l, nullptr, L.norm1, xs, sh, tid, warp, lane);
       }
       float* ysq = fs + 3 * kConsumerThreads;
-      ConvEpi ce{fs, b, p.convw, H, qk_rows, p.dk, h_lo, p.ybuf, ysq};
+      ConvEpi ce{fs, b, p.convw, Q4 ? rb : 2 * H, qk_rows, p.dk, h_lo, p.ybuf, ysq};
       if (dn) {
         if (tid < nconv) {
 #pragma unroll
@@ -785,13 +993,28 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
       }
       const int rb_in = dn ? rb + 16 : rb;
       const int rpc = kSlotBytes / rb_in;
-      XReg<XK> xr;
-      load_xreg<XK>(xr, xs, H, lane);
-      for (int r0 = 0; r0 < e - b; r0 += rpc) {
-        const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
-        gemv_rows<XK>(ch, min(rpc, e - b - r0), rb_in, xr, xs, H, warp, lane, b + r0, dn ? p.C : kNoSplit,
-                      dn ? ringc : p.z, p.z, dn, ce);
-        release(p, sh, n, lane);
+      if constexpr (Q4) {
+        q4_xsum(xs, xsum, H, tid);
+        cons_sync(kConsumerThreads);
+        for (int r0 = 0; r0 < e - b; r0 += rpc) {
+          const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+          gemv_rows_q4(ch, min(rpc, e - b - r0), rb_in, H >> 8, xs, xsum, qpart, warp, lane, tid, [&](int r, float v) {
+            const int g = b + r0 + r;
+            if (!dn) p.z[g] = v;
+            else if (g < p.C) conv_epilogue(ce, g, v, ch + static_cast<size_t>(r) * rb_in, ringc);
+            else p.z[g - p.C] = v;
+          });
+          release<NS>(p, sh, n, lane);
+        }
+      } else {
+        XReg<XK> xr;
+        load_xreg<XK>(xr, xs, H, lane);
+        for (int r0 = 0; r0 < e - b; r0 += rpc) {
+          const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+          gemv_rows<XK>(ch, min(rpc, e - b - r0), rb_in, xr, xs, H, warp, lane, b + r0, dn ? p.C : kNoSplit,
+                        dn ? ringc : p.z, p.z, dn, ce);
+          release<NS>(p, sh, n, lane);
+        }
       }
       if (n_ss > 0) {   // this CTA's share of the per-head sums of squares of q and k
         cons_sync(kConsumerThreads);
@@ -865,7 +1088,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
         // S rows: S = a S; u = S k; S += b (v - u) k^T; o = S q
         const int srb = p.dk * 4, srpc = kSlotBytes / srb, vpl = p.dk / 32;
         for (int r0 = 0; r0 < nrows; r0 += srpc) {
-          const float* ch = reinterpret_cast<const float*>(acquire(p, sh, ring, n, tid, lane));
+          const float* ch = reinterpret_cast<const float*>(acquire<NS>(p, sh, ring, n, tid, lane));
           const int nr = min(srpc, nrows - r0);
           for (int r = warp; r < nr; r += kConsumerWarps) {
             const int lr = r0 + r;
@@ -899,17 +1122,27 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
             o = warp_sum(o);
             if (lane == 0) oc[lr] = o;
           }
-          release(p, sh, n, lane);
+          release<NS>(p, sh, n, lane);
         }
         cons_sync(kConsumerThreads);
-        const int rpc = kSlotBytes / rb;
-        for (int r0 = 0; r0 < nrows; r0 += rpc) {
-          const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
-          splitk_rows<MG>(ch, min(rpc, nrows - r0), rb, oc + r0, H, acc, tid);
-          release(p, sh, n, lane);
+        if constexpr (Q4) {
+          for (int lr = tid; lr < nrows; lr += kConsumerThreads) __stcg(p.obuf + g0 + lr, oc[lr]);
+        } else {
+          const int rpc = kSlotBytes / rb;
+          for (int r0 = 0; r0 < nrows; r0 += rpc) {
+            const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+            splitk_rows<MG>(ch, min(rpc, nrows - r0), rb, oc + r0, H, acc, tid);
+            release<NS>(p, sh, n, lane);
+          }
         }
       }
-      residual_add<MG>(p, H, 2 * l, nrows > 0, acc, tid);
+      if constexpr (Q4) {   // out-projection rows over the whole mixer output
+        if (!grid_barrier(p, sh, ++nbar, tid)) return;
+        q4_rows_to_residual<NS>(p, sh, ring, n, p.obuf, p.Hd * p.dv, p.rb_dn_out, 2 * l, xs, xsum, qpart, tid, warp,
+                                lane);
+      } else {
+        residual_add<MG>(p, H, 2 * l, nrows > 0, acc, tid);
+      }
     } else {
       // ---- phase 2 (attention): RoPE, KV append, split-K partial softmax over this CTA's positions ----
       if (rg.au_valid) {
@@ -963,7 +1196,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
         for (int sb = p0; sb < q1; sb += kAttnSub) {
           const int np = min(kAttnSub, q1 - sb);
           {   // scores q_t . K[pp] from the K rows in shared memory, one warp per row
-            const uint16_t* kch = reinterpret_cast<const uint16_t*>(acquire(p, sh, ring, n, tid, lane));
+            const uint16_t* kch = reinterpret_cast<const uint16_t*>(acquire<NS>(p, sh, ring, n, tid, lane));
             for (int pp = warp; pp < np; pp += kConsumerWarps) {
               const uint16_t* krow = kch + static_cast<size_t>(pp) * D + lane * dpl;
               float kf[8];
@@ -1002,13 +1235,13 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
                   if (t < grp) sc[t * kAttnSub + pp] = dd[t];
               }
             }
-            release(p, sh, n, lane);
+            release<NS>(p, sh, n, lane);
           }
           cons_sync(kConsumerThreads);
           softmax_block(sc, mlc, grp, np, warp, lane);
           cons_sync(kConsumerThreads);
           {   // values: thread d accumulates sum_pp p[pp] V[pp][d]
-            const uint16_t* vch = reinterpret_cast<const uint16_t*>(acquire(p, sh, ring, n, tid, lane));
+            const uint16_t* vch = reinterpret_cast<const uint16_t*>(acquire<NS>(p, sh, ring, n, tid, lane));
             if (tid < D) {
               float vsum[8];
 #pragma unroll
@@ -1039,7 +1272,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
               for (int t = 0; t < 8; ++t)
                 if (t < grp) oacc[t] = oacc[t] * mlc[3 * t + 2] + vsum[t];
             }
-            release(p, sh, n, lane);
+            release<NS>(p, sh, n, lane);
           }
           cons_sync(kConsumerThreads);
         }
@@ -1125,14 +1358,24 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
           if (lane == 0) oc[cc] = o * gte[cc];
         }
         cons_sync(kConsumerThreads);
-        const int rpc = kSlotBytes / rb;
-        for (int r0 = 0; r0 < ncol; r0 += rpc) {
-          const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
-          splitk_rows<MG>(ch, min(rpc, ncol - r0), rb, oc + r0, H, acc, tid);
-          release(p, sh, n, lane);
+        if constexpr (Q4) {
+          for (int cc = tid; cc < ncol; cc += kConsumerThreads) __stcg(p.obuf + c0 + cc, oc[cc]);
+        } else {
+          const int rpc = kSlotBytes / rb;
+          for (int r0 = 0; r0 < ncol; r0 += rpc) {
+            const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+            splitk_rows<MG>(ch, min(rpc, ncol - r0), rb, oc + r0, H, acc, tid);
+            release<NS>(p, sh, n, lane);
+          }
         }
       }
-      residual_add<MG>(p, H, 2 * l, ncol > 0, acc, tid);
+      if constexpr (Q4) {
+        if (!grid_barrier(p, sh, ++nbar, tid)) return;
+        q4_rows_to_residual<NS>(p, sh, ring, n, p.obuf, p.Hq * p.D, p.rb_at_out, 2 * l, xs, xsum, qpart, tid, warp,
+                                lane);
+      } else {
+        residual_add<MG>(p, H, 2 * l, ncol > 0, acc, tid);
+      }
     }
 
     // ---- last phase: pre-MLP RMSNorm, SwiGLU gate/up, down-projection split-K ----
@@ -1143,30 +1386,52 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
       float4 acc[MG];
 #pragma unroll
       for (int k = 0; k < MG; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (Q4) {
+        q4_xsum(xs, xsum, H, tid);
+        cons_sync(kConsumerThreads);
+      }
       if (nj > 0) {
         float* gs = fs;
         float* us = fs + nj;
         const int rpc = kSlotBytes / rb;
-        XReg<XK> xr;
-        load_xreg<XK>(xr, xs, H, lane);
-        for (int half = 0; half < 2; ++half) {
-          float* out = half ? us : gs;
+        if constexpr (Q4) {
+          for (int half = 0; half < 2; ++half) {
+            float* out = half ? us : gs;
+            for (int r0 = 0; r0 < nj; r0 += rpc) {
+              const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+              gemv_rows_q4(ch, min(rpc, nj - r0), rb, H >> 8, xs, xsum, qpart, warp, lane, tid,
+                           [&](int r, float v) { out[r0 + r] = v; });
+              release<NS>(p, sh, n, lane);
+            }
+          }
+          for (int j = tid; j < nj; j += kConsumerThreads) __stcg(p.abuf + rg.f_b + j, siluf_(gs[j]) * us[j]);
+        } else {
+          XReg<XK> xr;
+          load_xreg<XK>(xr, xs, H, lane);
+          for (int half = 0; half < 2; ++half) {
+            float* out = half ? us : gs;
+            for (int r0 = 0; r0 < nj; r0 += rpc) {
+              const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+              gemv_rows<XK>(ch, min(rpc, nj - r0), rb, xr, xs, H, warp, lane, r0, kNoSplit, out, out);
+              release<NS>(p, sh, n, lane);
+            }
+          }
+          cons_sync(kConsumerThreads);
+          for (int j = tid; j < nj; j += kConsumerThreads) us[j] = siluf_(gs[j]) * us[j];
+          cons_sync(kConsumerThreads);
           for (int r0 = 0; r0 < nj; r0 += rpc) {
-            const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
-            gemv_rows<XK>(ch, min(rpc, nj - r0), rb, xr, xs, H, warp, lane, r0, kNoSplit, out, out);
-            release(p, sh, n, lane);
+            const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+            splitk_rows<MG>(ch, min(rpc, nj - r0), rb, us + r0, H, acc, tid);
+            release<NS>(p, sh, n, lane);
           }
         }
-        cons_sync(kConsumerThreads);
-        for (int j = tid; j < nj; j += kConsumerThreads) us[j] = siluf_(gs[j]) * us[j];
-        cons_sync(kConsumerThreads);
-        for (int r0 = 0; r0 < nj; r0 += rpc) {
-          const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
-          splitk_rows<MG>(ch, min(rpc, nj - r0), rb, us + r0, H, acc, tid);
-          release(p, sh, n, lane);
-        }
       }
-      residual_add<MG>(p, H, 2 * l + 1, nj > 0, acc, tid);
+      if constexpr (Q4) {   // down-projection rows over the whole activation
+        if (!grid_barrier(p, sh, ++nbar, tid)) return;
+        q4_rows_to_residual<NS>(p, sh, ring, n, p.abuf, p.F, p.rb_ffn, 2 * l + 1, xs, xsum, qpart, tid, warp, lane);
+      } else {
+        residual_add<MG>(p, H, 2 * l + 1, nj > 0, acc, tid);
+      }
     }
   }
 
@@ -1181,10 +1446,35 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     int bi = 0x7FFFFFFF;
     const int v0 = rg.v_b, nv = rg.v_e - rg.v_b;
     const int rpc = kSlotBytes / rb;
+    if constexpr (Q4) {
+      q4_xsum(xs, xsum, H, tid);
+      cons_sync(kConsumerThreads);
+      for (int r0 = 0; r0 < nv; r0 += rpc) {
+        const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
+        gemv_rows_q4(ch, min(rpc, nv - r0), rb, H >> 8, xs, xsum, qpart, warp, lane, tid, [&](int r, float v) {
+          const int idx = v0 + r0 + r;
+          if (p.logits) __stcg(p.logits + idx, v);
+          if (v > bv || (v == bv && idx < bi)) {
+            bv = v;
+            bi = idx;
+          }
+        });
+        release<NS>(p, sh, n, lane);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {   // warp's best (lowest index among equal values)
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+    }
     XReg<XK> xr;
-    load_xreg<XK>(xr, xs, H, lane);
-    for (int r0 = 0; r0 < nv; r0 += rpc) {
-      const uint8_t* ch = acquire(p, sh, ring, n, tid, lane);
+    if constexpr (!Q4) load_xreg<XK>(xr, xs, H, lane);
+    for (int r0 = 0; r0 < (Q4 ? 0 : nv); r0 += rpc) {
+      const uint8_t* ch = acquire<NS>(p, sh, ring, n, tid, lane);
       const int nr = min(rpc, nv - r0);
       for (int r = warp; r < nr; r += 4 * kConsumerWarps) {
         int rr[4];
@@ -1207,7 +1497,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
           }
         }
       }
-      release(p, sh, n, lane);
+      release<NS>(p, sh, n, lane);
     }
     if (lane == 0) {
       sh->best_v[warp] = bv;
@@ -1244,17 +1534,24 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
 
 constexpr size_t kSmemLimit = 232448;
 
-size_t decode_scratch_floats(int H) {
-  const size_t fixed = static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + static_cast<size_t>(H) * 4;
+// Shared memory before the scratch: the ring, Shared, the staged input vector and, with
+// Q4 weights (2 ring slots), its per-lane sums and the row partial sums.
+static size_t decode_fixed_bytes(int H, bool q4, int xcap) {
+  if (!q4) return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + static_cast<size_t>(H) * 4;
+  return 2 * static_cast<size_t>(kSlotBytes) + sizeof(Shared) + static_cast<size_t>(xcap) * 4 +
+         static_cast<size_t>(xcap / 8) * 4 + static_cast<size_t>(kQ4PartFloats) * 4;
+}
+
+size_t decode_scratch_floats(int H, bool q4, int xcap) {
+  const size_t fixed = decode_fixed_bytes(H, q4, xcap);
   if (fixed >= kSmemLimit) return 0;
   size_t f = (kSmemLimit - fixed) / 4;
   f &= ~static_cast<size_t>(3);
   return f > 8192 ? 8192 : f;
 }
 
-size_t decode_smem_bytes(int H) {
-  return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + static_cast<size_t>(H) * 4 +
-         decode_scratch_floats(H) * 4;
+size_t decode_smem_bytes(int H, bool q4, int xcap) {
+  return decode_fixed_bytes(H, q4, xcap) + decode_scratch_floats(H, q4, xcap) * 4;
 }
 
 int decode_max_splits(int grid, int hkv) {
@@ -1262,11 +1559,11 @@ int decode_max_splits(int grid, int hkv) {
   return per < 1 ? 1 : per;
 }
 
-template <int HK>
+template <int HK, bool Q4>
 cudaError_t launch_hk(const DecodeParams& p, int grid, cudaStream_t s) {
-  static bool attr_set = false;
+  static bool attr_set = false;   // per process; the attribute is the same on every device
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(mk_decode_kernel<HK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(mk_decode_kernel<HK, Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kSmemLimit));
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -1274,21 +1571,22 @@ cudaError_t launch_hk(const DecodeParams& p, int grid, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = decode_smem_bytes(p.H);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, Q4, p.xcap);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mk_decode_kernel<HK>, p);
+  return cudaLaunchKernelEx(&cfg, mk_decode_kernel<HK, Q4>, p);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s) {
-  if (p.H == 1024) return launch_hk<4>(p, grid, s);
-  if (p.H == 256) return launch_hk<1>(p, grid, s);
-  if (p.H == 2048) return launch_hk<8>(p, grid, s);
-  return launch_hk<0>(p, grid, s);
+  if (p.q4) return launch_hk<0, true>(p, grid, s);
+  if (p.H == 1024) return launch_hk<4, false>(p, grid, s);
+  if (p.H == 256) return launch_hk<1, false>(p, grid, s);
+  if (p.H == 2048) return launch_hk<8, false>(p, grid, s);
+  return launch_hk<0, false>(p, grid, s);
 }
 
 }  // namespace mk

@@ -32,6 +32,11 @@ struct LayerW {
   const uint8_t* w_gate;    // [F][row_bytes]
   const uint8_t* w_up;      // [F][row_bytes]
   const uint8_t* w_downT;   // [F][row_bytes]           transposed: row j = column j of W_down
+  // Q4_K-style weights (row-major, 144-byte super-blocks along the input dim): the
+  // out-projection [H][K_mix] and the down-projection [H][F]; the fields above then hold
+  // Q4 rows of the in-projection, gate and up.
+  const uint8_t* w_out_q4;
+  const uint8_t* w_down_q4;
 };
 
 struct DecodeParams {
@@ -74,10 +79,19 @@ struct DecodeParams {
   int trace_cap;
   // how far (bytes per CTA) the L2 prefetch cursor runs ahead of the shared-memory fill
   int prefetch_bytes;
+  // Q4_K-style weights: row_bytes is then (H / 256) * 144, and the out- and down-projections
+  // are split over output rows (their inputs staged from obuf / abuf)
+  int q4;
+  int rb_dn_out, rb_at_out, rb_ffn;   // Q4 row bytes of W_out (DeltaNet, attention) and W_down
+  int xcap;                           // floats of the staged input vector in shared memory
+  float* obuf;                        // [max(Hd dv, Hq D)] mixer output (Q4)
+  float* abuf;                        // [F] SwiGLU activation (Q4)
 };
 
-size_t decode_smem_bytes(int H);
-size_t decode_scratch_floats(int H);   // fp32 scratch per CTA left after the ring and xs
+size_t decode_smem_bytes(int H, bool q4 = false, int xcap = 0);
+size_t decode_scratch_floats(int H, bool q4 = false, int xcap = 0);   // fp32 scratch per CTA left after the ring, xs (and the Q4 tables)
+constexpr int kQ4Block = 144;          // bytes per 256-weight super-block
+constexpr int kQ4PartFloats = 512;     // shared-memory partial sums of the Q4 row products
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s);
 int decode_max_splits(int grid, int hkv);
 

@@ -91,6 +91,8 @@ class Model:
             arr[i].ndim = t.dim()
             for d in range(min(4, t.dim())):
                 arr[i].shape[d] = t.shape[d]
+            if arr[i].dtype == _abi.MK_DT_Q4K and t.dim() == 2:
+                arr[i].shape[1] = t.shape[1] // 144 * 256     # logical columns of the 144-byte super-blocks
             arr[i].data = t.data_ptr()
             arr[i].bytes = t.numel() * t.element_size()
         handle = C.c_void_p()

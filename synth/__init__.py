@@ -114,7 +114,18 @@ MINI = _preset("mini", n_layers=4, pattern="DDDA", hidden=32, vocab=64, rms_eps=
                at_q_heads=2, at_kv_heads=1, at_head_dim=8, rope_theta=1e7, at_out_gate=1,
                ffn=48, seed=7)
 
-CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI)}
+# 4-bit test shapes: the tiny model in the 4-bit format, and a mid-size model with the
+# 27B model's head shapes (dk = dv = 128, gated attention) that the oracle runs in seconds.
+TINY_Q4 = _preset("tiny-q4", n_layers=4, pattern="DDDA", hidden=256, vocab=4096, rms_eps=1e-6,
+                  dn_heads=4, dn_dk=64, dn_dv=64, conv_width=4,
+                  at_q_heads=4, at_kv_heads=1, at_head_dim=64, rope_theta=1e7, at_out_gate=0,
+                  ffn=768, weight_format=W_Q4K, seed=10)
+MID_Q4 = _preset("mid-q4", n_layers=8, pattern="DDDA" * 2, hidden=1024, vocab=32768, rms_eps=1e-6,
+                 dn_heads=8, dn_dk=128, dn_dv=128, conv_width=4,
+                 at_q_heads=8, at_kv_heads=2, at_head_dim=128, rope_theta=1e7, at_out_gate=1,
+                 ffn=3072, weight_format=W_Q4K, seed=11)
+
+CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI, TINY_Q4, MID_Q4)}
 
 
 def with_changes(cfg: ModelConfig, **kw) -> ModelConfig:
