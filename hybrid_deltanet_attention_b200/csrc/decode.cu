@@ -782,28 +782,54 @@ __device__ __forceinline__ void softmax_block(float* sc, float* mlc, int grp, in
 // 32 j + 16 + 4 (l % 4) + t (high nibbles), t = 0..3, whose x values are xl and xh and
 // whose x sum is xsv. With w = (d sc_j) q - (dmin m_j) the lane's share of the product is
 // (d sc_j) sum(q x) - (dmin m_j) sum(x); d sc_j and dmin m_j are exact in fp32.
-__device__ __forceinline__ float q4_part(const uint8_t* blk, int j, int part, const float4& xl, const float4& xh,
+// Lane constants of q4_part: which 32-bit words of the 6-bit field stream hold the
+// lane's sc_j and m_j, and the shift inside the word pair.
+struct Q4Lane {
+  int j, part;
+  int sc_w, sc_sh;   // sc_j at stream bit 6j
+  int m_w, m_sh;     // m_j at stream bit 48 + 6j
+};
+__device__ __forceinline__ Q4Lane q4_lane(int lane) {
+  Q4Lane q;
+  q.j = lane >> 2;
+  q.part = lane & 3;
+  const int bs = 6 * q.j, bm = 48 + 6 * q.j;
+  q.sc_w = bs >> 5;
+  q.sc_sh = bs & 31;
+  q.m_w = bm >> 5;
+  q.m_sh = bm & 31;
+  return q;
+}
+
+// 1 + q/16 for the 4-bit field of c whose lowest bit is `bit` (exact in fp32).
+template <int BIT>
+__device__ __forceinline__ float q4_unit(uint32_t c) {
+  const uint32_t v = BIT <= 19 ? (c << (19 - BIT)) : (c >> (BIT - 19));
+  return __uint_as_float((v & 0x00780000u) | 0x3F800000u);
+}
+
+__device__ __forceinline__ float q4_part(const uint8_t* blk, const Q4Lane& ql, const float4& xl, const float4& xh,
                                          float xsv) {
   const uint32_t dd = *reinterpret_cast<const uint32_t*>(blk);
   const uint32_t f0 = *reinterpret_cast<const uint32_t*>(blk + 4);
   const uint32_t f1 = *reinterpret_cast<const uint32_t*>(blk + 8);
   const uint32_t f2 = *reinterpret_cast<const uint32_t*>(blk + 12);
-  const uint32_t c = *reinterpret_cast<const uint32_t*>(blk + 16 + 16 * j + 4 * part);
-  const uint64_t lo = static_cast<uint64_t>(f0) | (static_cast<uint64_t>(f1) << 32);
-  const uint64_t hi = static_cast<uint64_t>(f1) | (static_cast<uint64_t>(f2) << 32);
-  const float sc = static_cast<float>(static_cast<uint32_t>(lo >> (6 * j)) & 63u);
-  const float mm = static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * j)) & 63u);
-  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) * sc;
-  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) * mm;
-  float qx = static_cast<float>(c & 15u) * xl.x;
-  qx = fmaf(static_cast<float>((c >> 8) & 15u), xl.y, qx);
-  qx = fmaf(static_cast<float>((c >> 16) & 15u), xl.z, qx);
-  qx = fmaf(static_cast<float>((c >> 24) & 15u), xl.w, qx);
-  qx = fmaf(static_cast<float>((c >> 4) & 15u), xh.x, qx);
-  qx = fmaf(static_cast<float>((c >> 12) & 15u), xh.y, qx);
-  qx = fmaf(static_cast<float>((c >> 20) & 15u), xh.z, qx);
-  qx = fmaf(static_cast<float>((c >> 28) & 15u), xh.w, qx);
-  return fmaf(s, qx, -mn * xsv);
+  const uint32_t c = *reinterpret_cast<const uint32_t*>(blk + 16 + 16 * ql.j + 4 * ql.part);
+  const uint32_t sc = __funnelshift_r(ql.sc_w ? f1 : f0, ql.sc_w ? f2 : f1, ql.sc_sh) & 63u;
+  const uint32_t mm = __funnelshift_r(ql.m_w == 1 ? f1 : f2, ql.m_w == 1 ? f2 : 0u, ql.m_sh) & 63u;
+  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) * static_cast<float>(sc);
+  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) * static_cast<float>(mm);
+  // sum (1 + q/16) x over the lane's 8 weights; sum q x = 16 (that - sum x)
+  float u = q4_unit<0>(c) * xl.x;
+  u = fmaf(q4_unit<8>(c), xl.y, u);
+  u = fmaf(q4_unit<16>(c), xl.z, u);
+  u = fmaf(q4_unit<24>(c), xl.w, u);
+  u = fmaf(q4_unit<4>(c), xh.x, u);
+  u = fmaf(q4_unit<12>(c), xh.y, u);
+  u = fmaf(q4_unit<20>(c), xh.z, u);
+  u = fmaf(q4_unit<28>(c), xh.w, u);
+  const float s16 = 16.0f * s;
+  return fmaf(s16, u, -(s16 + mn) * xsv);
 }
 
 // xsum[sb * 32 + l] = the sum of the 8 x values lane l pairs with in super-block sb.
@@ -828,7 +854,8 @@ __device__ __forceinline__ void gemv_rows_q4(const uint8_t* chunk, int nrows, in
   const int WK = nsb >= 8 ? 8 : (nsb >= 4 ? 4 : (nsb >= 2 ? 2 : 1));
   const int RS = kConsumerWarps / WK;
   const int ks = warp % WK, rs = warp / WK;
-  const int j = lane >> 2, part = lane & 3;
+  const Q4Lane ql = q4_lane(lane);
+  const int j = ql.j, part = ql.part;
   for (int r0 = rs; r0 < nrows; r0 += 4 * RS) {
     const uint8_t* rp[4];
     bool live[4];
@@ -845,7 +872,7 @@ __device__ __forceinline__ void gemv_rows_q4(const uint8_t* chunk, int nrows, in
       const float4 xh = *reinterpret_cast<const float4*>(xb + 16);
       const float xsv = xsum[sb * 32 + lane];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[q] += q4_part(rp[q] + static_cast<size_t>(sb) * kQ4Block, j, part, xl, xh, xsv);
+      for (int q = 0; q < 4; ++q) acc[q] += q4_part(rp[q] + static_cast<size_t>(sb) * kQ4Block, ql, xl, xh, xsv);
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
