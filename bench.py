@@ -503,30 +503,6 @@ def run_prefill(args):
     return 0
 
 
-def device_q4_weights(cfg, dev, seed):
-    """Weights of the 4-bit model for timing: every Q4 super-block generated on the device
-    (uniform codes and 6-bit fields, fp16 d and dmin in [2^-15, 2^-14)), gains and conv taps
-    from the seeded stream. Parity at these head shapes is tested on the mid-size 4-bit model;
-    this only sizes the work (14.4 GB of 4-bit weights)."""
-    import torch
-    import synth
-    g = torch.Generator(device=dev)
-    g.manual_seed(seed)
-    out = {}
-    for name, shape, init in synth.tensor_specs(cfg):
-        if synth.is_quantized(cfg, name, shape):
-            rows, cols = shape
-            nb = cols // 256
-            t = torch.randint(0, 256, (rows, nb, 144), dtype=torch.uint8, device=dev, generator=g)
-            dd = ((torch.rand((rows, nb, 2), device=dev, generator=g) + 1.0) * 2.0 ** -15).to(torch.float16)
-            t[:, :, 0:4] = dd.view(torch.uint8).reshape(rows, nb, 4)
-            out[name] = t.reshape(rows, nb * 144)
-        else:
-            x = synth._draw_f32(cfg, seed, name, shape, init)
-            out[name] = torch.from_numpy(synth.f32_to_bf16_bits(x).view(np.int16)).to(dev).view(torch.bfloat16)
-    return out
-
-
 def run_27b(args):
     """27B-shaped 4-bit model: plain greedy decode after a 1024-token context, and
     speculative verify passes of K = 5 drafts (80 % equal to the model's greedy token)."""
@@ -539,7 +515,7 @@ def run_27b(args):
     dev = torch.device("cuda", local)
     CTX, K, TGP = 1024, 5, 32
     n_pass = max(4, args.steps)
-    m = hda.Model(cfg, device_q4_weights(cfg, dev, cfg.seed), max_ctx=CTX + TGP + (K + 1) * (n_pass + args.warmup + 2) + 16,
+    m = hda.Model(cfg, synth.device_q4_weights(cfg, dev, cfg.seed), max_ctx=CTX + TGP + (K + 1) * (n_pass + args.warmup + 2) + 16,
                   max_draft=K)
     torch.cuda.empty_cache()
     ctx = torch.from_numpy(synth.make_prompt(cfg, CTX, tag="ctx1024")).to(dev)

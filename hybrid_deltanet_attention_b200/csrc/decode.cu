@@ -107,12 +107,12 @@ __device__ void compute_ranges(const DecodeParams& p, int cta, int G, int pos, R
 // below kTraceChunks: phase boundaries; from kTraceChunks: chunk n issued (4n), warp 0
 // starts waiting for it (4n+1), has it (4n+2), is done with it (4n+3).
 constexpr int kTraceChunks = 512;
-__device__ __forceinline__ void trace_at(const DecodeParams& p, int idx) {
-  if (p.trace && blockIdx.x == 0 && idx < p.trace_cap) p.trace[idx] = clock64();
-}
 // From kTraceGrid: every CTA stamps %globaltimer (ns) when it arrives at grid barrier k
 // (entry kTraceGrid + 2 (k G + cta)) and when it leaves it (the next entry).
-constexpr int kTraceGrid = 8192;
+constexpr int kTraceGrid = 16384;
+__device__ __forceinline__ void trace_at(const DecodeParams& p, int idx) {
+  if (p.trace && blockIdx.x == 0 && idx < p.trace_cap && idx < kTraceGrid) p.trace[idx] = clock64();
+}
 __device__ __forceinline__ void trace_grid(const DecodeParams& p, unsigned k, int leave) {
   if (!p.trace) return;
   const long long ix = kTraceGrid + 2ll * (static_cast<long long>(k) * gridDim.x + blockIdx.x) + leave;

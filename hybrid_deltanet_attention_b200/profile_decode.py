@@ -26,6 +26,8 @@ def main():
     ap.add_argument("--steps", type=int, default=4)
     ap.add_argument("--trace", action="store_true")
     ap.add_argument("--mhz", type=float, default=1965.0, help="SM clock used to convert trace cycles to us")
+    ap.add_argument("--device-weights", action="store_true",
+                    help="4-bit models: generate the blocks on the device (timing only, see synth.device_q4_weights)")
     args = ap.parse_args()
 
     import numpy as np
@@ -35,12 +37,16 @@ def main():
 
     cfg = synth.CONFIGS[args.model]
     dev = torch.device("cuda", 0)
-    m = hda.Model(cfg, hda.weights_to_device(synth.make_weights(cfg), dev), max_ctx=args.prompt + args.steps + 8)
+    weights = (synth.device_q4_weights(cfg, dev, cfg.seed) if args.device_weights
+               else hda.weights_to_device(synth.make_weights(cfg), dev))
+    m = hda.Model(cfg, weights, max_ctx=args.prompt + args.steps + 8)
+    del weights
     tok = torch.empty(args.steps + 1, dtype=torch.int32, device=dev)
     m.prefill(torch.from_numpy(synth.make_prompt(cfg, args.prompt)).to(dev), next_token=tok[0:1])
-    nbar = sum(3 if k == "D" else 4 for k in cfg.pattern)
+    q4 = cfg.weight_format == synth.W_Q4K
+    nbar = sum((5 if q4 else 3) if k == "D" else (6 if q4 else 4) for k in cfg.pattern)
     G = int(m.sizes.grid_ctas)
-    buf = torch.zeros(8192 + 2 * (nbar + 1) * G, dtype=torch.int64, device=dev) if args.trace else None
+    buf = torch.zeros(16384 + 2 * (nbar + 1) * G, dtype=torch.int64, device=dev) if args.trace else None
     for i in range(args.steps):
         if buf is not None and i == args.steps - 1:
             m.phase_trace(buf)
@@ -51,7 +57,7 @@ def main():
         raise SystemExit(f"device error word 0x{err:x}")
     if buf is not None:
         raw = buf.cpu().numpy()
-        t = raw[:8192].astype("float64") * (1000.0 / args.mhz)      # cycles -> ns
+        t = raw[:16384].astype("float64") * (1000.0 / args.mhz)      # cycles -> ns
         exits = [t[0]] + [t[2 * k] for k in range(1, nbar + 1)]
         arrivals = [t[2 * k - 1] for k in range(1, nbar + 1)]
         end = t[2 * nbar + 1]
@@ -59,8 +65,12 @@ def main():
         waits = [(exits[k] - arrivals[k - 1]) / 1e3 for k in range(1, nbar + 1)]
         names = []
         for li, kind in enumerate(cfg.pattern):
-            names += [f"L{li}.in", f"L{li}.dn+out", f"L{li}.mlp"] if kind == "D" else \
-                     [f"L{li}.in", f"L{li}.attn", f"L{li}.attn_out", f"L{li}.mlp"]
+            if q4:
+                names += [f"L{li}.in", f"L{li}.dn", f"L{li}.out", f"L{li}.gateup", f"L{li}.down"] if kind == "D" else \
+                         [f"L{li}.in", f"L{li}.attn", f"L{li}.attn_out", f"L{li}.out", f"L{li}.gateup", f"L{li}.down"]
+            else:
+                names += [f"L{li}.in", f"L{li}.dn+out", f"L{li}.mlp"] if kind == "D" else \
+                         [f"L{li}.in", f"L{li}.attn", f"L{li}.attn_out", f"L{li}.mlp"]
         names.append("lm_head")
         rows = [{"phase": n, "us": round(p, 2), "barrier_wait_us": round(w, 2) if i < len(waits) else None}
                 for i, (n, p, w) in enumerate(zip(names, phases, waits + [0.0]))]
@@ -74,7 +84,7 @@ def main():
         # all CTAs (global timer, ns): per phase kind, the work (median arrival - median
         # exit of the previous barrier), the skew (last arrival - median arrival) and the
         # propagation (median exit - last arrival)
-        grid = raw[8192:8192 + 2 * (nbar + 1) * G].astype("float64").reshape(nbar + 1, G, 2)
+        grid = raw[16384:16384 + 2 * (nbar + 1) * G].astype("float64").reshape(nbar + 1, G, 2)
         kinds = {}
         for k in range(1, nbar + 1):
             a, e = grid[k, :, 0], grid[k, :, 1]

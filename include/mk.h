@@ -226,9 +226,9 @@ int mk_sync_status(mk_model* m, void* stream, int32_t* dev_err);
  * exit from grid barrier k (entries 2k-1, 2k) and when its LM-head slice is done
  * (entry 2*n_barriers+1); from entry 512 on, chunk n of its weight stream was issued
  * (512+4n), consumer warp 0 started waiting for it (513+4n), had it (514+4n) and was
- * done with it (515+4n); from entry 8192 on, every CTA c records the global timer (ns)
- * when it arrives at grid barrier k (8192 + 2(k*grid + c)) and when it leaves it (the
- * entry after). Entries at or past `capacity` are not written. Pass NULL to stop. The
+ * done with it (515+4n; chunks past entry 16383 are not recorded); from entry 16384 on,
+ * every CTA c records the global timer (ns) when it arrives at grid barrier k
+ * (16384 + 2(k*grid + c)) and when it leaves it (the entry after). Entries at or past `capacity` are not written. Pass NULL to stop. The
  * buffer stays the caller's. */
 int mk_phase_trace(mk_model* m, uint64_t* d_trace, int32_t capacity);
 

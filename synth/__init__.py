@@ -344,3 +344,27 @@ def long_context_state(cfg: ModelConfig, n_pos: int, seed: int = 3):
         s = stream(seed, f"state.S.{i}").standard_normal((cfg.dn_heads, cfg.dn_dv, cfg.dn_dk), dtype=np.float32)
         ss.append((s * np.float32(0.1)).astype(np.float32))
     return ks, vs, ss
+
+
+# ---------------------------------------------------------------- device-side 4-bit blocks
+def device_q4_weights(cfg: ModelConfig, dev, seed: int):
+    """Weights of the 4-bit model for timing: every Q4 super-block generated on the device
+    (uniform codes and 6-bit fields, fp16 d and dmin in [2^-15, 2^-14)), gains and conv taps
+    from the seeded stream. Parity at these head shapes is tested on the mid-size 4-bit model;
+    this only sizes the work (14.4 GB of 4-bit weights)."""
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    out = {}
+    for name, shape, init in tensor_specs(cfg):
+        if is_quantized(cfg, name, shape):
+            rows, cols = shape
+            nb = cols // 256
+            t = torch.randint(0, 256, (rows, nb, 144), dtype=torch.uint8, device=dev, generator=g)
+            dd = ((torch.rand((rows, nb, 2), device=dev, generator=g) + 1.0) * 2.0 ** -15).to(torch.float16)
+            t[:, :, 0:4] = dd.view(torch.uint8).reshape(rows, nb, 4)
+            out[name] = t.reshape(rows, nb * 144)
+        else:
+            x = _draw_f32(cfg, seed, name, shape, init)
+            out[name] = torch.from_numpy(f32_to_bf16_bits(x).view(np.int16)).to(dev).view(torch.bfloat16)
+    return out
