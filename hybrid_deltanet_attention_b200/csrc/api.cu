@@ -237,7 +237,7 @@ struct Layout {
   int max_splits;
   // batched prefill workspace
   int pf_rows;
-  size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec;
+  size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec, pf_apart, pf_splitk, pf_best;
   // batched verify saves
   int vf_rows;
   size_t vf_delta, vf_k, vf_g, vf_raw, vf_logits, vf_greedy;
@@ -361,6 +361,11 @@ Layout make_layout(const mk_config& c, int grid) {
     L.pf_p = off; off = align256(off + nch * c.dn_heads * 64 * 64 * 4);
     L.pf_gam = off; off = align256(off + T * c.dn_heads * 4);
     L.pf_dec = off; off = align256(off + T * c.dn_heads * 4);
+    L.pf_apart = off;
+    off = align256(off + std::min<size_t>(T, mk::kAttnSplitRows) * c.at_q_heads * mk::kAttnMaxSplit *
+                             (static_cast<size_t>(c.at_head_dim) + 2) * 4);
+    L.pf_splitk = off; off = align256(off + static_cast<size_t>(mk::kSplitKFloats) * 4);
+    L.pf_best = off; off = align256(off + T * 8);
   }
   L.vf_rows = (L.pf_rows > 0 && c.max_draft > 0 && c.max_draft + 1 <= std::min(64, L.pf_rows)) ? c.max_draft + 1 : 0;
   if (L.vf_rows > 0) {
@@ -703,6 +708,9 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     m->pf.p = reinterpret_cast<float*>(W + L.pf_p);
     m->pf.gam = reinterpret_cast<float*>(W + L.pf_gam);
     m->pf.dec = reinterpret_cast<float*>(W + L.pf_dec);
+    m->pf.apart = reinterpret_cast<float*>(W + L.pf_apart);
+    m->pf.splitk = reinterpret_cast<float*>(W + L.pf_splitk);
+    m->pf.best = reinterpret_cast<unsigned long long*>(W + L.pf_best);
   }
   m->vf.rows = L.vf_rows;
   if (L.vf_rows > 0) {

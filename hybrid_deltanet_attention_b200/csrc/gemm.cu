@@ -20,6 +20,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 
@@ -59,14 +60,23 @@ template <int BN>
 __global__ void __launch_bounds__(192, 1)
     linear_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                   const __grid_constant__ CUtensorMap tb, float* __restrict__ C, long long ldc, int M, int N, int K,
-                  int accumulate, int* err) {
+                  int accumulate, int* err, float* __restrict__ ws) {
   using S = GemmShape<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmBars* gb = reinterpret_cast<GemmBars*>(smem + S::kRingBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
-  const int nk = K / kBK;
+  // split-K: CTA z takes K blocks [kb0, kb1) and writes its partial tile to ws[z] ([M][N])
+  const int nkall = K / kBK, nz = gridDim.z, z = blockIdx.z;
+  const int kb0 = static_cast<int>((static_cast<long long>(nkall) * z) / nz);
+  const int kb1 = static_cast<int>((static_cast<long long>(nkall) * (z + 1)) / nz);
+  const int nk = kb1 - kb0;
+  if (nz > 1) {
+    C = ws + static_cast<long long>(z) * M * N;
+    ldc = N;
+    accumulate = 0;
+  }
   auto a_hi = [&](int s) { return smem + s * S::kStageBytes; };
   auto a_lo = [&](int s) { return smem + s * S::kStageBytes + S::kABytes; };
   auto b_t = [&](int s) { return smem + s * S::kStageBytes + 2 * S::kABytes; };
@@ -104,9 +114,9 @@ __global__ void __launch_bounds__(192, 1)
           break;
         }
         mbar_arrive_expect_tx(&gb->full[s], S::kStageBytes);
-        tc::tma_load_2d(a_hi(s), &ta_hi, kb * kBK, m0, &gb->full[s]);
-        tc::tma_load_2d(a_lo(s), &ta_lo, kb * kBK, m0, &gb->full[s]);
-        tc::tma_load_2d(b_t(s), &tb, kb * kBK, n0, &gb->full[s]);
+        tc::tma_load_2d(a_hi(s), &ta_hi, (kb0 + kb) * kBK, m0, &gb->full[s]);
+        tc::tma_load_2d(a_lo(s), &ta_lo, (kb0 + kb) * kBK, m0, &gb->full[s]);
+        tc::tma_load_2d(b_t(s), &tb, (kb0 + kb) * kBK, n0, &gb->full[s]);
         ++issued;
       }
       int never = 0;   // let the copies this lane issued land before the CTA ends (bounded)
@@ -177,6 +187,19 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// C[m][n] (+)= sum_z ws[z][m][n], z in order (deterministic).
+__global__ void splitk_reduce(const float* __restrict__ ws, int nz, int M, int N, float* __restrict__ C, long long ldc,
+                              int accumulate) {
+  const long long total = static_cast<long long>(M) * N;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long m = i / N, n = i % N;
+    float v = accumulate ? C[m * ldc + n] : 0.f;
+    for (int z = 0; z < nz; ++z) v += ws[z * total + i];
+    C[m * ldc + n] = v;
+  }
+}
+
 __global__ void split_bf16_kernel(const float* __restrict__ x, long long ldx, uint16_t* __restrict__ hi,
                                   uint16_t* __restrict__ lo, int M, int K) {
   const long long total = static_cast<long long>(M) * K;
@@ -219,21 +242,72 @@ bool make_map(CUtensorMap* map, const void* base, long long rows, long long cols
   return r == CUDA_SUCCESS;
 }
 
+// Tensor maps are plain host structs that depend only on (base, rows, cols, stride, box);
+// the prefill and verify passes reuse the same few hundred, so they are encoded once.
+struct MapKey {
+  const void* base;
+  long long rows, cols, stride;
+  int box;
+  bool operator<(const MapKey& o) const {
+    if (base != o.base) return base < o.base;
+    if (rows != o.rows) return rows < o.rows;
+    if (cols != o.cols) return cols < o.cols;
+    if (stride != o.stride) return stride < o.stride;
+    return box < o.box;
+  }
+};
+
+bool cached_map(CUtensorMap* map, const void* base, long long rows, long long cols, long long stride_bytes, int box) {
+  static std::mutex mu;
+  static std::map<MapKey, CUtensorMap> cache;
+  const MapKey k{base, rows, cols, stride_bytes, box};
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(k);
+  if (it != cache.end()) {
+    *map = it->second;
+    return true;
+  }
+  if (!make_map(map, base, rows, cols, stride_bytes, box)) return false;
+  if (cache.size() > 65536) cache.clear();   // bound the cache (device buffers come and go)
+  cache.emplace(k, *map);
+  return true;
+}
+
 template <int BN>
 cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
   using S = GemmShape<BN>;
   CUtensorMap ma_hi, ma_lo, mb;
-  if (!make_map(&ma_hi, a.x_hi, a.M, a.K, static_cast<long long>(a.K) * 2, kBM) ||
-      !make_map(&ma_lo, a.x_lo, a.M, a.K, static_cast<long long>(a.K) * 2, kBM) ||
-      !make_map(&mb, a.w, a.N, a.K, a.ldw_bytes, BN))
+  if (!cached_map(&ma_hi, a.x_hi, a.M, a.K, static_cast<long long>(a.K) * 2, kBM) ||
+      !cached_map(&ma_lo, a.x_lo, a.M, a.K, static_cast<long long>(a.K) * 2, kBM) ||
+      !cached_map(&mb, a.w, a.N, a.K, a.ldw_bytes, BN))
     return cudaErrorInvalidValue;
-  const cudaError_t attr =
-      cudaFuncSetAttribute(linear_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
-  if (attr != cudaSuccess) return attr;
+  static bool attr_set = false;   // per process; the attribute is the same on every device
+  if (!attr_set) {
+    const cudaError_t attr =
+        cudaFuncSetAttribute(linear_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    attr_set = true;
+  }
   dim3 grid((a.N + BN - 1) / BN, (a.M + kBM - 1) / kBM);
+  // split K when the tile grid leaves most SMs idle (few tokens) and the workspace holds it
+  const int tiles = static_cast<int>(grid.x * grid.y), nk = a.K / kBK;
+  int nz = 1;
+  if (a.ws && grid.y == 1 && tiles < 148 && nk >= 6) {   // few tokens (one M tile) and few N tiles
+    nz = std::min({(148 + tiles - 1) / tiles, nk / 3, 16});   // about one wave, >= 3 K blocks per CTA
+    const long long need = static_cast<long long>(a.M) * a.N;
+    while (nz > 1 && need * nz > a.ws_floats) --nz;
+  }
+  grid.z = nz;
   linear_kernel<BN><<<grid, 192, S::kSmemBytes, s>>>(ma_hi, ma_lo, mb, a.c, a.ldc, a.M, a.N, a.K, a.accumulate,
-                                                     a.err);
-  return cudaGetLastError();
+                                                     a.err, a.ws);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && nz > 1) {
+    const long long total = static_cast<long long>(a.M) * a.N;
+    const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 8));
+    splitk_reduce<<<blocks, 256, 0, s>>>(a.ws, nz, a.M, a.N, a.c, a.ldc, a.accumulate);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace
@@ -253,7 +327,8 @@ cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s) {
       (reinterpret_cast<uintptr_t>(a.x_hi) & 15) || (reinterpret_cast<uintptr_t>(a.x_lo) & 15) ||
       (reinterpret_cast<uintptr_t>(a.w) & 15))
     return cudaErrorInvalidValue;
-  return a.N >= 2048 ? launch_bn<256>(a, s) : launch_bn<128>(a, s);
+  // 256-wide tiles for many tokens and wide outputs; 128-wide for few tokens (more CTAs to split over)
+  return (a.N >= 2048 && a.M > kBM) ? launch_bn<256>(a, s) : launch_bn<128>(a, s);
 }
 
 }  // namespace mk

@@ -97,6 +97,10 @@ int decode_max_splits(int grid, int hkv);
 
 // prefill linear layers on the tensor cores (gemm.cu): C[m][n] (+)= sum_k X[m][k] W[n][k]
 // with X given as its bf16 high and low parts.
+constexpr int kAttnMaxSplit = 32;     // key splits per token of the prefill attention for few-token passes
+constexpr int kAttnSplitRows = 148;   // tokens up to which the split workspace is sized
+constexpr long long kSplitKFloats = 8ll << 20;   // split-K partial workspace of the linear layers (32 MB)
+
 struct LinearArgs {
   const uint16_t* x_hi;     // bf16 [M][K], row stride K
   const uint16_t* x_lo;
@@ -107,6 +111,8 @@ struct LinearArgs {
   int M, N, K;              // K a multiple of 64
   int accumulate;
   int* err;
+  float* ws = nullptr;      // optional split-K partials (when the tile grid is smaller than the GPU)
+  long long ws_floats = 0;
 };
 cudaError_t launch_split_bf16(const float* x, long long ldx, uint16_t* hi, uint16_t* lo, int M, int K, cudaStream_t s);
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s);

@@ -25,6 +25,9 @@ struct mk_prefill_ws {
   float* p = nullptr;        // [chunks][Hd][64][64] chunked delta rule: masked decayed Q K^T
   float* gam = nullptr;      // [rows][Hd]
   float* dec = nullptr;      // [rows][Hd]
+  float* apart = nullptr;    // [min(rows, kAttnSplitRows)][Hq][kAttnMaxSplit][D + 2] attention key-split partials
+  float* splitk = nullptr;   // [kSplitKFloats] split-K partials of the linear layers
+  unsigned long long* best = nullptr;   // [rows] packed (value, index) row maxima of the verify logits
 };
 
 struct mk_prefill_layer {   // K-major copies of the projections the decode kernel keeps transposed

@@ -116,6 +116,53 @@ __global__ void dn_prep(const float* __restrict__ z, int ldz, const int* __restr
   }
 }
 
+// The same on a (token, vector) grid: vector v < 2 Hd is one q or k head (conv + SiLU +
+// L2 norm over its dk <= 128 channels), then blocks of 128 v channels, then the gates.
+// Enough CTAs for a few-token pass (a verify pass has T = K + 1).
+__global__ void __launch_bounds__(128) dn_prep_wide(const float* __restrict__ z, int ldz, const int* __restrict__ posp,
+                                                    int off, const float* __restrict__ ring, int W, int C, int Hd, int dk,
+                                                    int dv, const uint16_t* __restrict__ taps, float* __restrict__ y,
+                                                    int ldy) {
+  __shared__ float red[4];
+  const int t = blockIdx.x, vec = blockIdx.y, tid = threadIdx.x;
+  const int pos0 = *posp + off;
+  const int nqk = 2 * Hd, nvb = (Hd * dv + 127) / 128;
+  auto conv = [&](int c) -> float {
+    float acc = 0.f;
+    for (int j = 0; j < W; ++j) {
+      const int s = t - (W - 1) + j;
+      float x;
+      if (s >= 0) x = z[static_cast<long long>(s) * ldz + c];
+      else {
+        const int p = pos0 + s;
+        x = p >= 0 ? ring[static_cast<long long>(p % W) * C + c] : 0.f;
+      }
+      acc = fmaf(bf16_to_f(taps[static_cast<long long>(c) * W + j]), x, acc);
+    }
+    return siluf_(acc);
+  };
+  float* yr = y + static_cast<long long>(t) * ldy;
+  if (vec < nqk) {
+    const int c = vec * dk + tid;
+    const float v = tid < dk ? conv(c) : 0.f;
+    const float ss = warp_sum(v * v);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    __syncthreads();
+    const float inv = 1.0f / sqrtf(red[0] + red[1] + red[2] + red[3] + 1e-6f);
+    if (tid < dk) yr[c] = v * inv;
+  } else if (vec < nqk + nvb) {
+    const int c = 2 * Hd * dk + (vec - nqk) * 128 + tid;
+    if (c < C) yr[c] = conv(c);
+  } else {
+    for (int hh = tid; hh < Hd; hh += blockDim.x) {
+      const float al = z[static_cast<long long>(t) * ldz + C + hh];
+      const float be = z[static_cast<long long>(t) * ldz + C + Hd + hh];
+      yr[C + hh] = -(fmaxf(al, 0.f) + log1pf(expf(-fabsf(al))));
+      yr[C + Hd + hh] = sigmoidf_(be);
+    }
+  }
+}
+
 // Conv history after the batch: the raw inputs of the last W-1 positions go to their ring slots.
 __global__ void conv_history_update(const float* __restrict__ z, int ldz, int T, const int* __restrict__ posp, int off,
                                     float* __restrict__ ring, int W, int C) {
@@ -164,7 +211,7 @@ __global__ void at_prep(const float* __restrict__ z, int ldz, const int* __restr
 __global__ void gate_split(const float* __restrict__ o, int ldo, const float* __restrict__ gate, int ldg, int n,
                            uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
   const int t = blockIdx.x;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+  for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < n; i += gridDim.y * blockDim.x) {
     float v = o[static_cast<long long>(t) * ldo + i];
     if (gate) v *= sigmoidf_(gate[static_cast<long long>(t) * ldg + i]);
     put_split(xhi, xlo, static_cast<long long>(t) * n + i, v);
@@ -175,7 +222,7 @@ __global__ void gate_split(const float* __restrict__ o, int ldo, const float* __
 __global__ void act_split(const float* __restrict__ gu, int F, uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
   const int t = blockIdx.x;
   const float* r = gu + static_cast<long long>(t) * 2 * F;
-  for (int i = threadIdx.x; i < F; i += blockDim.x)
+  for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < F; i += gridDim.y * blockDim.x)
     put_split(xhi, xlo, static_cast<long long>(t) * F + i, siluf_(r[i]) * r[F + i]);
 }
 
@@ -381,6 +428,45 @@ __global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S 
 // shared-memory traffic (rows padded by 4 floats: 16-byte aligned, conflict-free for the
 // access patterns below), 4 x 4 output tiles per thread, and the forward substitution on
 // a right-hand-side column held in registers.
+// Forward substitution (I + A) X = RHS for the first CH rows of a chunk (CH >= n), column
+// j of X held in registers; writes the U (j < DV) or W column.
+template <int CH, int DK, int DV>
+__device__ __forceinline__ void wy_fsub(const WyBufs& b, const float* K, const float* A, const float* g,
+                                        const float* bb, int t0, int n, int h, int j, int vo) {
+  constexpr int KP = DK + 4, AP = kChunk + 4;
+  const int Hd = b.Hd;
+  float x[CH];
+#pragma unroll
+  for (int r = 0; r < CH; ++r) {
+    float v = 0.f;
+    if (r < n) {
+      v = (j < DV) ? b.y[static_cast<long long>(t0 + r) * b.ldy + vo + j] : expf(g[r]) * K[r * KP + (j - DV)];
+      v *= bb[r];
+    }
+    x[r] = v;
+  }
+#pragma unroll
+  for (int r = 1; r < CH; ++r) {
+    float acc = x[r];
+#pragma unroll
+    for (int s4 = 0; s4 < r; s4 += 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(A + r * AP + s4);
+      acc = fmaf(-a4.x, x[s4], acc);
+      if (s4 + 1 < r) acc = fmaf(-a4.y, x[s4 + 1], acc);
+      if (s4 + 2 < r) acc = fmaf(-a4.z, x[s4 + 2], acc);
+      if (s4 + 3 < r) acc = fmaf(-a4.w, x[s4 + 3], acc);
+    }
+    x[r] = acc;
+  }
+#pragma unroll
+  for (int r = 0; r < CH; ++r) {
+    if (r < n) {
+      if (j < DV) b.u[static_cast<long long>(t0 + r) * Hd * DV + h * DV + j] = x[r];
+      else b.w[static_cast<long long>(t0 + r) * Hd * DK + h * DK + (j - DV)] = x[r];
+    }
+  }
+}
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
   constexpr int KP = DK + 4, AP = kChunk + 4, XW = DV + DK;
@@ -467,37 +553,8 @@ __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
   __syncthreads();
   // (I + A) X = [diag(b) V | diag(b gamma) K]: column j of X in registers
   if (tid < XW) {
-    const int j = tid;
-    float x[kChunk];
-#pragma unroll
-    for (int r = 0; r < kChunk; ++r) {
-      float v = 0.f;
-      if (r < n) {
-        v = (j < DV) ? b.y[static_cast<long long>(t0 + r) * b.ldy + vo + j] : expf(g[r]) * K[r * KP + (j - DV)];
-        v *= bb[r];
-      }
-      x[r] = v;
-    }
-#pragma unroll
-    for (int r = 1; r < kChunk; ++r) {
-      float acc = x[r];
-#pragma unroll
-      for (int s4 = 0; s4 < r; s4 += 4) {
-        const float4 a4 = *reinterpret_cast<const float4*>(A + r * AP + s4);
-        acc = fmaf(-a4.x, x[s4], acc);
-        if (s4 + 1 < r) acc = fmaf(-a4.y, x[s4 + 1], acc);
-        if (s4 + 2 < r) acc = fmaf(-a4.z, x[s4 + 2], acc);
-        if (s4 + 3 < r) acc = fmaf(-a4.w, x[s4 + 3], acc);
-      }
-      x[r] = acc;
-    }
-#pragma unroll
-    for (int r = 0; r < kChunk; ++r) {
-      if (r < n) {
-        if (j < DV) b.u[static_cast<long long>(t0 + r) * Hd * DV + h * DV + j] = x[r];
-        else b.w[static_cast<long long>(t0 + r) * Hd * DK + h * DK + (j - DV)] = x[r];
-      }
-    }
+    if (n <= 16) wy_fsub<16, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo);
+    else wy_fsub<kChunk, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo);
   }
   if (tid < n) {
     b.gam[static_cast<long long>(t0 + tid) * Hd + h] = expf(g[tid]);
@@ -660,14 +717,20 @@ size_t wy_state_smem(int dk) {
 // One CTA per (query token t, kv head g): the Hq/Hkv query heads of group g attend to the
 // cached positions 0 .. pos0+t in blocks of 64 keys with an online softmax.
 constexpr int kKeyBlock = 64;
+constexpr int kMaxDraftRows = 17;   // max_draft <= 16
 
+// With nsplit > 1 (few tokens: T * Hkv CTAs would leave most SMs idle) CTA z takes the
+// z-th of nsplit equal ranges of the token's keys and writes its unnormalised partial
+// (acc[D], m, l per query head) to part [T][Hq][nsplit][D + 2]; attn_combine merges them.
 __global__ void __launch_bounds__(256) attn_prefill(const float* __restrict__ q, int ldq, const uint16_t* __restrict__ kc,
                                                     const uint16_t* __restrict__ vc, const int* __restrict__ posp,
                                                     int off, int Hq, int Hkv, int D, int max_ctx, float* __restrict__ o,
-                                                    int ldo) {
+                                                    int ldo, int nsplit, float* __restrict__ part) {
   extern __shared__ float sm[];
-  const int t = blockIdx.x, g = blockIdx.y, grp = Hq / Hkv;
-  const int nkeys = min(*posp + off + t + 1, max_ctx);
+  const int t = blockIdx.x, g = blockIdx.y, grp = Hq / Hkv, z = blockIdx.z;
+  const int nall = min(*posp + off + t + 1, max_ctx);
+  const int ks = ((nall + nsplit - 1) / nsplit + kKeyBlock - 1) / kKeyBlock * kKeyBlock;
+  const int kbeg = min(nall, z * ks), nkeys = min(nall, kbeg + ks);
   float* qs = sm;                                   // [grp][D]
   float* sc = qs + grp * D;                         // [grp][64]
   float* ml = sc + grp * kKeyBlock;                 // [grp][3]: m, l, corr
@@ -686,7 +749,7 @@ __global__ void __launch_bounds__(256) attn_prefill(const float* __restrict__ q,
   for (int u = 0; u < 8; ++u) acc[u] = 0.f;
   const uint16_t* kg = kc + static_cast<long long>(g) * max_ctx * D;
   const uint16_t* vg = vc + static_cast<long long>(g) * max_ctx * D;
-  for (int p0 = 0; p0 < nkeys; p0 += kKeyBlock) {
+  for (int p0 = kbeg; p0 < nkeys; p0 += kKeyBlock) {
     const int np = min(kKeyBlock, nkeys - p0);
     __syncthreads();
     for (int idx = threadIdx.x; idx < np * D / 8; idx += blockDim.x) {
@@ -749,10 +812,45 @@ __global__ void __launch_bounds__(256) attn_prefill(const float* __restrict__ q,
     }
   }
   __syncthreads();
+  if (nsplit > 1) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u < grp) part[((static_cast<long long>(t) * Hq + g * grp + u) * nsplit + z) * (D + 2) + d] = acc[u];
+    }
+    if (threadIdx.x < grp) {
+      float* pp = part + ((static_cast<long long>(t) * Hq + g * grp + threadIdx.x) * nsplit + z) * (D + 2);
+      pp[D] = ml[3 * threadIdx.x];
+      pp[D + 1] = ml[3 * threadIdx.x + 1];
+    }
+    return;
+  }
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
 #pragma unroll
     for (int u = 0; u < 8; ++u)
       if (u < grp) o[static_cast<long long>(t) * ldo + (g * grp + u) * D + d] = acc[u] / ml[3 * u + 1];
+  }
+}
+
+// o[t][hq] = sum_z e^{m_z - M} acc_z / sum_z e^{m_z - M} l_z over the key splits (empty
+// splits carry m = -inf, l = 0).
+__global__ void attn_combine(const float* __restrict__ part, int nsplit, int Hq, int D, float* __restrict__ o, int ldo) {
+  const int t = blockIdx.x, hq = blockIdx.y;
+  const float* pp = part + (static_cast<long long>(t) * Hq + hq) * nsplit * (D + 2);
+  float M = -INFINITY;
+  for (int z = 0; z < nsplit; ++z) M = fmaxf(M, pp[z * (D + 2) + D]);
+  float L = 0.f;
+  for (int z = 0; z < nsplit; ++z) {
+    const float mz = pp[z * (D + 2) + D];
+    if (mz > -INFINITY) L += expf(mz - M) * pp[z * (D + 2) + D + 1];
+  }
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float acc = 0.f;
+    for (int z = 0; z < nsplit; ++z) {
+      const float mz = pp[z * (D + 2) + D];
+      if (mz > -INFINITY) acc = fmaf(expf(mz - M), pp[z * (D + 2) + d], acc);
+    }
+    o[static_cast<long long>(t) * ldo + hq * D + d] = acc / L;
   }
 }
 
@@ -773,12 +871,16 @@ __global__ void advance_pos(int* pos, int n, int max_ctx) {
   *pos = min(*pos + n, max_ctx);
 }
 
-// Greedy token of each logits row (lowest index among equal maxima).
-__global__ void row_argmax(const float* __restrict__ logits, int V, int32_t* __restrict__ out) {
-  __shared__ unsigned long long best[32];
+// Greedy token of each logits row (lowest index among equal maxima): CTA (t, c) scans
+// slice c of row t and folds its best packed (value, index) key into best[t] (zeroed
+// before); the maximum is the same in any order.
+__global__ void row_argmax(const float* __restrict__ logits, int V, unsigned long long* __restrict__ best) {
+  __shared__ unsigned long long wb[32];
   const float* r = logits + static_cast<long long>(blockIdx.x) * V;
+  const int per = (V + gridDim.y - 1) / gridDim.y;
+  const int i0 = blockIdx.y * per, i1 = min(V, i0 + per);
   unsigned long long b = 0;
-  for (int i = threadIdx.x; i < V; i += blockDim.x) {
+  for (int i = i0 + threadIdx.x; i < i1; i += blockDim.x) {
     const unsigned long long k = pack_argmax(r[i], i);
     b = k > b ? k : b;
   }
@@ -786,12 +888,11 @@ __global__ void row_argmax(const float* __restrict__ logits, int V, int32_t* __r
     const unsigned long long x = __shfl_xor_sync(0xffffffffu, b, o);
     b = x > b ? x : b;
   }
-  if ((threadIdx.x & 31) == 0) best[threadIdx.x >> 5] = b;
+  if ((threadIdx.x & 31) == 0) wb[threadIdx.x >> 5] = b;
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w) b = best[w] > b ? best[w] : b;
-    b = best[0] > b ? best[0] : b;
-    out[blockIdx.x] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(b & 0xFFFFFFFFull));
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) b = wb[w] > b ? wb[w] : b;
+    atomicMax(best + blockIdx.x, b);
   }
 }
 
@@ -829,8 +930,14 @@ __global__ void advance_pos_accepted(int* pos, const int* n_acc, int max_ctx) {
   *pos = min(*pos + *n_acc + 1, max_ctx);
 }
 
-__global__ void accept_prefix(const int* tokens, const int* g, int K, int* n_out, int* n_acc, int* out) {
+__global__ void accept_prefix(const int* tokens, const unsigned long long* best, int K, int* n_out, int* n_acc, int* out,
+                              int* greedy) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int g[kMaxDraftRows];
+  for (int i = 0; i <= K; ++i) {
+    g[i] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best[i] & 0xFFFFFFFFull));
+    greedy[i] = g[i];
+  }
   int n = 0;
   while (n < K && tokens[1 + n] == g[n]) ++n;
   for (int i = 0; i < n; ++i) out[i] = tokens[1 + i];
@@ -857,7 +964,7 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
   };
   auto linear = [&](const void* w, long long ldw, int N, int K, float* out, long long ldc, int acc) {
     if (e != cudaSuccess) return;
-    LinearArgs a{pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, b.err};
+    LinearArgs a{pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, b.err, pf.splitk, kSplitKFloats};
     e = launch_linear(a, s);
     ++m->launches;
   };
@@ -875,7 +982,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       float* ring = b.conv_ring + static_cast<size_t>(di) * Wc * C;
       ++di;
       linear(L.w_in, 2LL * H + 16, rows, H, pf.z, rows, 0);
-      dn_prep<<<T, kPT, C * sizeof(float), s>>>(pf.z, rows, b.pos, off, ring, Wc, C, Hd, dk, L.conv, pf.y, rows);
+      dn_prep_wide<<<dim3(T, 2 * Hd + (Hd * dv + 127) / 128 + 1), 128, 0, s>>>(pf.z, rows, b.pos, off, ring, Wc, C, Hd,
+                                                                              dk, dv, L.conv, pf.y, rows);
       chk();
       WyBufs wy{pf.y, rows, pf.u, pf.w, pf.p, pf.gam, pf.dec, pf.o, T, Hd, dk, dv, nullptr, nullptr, nullptr, 0};
       if (vs) {
@@ -906,7 +1014,7 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         wy_state<<<dim3(Hd, dv / kRowGroup), 256, wy_state_smem(dk), s>>>(wy, S);
       }
       chk();
-      gate_split<<<T, kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo);
+      gate_split<<<dim3(T, (Hd * dv + 1023) / 1024), kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo);
       chk();
       linear(PL.w_out, 2LL * Hd * dv, H, Hd * dv, pf.h, H, 1);
     } else {
@@ -918,10 +1026,18 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       at_prep<<<T, kPT, 0, s>>>(pf.z, rows, b.pos, off, b.inv_freq, Hq, Hkv, D, c.at_out_gate, kc, vc, c.max_ctx,
                                  pf.y, qd);
       chk();
-      attn_prefill<<<dim3(T, Hkv), 256, attn_prefill_smem(Hq / Hkv, D), s>>>(pf.y, qd, kc, vc, b.pos, off, Hq, Hkv,
-                                                                              D, c.max_ctx, pf.o, qd);
+      // key splits when T * Hkv CTAs would leave most of the GPU idle (verify passes, short prompts)
+      int nsplit = 1;
+      if (T * Hkv < 148 && T <= kAttnSplitRows) nsplit = std::min(kAttnMaxSplit, (296 + T * Hkv - 1) / (T * Hkv));
+      attn_prefill<<<dim3(T, Hkv, nsplit), 256, attn_prefill_smem(Hq / Hkv, D), s>>>(
+          pf.y, qd, kc, vc, b.pos, off, Hq, Hkv, D, c.max_ctx, pf.o, qd, nsplit, pf.apart);
       chk();
-      gate_split<<<T, kPT, 0, s>>>(pf.o, qd, c.at_out_gate ? pf.z + qd : nullptr, rows, qd, pf.xhi, pf.xlo);
+      if (nsplit > 1) {
+        attn_combine<<<dim3(T, Hq), std::min(D, 256), 0, s>>>(pf.apart, nsplit, Hq, D, pf.o, qd);
+        chk();
+      }
+      gate_split<<<dim3(T, (qd + 1023) / 1024), kPT, 0, s>>>(pf.o, qd, c.at_out_gate ? pf.z + qd : nullptr, rows, qd,
+                                                             pf.xhi, pf.xlo);
       chk();
       linear(PL.w_out, 2LL * qd, H, qd, pf.h, H, 1);
     }
@@ -930,7 +1046,7 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
     chk();
     linear(L.w_gate, 2LL * H, F, H, pf.z, 2LL * F, 0);
     linear(L.w_up, 2LL * H, F, H, pf.z + F, 2LL * F, 0);
-    act_split<<<T, kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
+    act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
     chk();
     linear(PL.w_down, 2LL * F, H, F, pf.h, H, 1);
   }
@@ -940,6 +1056,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
 }  // namespace
 
 cudaError_t set_prefill_smem_limits() {
+  static bool done = false;   // per process; the attributes are the same on every device
+  if (done) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(wy_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
@@ -948,6 +1066,7 @@ cudaError_t set_prefill_smem_limits() {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess) done = true;
   return e;
 }
 
@@ -1012,13 +1131,14 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
     e = mk::launch_linear(a, s);
     ++m->launches;
   }
+  if (e == cudaSuccess) e = cudaMemsetAsync(m->pf.best, 0, sizeof(unsigned long long) * T, s);
   if (e == cudaSuccess) {
-    mk::row_argmax<<<T, 256, 0, s>>>(logits, c.vocab, vs.greedy);
+    mk::row_argmax<<<dim3(T, 64), 256, 0, s>>>(logits, c.vocab, m->pf.best);
     chk();
   }
   // 3. longest matching prefix plus the bonus token
   if (e == cudaSuccess) {
-    mk::accept_prefix<<<1, 32, 0, s>>>(d_tokens, vs.greedy, K, m->ws_n, d_n_accepted, d_out_tokens);
+    mk::accept_prefix<<<1, 32, 0, s>>>(d_tokens, m->pf.best, K, m->ws_n, d_n_accepted, d_out_tokens, vs.greedy);
     chk();
   }
   // 4. commit: DeltaNet states and conv histories of the accepted prefix, then the position
