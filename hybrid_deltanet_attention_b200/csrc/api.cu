@@ -238,6 +238,8 @@ struct Layout {
   // batched prefill workspace
   int pf_rows;
   size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec, pf_apart, pf_splitk, pf_best;
+  size_t pf_sbuf, pf_phi, pf_plo, pf_vt;
+  long long pf_nk;
   // batched verify saves
   int vf_rows;
   size_t vf_delta, vf_k, vf_g, vf_raw, vf_logits, vf_greedy;
@@ -366,6 +368,14 @@ Layout make_layout(const mk_config& c, int grid) {
                              (static_cast<size_t>(c.at_head_dim) + 2) * 4);
     L.pf_splitk = off; off = align256(off + static_cast<size_t>(mk::kSplitKFloats) * 4);
     L.pf_best = off; off = align256(off + T * 8);
+    L.pf_nk = na ? std::min<long long>(8192, (static_cast<long long>(c.max_ctx) + 63) / 64 * 64) : 0;
+    if (L.pf_nk > 0) {
+      const size_t nk = static_cast<size_t>(L.pf_nk);
+      L.pf_sbuf = off; off = align256(off + T * nk * 4);
+      L.pf_phi = off; off = align256(off + T * nk * 2);
+      L.pf_plo = off; off = align256(off + T * nk * 2);
+      L.pf_vt = off; off = align256(off + static_cast<size_t>(c.at_head_dim) * nk * 2);
+    }
   }
   L.vf_rows = (L.pf_rows > 0 && c.max_draft > 0 && c.max_draft + 1 <= std::min(64, L.pf_rows)) ? c.max_draft + 1 : 0;
   if (L.vf_rows > 0) {
@@ -430,6 +440,7 @@ int launch_step(mk_model* m, const int32_t* in_tok, int32_t* out_tok, float* log
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   ++m->launches;
   ++m->pos_hint;
+  ++m->pos_max;
   return MK_OK;
 }
 
@@ -511,6 +522,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   m->device = dev;
   m->launches = 0;
   m->pos_hint = 0;
+  m->pos_max = 0;
 
   auto copy = [&](const std::string& nm, size_t dst_off) -> cudaError_t {
     const mk_tensor* t = got[nm];
@@ -711,6 +723,13 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     m->pf.apart = reinterpret_cast<float*>(W + L.pf_apart);
     m->pf.splitk = reinterpret_cast<float*>(W + L.pf_splitk);
     m->pf.best = reinterpret_cast<unsigned long long*>(W + L.pf_best);
+    m->pf.nk_max = L.pf_nk;
+    if (L.pf_nk > 0) {
+      m->pf.sbuf = reinterpret_cast<float*>(W + L.pf_sbuf);
+      m->pf.phi = reinterpret_cast<uint16_t*>(W + L.pf_phi);
+      m->pf.plo = reinterpret_cast<uint16_t*>(W + L.pf_plo);
+      m->pf.vt = reinterpret_cast<uint16_t*>(W + L.pf_vt);
+    }
   }
   m->vf.rows = L.vf_rows;
   if (L.vf_rows > 0) {
@@ -732,6 +751,7 @@ int mk_reset_state(mk_model* m, void* stream) {
   if (e == cudaSuccess) e = cudaMemsetAsync(m->ws, 0, kResetBytes, s);   // sync words and per-head norms
   if (e != cudaSuccess) return cuda_fail(e, "reset");
   m->pos_hint = 0;
+  m->pos_max = 0;
   return MK_OK;
 }
 
@@ -743,6 +763,7 @@ int mk_set_position(mk_model* m, int32_t pos, void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "set position");
   ++m->launches;
   m->pos_hint = pos;
+  m->pos_max = pos;
   return MK_OK;
 }
 
@@ -823,6 +844,7 @@ int mk_verify_drafts(mk_model* m, const int32_t* d_tokens, int32_t K, int32_t* d
     ++m->launches;
   }
   m->pos_hint = pos0 + 1;   // at least one position is always committed; the exact count is on the device
+  m->pos_max = pos0 + K + 1;
   return MK_OK;
 }
 

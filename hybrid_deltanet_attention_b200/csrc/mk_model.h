@@ -28,6 +28,13 @@ struct mk_prefill_ws {
   float* apart = nullptr;    // [min(rows, kAttnSplitRows)][Hq][kAttnMaxSplit][D + 2] attention key-split partials
   float* splitk = nullptr;   // [kSplitKFloats] split-K partials of the linear layers
   unsigned long long* best = nullptr;   // [rows] packed (value, index) row maxima of the verify logits
+  // attention as two GEMMs: scores [rows][nk_max] fp32, probabilities as bf16 high/low
+  // parts [rows][nk_max], V^T [D][nk_max]
+  long long nk_max = 0;
+  float* sbuf = nullptr;
+  uint16_t* phi = nullptr;
+  uint16_t* plo = nullptr;
+  uint16_t* vt = nullptr;
 };
 
 struct mk_prefill_layer {   // K-major copies of the projections the decode kernel keeps transposed
@@ -65,7 +72,8 @@ struct mk_model {
   mk::DecodeParams base;
   std::vector<mk::LayerW> layers_host;
   int64_t launches;
-  int64_t pos_hint;      // host shadow of the device position (calls through this handle)
+  int64_t pos_hint;      // host shadow of the device position (calls through this handle); a lower bound
+  int64_t pos_max;       // an upper bound of the device position (verify passes commit 1..K+1 tokens)
   // workspace sub-buffers used by the host-side drivers
   int32_t* ws_tok;       // [max_ctx + 8] token staging for prefill / generate
   int32_t* ws_g;         // [max_draft + 1] greedy tokens of a verify pass

@@ -97,6 +97,7 @@ int mk_decode_step_noalloc(mk_model* m, const int32_t* d_in_token, int32_t* d_ou
   if (e != cudaSuccess) return fail(MK_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
   ++m->launches;
   ++m->pos_hint;
+  ++m->pos_max;
   return MK_OK;
 }
 

@@ -713,11 +713,60 @@ size_t wy_state_smem(int dk) {
                           kChunk * kRowGroup + kChunk * 17 + 2 * kChunk);
 }
 
+// ------------------------------------------------------------------ attention as two GEMMs
+// For long prompts, per query head: S = Q K^T (tcgen05 linear layer over the cached keys),
+// P = causal softmax(S) written as bf16 high/low parts, O = P V (second linear layer
+// against V^T). Keys past a row's position are masked in the softmax; P is zero there.
+__device__ __forceinline__ float block_max(float v, float* red) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = (l < static_cast<int>(blockDim.x >> 5)) ? red[l] : -INFINITY;
+  return warp_max(t);
+}
+
+__global__ void attn_softmax_split(const float* __restrict__ S, int nk, const int* __restrict__ posp, int off,
+                                   uint16_t* __restrict__ phi, uint16_t* __restrict__ plo) {
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  const int last = min(*posp + off + t, nk - 1);   // keys 0 .. last
+  const float* r = S + static_cast<long long>(t) * nk;
+  float mx = -INFINITY;
+  for (int j = threadIdx.x; j <= last; j += blockDim.x) mx = fmaxf(mx, r[j]);
+  mx = block_max(mx, red);
+  float sum = 0.f;
+  for (int j = threadIdx.x; j <= last; j += blockDim.x) sum += expf(r[j] - mx);
+  sum = block_sum(sum, red);
+  const float inv = 1.0f / sum;
+  for (int j = threadIdx.x; j < nk; j += blockDim.x)
+    put_split(phi, plo, static_cast<long long>(t) * nk + j, j <= last ? expf(r[j] - mx) * inv : 0.f);
+}
+
+// VT[d][j] = V[j][d] for the keys up to the pass's last position, zero past it.
+__global__ void v_transpose(const uint16_t* __restrict__ vg, int D, int nk, const int* __restrict__ posp, int last_off,
+                            int max_ctx, uint16_t* __restrict__ vt) {
+  __shared__ uint16_t tile[32][33];
+  const int last = min(*posp + last_off, max_ctx - 1);
+  const int j0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
+  for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+    const int j = j0 + k, d = d0 + threadIdx.x;
+    tile[k][threadIdx.x] = (j <= last && d < D) ? vg[static_cast<long long>(j) * D + d] : 0;
+  }
+  __syncthreads();
+  for (int k = threadIdx.y; k < 32; k += blockDim.y) {
+    const int d = d0 + k, j = j0 + threadIdx.x;
+    if (d < D && j < nk) vt[static_cast<long long>(d) * nk + j] = tile[threadIdx.x][k];
+  }
+}
+
 // ------------------------------------------------------------------ causal attention
 // One CTA per (query token t, kv head g): the Hq/Hkv query heads of group g attend to the
 // cached positions 0 .. pos0+t in blocks of 64 keys with an online softmax.
 constexpr int kKeyBlock = 64;
 constexpr int kMaxDraftRows = 17;   // max_draft <= 16
+constexpr int kGemmAttnMinRows = 64;   // prompts from this many tokens run attention as two GEMMs
 
 // With nsplit > 1 (few tokens: T * Hkv CTAs would leave most SMs idle) CTA z takes the
 // z-th of nsplit equal ranges of the token's keys and writes its unnormalised partial
@@ -1026,15 +1075,46 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       at_prep<<<T, kPT, 0, s>>>(pf.z, rows, b.pos, off, b.inv_freq, Hq, Hkv, D, c.at_out_gate, kc, vc, c.max_ctx,
                                  pf.y, qd);
       chk();
-      // key splits when T * Hkv CTAs would leave most of the GPU idle (verify passes, short prompts)
-      int nsplit = 1;
-      if (T * Hkv < 148 && T <= kAttnSplitRows) nsplit = std::min(kAttnMaxSplit, (296 + T * Hkv - 1) / (T * Hkv));
-      attn_prefill<<<dim3(T, Hkv, nsplit), 256, attn_prefill_smem(Hq / Hkv, D), s>>>(
-          pf.y, qd, kc, vc, b.pos, off, Hq, Hkv, D, c.max_ctx, pf.o, qd, nsplit, pf.apart);
-      chk();
-      if (nsplit > 1) {
-        attn_combine<<<dim3(T, Hq), std::min(D, 256), 0, s>>>(pf.apart, nsplit, Hq, D, pf.o, qd);
+      const long long nk_gemm = (m->pos_max + off + T + 63) / 64 * 64;   // covers every key of the pass
+      if (T >= kGemmAttnMinRows && pf.sbuf && nk_gemm <= pf.nk_max) {
+        const int nk = static_cast<int>(nk_gemm);
+        const int grp = Hq / Hkv;
+        for (int g = 0; g < Hkv && e == cudaSuccess; ++g) {
+          v_transpose<<<dim3(nk / 32, (D + 31) / 32), dim3(32, 8), 0, s>>>(
+              vc + static_cast<size_t>(g) * c.max_ctx * D, D, nk, b.pos, off + T - 1, c.max_ctx, pf.vt);
+          chk();
+          for (int u = 0; u < grp && e == cudaSuccess; ++u) {
+            const int hq = g * grp + u;
+            e = launch_split_bf16(pf.y + static_cast<size_t>(hq) * D, qd, pf.xhi, pf.xlo, T, D, s);
+            ++m->launches;
+            if (e == cudaSuccess) {   // S = Q K^T over the cached keys (rows past max_ctx read as zero)
+              LinearArgs a{pf.xhi, pf.xlo, kc + static_cast<size_t>(g) * c.max_ctx * D, 2LL * D, pf.sbuf, nk, T,
+                           std::min(nk, c.max_ctx), D, 0, b.err, pf.splitk, kSplitKFloats};
+              e = launch_linear(a, s);
+              ++m->launches;
+            }
+            if (e != cudaSuccess) break;
+            attn_softmax_split<<<T, kPT, 0, s>>>(pf.sbuf, nk, b.pos, off, pf.phi, pf.plo);
+            chk();
+            if (e == cudaSuccess) {   // O = P V
+              LinearArgs a{pf.phi, pf.plo, pf.vt, 2LL * nk, pf.o + static_cast<size_t>(hq) * D, qd, T, D, nk, 0, b.err,
+                           pf.splitk, kSplitKFloats};
+              e = launch_linear(a, s);
+              ++m->launches;
+            }
+          }
+        }
+      } else {
+        // key splits when T * Hkv CTAs would leave most of the GPU idle (verify passes, short prompts)
+        int nsplit = 1;
+        if (T * Hkv < 148 && T <= kAttnSplitRows) nsplit = std::min(kAttnMaxSplit, (296 + T * Hkv - 1) / (T * Hkv));
+        attn_prefill<<<dim3(T, Hkv, nsplit), 256, attn_prefill_smem(Hq / Hkv, D), s>>>(
+            pf.y, qd, kc, vc, b.pos, off, Hq, Hkv, D, c.max_ctx, pf.o, qd, nsplit, pf.apart);
         chk();
+        if (nsplit > 1) {
+          attn_combine<<<dim3(T, Hq), std::min(D, 256), 0, s>>>(pf.apart, nsplit, Hq, D, pf.o, qd);
+          chk();
+        }
       }
       gate_split<<<dim3(T, (qd + 1023) / 1024), kPT, 0, s>>>(pf.o, qd, c.at_out_gate ? pf.z + qd : nullptr, rows, qd,
                                                              pf.xhi, pf.xlo);
@@ -1100,6 +1180,7 @@ int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t
     return MK_ERR_CUDA;
   }
   m->pos_hint += n;
+  m->pos_max += n;
   return MK_OK;
 }
 
@@ -1166,5 +1247,6 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
     return MK_ERR_CUDA;
   }
   m->pos_hint += 1;   // at least one position is always committed; the exact count is on the device
+  m->pos_max += T;
   return MK_OK;
 }
