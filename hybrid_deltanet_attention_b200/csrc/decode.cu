@@ -1609,7 +1609,11 @@ cudaError_t launch_hk(const DecodeParams& p, int grid, cudaStream_t s) {
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s) {
-  if (p.q4) return launch_hk<0, true>(p, grid, s);
+  if (p.q4) {
+    if (p.H == 1024) return launch_hk<4, true>(p, grid, s);
+    if (p.H == 5120) return launch_hk<20, true>(p, grid, s);
+    return launch_hk<0, true>(p, grid, s);
+  }
   if (p.H == 1024) return launch_hk<4, false>(p, grid, s);
   if (p.H == 256) return launch_hk<1, false>(p, grid, s);
   if (p.H == 2048) return launch_hk<8, false>(p, grid, s);
