@@ -817,19 +817,22 @@ __device__ __forceinline__ float q4_part(const uint8_t* blk, const Q4Lane& ql, c
   const uint32_t c = *reinterpret_cast<const uint32_t*>(blk + 16 + 16 * ql.j + 4 * ql.part);
   const uint32_t sc = __funnelshift_r(ql.sc_w ? f1 : f0, ql.sc_w ? f2 : f1, ql.sc_sh) & 63u;
   const uint32_t mm = __funnelshift_r(ql.m_w == 1 ? f1 : f2, ql.m_w == 1 ? f2 : 0u, ql.m_sh) & 63u;
-  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) * static_cast<float>(sc);
-  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) * static_cast<float>(mm);
-  // sum (1 + q/16) x over the lane's 8 weights; sum q x = 16 (that - sum x)
-  float u = q4_unit<0>(c) * xl.x;
-  u = fmaf(q4_unit<8>(c), xl.y, u);
-  u = fmaf(q4_unit<16>(c), xl.z, u);
-  u = fmaf(q4_unit<24>(c), xl.w, u);
-  u = fmaf(q4_unit<4>(c), xh.x, u);
-  u = fmaf(q4_unit<12>(c), xh.y, u);
-  u = fmaf(q4_unit<20>(c), xh.z, u);
-  u = fmaf(q4_unit<28>(c), xh.w, u);
+  // small integers to float through the exponent field: 2^23 + v is exact for v < 2^23
+  const float scf = __uint_as_float(0x4B000000u | sc) - 8388608.0f;
+  const float mmf = __uint_as_float(0x4B000000u | mm) - 8388608.0f;
+  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) * scf;
+  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) * mmf;
+  // sum (1 + q/16) x over the lane's 8 weights (two chains); sum q x = 16 (that - sum x)
+  float u0 = q4_unit<0>(c) * xl.x;
+  float u1 = q4_unit<4>(c) * xh.x;
+  u0 = fmaf(q4_unit<8>(c), xl.y, u0);
+  u1 = fmaf(q4_unit<12>(c), xh.y, u1);
+  u0 = fmaf(q4_unit<16>(c), xl.z, u0);
+  u1 = fmaf(q4_unit<20>(c), xh.z, u1);
+  u0 = fmaf(q4_unit<24>(c), xl.w, u0);
+  u1 = fmaf(q4_unit<28>(c), xh.w, u1);
   const float s16 = 16.0f * s;
-  return fmaf(s16, u, -(s16 + mn) * xsv);
+  return fmaf(s16, u0 + u1, -(s16 + mn) * xsv);
 }
 
 // xsum[sb * 32 + l] = the sum of the 8 x values lane l pairs with in super-block sb.

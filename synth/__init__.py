@@ -125,7 +125,11 @@ MID_Q4 = _preset("mid-q4", n_layers=8, pattern="DDDA" * 2, hidden=1024, vocab=32
                  at_q_heads=8, at_kv_heads=2, at_head_dim=128, rope_theta=1e7, at_out_gate=1,
                  ffn=3072, weight_format=W_Q4K, seed=11)
 
-CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI, TINY_Q4, MID_Q4)}
+# Four layers of the 27B shape (one [D,D,D,A] block): the 27B kernels on a small case
+# (about 1.4 GB of 4-bit weights), for profiling.
+QWEN_27B_4L = dataclasses.replace(QWEN_27B, name="27b-4l", n_layers=4, pattern="DDDA")
+
+CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI, TINY_Q4, MID_Q4, QWEN_27B_4L)}
 
 
 def with_changes(cfg: ModelConfig, **kw) -> ModelConfig:
