@@ -9,13 +9,16 @@
 // keeps its activations at.
 //
 // One CTA computes one 128 x BN tile of C:
-//   warp 0   allocates BN TMEM columns; its lane 0 is the TMA producer: per 64-wide K
-//            block it loads Xhi, Xlo [128 x 64] and W [BN x 64] (128-byte swizzled) into a
-//            4-stage shared-memory ring;
-//   warp 1   lane 0 issues tcgen05.mma (M = 128, N = BN, K = 16; 8 per K block) and
-//            commits each stage back to the producer, then the accumulator;
-//   warps 2-5 read the accumulator rows from TMEM (warp w owns lanes 32 (w % 4) ..) and
-//            store (or add into) C.
+// persistent CTAs (at most one per SM) walk the tiles (and K splits):
+//   warp 0   allocates 2 x BN TMEM columns (two accumulators); its lane 0 is the TMA
+//            producer: per 64-wide K block it loads Xhi, Xlo [128 x 64] and W [BN x 64]
+//            (128-byte swizzled) into a 3-4 stage shared-memory ring;
+//   warp 1   lane 0 issues tcgen05.mma (M = 128, N = BN, K = 16; 8 per K block) into the
+//            tile's accumulator, commits each stage back to the producer and the finished
+//            accumulator to the epilogue;
+//   warps 2-5 read the accumulator rows from TMEM (warp w owns lanes 32 (w % 4) ..), store
+//            (or add into) C, and hand the accumulator back, while the next tile's MMAs run
+//            in the other one.
 // Every wait has a time limit; on expiry the CTA latches an error bit and winds down.
 #include <algorithm>
 #include <cstdio>
@@ -51,42 +54,49 @@ struct GemmShape {
 struct GemmBars {
   uint64_t full[4];
   uint64_t empty[4];
-  uint64_t acc;
+  uint64_t acc_full[2];    // accumulator buffer b holds a finished tile
+  uint64_t acc_empty[2];   // the epilogue has drained buffer b
   uint32_t tmem;
   int abort;
 };
 
+// Persistent: CTA c walks the work items c, c + grid, ... (item = (N tile, M tile, K split)),
+// with two TMEM accumulators so that the epilogue of one item overlaps the MMAs of the next.
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
     linear_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                   const __grid_constant__ CUtensorMap tb, float* __restrict__ C, long long ldc, int M, int N, int K,
-                  int accumulate, int* err, float* __restrict__ ws) {
+                  int accumulate, int* err, float* __restrict__ ws, int nz) {
   using S = GemmShape<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   GemmBars* gb = reinterpret_cast<GemmBars*>(smem + S::kRingBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
-  // split-K: CTA z takes K blocks [kb0, kb1) and writes its partial tile to ws[z] ([M][N])
-  const int nkall = K / kBK, nz = gridDim.z, z = blockIdx.z;
-  const int kb0 = static_cast<int>((static_cast<long long>(nkall) * z) / nz);
-  const int kb1 = static_cast<int>((static_cast<long long>(nkall) * (z + 1)) / nz);
-  const int nk = kb1 - kb0;
-  if (nz > 1) {
-    C = ws + static_cast<long long>(z) * M * N;
-    ldc = N;
-    accumulate = 0;
-  }
+  const int tiles_n = (N + BN - 1) / BN, tiles_m = (M + kBM - 1) / kBM;
+  const int items = tiles_n * tiles_m * nz;
+  const int nkall = K / kBK;
   auto a_hi = [&](int s) { return smem + s * S::kStageBytes; };
   auto a_lo = [&](int s) { return smem + s * S::kStageBytes + S::kABytes; };
   auto b_t = [&](int s) { return smem + s * S::kStageBytes + 2 * S::kABytes; };
+  // item -> tile origin and K-block range (split z takes [kb0, kb1))
+  auto decode = [&](int w, int& n0, int& m0, int& z, int& kb0, int& kb1) {
+    const int tn = w % tiles_n, rest = w / tiles_n;
+    n0 = tn * BN;
+    m0 = (rest % tiles_m) * kBM;
+    z = rest / tiles_m;
+    kb0 = static_cast<int>((static_cast<long long>(nkall) * z) / nz);
+    kb1 = static_cast<int>((static_cast<long long>(nkall) * (z + 1)) / nz);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::kStages; ++s) {
       mbar_init(&gb->full[s], 1);
       mbar_init(&gb->empty[s], 1);
     }
-    mbar_init(&gb->acc, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&gb->acc_full[b], 1);
+      mbar_init(&gb->acc_empty[b], 4);   // one arrival per epilogue warp
+    }
     gb->abort = 0;
     fence_barrier_init();
     tc::prefetch_tensormap(&ta_hi);
@@ -94,7 +104,7 @@ __global__ void __launch_bounds__(192, 1)
     tc::prefetch_tensormap(&tb);
   }
   if (warp == 0) {
-    tc::tmem_alloc(&gb->tmem, BN);
+    tc::tmem_alloc(&gb->tmem, 2 * BN);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -104,67 +114,102 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort = &gb->abort;
 
   if (warp == 0) {
-    if (lane == 0) {   // ---- TMA producer
-      int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S::kStages;
-        if (kb >= S::kStages && !mbar_wait(&gb->empty[s], ((kb / S::kStages) - 1) & 1, abort, kGemmWaitNs)) {
-          if (!*abort) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
-          *abort = 1;
-          break;
+    if (lane == 0) {   // ---- TMA producer: one running K-block counter over all items
+      uint32_t kc = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+        int n0, m0, z, kb0, kb1;
+        decode(w, n0, m0, z, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++kc) {
+          const int s = kc % S::kStages;
+          if (kc >= static_cast<uint32_t>(S::kStages) &&
+              !mbar_wait(&gb->empty[s], ((kc / S::kStages) - 1) & 1, abort, kGemmWaitNs)) {
+            if (!*abort) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
+            *abort = 1;
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&gb->full[s], S::kStageBytes);
+          tc::tma_load_2d(a_hi(s), &ta_hi, kb * kBK, m0, &gb->full[s]);
+          tc::tma_load_2d(a_lo(s), &ta_lo, kb * kBK, m0, &gb->full[s]);
+          tc::tma_load_2d(b_t(s), &tb, kb * kBK, n0, &gb->full[s]);
         }
-        mbar_arrive_expect_tx(&gb->full[s], S::kStageBytes);
-        tc::tma_load_2d(a_hi(s), &ta_hi, (kb0 + kb) * kBK, m0, &gb->full[s]);
-        tc::tma_load_2d(a_lo(s), &ta_lo, (kb0 + kb) * kBK, m0, &gb->full[s]);
-        tc::tma_load_2d(b_t(s), &tb, (kb0 + kb) * kBK, n0, &gb->full[s]);
-        ++issued;
       }
       int never = 0;   // let the copies this lane issued land before the CTA ends (bounded)
-      for (int kb = issued > S::kStages ? issued - S::kStages : 0; kb < issued; ++kb)
-        mbar_wait(&gb->full[kb % S::kStages], (kb / S::kStages) & 1, &never, kGemmWaitNs / 5);
+      for (uint32_t k = kc > static_cast<uint32_t>(S::kStages) ? kc - S::kStages : 0; k < kc; ++k)
+        mbar_wait(&gb->full[k % S::kStages], (k / S::kStages) & 1, &never, kGemmWaitNs / 5);
     }
   } else if (warp == 1) {
     if (lane == 0) {   // ---- MMA issuer
       constexpr uint32_t idesc = tc::idesc_bf16_f32(kBM, BN);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S::kStages;
-        if (!mbar_wait(&gb->full[s], (kb / S::kStages) & 1, abort, kGemmWaitNs)) {
+      uint32_t kc = 0;
+      bool ok = true;
+      int i = 0;
+      for (int w = blockIdx.x; w < items && ok; w += gridDim.x, ++i) {
+        int n0, m0, z, kb0, kb1;
+        decode(w, n0, m0, z, kb0, kb1);
+        const int buf = i & 1;
+        if (i >= 2 && !mbar_wait(&gb->acc_empty[buf], ((i >> 1) - 1) & 1, abort, kGemmWaitNs)) {
           if (!*abort) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
           *abort = 1;
           break;
         }
         tc::fence_after_sync();
+        const uint32_t acc = tmem + static_cast<uint32_t>(buf * BN);
+        for (int kb = kb0; kb < kb1; ++kb, ++kc) {
+          const int s = kc % S::kStages;
+          if (!mbar_wait(&gb->full[s], (kc / S::kStages) & 1, abort, kGemmWaitNs)) {
+            if (!*abort) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
+            *abort = 1;
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t bd = tc::desc_kmajor_sw128(b_t(s) + kk * 32);
-          tc::mma_bf16(tmem, tc::desc_kmajor_sw128(a_hi(s) + kk * 32), bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-          tc::mma_bf16(tmem, tc::desc_kmajor_sw128(a_lo(s) + kk * 32), bd, idesc, 1u);
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t bd = tc::desc_kmajor_sw128(b_t(s) + kk * 32);
+            tc::mma_bf16(acc, tc::desc_kmajor_sw128(a_hi(s) + kk * 32), bd, idesc, (kb > kb0 || kk) ? 1u : 0u);
+            tc::mma_bf16(acc, tc::desc_kmajor_sw128(a_lo(s) + kk * 32), bd, idesc, 1u);
+          }
+          tc::mma_commit(&gb->empty[s]);
         }
-        tc::mma_commit(&gb->empty[s]);
+        tc::mma_commit(&gb->acc_full[buf]);   // arrives once every MMA issued so far has completed
       }
-      tc::mma_commit(&gb->acc);   // arrives once every MMA issued above has completed
     }
   } else {   // ---- epilogue: warps 2..5
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const bool ok = mbar_wait(&gb->acc, 0, abort, kGemmWaitNs);
-    tc::fence_after_sync();
-    if (!ok && lane == 0) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
-    if (__all_sync(0xffffffffu, ok) && !*abort) {
+    int i = 0;
+    for (int w = blockIdx.x; w < items; w += gridDim.x, ++i) {
+      int n0, m0, z, kb0, kb1;
+      decode(w, n0, m0, z, kb0, kb1);
+      const int buf = i & 1;
+      const bool okw = mbar_wait(&gb->acc_full[buf], (i >> 1) & 1, abort, kGemmWaitNs);
+      tc::fence_after_sync();
+      if (!okw && lane == 0) atomicOr(err, MK_DEVERR_PIPE_TIMEOUT);
+      if (!__all_sync(0xffffffffu, okw) || *abort) break;
+      float* Cz = C;
+      long long ldz = ldc;
+      int accz = accumulate;
+      if (nz > 1) {
+        Cz = ws + static_cast<long long>(z) * M * N;
+        ldz = N;
+        accz = 0;
+      }
       const int m = m0 + row;
-      float* crow = C + static_cast<long long>(m) * ldc + n0;
-      const bool vec = (ldc % 4 == 0) && ((reinterpret_cast<uintptr_t>(C) & 15) == 0);
+      float* crow = Cz + static_cast<long long>(m) * ldz + n0;
+      const bool vec = (ldz % 4 == 0) && ((reinterpret_cast<uintptr_t>(Cz) & 15) == 0);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
         float v[16];
-        tc::tmem_ld16(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+        tc::tmem_ld16(tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
         if (m < M) {
           if (vec && n0 + c0 + 16 <= N) {
             float4* d4 = reinterpret_cast<float4*>(crow + c0);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               float4 o = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-              if (accumulate) {
+              if (accz) {
                 const float4 c = d4[j];
                 o.x += c.x; o.y += c.y; o.z += c.z; o.w += c.w;
               }
@@ -173,17 +218,20 @@ __global__ void __launch_bounds__(192, 1)
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (n0 + c0 + j < N) crow[c0 + j] = accumulate ? crow[c0 + j] + v[j] : v[j];
+              if (n0 + c0 + j < N) crow[c0 + j] = accz ? crow[c0 + j] + v[j] : v[j];
           }
         }
       }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&gb->acc_empty[buf]);
     }
   }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, BN);
+    tc::tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -297,9 +345,10 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
     const long long need = static_cast<long long>(a.M) * a.N;
     while (nz > 1 && need * nz > a.ws_floats) --nz;
   }
-  grid.z = nz;
-  linear_kernel<BN><<<grid, 192, S::kSmemBytes, s>>>(ma_hi, ma_lo, mb, a.c, a.ldc, a.M, a.N, a.K, a.accumulate,
-                                                     a.err, a.ws);
+  const int items = tiles * nz;
+  const int nctas = std::min(items, 148);
+  linear_kernel<BN><<<nctas, 192, S::kSmemBytes, s>>>(ma_hi, ma_lo, mb, a.c, a.ldc, a.M, a.N, a.K, a.accumulate,
+                                                      a.err, a.ws, nz);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && nz > 1) {
     const long long total = static_cast<long long>(a.M) * a.N;
