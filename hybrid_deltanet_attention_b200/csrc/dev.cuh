@@ -113,6 +113,24 @@ __device__ __forceinline__ void red_add_v4(float4* p, float4 v) {
                : "memory");
 }
 
+// Asynchronous global -> shared copies that do not stall the issuing thread. Bytes of the
+// destination past src_bytes are zero-filled (src_bytes 0 writes zeros; src must still be a
+// valid address). Completion is per thread: cp_async_wait<N>() returns once at most N of the
+// thread's committed groups are pending; a block barrier after it publishes the data.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // RoPE angle pos * inv_freq reduced to [-pi, pi] in double, then sin/cos in fp32.
 __device__ __forceinline__ void rope_cs(double ang, float& c, float& s) {
   const double two_pi = 6.283185307179586476925286766559;

@@ -447,16 +447,16 @@ __device__ __forceinline__ void wy_fsub(const WyBufs& b, const float* K, const f
   }
 #pragma unroll
   for (int r = 1; r < CH; ++r) {
-    float acc = x[r];
+    float a0 = x[r], a1 = 0.f, a2 = 0.f, a3 = 0.f;   // four partial chains
 #pragma unroll
     for (int s4 = 0; s4 < r; s4 += 4) {
       const float4 a4 = *reinterpret_cast<const float4*>(A + r * AP + s4);
-      acc = fmaf(-a4.x, x[s4], acc);
-      if (s4 + 1 < r) acc = fmaf(-a4.y, x[s4 + 1], acc);
-      if (s4 + 2 < r) acc = fmaf(-a4.z, x[s4 + 2], acc);
-      if (s4 + 3 < r) acc = fmaf(-a4.w, x[s4 + 3], acc);
+      a0 = fmaf(-a4.x, x[s4], a0);
+      if (s4 + 1 < r) a1 = fmaf(-a4.y, x[s4 + 1], a1);
+      if (s4 + 2 < r) a2 = fmaf(-a4.z, x[s4 + 2], a2);
+      if (s4 + 3 < r) a3 = fmaf(-a4.w, x[s4 + 3], a3);
     }
-    x[r] = acc;
+    x[r] = (a0 + a1) + (a2 + a3);
   }
 #pragma unroll
   for (int r = 0; r < CH; ++r) {
@@ -482,22 +482,21 @@ __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
   const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
   const int qo = h * DK, ko = Hd * DK + h * DK, vo = 2 * Hd * DK + h * DV;
   const int C = 2 * Hd * DK + Hd * DV;
-  for (int idx = tid; idx < kChunk * DK / 4; idx += 256) {
+  for (int idx = tid; idx < kChunk * DK / 4; idx += 256) {   // rows past the prompt read as zero
     const int r = idx / (DK / 4), j4 = idx % (DK / 4);
-    float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), qv = kv;
-    if (r < n) {
-      const float* yr = b.y + static_cast<long long>(t0 + r) * b.ldy;
-      kv = *reinterpret_cast<const float4*>(yr + ko + 4 * j4);
-      qv = *reinterpret_cast<const float4*>(yr + qo + 4 * j4);
-    }
-    *reinterpret_cast<float4*>(K + r * KP + 4 * j4) = kv;
-    *reinterpret_cast<float4*>(Q + r * KP + 4 * j4) = qv;
+    const float* yr = b.y + static_cast<long long>(t0 + min(r, n - 1)) * b.ldy;
+    const uint32_t nb = r < n ? 16u : 0u;
+    cp_async16(K + r * KP + 4 * j4, yr + ko + 4 * j4, nb);
+    cp_async16(Q + r * KP + 4 * j4, yr + qo + 4 * j4, nb);
   }
-  if (tid < kChunk) {
-    const float* yr = b.y + static_cast<long long>(t0 + tid) * b.ldy;
-    g[tid] = tid < n ? yr[C + h] : 0.f;
-    bb[tid] = tid < n ? yr[C + Hd + h] : 0.f;
+  if (tid < 2 * kChunk) {
+    const int r = tid & (kChunk - 1);
+    const float* yr = b.y + static_cast<long long>(t0 + min(r, n - 1)) * b.ldy;
+    if (tid < kChunk) cp_async4(g + r, yr + C + h, r < n ? 4u : 0u);
+    else cp_async4(bb + r, yr + C + Hd + h, r < n ? 4u : 0u);
   }
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
   if (tid < 32) {   // inclusive prefix sum of log a over the chunk (two values per lane)
     float v0 = g[2 * tid], v1 = g[2 * tid + 1];
@@ -569,6 +568,10 @@ __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
   }
 }
 
+// Inputs of one chunk are fetched with cp.async in three groups so that their L2 latency
+// hides behind the previous phase: W, Q, U, gamma and the decay factors of chunk c+1 are
+// issued once chunk c's Delta is formed, P of chunk c+1 once chunk c's outputs are written,
+// and K of chunk c at the top of its own iteration (K is read last, by the state update).
 template <int DK, int DV>
 __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict__ S) {
   constexpr int KP = DK + 4, AP = kChunk + 4, RG = kRowGroup;
@@ -580,49 +583,67 @@ __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict
   float* Pc = Kc + kChunk * KP;               // [64][AP]
   float* DT = Pc + kChunk * AP;               // [16][AP]  Delta^T
   float* Uc = DT + RG * AP;                   // [64][16]
-  float* gm = Uc + kChunk * RG;               // [64]
-  float* dc = gm + kChunk;                    // [64]
+  float* gmb = Uc + kChunk * RG;              // [2][64] gamma, by chunk parity
+  float* dcb = gmb + 2 * kChunk;              // [2][64] e^{g_last - g_r}, by chunk parity
   const int Hd = b.Hd, tid = threadIdx.x;
   const int h = blockIdx.x, i0 = blockIdx.y * RG;
   float* Sg = S + (static_cast<long long>(h) * DV + i0) * DK;
-  for (int idx = tid; idx < RG * DK / 4; idx += 256) {
-    const int i = idx / (DK / 4), j4 = idx % (DK / 4);
-    *reinterpret_cast<float4*>(S0 + i * KP + 4 * j4) = *reinterpret_cast<const float4*>(Sg + i * DK + 4 * j4);
-  }
   const int qo = h * DK, ko = Hd * DK + h * DK;
   const int nch = (b.T + kChunk - 1) / kChunk;
-  const int rg = tid >> 4, ti = tid & 15;       // rows rg + 16 a of the chunk, column ti of the group
-  for (int ch = 0; ch < nch; ++ch) {
-    const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
-    __syncthreads();
+  const bool upd = !b.keep_state;
+  // W, Q, U, gamma, decay of chunk c (rows past the prompt read as zero)
+  auto fetch_wqu = [&](int c) {
+    const int t0 = c * kChunk, n = min(kChunk, b.T - t0);
     for (int idx = tid; idx < kChunk * DK / 4; idx += 256) {
       const int r = idx / (DK / 4), j4 = idx % (DK / 4);
-      float4 wv = make_float4(0.f, 0.f, 0.f, 0.f), qv = wv, kv = wv;
-      if (r < n) {
-        const long long t = t0 + r;
-        wv = *reinterpret_cast<const float4*>(b.w + t * Hd * DK + h * DK + 4 * j4);
-        qv = *reinterpret_cast<const float4*>(b.y + t * b.ldy + qo + 4 * j4);
-        kv = *reinterpret_cast<const float4*>(b.y + t * b.ldy + ko + 4 * j4);
-      }
-      *reinterpret_cast<float4*>(Wc + r * KP + 4 * j4) = wv;
-      *reinterpret_cast<float4*>(Qc + r * KP + 4 * j4) = qv;
-      *reinterpret_cast<float4*>(Kc + r * KP + 4 * j4) = kv;
-    }
-    const float* P = b.p + (static_cast<long long>(ch) * Hd + h) * kChunk * kChunk;
-    for (int idx = tid; idx < kChunk * kChunk / 4; idx += 256) {
-      const int r = idx / (kChunk / 4), s4 = idx % (kChunk / 4);
-      *reinterpret_cast<float4*>(Pc + r * AP + 4 * s4) = *reinterpret_cast<const float4*>(P + r * kChunk + 4 * s4);
+      const long long t = t0 + min(r, n - 1);
+      const uint32_t nb = r < n ? 16u : 0u;
+      cp_async16(Wc + r * KP + 4 * j4, b.w + t * Hd * DK + h * DK + 4 * j4, nb);
+      cp_async16(Qc + r * KP + 4 * j4, b.y + t * b.ldy + qo + 4 * j4, nb);
     }
     {
       const int r = tid >> 2, q4 = tid & 3;   // 64 rows x 4 float4 of U
-      float4 uv = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < n) uv = *reinterpret_cast<const float4*>(b.u + static_cast<long long>(t0 + r) * Hd * DV + h * DV + i0 + 4 * q4);
-      *reinterpret_cast<float4*>(Uc + r * RG + 4 * q4) = uv;
+      const long long t = t0 + min(r, n - 1);
+      cp_async16(Uc + r * RG + 4 * q4, b.u + t * Hd * DV + h * DV + i0 + 4 * q4, r < n ? 16u : 0u);
     }
-    if (tid < kChunk) {
-      gm[tid] = tid < n ? b.gam[static_cast<long long>(t0 + tid) * Hd + h] : 0.f;
-      dc[tid] = tid < n ? b.dec[static_cast<long long>(t0 + tid) * Hd + h] : 0.f;
+    if (tid < 2 * kChunk) {
+      const int r = tid & (kChunk - 1);
+      const long long t = t0 + min(r, n - 1);
+      const uint32_t nb = r < n ? 4u : 0u;
+      if (tid < kChunk) cp_async4(gmb + (c & 1) * kChunk + r, b.gam + t * Hd + h, nb);
+      else cp_async4(dcb + (c & 1) * kChunk + r, b.dec + t * Hd + h, nb);
     }
+  };
+  auto fetch_p = [&](int c) {   // P is stored for all 64 rows of every chunk
+    const float* P = b.p + (static_cast<long long>(c) * Hd + h) * kChunk * kChunk;
+    for (int idx = tid; idx < kChunk * kChunk / 4; idx += 256) {
+      const int r = idx / (kChunk / 4), s4 = idx % (kChunk / 4);
+      cp_async16(Pc + r * AP + 4 * s4, P + r * kChunk + 4 * s4, 16u);
+    }
+  };
+  for (int idx = tid; idx < RG * DK / 4; idx += 256) {
+    const int i = idx / (DK / 4), j4 = idx % (DK / 4);
+    cp_async16(S0 + i * KP + 4 * j4, Sg + i * DK + 4 * j4, 16u);
+  }
+  fetch_wqu(0);
+  cp_async_commit();
+  fetch_p(0);
+  cp_async_commit();
+  const int rg = tid >> 4, ti = tid & 15;       // rows rg + 16 a of the chunk, column ti of the group
+  for (int ch = 0; ch < nch; ++ch) {
+    const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
+    const float* gm = gmb + (ch & 1) * kChunk;
+    const float* dc = dcb + (ch & 1) * kChunk;
+    __syncthreads();   // Kc is free: the previous state update is done
+    if (upd) {
+      for (int idx = tid; idx < kChunk * DK / 4; idx += 256) {
+        const int r = idx / (DK / 4), j4 = idx % (DK / 4);
+        const long long t = t0 + min(r, n - 1);
+        cp_async16(Kc + r * KP + 4 * j4, b.y + t * b.ldy + ko + 4 * j4, r < n ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+    cp_async_wait<2>();   // W, Q, U, gamma, decay of this chunk (and S0 before the first)
     __syncthreads();
     // Delta = U - W S0^T and Q S0^T, rows rg + 16 a, column ti
     float dw[4] = {0.f, 0.f, 0.f, 0.f}, dq[4] = {0.f, 0.f, 0.f, 0.f};
@@ -644,7 +665,10 @@ __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict
       DT[ti * AP + r] = d;
       if (b.save_delta && r < n) b.save_delta[static_cast<long long>(t0 + r) * Hd * DV + h * DV + i0 + ti] = d;
     }
-    __syncthreads();
+    cp_async_wait<1>();   // P of this chunk
+    __syncthreads();      // Delta and P visible; W, Q, U free
+    if (ch + 1 < nch) fetch_wqu(ch + 1);
+    cp_async_commit();
     // o_r = gamma_r (Q S0^T)_r + sum_s P[r][s] Delta_s   (P is zero above the diagonal)
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
@@ -658,13 +682,18 @@ __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict
       }
       if (r < n) b.o[static_cast<long long>(t0 + r) * Hd * DV + h * DV + i0 + ti] = acc;
     }
-    if (b.keep_state) continue;
-    __syncthreads();
-    for (int idx = tid; idx < RG * kChunk; idx += 256) {   // Delta_r scaled by e^{g_{n-1} - g_r}
-      const int i = idx / kChunk, r = idx % kChunk;
-      DT[i * AP + r] *= dc[r];
+    __syncthreads();      // P and the unscaled Delta are consumed
+    if (ch + 1 < nch) fetch_p(ch + 1);
+    cp_async_commit();
+    if (upd) {
+      for (int idx = tid; idx < RG * kChunk; idx += 256) {   // Delta_r scaled by e^{g_{n-1} - g_r}
+        const int i = idx / kChunk, r = idx % kChunk;
+        DT[i * AP + r] *= dc[r];
+      }
     }
+    cp_async_wait<2>();   // K of this chunk
     __syncthreads();
+    if (!upd) continue;
     // S0 <- gamma_{n-1} S0 + sum_r (dec_r Delta_r) k_r^T: row ti2, float4 columns jq, jq + 16, ...
     const float gl = gm[n - 1];
     const int ti2 = tid >> 4, jq = tid & 15;
@@ -689,6 +718,7 @@ __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict
       *reinterpret_cast<float4*>(S0 + ti2 * KP + j) = acc;   // only this thread touches these elements here
     }
   }
+  cp_async_wait<0>();
   __syncthreads();
   if (b.keep_state) return;
   for (int idx = tid; idx < RG * DK / 4; idx += 256) {
@@ -698,11 +728,11 @@ __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict
 }
 
 template <int DK, int DV>
-size_t wy_fast_smem() {
+size_t wy_fast_smem(bool state_pass) {
   const size_t prep = sizeof(float) * (2 * kChunk * (DK + 4) + kChunk * (kChunk + 4) + 2 * kChunk);
   const size_t state = sizeof(float) * (kRowGroup * (DK + 4) + 3 * kChunk * (DK + 4) + kChunk * (kChunk + 4) +
-                                        kRowGroup * (kChunk + 4) + kChunk * kRowGroup + 2 * kChunk);
-  return prep > state ? prep : state;
+                                        kRowGroup * (kChunk + 4) + kChunk * kRowGroup + 4 * kChunk);
+  return state_pass ? state : prep;
 }
 
 size_t wy_prep_smem(int dk, int dv) {
@@ -1031,8 +1061,12 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       float* ring = b.conv_ring + static_cast<size_t>(di) * Wc * C;
       ++di;
       linear(L.w_in, 2LL * H + 16, rows, H, pf.z, rows, 0);
-      dn_prep_wide<<<dim3(T, 2 * Hd + (Hd * dv + 127) / 128 + 1), 128, 0, s>>>(pf.z, rows, b.pos, off, ring, Wc, C, Hd,
-                                                                              dk, dv, L.conv, pf.y, rows);
+      if (T <= 64) {   // few tokens: a (token, vector) grid keeps the GPU busy
+        dn_prep_wide<<<dim3(T, 2 * Hd + (Hd * dv + 127) / 128 + 1), 128, 0, s>>>(pf.z, rows, b.pos, off, ring, Wc, C,
+                                                                                Hd, dk, dv, L.conv, pf.y, rows);
+      } else {
+        dn_prep<<<T, kPT, C * sizeof(float), s>>>(pf.z, rows, b.pos, off, ring, Wc, C, Hd, dk, L.conv, pf.y, rows);
+      }
       chk();
       WyBufs wy{pf.y, rows, pf.u, pf.w, pf.p, pf.gam, pf.dec, pf.o, T, Hd, dk, dv, nullptr, nullptr, nullptr, 0};
       if (vs) {
@@ -1049,14 +1083,14 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         chk();
       }
       const int nch = (T + kChunk - 1) / kChunk;
-      if (dk == 128 && dv == 128) {
-        wy_prep_fast<128, 128><<<dim3(nch, Hd), 256, wy_fast_smem<128, 128>(), s>>>(wy);
+      if (dk == 128 && dv == 128 && rows % 4 == 0) {   // 16-byte rows of q, k
+        wy_prep_fast<128, 128><<<dim3(nch, Hd), 256, wy_fast_smem<128, 128>(false), s>>>(wy);
         chk();
-        wy_state_fast<128, 128><<<dim3(Hd, dv / kRowGroup), 256, wy_fast_smem<128, 128>(), s>>>(wy, S);
-      } else if (dk == 64 && dv == 64) {
-        wy_prep_fast<64, 64><<<dim3(nch, Hd), 256, wy_fast_smem<64, 64>(), s>>>(wy);
+        wy_state_fast<128, 128><<<dim3(Hd, dv / kRowGroup), 256, wy_fast_smem<128, 128>(true), s>>>(wy, S);
+      } else if (dk == 64 && dv == 64 && rows % 4 == 0) {
+        wy_prep_fast<64, 64><<<dim3(nch, Hd), 256, wy_fast_smem<64, 64>(false), s>>>(wy);
         chk();
-        wy_state_fast<64, 64><<<dim3(Hd, dv / kRowGroup), 256, wy_fast_smem<64, 64>(), s>>>(wy, S);
+        wy_state_fast<64, 64><<<dim3(Hd, dv / kRowGroup), 256, wy_fast_smem<64, 64>(true), s>>>(wy, S);
       } else {
         wy_prep<<<dim3(nch, Hd), 256, wy_prep_smem(dk, dv), s>>>(wy);
         chk();
