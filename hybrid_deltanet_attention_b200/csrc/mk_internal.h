@@ -14,7 +14,7 @@ constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kSlotBytes = 65536;
 constexpr int kSlots = 3;
 constexpr int kAttnSub = 64;          // positions per online-softmax sub-block
-constexpr int kResCopies = 8;          // copies of each residual delta (CTA c adds into copy c % 8)
+constexpr int kResCopies = 2;          // copies of each residual delta (CTA c adds into copy c % 2)
 constexpr int kAttnMinChunk = 16;     // smallest split-K chunk of the KV cache
 
 enum LayerKind : int { kDeltaNet = 0, kAttention = 1 };

@@ -35,6 +35,8 @@ struct mk_prefill_ws {
   uint16_t* phi = nullptr;
   uint16_t* plo = nullptr;
   uint16_t* vt = nullptr;
+  // chunked delta rule on the tensor cores: bf16 operand images [chunks][Hd][bytes per image]
+  uint8_t* img = nullptr;
 };
 
 struct mk_prefill_layer {   // K-major copies of the projections the decode kernel keeps transposed

@@ -23,6 +23,7 @@
 #include "dev.cuh"
 #include "mk_internal.h"
 #include "mk_model.h"
+#include "tc.cuh"
 
 namespace mk {
 namespace {
@@ -254,7 +255,38 @@ struct WyBufs {
   float* save_k;     // [T][Hd dk] or null
   float* save_delta; // [T][Hd dv] or null
   int keep_state;
+  // tensor-core state pass: bf16 operand images per (chunk, head), see WyImg; null = fp32 w, p
+  uint8_t* img;
+  int* err;          // device error word (tensor-core state pass)
 };
+
+// Operand images of one (chunk, head) for the tensor-core state pass: bf16 high and low
+// parts of K-major, 128-byte-swizzled tiles (64 bf16 of K per 128-byte row, the layout a
+// 128-byte-swizzled TMA load writes), so that one bulk copy stages each:
+//   A1 [part][dk/64 K blocks][128 rows]: rows 0..63 gamma_r q_r, rows 64..127 w_r (K = dk)
+//   P  [part][64 rows]:  P[r][s] (K = s)
+//   KT [part][128 rows]: row j holds k_r[j] over r (K = r); rows j >= dk are zero
+template <int DK>
+struct WyImg {
+  static constexpr uint32_t kA1 = 2u * (DK / 64) * 16384u;
+  static constexpr uint32_t kP = 2u * 8192u;
+  static constexpr uint32_t kKT = 2u * 16384u;
+  static constexpr uint32_t kBytes = kA1 + kP + kKT;
+};
+
+// Eight floats as bf16 high parts (hi) and the bf16 of the remainders (lo).
+__device__ __forceinline__ void split8_bf16(const float* v, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint16_t h0 = f_to_bf16(v[2 * q]), h1 = f_to_bf16(v[2 * q + 1]);
+    const uint16_t l0 = f_to_bf16(v[2 * q] - bf16_to_f(h0)), l1 = f_to_bf16(v[2 * q + 1] - bf16_to_f(h1));
+    h[q] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+    l[q] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
 
 __global__ void __launch_bounds__(256) wy_prep(WyBufs b) {
   extern __shared__ float sm[];
@@ -429,10 +461,11 @@ __global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S 
 // access patterns below), 4 x 4 output tiles per thread, and the forward substitution on
 // a right-hand-side column held in registers.
 // Forward substitution (I + A) X = RHS for the first CH rows of a chunk (CH >= n), column
-// j of X held in registers; writes the U (j < DV) or W column.
+// j of X held in registers; writes the U (j < DV) or W column (W into wst [64][DK + 4] in
+// shared memory when wst is set).
 template <int CH, int DK, int DV>
 __device__ __forceinline__ void wy_fsub(const WyBufs& b, const float* K, const float* A, const float* g,
-                                        const float* bb, int t0, int n, int h, int j, int vo) {
+                                        const float* bb, int t0, int n, int h, int j, int vo, float* wst) {
   constexpr int KP = DK + 4, AP = kChunk + 4;
   const int Hd = b.Hd;
   float x[CH];
@@ -460,7 +493,9 @@ __device__ __forceinline__ void wy_fsub(const WyBufs& b, const float* K, const f
   }
 #pragma unroll
   for (int r = 0; r < CH; ++r) {
-    if (r < n) {
+    if (j >= DV && wst) {
+      wst[r * KP + (j - DV)] = x[r];   // rows past n are zero
+    } else if (r < n) {
       if (j < DV) b.u[static_cast<long long>(t0 + r) * Hd * DV + h * DV + j] = x[r];
       else b.w[static_cast<long long>(t0 + r) * Hd * DK + h * DK + (j - DV)] = x[r];
     }
@@ -477,6 +512,7 @@ __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
   float* A = Q + kChunk * KP;                 // [64][AP]
   float* g = A + kChunk * AP;                 // [64]
   float* bb = g + kChunk;                     // [64]
+  float* Ps = bb + kChunk;                    // [64][AP] P, staged for the operand images
   const int Hd = b.Hd, tid = threadIdx.x;
   const int ch = blockIdx.x, h = blockIdx.y;
   const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
@@ -546,14 +582,70 @@ __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
         const bool live = r < n;
         const float e = (s2 <= r && live) ? expf(g[r] - g[s2]) : 0.f;
         A[r * AP + s2] = (s2 < r) ? bb[r] * e * akk[a][c] : 0.f;
-        P[r * kChunk + s2] = e * aqk[a][c];
+        if (b.img) Ps[r * AP + s2] = e * aqk[a][c];
+        else P[r * kChunk + s2] = e * aqk[a][c];
       }
   }
   __syncthreads();
+  uint8_t* img = b.img ? b.img + (static_cast<size_t>(ch) * Hd + h) * WyImg<DK>::kBytes : nullptr;
+  if (img) {   // gamma Q (A1 rows 0..63), P, K^T as bf16 high / low tiles
+    constexpr int KB = DK / 64;
+    uint8_t* a1 = img;
+    uint8_t* pi = img + WyImg<DK>::kA1;
+    uint8_t* kt = pi + WyImg<DK>::kP;
+    float v[8];
+    uint4 hv, lv;
+    for (int idx = tid; idx < kChunk * (DK / 8); idx += 256) {
+      const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
+      const float gr = expf(g[r]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = gr * Q[r * KP + 8 * c8 + u];
+      split8_bf16(v, hv, lv);
+      const uint32_t off = r * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4);
+      *reinterpret_cast<uint4*>(a1 + kb * 16384 + off) = hv;
+      *reinterpret_cast<uint4*>(a1 + (KB + kb) * 16384 + off) = lv;
+    }
+    for (int idx = tid; idx < kChunk * 8; idx += 256) {
+      const int r = idx >> 3, c = idx & 7;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = Ps[r * AP + 8 * c + u];
+      split8_bf16(v, hv, lv);
+      const uint32_t off = r * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4);
+      *reinterpret_cast<uint4*>(pi + off) = hv;
+      *reinterpret_cast<uint4*>(pi + 8192 + off) = lv;
+    }
+    for (int idx = tid; idx < 128 * 8; idx += 256) {   // row j of K^T: k_r[j] over the chunk's r
+      const int j = idx & 127, c = idx >> 7;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = j < DK ? K[(8 * c + u) * KP + j] : 0.f;
+      split8_bf16(v, hv, lv);
+      const uint32_t off = j * 128u + ((static_cast<uint32_t>(c) ^ (j & 7u)) << 4);
+      *reinterpret_cast<uint4*>(kt + off) = hv;
+      *reinterpret_cast<uint4*>(kt + 16384 + off) = lv;
+    }
+    __syncthreads();   // Q is consumed: W is staged in its place
+  }
   // (I + A) X = [diag(b) V | diag(b gamma) K]: column j of X in registers
   if (tid < XW) {
-    if (n <= 16) wy_fsub<16, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo);
-    else wy_fsub<kChunk, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo);
+    float* wst = img ? Q : nullptr;
+    if (n <= 16) wy_fsub<16, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo, wst);
+    else wy_fsub<kChunk, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo, wst);
+  }
+  if (img) {   // W (A1 rows 64..127)
+    constexpr int KB = DK / 64;
+    __syncthreads();
+    float v[8];
+    uint4 hv, lv;
+    for (int idx = tid; idx < kChunk * (DK / 8); idx += 256) {
+      const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = r < n ? Q[r * KP + 8 * c8 + u] : 0.f;   // rows past n: zero
+      split8_bf16(v, hv, lv);
+      const uint32_t row = 64u + r;
+      const uint32_t off = row * 128u + ((static_cast<uint32_t>(c) ^ (row & 7u)) << 4);
+      *reinterpret_cast<uint4*>(img + kb * 16384 + off) = hv;
+      *reinterpret_cast<uint4*>(img + (KB + kb) * 16384 + off) = lv;
+    }
   }
   if (tid < n) {
     b.gam[static_cast<long long>(t0 + tid) * Hd + h] = expf(g[tid]);
@@ -727,9 +819,273 @@ __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict
   }
 }
 
+// State pass on the tensor cores (chunks of 64, two or more per pass). CTA (head h, rows
+// i0 .. i0 + 15 of S), 128 threads; thread t owns TMEM lane t. Per chunk, with every
+// product taken as hi*hi + hi*lo + lo*hi of bf16 parts into fp32 (tcgen05.mma, M = 128,
+// N = 16, K = 16):
+//   A: D1 = [gamma Q; W] S0^T                   (lanes 0..63: gamma Q S0^T, 64..127: W S0^T)
+//   Delta = U - W S0^T (lanes 64..127), written as bf16 tiles Delta^T, (dec Delta)^T
+//   B: D1[0..63] += P Delta                     (o; the P tile's M = 128 operand spans the
+//                                                next 64 rows of the image, whose products
+//                                                land in lanes 64..127, which are not read)
+//   C: D3 = gamma_last S0^T + K^T (dec Delta)   (S^T accumulates in TMEM across chunks)
+// then S1 = D3 is copied to the S0 operand tile and pre-scaled by the next chunk's
+// gamma_last. Operand images arrive by bulk copies: A1 of the next chunk as soon as phase
+// A has consumed it, P and K^T two chunks ahead (double buffer); U and the decay factors
+// by cp.async. Every wait has a time limit; on expiry the CTA latches an error and stops.
+struct WyTcBars {
+  uint64_t a1, pk[2], mma;
+  uint32_t tmem;
+  int abort;
+};
+constexpr uint64_t kWyWaitNs = 1000000000ull;
+
+template <int DK>
+constexpr size_t wy_tc_smem() {
+  return WyImg<DK>::kA1 + 2ull * (WyImg<DK>::kP + WyImg<DK>::kKT) + 2ull * (DK / 64) * 2048 + 2 * 4096 +
+         sizeof(float) * (2 * kChunk * kRowGroup + 2 * kChunk + 128) + sizeof(WyTcBars) + 1024;
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restrict__ S) {
+  using I = WyImg<DK>;
+  constexpr int KB = DK / 64, RG = kRowGroup;
+  constexpr uint32_t kPK = I::kP + I::kKT, kB1 = 2u * KB * 2048u;
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(128, 16);
+  extern __shared__ uint8_t wy_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wy_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* A1 = sm;
+  uint8_t* PK0 = A1 + I::kA1;
+  uint8_t* B1 = PK0 + 2 * kPK;
+  uint8_t* B2 = B1 + kB1;
+  uint8_t* B3 = B2 + 4096;
+  float* Ub = reinterpret_cast<float*>(B3 + 4096);   // [2][64][16]
+  float* dcb = Ub + 2 * kChunk * RG;                 // [2][64]
+  float* gl = dcb + 2 * kChunk;                      // [128] gamma at each chunk's last row
+  WyTcBars* bars = reinterpret_cast<WyTcBars*>(gl + 128);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int Hd = b.Hd, h = blockIdx.x, i0 = blockIdx.y * RG;
+  const int nch = (b.T + kChunk - 1) / kChunk;
+  auto img_at = [&](int c) { return b.img + (static_cast<size_t>(c) * Hd + h) * I::kBytes; };
+  volatile int* abort = &bars->abort;
+
+  if (tid == 0) {
+    mbar_init(&bars->a1, 1);
+    mbar_init(&bars->pk[0], 1);
+    mbar_init(&bars->pk[1], 1);
+    mbar_init(&bars->mma, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&bars->tmem, 32);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+  const uint32_t d1 = bars->tmem + lane_off, d3 = bars->tmem + 16 + lane_off;
+
+  int n_a1 = 0, n_pk[2] = {0, 0};   // bulk copies issued per barrier (thread 0)
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&bars->a1, I::kA1);
+    tc::bulk_load(A1, img_at(0), I::kA1, &bars->a1);
+    n_a1 = 1;
+    for (int c = 0; c < 2 && c < nch; ++c) {
+      mbar_arrive_expect_tx(&bars->pk[c], kPK);
+      tc::bulk_load(PK0 + c * kPK, img_at(c) + I::kA1, kPK, &bars->pk[c]);
+      n_pk[c] = 1;
+    }
+  }
+  auto fetch_ud = [&](int c) {   // U columns i0.., decay of chunk c (rows past the prompt read as zero)
+    const int t0 = c * kChunk, n = min(kChunk, b.T - t0);
+    float* U = Ub + (c & 1) * kChunk * RG;
+    for (int idx = tid; idx < kChunk * RG / 4; idx += 128) {
+      const int r = idx >> 2, q4 = idx & 3;
+      const long long t = t0 + min(r, n - 1);
+      cp_async16(U + r * RG + 4 * q4, b.u + t * Hd * DV + h * DV + i0 + 4 * q4, r < n ? 16u : 0u);
+    }
+    if (tid < kChunk) {
+      const long long t = t0 + min(tid, n - 1);
+      cp_async4(dcb + (c & 1) * kChunk + tid, b.dec + t * Hd + h, tid < n ? 4u : 0u);
+    }
+  };
+  fetch_ud(0);
+  cp_async_commit();
+  for (int c = tid; c < nch; c += 128) {
+    const int tl = min(b.T, (c + 1) * kChunk) - 1;
+    gl[c] = b.gam[static_cast<long long>(tl) * Hd + h];
+  }
+  // S0 operand tile (rows i of S, K = dk) from thread j = column j, bf16 high and low parts
+  auto put_s = [&](const float* sv) {
+    if (tid < DK) {
+      const int kb = tid >> 6, kk = tid & 63;
+#pragma unroll
+      for (int i = 0; i < RG; ++i) {
+        const uint16_t hi = f_to_bf16(sv[i]), lo = f_to_bf16(sv[i] - bf16_to_f(hi));
+        const uint32_t off = tc::sw128_offset(i, kk);
+        *reinterpret_cast<uint16_t*>(B1 + kb * 2048 + off) = hi;
+        *reinterpret_cast<uint16_t*>(B1 + (KB + kb) * 2048 + off) = lo;
+      }
+    }
+  };
+  float sv[RG];
+#pragma unroll
+  for (int i = 0; i < RG; ++i)
+    sv[i] = tid < DK ? S[(static_cast<long long>(h) * DV + i0 + i) * DK + tid] : 0.f;
+  __syncthreads();   // gl
+  put_s(sv);
+  {
+    float v[RG];
+#pragma unroll
+    for (int i = 0; i < RG; ++i) v[i] = gl[0] * sv[i];
+    tc::tmem_st16(d3, v);
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+
+  uint32_t mph = 0;
+  for (int ch = 0; ch < nch; ++ch) {
+    const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
+    // ---- A: D1 = [gamma Q; W] S0^T
+    if (tid == 0) {
+      if (!mbar_wait(&bars->a1, ch & 1, abort, kWyWaitNs)) {
+        if (!*abort) atomicOr(b.err, MK_DEVERR_PIPE_TIMEOUT);
+        *abort = 1;
+      } else {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ah = tc::desc_kmajor_sw128(A1 + kb * 16384 + kk * 32);
+            const uint64_t al = tc::desc_kmajor_sw128(A1 + (KB + kb) * 16384 + kk * 32);
+            const uint64_t bh = tc::desc_kmajor_sw128(B1 + kb * 2048 + kk * 32);
+            const uint64_t bl = tc::desc_kmajor_sw128(B1 + (KB + kb) * 2048 + kk * 32);
+            tc::mma_bf16(d1 - lane_off, ah, bh, idesc, (kb | kk) ? 1u : 0u);
+            tc::mma_bf16(d1 - lane_off, ah, bl, idesc, 1u);
+            tc::mma_bf16(d1 - lane_off, al, bh, idesc, 1u);
+          }
+        tc::mma_commit(&bars->mma);
+      }
+    }
+    if (!mbar_wait(&bars->mma, mph, abort, kWyWaitNs)) *abort = 1;
+    mph ^= 1u;
+    tc::fence_after_sync();
+    if (tid == 0 && ch + 1 < nch && !*abort) {   // A1 is consumed: stage the next chunk's
+      mbar_arrive_expect_tx(&bars->a1, I::kA1);
+      tc::bulk_load(A1, img_at(ch + 1), I::kA1, &bars->a1);
+      ++n_a1;
+    }
+    if (ch + 1 < nch) fetch_ud(ch + 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();   // U and the decay factors of this chunk
+    if (*abort) break;
+    // ---- Delta = U - W S0^T; the tiles Delta^T and (dec Delta)^T (row i, K = token r)
+    if (warp >= 2) {
+      const int r = tid - 64;
+      float ws[RG];
+      tc::tmem_ld16(d1, ws);
+      const float* U = Ub + (ch & 1) * kChunk * RG;
+      const float dr = dcb[(ch & 1) * kChunk + r];
+#pragma unroll
+      for (int i = 0; i < RG; ++i) {
+        const float d = U[r * RG + i] - ws[i];
+        const float dd = dr * d;
+        const uint32_t off = tc::sw128_offset(i, r);
+        const uint16_t h1 = f_to_bf16(d), h2 = f_to_bf16(dd);
+        *reinterpret_cast<uint16_t*>(B2 + off) = h1;
+        *reinterpret_cast<uint16_t*>(B2 + 2048 + off) = f_to_bf16(d - bf16_to_f(h1));
+        *reinterpret_cast<uint16_t*>(B3 + off) = h2;
+        *reinterpret_cast<uint16_t*>(B3 + 2048 + off) = f_to_bf16(dd - bf16_to_f(h2));
+      }
+    }
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- B: D1[0..63] += P Delta;  C: D3 += K^T (dec Delta)
+    if (tid == 0) {
+      if (!mbar_wait(&bars->pk[ch & 1], (ch >> 1) & 1, abort, kWyWaitNs)) {
+        if (!*abort) atomicOr(b.err, MK_DEVERR_PIPE_TIMEOUT);
+        *abort = 1;
+      } else {
+        tc::fence_after_sync();
+        const uint8_t* PK = PK0 + (ch & 1) * kPK;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ph = tc::desc_kmajor_sw128(PK + kk * 32);
+          const uint64_t pl = tc::desc_kmajor_sw128(PK + 8192 + kk * 32);
+          const uint64_t dh = tc::desc_kmajor_sw128(B2 + kk * 32);
+          const uint64_t dl = tc::desc_kmajor_sw128(B2 + 2048 + kk * 32);
+          tc::mma_bf16(d1 - lane_off, ph, dh, idesc, 1u);
+          tc::mma_bf16(d1 - lane_off, ph, dl, idesc, 1u);
+          tc::mma_bf16(d1 - lane_off, pl, dh, idesc, 1u);
+          const uint64_t kh = tc::desc_kmajor_sw128(PK + I::kP + kk * 32);
+          const uint64_t kl = tc::desc_kmajor_sw128(PK + I::kP + 16384 + kk * 32);
+          const uint64_t eh = tc::desc_kmajor_sw128(B3 + kk * 32);
+          const uint64_t el = tc::desc_kmajor_sw128(B3 + 2048 + kk * 32);
+          tc::mma_bf16(d3 - lane_off, kh, eh, idesc, 1u);
+          tc::mma_bf16(d3 - lane_off, kh, el, idesc, 1u);
+          tc::mma_bf16(d3 - lane_off, kl, eh, idesc, 1u);
+        }
+        tc::mma_commit(&bars->mma);
+      }
+    }
+    if (!mbar_wait(&bars->mma, mph, abort, kWyWaitNs)) *abort = 1;
+    mph ^= 1u;
+    tc::fence_after_sync();
+    if (tid == 0 && ch + 2 < nch && !*abort) {   // this P / K^T buffer is consumed
+      mbar_arrive_expect_tx(&bars->pk[ch & 1], kPK);
+      tc::bulk_load(PK0 + (ch & 1) * kPK, img_at(ch + 2) + I::kA1, kPK, &bars->pk[ch & 1]);
+      ++n_pk[ch & 1];
+    }
+    __syncthreads();
+    if (*abort) break;
+    // ---- outputs of this chunk (lanes 0..63) and the state after it
+    if (warp < 2) {   // every lane of the warp takes part in the load
+      float o[RG];
+      tc::tmem_ld16(d1, o);
+      if (tid < n) {
+        float4* dst = reinterpret_cast<float4*>(b.o + static_cast<long long>(t0 + tid) * Hd * DV + h * DV + i0);
+#pragma unroll
+        for (int q = 0; q < RG / 4; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+    }
+    tc::tmem_ld16(d3, sv);
+    if (ch + 1 < nch) {
+      put_s(sv);
+      float v[RG];
+#pragma unroll
+      for (int i = 0; i < RG; ++i) v[i] = gl[ch + 1] * sv[i];
+      tc::tmem_st16(d3, v);
+    } else if (tid < DK) {
+#pragma unroll
+      for (int i = 0; i < RG; ++i) S[(static_cast<long long>(h) * DV + i0 + i) * DK + tid] = sv[i];
+    }
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+  }
+  cp_async_wait<0>();
+  if (tid == 0) {   // let issued bulk copies land before the CTA ends (bounded)
+    int never = 0;
+    if (n_a1 > 0) mbar_wait(&bars->a1, (n_a1 - 1) & 1, &never, kWyWaitNs / 5);
+    for (int c = 0; c < 2; ++c)
+      if (n_pk[c] > 0) mbar_wait(&bars->pk[c], (n_pk[c] - 1) & 1, &never, kWyWaitNs / 5);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(bars->tmem, 32);
+}
+
 template <int DK, int DV>
 size_t wy_fast_smem(bool state_pass) {
-  const size_t prep = sizeof(float) * (2 * kChunk * (DK + 4) + kChunk * (kChunk + 4) + 2 * kChunk);
+  const size_t prep = sizeof(float) * (2 * kChunk * (DK + 4) + 2 * kChunk * (kChunk + 4) + 2 * kChunk);
   const size_t state = sizeof(float) * (kRowGroup * (DK + 4) + 3 * kChunk * (DK + 4) + kChunk * (kChunk + 4) +
                                         kRowGroup * (kChunk + 4) + kChunk * kRowGroup + 4 * kChunk);
   return state_pass ? state : prep;
@@ -1083,7 +1439,21 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         chk();
       }
       const int nch = (T + kChunk - 1) / kChunk;
-      if (dk == 128 && dv == 128 && rows % 4 == 0) {   // 16-byte rows of q, k
+      // two or more chunks of a prompt: the state pass on the tensor cores
+      const bool tcs = !vs && pf.img && nch >= 2 && nch <= 128 && dk == dv && (dk == 128 || dk == 64) && rows % 4 == 0;
+      if (tcs) {
+        wy.img = pf.img;
+        wy.err = b.err;
+        if (dk == 128) {
+          wy_prep_fast<128, 128><<<dim3(nch, Hd), 256, wy_fast_smem<128, 128>(false), s>>>(wy);
+          chk();
+          wy_state_tc<128, 128><<<dim3(Hd, dv / kRowGroup), 128, wy_tc_smem<128>(), s>>>(wy, S);
+        } else {
+          wy_prep_fast<64, 64><<<dim3(nch, Hd), 256, wy_fast_smem<64, 64>(false), s>>>(wy);
+          chk();
+          wy_state_tc<64, 64><<<dim3(Hd, dv / kRowGroup), 128, wy_tc_smem<64>(), s>>>(wy, S);
+        }
+      } else if (dk == 128 && dv == 128 && rows % 4 == 0) {   // 16-byte rows of q, k
         wy_prep_fast<128, 128><<<dim3(nch, Hd), 256, wy_fast_smem<128, 128>(false), s>>>(wy);
         chk();
         wy_state_fast<128, 128><<<dim3(Hd, dv / kRowGroup), 256, wy_fast_smem<128, 128>(true), s>>>(wy, S);
@@ -1180,6 +1550,12 @@ cudaError_t set_prefill_smem_limits() {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(wy_state_tc<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(wy_tc_smem<128>()));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(wy_state_tc<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(wy_tc_smem<64>()));
   if (e == cudaSuccess) done = true;
   return e;
 }
