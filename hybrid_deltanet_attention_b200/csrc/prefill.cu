@@ -29,6 +29,7 @@ namespace mk {
 namespace {
 
 constexpr int kPT = 256;    // threads of the row kernels
+constexpr int kPrepMaxConv = 4;   // causal conv width limit (checked at load)
 
 __device__ __forceinline__ float block_sum(float v, float* red) {
   v = warp_sum(v);
@@ -115,6 +116,64 @@ __global__ void dn_prep(const float* __restrict__ z, int ldz, const int* __restr
     yr[C + hh] = -(fmaxf(al, 0.f) + log1pf(expf(-fabsf(al))));
     yr[C + Hd + hh] = sigmoidf_(be);
   }
+}
+
+// The same with one warp per (token, 128-channel block) and four channels per lane
+// (float4 loads of z, the ring and the outputs; C a multiple of 128, dk 64 or 128, row
+// strides multiples of 4 floats). The q / k norms reduce over the dk / 4 lanes of a head
+// with shuffles. CTA = 8 consecutive tokens of one block, so the W overlapping z rows a
+// token reads are mostly L1 hits; block C / 128 holds the gates.
+__global__ void __launch_bounds__(256) dn_prep_v4(const float* __restrict__ z, int ldz, int T,
+                                                  const int* __restrict__ posp, int off, const float* __restrict__ ring,
+                                                  int W, int C, int Hd, int dk, const uint16_t* __restrict__ taps,
+                                                  float* __restrict__ y, int ldy) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  const float* zt = z + static_cast<long long>(t) * ldz;
+  float* yr = y + static_cast<long long>(t) * ldy;
+  if (static_cast<int>(blockIdx.y) * 128 >= C) {   // gates
+    for (int hh = lane; hh < Hd; hh += 32) {
+      const float al = zt[C + hh], be = zt[C + Hd + hh];
+      yr[C + hh] = -(fmaxf(al, 0.f) + log1pf(expf(-fabsf(al))));
+      yr[C + Hd + hh] = sigmoidf_(be);
+    }
+    return;
+  }
+  const int pos0 = *posp + off;
+  const int c0 = blockIdx.y * 128 + 4 * lane;
+  float x[kPrepMaxConv][4];
+#pragma unroll
+  for (int j = 0; j < kPrepMaxConv; ++j) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < W) {
+      const int s = t - (W - 1) + j;
+      if (s >= 0) {
+        v = *reinterpret_cast<const float4*>(z + static_cast<long long>(s) * ldz + c0);
+      } else {
+        const int p = pos0 + s;
+        if (p >= 0) v = *reinterpret_cast<const float4*>(ring + static_cast<long long>(p % W) * C + c0);
+      }
+    }
+    x[j][0] = v.x; x[j][1] = v.y; x[j][2] = v.z; x[j][3] = v.w;
+  }
+  float o[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < kPrepMaxConv; ++j)
+      if (j < W) acc = fmaf(bf16_to_f(taps[static_cast<long long>(c0 + u) * W + j]), x[j][u], acc);
+    o[u] = siluf_(acc);
+  }
+  if (c0 < 2 * Hd * dk) {   // q or k channel: L2 norm over the head (dk / 4 lanes, aligned)
+    float ss = o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3];
+    for (int m = dk / 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+    const float nr = 1.0f / sqrtf(ss + 1e-6f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) o[u] *= nr;
+  }
+  *reinterpret_cast<float4*>(yr + c0) = make_float4(o[0], o[1], o[2], o[3]);
 }
 
 // The same on a (token, vector) grid: vector v < 2 Hd is one q or k head (conv + SiLU +
@@ -1417,7 +1476,10 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       float* ring = b.conv_ring + static_cast<size_t>(di) * Wc * C;
       ++di;
       linear(L.w_in, 2LL * H + 16, rows, H, pf.z, rows, 0);
-      if (T <= 64) {   // few tokens: a (token, vector) grid keeps the GPU busy
+      if (C % 128 == 0 && (dk == 64 || dk == 128) && rows % 4 == 0 && Wc <= kPrepMaxConv) {
+        dn_prep_v4<<<dim3((T + 7) / 8, C / 128 + 1), 256, 0, s>>>(pf.z, rows, T, b.pos, off, ring, Wc, C, Hd, dk, L.conv,
+                                                                   pf.y, rows);
+      } else if (T <= 64) {   // few tokens: a (token, vector) grid keeps the GPU busy
         dn_prep_wide<<<dim3(T, 2 * Hd + (Hd * dv + 127) / 128 + 1), 128, 0, s>>>(pf.z, rows, b.pos, off, ring, Wc, C,
                                                                                 Hd, dk, dv, L.conv, pf.y, rows);
       } else {
