@@ -19,6 +19,8 @@
 #include <cmath>
 #include <string>
 
+#include <cuda_fp16.h>
+
 #include "../../include/mk.h"
 #include "dev.cuh"
 #include "mk_internal.h"
@@ -59,9 +61,10 @@ __global__ void embed_rows(const int32_t* __restrict__ tok, int T, const uint16_
     h[static_cast<long long>(t) * H + i] = ok ? bf16_to_f(embed[static_cast<long long>(id) * H + i]) : 0.f;
 }
 
-// x[t] = h[t] / sqrt(mean(h[t]^2) + eps) * gamma, written as bf16 high/low parts.
+// x[t] = h[t] / sqrt(mean(h[t]^2) + eps) * gamma, written as bf16 high/low parts (and as
+// fp32 into xf when set: the input of the 4-bit linear layers).
 __global__ void rms_split(const float* __restrict__ h, int H, const uint16_t* __restrict__ gamma, float eps,
-                          uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
+                          uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo, float* __restrict__ xf = nullptr) {
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* row = h + static_cast<long long>(t) * H;
@@ -69,8 +72,147 @@ __global__ void rms_split(const float* __restrict__ h, int H, const uint16_t* __
   for (int i = threadIdx.x; i < H; i += blockDim.x) ss += row[i] * row[i];
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / static_cast<float>(H) + eps);
-  for (int i = threadIdx.x; i < H; i += blockDim.x)
-    put_split(xhi, xlo, static_cast<long long>(t) * H + i, row[i] * inv * bf16_to_f(gamma[i]));
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    const float v = row[i] * inv * bf16_to_f(gamma[i]);
+    put_split(xhi, xlo, static_cast<long long>(t) * H + i, v);
+    if (xf) xf[static_cast<long long>(t) * H + i] = v;
+  }
+}
+
+// h[t] = E[tok[t]] for 4-bit embedding rows (w = d sc q - dmin m per 32-weight sub-block).
+__global__ void embed_rows_q4(const int32_t* __restrict__ tok, int T, const uint8_t* __restrict__ embed, int rb,
+                              int H, int V, float* __restrict__ h, int* err) {
+  const int t = blockIdx.x;
+  const int id = tok[t];
+  const bool ok = id >= 0 && id < V;
+  if (!ok && threadIdx.x == 0) atomicOr(err, MK_DEVERR_BAD_TOKEN);
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float v = 0.f;
+    if (ok) {
+      const uint8_t* blk = embed + static_cast<long long>(id) * rb + (i >> 8) * 144;
+      const int e = i & 255, jb = e >> 5, w = e & 31;
+      const uint32_t dd = *reinterpret_cast<const uint32_t*>(blk);
+      const uint64_t lo = static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 4)) |
+                          (static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 8)) << 32);
+      const uint64_t hi = static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 8)) |
+                          (static_cast<uint64_t>(*reinterpret_cast<const uint32_t*>(blk + 12)) << 32);
+      const float sc = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) *
+                       static_cast<float>(static_cast<uint32_t>(lo >> (6 * jb)) & 63u);
+      const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) *
+                       static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * jb)) & 63u);
+      const uint32_t q = (blk[16 + 16 * jb + (w & 15)] >> (4 * (w >> 4))) & 15u;
+      v = fmaf(sc, static_cast<float>(q), -mn);
+    }
+    h[static_cast<long long>(t) * H + i] = v;
+  }
+}
+
+// C[t][n] (+)= sum_k X[t][k] W[n][k] with 4-bit rows W (Q4_K-style 144-byte super-blocks of
+// 256 weights along k: fp16 d, dmin; 6-bit sub-block scales and mins; 4-bit codes) and fp32
+// X [T][K] (row stride ldx). A warp takes RW rows at a time; lane l dequantises the 8
+// weights k = 256 sb + 8 l .. + 7 of every super-block sb of each row and applies them to
+// the TT tokens of its CTA (grid.y walks token tiles), so one load of the activations
+// serves RW rows and the weights are read once per token tile.
+constexpr int kQ4Rows = 4;
+__device__ __forceinline__ void q4_lane_weights(const uint8_t* blk, int jb, int cb, int sh, float* w) {
+  const uint4 hd = *reinterpret_cast<const uint4*>(blk);
+  const uint2 cw = *reinterpret_cast<const uint2*>(blk + cb);
+  const uint64_t lo = static_cast<uint64_t>(hd.y) | (static_cast<uint64_t>(hd.z) << 32);
+  const uint64_t hi = static_cast<uint64_t>(hd.z) | (static_cast<uint64_t>(hd.w) << 32);
+  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu))) *
+                  static_cast<float>(static_cast<uint32_t>(lo >> (6 * jb)) & 63u);
+  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16))) *
+                   static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * jb)) & 63u);
+  // code q as a float: the low mantissa bits of 2^23 + q, minus 2^23 (exact)
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float q0 = __uint_as_float(0x4B000000u | ((cw.x >> (8 * u + sh)) & 15u)) - 8388608.f;
+    const float q1 = __uint_as_float(0x4B000000u | ((cw.y >> (8 * u + sh)) & 15u)) - 8388608.f;
+    w[u] = fmaf(s, q0, -mn);
+    w[4 + u] = fmaf(s, q1, -mn);
+  }
+}
+
+constexpr int kQ4Depth = 6;   // super-blocks per row a warp keeps in flight (cp.async ring)
+
+template <int TT>
+__global__ void __launch_bounds__(256) q4_linear_kernel(const float* __restrict__ X, long long ldx,
+                                                        const uint8_t* __restrict__ W, long long ldw,
+                                                        float* __restrict__ Cm, long long ldc, int T, int N, int K,
+                                                        int accumulate) {
+  constexpr int RW = kQ4Rows, DEP = kQ4Depth, CH = 144 / 16;
+  extern __shared__ __align__(16) uint8_t q4s[];   // per warp: [DEP][RW][144]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = q4s + warp * DEP * RW * 144;
+  const int t0 = blockIdx.y * TT, tn = min(TT, T - t0);
+  const int nsb = K >> 8;
+  const int jb = lane >> 2, q = lane & 3;
+  const int cb = 16 + 16 * jb + 8 * (q & 1);   // this lane's 8 code bytes in a super-block
+  const int sh = 4 * (q >> 1);                 // low (weights 0..15) or high (16..31) nibbles
+  const float* xt = X + static_cast<long long>(t0) * ldx + 8 * lane;
+  for (int n0 = (blockIdx.x * 8 + warp) * RW; n0 < N; n0 += gridDim.x * 8 * RW) {
+    const uint8_t* rows[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r) rows[r] = W + static_cast<long long>(min(n0 + r, N - 1)) * ldw;
+    // the warp's RW rows of super-block sb into ring slot sb % DEP (16-byte pieces over the lanes)
+    auto issue = [&](int sb) {
+      if (sb < nsb) {
+        uint8_t* slot = ring + (sb % DEP) * RW * 144;
+        for (int i = lane; i < RW * CH; i += 32) {
+          const int r = i / CH, c = i % CH;
+          cp_async16(slot + r * 144 + c * 16, rows[r] + sb * 144 + c * 16, 16u);
+        }
+      }
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int p = 0; p < DEP - 1; ++p) issue(p);
+    float acc[RW][TT];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt) acc[r][tt] = 0.f;
+    for (int sb = 0; sb < nsb; ++sb) {
+      issue(sb + DEP - 1);
+      cp_async_wait<DEP - 1>();
+      __syncwarp();
+      const uint8_t* slot = ring + (sb % DEP) * RW * 144;
+      float w[RW][8];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) q4_lane_weights(slot + r * 144, jb, cb, sh, w[r]);
+      const float* xk = xt + sb * 256;
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt) {
+        if (tt < tn) {
+          const float4 a = *reinterpret_cast<const float4*>(xk + tt * ldx);
+          const float4 c = *reinterpret_cast<const float4*>(xk + tt * ldx + 4);
+#pragma unroll
+          for (int r = 0; r < RW; ++r) {
+            float v = acc[r][tt];
+            v = fmaf(w[r][0], a.x, v); v = fmaf(w[r][1], a.y, v); v = fmaf(w[r][2], a.z, v); v = fmaf(w[r][3], a.w, v);
+            v = fmaf(w[r][4], c.x, v); v = fmaf(w[r][5], c.y, v); v = fmaf(w[r][6], c.z, v); v = fmaf(w[r][7], c.w, v);
+            acc[r][tt] = v;
+          }
+        }
+      }
+      __syncwarp();   // every lane is done with this slot before it is refilled
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+      float mine = 0.f;
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt) {
+        const float v = warp_sum(acc[r][tt]);
+        if (lane == tt) mine = v;
+      }
+      if (lane < tn && n0 + r < N) {
+        float* dst = Cm + static_cast<long long>(t0 + lane) * ldc + n0 + r;
+        *dst = accumulate ? *dst + mine : mine;
+      }
+    }
+  }
 }
 
 // DeltaNet token prep. z[t] = [q~ k~ v~ (C channels) | alpha (Hd) | beta (Hd)].
@@ -267,23 +409,28 @@ __global__ void at_prep(const float* __restrict__ z, int ldz, const int* __restr
   }
 }
 
-// x = o (* sigmoid(gate) when gate != null), as bf16 high/low parts [T][n].
+// x = o (* sigmoid(gate) when gate != null), as bf16 high/low parts [T][n] (and fp32 in xf).
 __global__ void gate_split(const float* __restrict__ o, int ldo, const float* __restrict__ gate, int ldg, int n,
-                           uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
+                           uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo, float* __restrict__ xf = nullptr) {
   const int t = blockIdx.x;
   for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < n; i += gridDim.y * blockDim.x) {
     float v = o[static_cast<long long>(t) * ldo + i];
     if (gate) v *= sigmoidf_(gate[static_cast<long long>(t) * ldg + i]);
     put_split(xhi, xlo, static_cast<long long>(t) * n + i, v);
+    if (xf) xf[static_cast<long long>(t) * n + i] = v;
   }
 }
 
-// act = SiLU(g) * u from gu[t] = [g (F) | u (F)], as bf16 high/low parts [T][F].
-__global__ void act_split(const float* __restrict__ gu, int F, uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
+// act = SiLU(g) * u from gu[t] = [g (F) | u (F)], as bf16 high/low parts [T][F] (and fp32 in xf).
+__global__ void act_split(const float* __restrict__ gu, int F, uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo,
+                          float* __restrict__ xf = nullptr) {
   const int t = blockIdx.x;
   const float* r = gu + static_cast<long long>(t) * 2 * F;
-  for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < F; i += gridDim.y * blockDim.x)
-    put_split(xhi, xlo, static_cast<long long>(t) * F + i, siluf_(r[i]) * r[F + i]);
+  for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < F; i += gridDim.y * blockDim.x) {
+    const float v = siluf_(r[i]) * r[F + i];
+    put_split(xhi, xlo, static_cast<long long>(t) * F + i, v);
+    if (xf) xf[static_cast<long long>(t) * F + i] = v;
+  }
 }
 
 // ------------------------------------------------------------------ chunked delta rule
@@ -1443,6 +1590,19 @@ __global__ void accept_prefix(const int* tokens, const unsigned long long* best,
 // One pass of every layer over T tokens at device position *pos + off. With vs (a verify
 // pass, T <= 64) the DeltaNet layers keep their state and conv history untouched and
 // save what the commit of an accepted prefix needs.
+// Row bytes of a 4-bit matrix with K inputs (K a multiple of 256).
+inline long long q4_row_bytes(long long K) { return (K / 256) * 144; }
+
+cudaError_t launch_q4_linear(const float* X, long long ldx, const void* W, long long ldw, float* C, long long ldc,
+                             int T, int N, int K, int accumulate, cudaStream_t s) {
+  if (T <= 0 || N <= 0) return cudaSuccess;
+  const int gx = std::min((N + 8 * kQ4Rows - 1) / (8 * kQ4Rows), 1184);
+  constexpr size_t smem = 8ull * kQ4Depth * kQ4Rows * 144;
+  q4_linear_kernel<8><<<dim3(gx, (T + 7) / 8), 256, smem, s>>>(X, ldx, static_cast<const uint8_t*>(W), ldw, C, ldc, T,
+                                                                N, K, accumulate);
+  return cudaGetLastError();
+}
+
 cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaStream_t s,
                          const mk_verify_ws* vs = nullptr) {
   const mk_config& c = m->cfg;
@@ -1456,19 +1616,29 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
     if (e == cudaSuccess) e = cudaGetLastError();
     ++m->launches;
   };
+  const bool q4 = b.q4 != 0;   // 4-bit weights: linear layers on the CUDA cores from fp32 inputs (pf.xf)
+  float* xf = q4 ? pf.xf : nullptr;
+  // ldw is the bf16 row stride; 4-bit rows take (K / 256) * 144 bytes plus the same tail
   auto linear = [&](const void* w, long long ldw, int N, int K, float* out, long long ldc, int acc) {
     if (e != cudaSuccess) return;
-    LinearArgs a{pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, b.err, pf.splitk, kSplitKFloats};
-    e = launch_linear(a, s);
+    if (q4) {
+      e = launch_q4_linear(pf.xf, K, w, q4_row_bytes(K) + (ldw - 2LL * K), out, ldc, T, N, K, acc, s);
+    } else {
+      LinearArgs a{pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, b.err, pf.splitk, kSplitKFloats};
+      e = launch_linear(a, s);
+    }
     ++m->launches;
   };
-  embed_rows<<<T, kPT, 0, s>>>(tok, T, reinterpret_cast<const uint16_t*>(b.embed), H, c.vocab, pf.h, b.err);
+  if (q4)
+    embed_rows_q4<<<T, kPT, 0, s>>>(tok, T, b.embed, b.row_bytes, H, c.vocab, pf.h, b.err);
+  else
+    embed_rows<<<T, kPT, 0, s>>>(tok, T, reinterpret_cast<const uint16_t*>(b.embed), H, c.vocab, pf.h, b.err);
   chk();
   int di = 0, ai = 0;
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     const LayerW& L = m->layers_host[l];
     const mk_prefill_layer& PL = m->pf_layers[l];
-    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm1, b.eps, pf.xhi, pf.xlo);
+    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm1, b.eps, pf.xhi, pf.xlo, xf);
     chk();
     if (L.kind == kDeltaNet) {
       const int rows = C + 2 * Hd;
@@ -1529,9 +1699,10 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         wy_state<<<dim3(Hd, dv / kRowGroup), 256, wy_state_smem(dk), s>>>(wy, S);
       }
       chk();
-      gate_split<<<dim3(T, (Hd * dv + 1023) / 1024), kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo);
+      gate_split<<<dim3(T, (Hd * dv + 1023) / 1024), kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo,
+                                                                   xf);
       chk();
-      linear(PL.w_out, 2LL * Hd * dv, H, Hd * dv, pf.h, H, 1);
+      linear(q4 ? L.w_out_q4 : PL.w_out, 2LL * Hd * dv, H, Hd * dv, pf.h, H, 1);
     } else {
       const int rows = b.at_in_rows;
       uint16_t* kc = b.kc + static_cast<size_t>(ai) * Hkv * c.max_ctx * D;
@@ -1583,18 +1754,18 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         }
       }
       gate_split<<<dim3(T, (qd + 1023) / 1024), kPT, 0, s>>>(pf.o, qd, c.at_out_gate ? pf.z + qd : nullptr, rows, qd,
-                                                             pf.xhi, pf.xlo);
+                                                             pf.xhi, pf.xlo, xf);
       chk();
-      linear(PL.w_out, 2LL * qd, H, qd, pf.h, H, 1);
+      linear(q4 ? L.w_out_q4 : PL.w_out, 2LL * qd, H, qd, pf.h, H, 1);
     }
     if (e != cudaSuccess) break;
-    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm2, b.eps, pf.xhi, pf.xlo);
+    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm2, b.eps, pf.xhi, pf.xlo, xf);
     chk();
     linear(L.w_gate, 2LL * H, F, H, pf.z, 2LL * F, 0);
     linear(L.w_up, 2LL * H, F, H, pf.z + F, 2LL * F, 0);
-    act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
+    act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo, xf);
     chk();
-    linear(PL.w_down, 2LL * F, H, F, pf.h, H, 1);
+    linear(q4 ? L.w_down_q4 : PL.w_down, 2LL * F, H, F, pf.h, H, 1);
   }
   return e;
 }
@@ -1676,10 +1847,14 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
   // 2. final norm, LM head on the tensor cores for all K + 1 positions, greedy tokens
   float* logits = d_logits ? d_logits : vs.logits;
   if (e == cudaSuccess) {
-    mk::rms_split<<<T, mk::kPT, 0, s>>>(m->pf.h, c.hidden, b.norm_f, b.eps, m->pf.xhi, m->pf.xlo);
+    mk::rms_split<<<T, mk::kPT, 0, s>>>(m->pf.h, c.hidden, b.norm_f, b.eps, m->pf.xhi, m->pf.xlo,
+                                         b.q4 ? m->pf.xf : nullptr);
     chk();
   }
-  if (e == cudaSuccess) {
+  if (e == cudaSuccess && b.q4) {   // 4-bit tied LM head
+    e = mk::launch_q4_linear(m->pf.xf, c.hidden, b.embed, b.row_bytes, logits, c.vocab, T, c.vocab, c.hidden, 0, s);
+    ++m->launches;
+  } else if (e == cudaSuccess) {
     mk::LinearArgs a{m->pf.xhi, m->pf.xlo, b.embed, 2LL * c.hidden, logits, c.vocab, T, c.vocab, c.hidden, 0, b.err};
     e = mk::launch_linear(a, s);
     ++m->launches;

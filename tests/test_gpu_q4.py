@@ -98,3 +98,46 @@ def test_tiny_q4_verify_matches_oracle():
         assert list(out.cpu().numpy()[:n_or + 1]) == list(committed)
         assert np.abs(logits.cpu().numpy() - z_or).max() <= LOGIT_MAX_ABS
         last = int(committed[-1])
+
+
+def test_mid_q4_batched_prefill_two_passes():
+    """A 70-token prompt on the mid-size 4-bit model: two batched passes (64 + 5 tokens,
+    4-bit linear layers on 8-token tiles) and the last token through the decode kernel."""
+    cfg = synth.MID_Q4
+    m, W = _setup(cfg, 128)
+    _teacher_forced(cfg, m, W, 70, 2, 128)
+
+
+def test_mid_q4_verify_one_pass():
+    """Speculative verify with 4-bit weights: K + 1 tokens in one pass over the weights,
+    acceptance and the DeltaNet state committed to the accepted prefix."""
+    cfg = synth.MID_Q4
+    m, W = _setup(cfg, 128, max_draft=5)
+    dev = torch.device("cuda")
+    K = 5
+    prompt = synth.make_prompt(cfg, 24, tag="q4mv")
+    m.reset()
+    st = oracle.new_state(cfg, 128)
+    oracle.prefill(cfg, W, st, prompt[:-1])
+    m.prefill(torch.from_numpy(prompt[:-1]).to(dev))
+    last = int(prompt[-1])
+    for ps in range(2):
+        greedy, _ = oracle.greedy_generate(cfg, W, st.copy(), last, K)
+        use, ids = synth.draft_choices(4, ps, K, cfg.vocab)
+        if ps == 0:
+            use[:] = True
+        drafts = synth.compose_drafts(greedy, use, ids, cfg.vocab)
+        n_or, committed, z_or = oracle.verify_drafts(cfg, W, st, last, drafts)
+        toks = torch.from_numpy(np.concatenate([[last], drafts]).astype(np.int32)).to(dev)
+        n_acc = torch.zeros(1, dtype=torch.int32, device=dev)
+        out = torch.full((K + 1,), -1, dtype=torch.int32, device=dev)
+        logits = torch.empty((K + 1, cfg.vocab), dtype=torch.float32, device=dev)
+        m.verify(toks, n_acc, out, logits)
+        assert m.sync() == 0
+        assert int(n_acc.item()) == n_or
+        assert list(out.cpu().numpy()[:n_or + 1]) == list(committed)
+        assert np.abs(logits.cpu().numpy() - z_or).max() <= LOGIT_MAX_ABS
+        S = m.S.cpu().numpy()
+        assert max(rel_frob(S[li], st.S[li]) for li in range(cfg.n_dn)) <= STATE_REL_FROB
+        assert int(m.pos_tensor.item()) == st.pos
+        last = int(committed[-1])
