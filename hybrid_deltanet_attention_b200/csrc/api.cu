@@ -238,7 +238,7 @@ struct Layout {
   // batched prefill workspace
   int pf_rows;
   size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec, pf_apart, pf_splitk, pf_best;
-  size_t pf_sbuf, pf_phi, pf_plo, pf_vt, pf_img = 0, pf_xf = 0;
+  size_t pf_sbuf, pf_phi, pf_plo, pf_vt, pf_img = 0;
   long long pf_nk;
   // batched verify saves
   int vf_rows;
@@ -368,7 +368,6 @@ Layout make_layout(const mk_config& c, int grid) {
                              (static_cast<size_t>(c.at_head_dim) + 2) * 4);
     L.pf_splitk = off; off = align256(off + static_cast<size_t>(mk::kSplitKFloats) * 4);
     L.pf_best = off; off = align256(off + T * 8);
-    if (is_q4(c)) { L.pf_xf = off; off = align256(off + T * kmax * 4); }
     if (nd > 0 && c.dn_dk == c.dn_dv && (c.dn_dk == 128 || c.dn_dk == 64)) {   // tensor-core chunked delta rule
       const size_t img = 2ull * (c.dn_dk / 64) * 16384 + 16384 + 32768;     // operand images per (chunk, head)
       L.pf_img = off; off = align256(off + nch * c.dn_heads * img);
@@ -730,7 +729,6 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     m->pf.best = reinterpret_cast<unsigned long long*>(W + L.pf_best);
     m->pf.nk_max = L.pf_nk;
     if (L.pf_img) m->pf.img = W + L.pf_img;
-    if (L.pf_xf) m->pf.xf = reinterpret_cast<float*>(W + L.pf_xf);
     if (L.pf_nk > 0) {
       m->pf.sbuf = reinterpret_cast<float*>(W + L.pf_sbuf);
       m->pf.phi = reinterpret_cast<uint16_t*>(W + L.pf_phi);

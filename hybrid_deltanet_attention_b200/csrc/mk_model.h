@@ -36,8 +36,7 @@ struct mk_prefill_ws {
   uint16_t* plo = nullptr;
   uint16_t* vt = nullptr;
   // chunked delta rule on the tensor cores: bf16 operand images [chunks][Hd][bytes per image]
-  uint8_t* img = nullptr;  float* xf = nullptr;       // [rows][Kmax] fp32 inputs of the 4-bit linear layers
-};
+  uint8_t* img = nullptr;};
 
 struct mk_prefill_layer {   // K-major copies of the projections the decode kernel keeps transposed
   const uint8_t* w_out;      // [H][K_mix] bf16

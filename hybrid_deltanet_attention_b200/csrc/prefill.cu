@@ -33,6 +33,9 @@ namespace {
 constexpr int kPT = 256;    // threads of the row kernels
 constexpr int kPrepMaxConv = 4;   // causal conv width limit (checked at load)
 
+// Threads of a row kernel: wide CTAs when a pass has few rows (verify, short tails).
+inline int rms_threads(int T) { return T < 64 ? 1024 : kPT; }
+
 __device__ __forceinline__ float block_sum(float v, float* red) {
   v = warp_sum(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -61,10 +64,9 @@ __global__ void embed_rows(const int32_t* __restrict__ tok, int T, const uint16_
     h[static_cast<long long>(t) * H + i] = ok ? bf16_to_f(embed[static_cast<long long>(id) * H + i]) : 0.f;
 }
 
-// x[t] = h[t] / sqrt(mean(h[t]^2) + eps) * gamma, written as bf16 high/low parts (and as
-// fp32 into xf when set: the input of the 4-bit linear layers).
+// x[t] = h[t] / sqrt(mean(h[t]^2) + eps) * gamma, written as bf16 high/low parts.
 __global__ void rms_split(const float* __restrict__ h, int H, const uint16_t* __restrict__ gamma, float eps,
-                          uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo, float* __restrict__ xf = nullptr) {
+                          uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* row = h + static_cast<long long>(t) * H;
@@ -75,7 +77,6 @@ __global__ void rms_split(const float* __restrict__ h, int H, const uint16_t* __
   for (int i = threadIdx.x; i < H; i += blockDim.x) {
     const float v = row[i] * inv * bf16_to_f(gamma[i]);
     put_split(xhi, xlo, static_cast<long long>(t) * H + i, v);
-    if (xf) xf[static_cast<long long>(t) * H + i] = v;
   }
 }
 
@@ -108,110 +109,165 @@ __global__ void embed_rows_q4(const int32_t* __restrict__ tok, int T, const uint
 }
 
 // C[t][n] (+)= sum_k X[t][k] W[n][k] with 4-bit rows W (Q4_K-style 144-byte super-blocks of
-// 256 weights along k: fp16 d, dmin; 6-bit sub-block scales and mins; 4-bit codes) and fp32
-// X [T][K] (row stride ldx). A warp takes RW rows at a time; lane l dequantises the 8
-// weights k = 256 sb + 8 l .. + 7 of every super-block sb of each row and applies them to
-// the TT tokens of its CTA (grid.y walks token tiles), so one load of the activations
-// serves RW rows and the weights are read once per token tile.
-constexpr int kQ4Rows = 4;
-__device__ __forceinline__ void q4_lane_weights(const uint8_t* blk, int jb, int cb, int sh, float* w) {
-  const uint4 hd = *reinterpret_cast<const uint4*>(blk);
-  const uint2 cw = *reinterpret_cast<const uint2*>(blk + cb);
-  const uint64_t lo = static_cast<uint64_t>(hd.y) | (static_cast<uint64_t>(hd.z) << 32);
-  const uint64_t hi = static_cast<uint64_t>(hd.z) | (static_cast<uint64_t>(hd.w) << 32);
-  const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu))) *
-                  static_cast<float>(static_cast<uint32_t>(lo >> (6 * jb)) & 63u);
-  const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16))) *
-                   static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * jb)) & 63u);
-  // code q as a float: the low mantissa bits of 2^23 + q, minus 2^23 (exact)
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float q0 = __uint_as_float(0x4B000000u | ((cw.x >> (8 * u + sh)) & 15u)) - 8388608.f;
-    const float q1 = __uint_as_float(0x4B000000u | ((cw.y >> (8 * u + sh)) & 15u)) - 8388608.f;
-    w[u] = fmaf(s, q0, -mn);
-    w[4 + u] = fmaf(s, q1, -mn);
-  }
+// 256 weights along k: fp16 d, dmin; 6-bit sub-block scales sc_j and mins m_j; 4-bit codes
+// q, w = d sc_j q - dmin m_j) for up to 8 tokens per CTA, on the tensor cores with
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate): the 32 weights of a sub-block enter as the
+// exact bf16 values 128 + q, the tokens' activations as their bf16 high and low parts, so
+//   sum_k w_k x_k = d sc_j (D_j - 128 X_j) - dmin m_j X_j,   D_j = sum_k (128 + q_k) x_k,
+// with X_j = sum_k x_k over the sub-block taken by the same MMA against a tile of ones.
+// A warp owns 32 rows (two m16 groups) and a slice of super-blocks (grid.y splits K when
+// the rows alone leave the GPU idle; partial sums go to a workspace and are reduced in a
+// fixed order); its rows stream through a private cp.async ring of 3 super-blocks.
+// Token tile: grid.z (8 tokens each).
+constexpr int kQ4Depth = 3;
+__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// bytes [b0, b1] of a code pair -> bf16x2 (128 + q(b0), 128 + q(b1)) of the low (hi4 = 0) or
+// high (hi4 = 1) nibbles
+__device__ __forceinline__ uint32_t q4_pair_bf16(uint32_t spread, int hi4) {
+  return ((hi4 ? (spread >> 4) : spread) & 0x000F000Fu) | 0x43004300u;
 }
 
-constexpr int kQ4Depth = 6;   // super-blocks per row a warp keeps in flight (cp.async ring)
-
-template <int TT>
-__global__ void __launch_bounds__(256) q4_linear_kernel(const float* __restrict__ X, long long ldx,
-                                                        const uint8_t* __restrict__ W, long long ldw,
-                                                        float* __restrict__ Cm, long long ldc, int T, int N, int K,
-                                                        int accumulate) {
-  constexpr int RW = kQ4Rows, DEP = kQ4Depth, CH = 144 / 16;
-  extern __shared__ __align__(16) uint8_t q4s[];   // per warp: [DEP][RW][144]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* ring = q4s + warp * DEP * RW * 144;
-  const int t0 = blockIdx.y * TT, tn = min(TT, T - t0);
+__global__ void __launch_bounds__(128) q4_linear_mma(const uint16_t* __restrict__ xhi, const uint16_t* __restrict__ xlo,
+                                                     int ldx, const uint8_t* __restrict__ W, long long ldw,
+                                                     float* __restrict__ out, long long ldo, int T, int N, int K,
+                                                     int sb_per_split, int accumulate) {
+  constexpr int DEP = kQ4Depth, CH = 144 / 16, RPW = 32;
+  extern __shared__ __align__(16) uint8_t q4m[];   // per warp: [DEP][32 rows][144]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  uint8_t* ring = q4m + warp * DEP * RPW * 144;
+  const int n0 = blockIdx.x * 128 + warp * RPW;
   const int nsb = K >> 8;
-  const int jb = lane >> 2, q = lane & 3;
-  const int cb = 16 + 16 * jb + 8 * (q & 1);   // this lane's 8 code bytes in a super-block
-  const int sh = 4 * (q >> 1);                 // low (weights 0..15) or high (16..31) nibbles
-  const float* xt = X + static_cast<long long>(t0) * ldx + 8 * lane;
-  for (int n0 = (blockIdx.x * 8 + warp) * RW; n0 < N; n0 += gridDim.x * 8 * RW) {
-    const uint8_t* rows[RW];
+  const int sbA = blockIdx.y * sb_per_split, sbB = min(nsb, sbA + sb_per_split);
+  const int t0 = blockIdx.z * 8;
+  const bool tok_ok = t0 + g < T;   // this lane's B column (token t0 + g)
+  const uint16_t* xh = xhi + static_cast<long long>(tok_ok ? t0 + g : 0) * ldx + 2 * c;
+  const uint16_t* xl = xlo + static_cast<long long>(tok_ok ? t0 + g : 0) * ldx + 2 * c;
+  const uint8_t* rowp[CH];   // the 16-byte pieces this lane copies: i = lane + 32 m of 32 rows x 9
+  int rowo[CH];
 #pragma unroll
-    for (int r = 0; r < RW; ++r) rows[r] = W + static_cast<long long>(min(n0 + r, N - 1)) * ldw;
-    // the warp's RW rows of super-block sb into ring slot sb % DEP (16-byte pieces over the lanes)
-    auto issue = [&](int sb) {
-      if (sb < nsb) {
-        uint8_t* slot = ring + (sb % DEP) * RW * 144;
-        for (int i = lane; i < RW * CH; i += 32) {
-          const int r = i / CH, c = i % CH;
-          cp_async16(slot + r * 144 + c * 16, rows[r] + sb * 144 + c * 16, 16u);
-        }
-      }
-      cp_async_commit();
-    };
+  for (int m = 0; m < CH; ++m) {
+    const int i = lane + 32 * m, r = i / CH, ch = i % CH;
+    rowp[m] = W + static_cast<long long>(min(n0 + r, N - 1)) * ldw + ch * 16;
+    rowo[m] = r * 144 + ch * 16;
+  }
+  auto issue = [&](int sb) {
+    if (sb < sbB) {
+      uint8_t* slot = ring + ((sb - sbA) % DEP) * RPW * 144;
 #pragma unroll
-    for (int p = 0; p < DEP - 1; ++p) issue(p);
-    float acc[RW][TT];
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-#pragma unroll
-      for (int tt = 0; tt < TT; ++tt) acc[r][tt] = 0.f;
-    for (int sb = 0; sb < nsb; ++sb) {
-      issue(sb + DEP - 1);
-      cp_async_wait<DEP - 1>();
-      __syncwarp();
-      const uint8_t* slot = ring + (sb % DEP) * RW * 144;
-      float w[RW][8];
-#pragma unroll
-      for (int r = 0; r < RW; ++r) q4_lane_weights(slot + r * 144, jb, cb, sh, w[r]);
-      const float* xk = xt + sb * 256;
-#pragma unroll
-      for (int tt = 0; tt < TT; ++tt) {
-        if (tt < tn) {
-          const float4 a = *reinterpret_cast<const float4*>(xk + tt * ldx);
-          const float4 c = *reinterpret_cast<const float4*>(xk + tt * ldx + 4);
-#pragma unroll
-          for (int r = 0; r < RW; ++r) {
-            float v = acc[r][tt];
-            v = fmaf(w[r][0], a.x, v); v = fmaf(w[r][1], a.y, v); v = fmaf(w[r][2], a.z, v); v = fmaf(w[r][3], a.w, v);
-            v = fmaf(w[r][4], c.x, v); v = fmaf(w[r][5], c.y, v); v = fmaf(w[r][6], c.z, v); v = fmaf(w[r][7], c.w, v);
-            acc[r][tt] = v;
-          }
-        }
-      }
-      __syncwarp();   // every lane is done with this slot before it is refilled
+      for (int m = 0; m < CH; ++m) cp_async16(slot + rowo[m], rowp[m] + static_cast<long long>(sb) * 144, 16u);
     }
-    cp_async_wait<0>();
+    cp_async_commit();
+  };
+  if (n0 < N) {
+#pragma unroll
+    for (int p = 0; p < DEP - 1; ++p) issue(sbA + p);
+  }
+  float acc[2][4];
+#pragma unroll
+  for (int gr = 0; gr < 2; ++gr)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[gr][i] = 0.f;
+  const uint32_t ones = 0x3F803F80u;   // bf16 1.0, 1.0
+  for (int sb = sbA; sb < sbB && n0 < N; ++sb) {
+    issue(sb + DEP - 1);
+    cp_async_wait<DEP - 1>();
     __syncwarp();
+    const uint8_t* slot = ring + ((sb - sbA) % DEP) * RPW * 144;
+    // my rows: rr = 0..3 -> row 16 (rr >> 1) + 8 (rr & 1) + g of the warp's 32
+    const uint8_t* rb[4];
+    uint4 hd[4];
 #pragma unroll
-    for (int r = 0; r < RW; ++r) {
-      float mine = 0.f;
+    for (int rr = 0; rr < 4; ++rr) {
+      rb[rr] = slot + ((rr >> 1) * 16 + (rr & 1) * 8 + g) * 144;
+      hd[rr] = *reinterpret_cast<const uint4*>(rb[rr]);
+    }
 #pragma unroll
-      for (int tt = 0; tt < TT; ++tt) {
-        const float v = warp_sum(acc[r][tt]);
-        if (lane == tt) mine = v;
+    for (int j = 0; j < 8; ++j) {
+      // codes of sub-block j: bytes (2c, 2c+1) and (2c+8, 2c+9) of each row, spread to [b0, 0, b1, 0]
+      uint32_t sp[4][2];
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const uint32_t w0 = *reinterpret_cast<const uint16_t*>(rb[rr] + 16 + 16 * j + 2 * c);
+        const uint32_t w1 = *reinterpret_cast<const uint16_t*>(rb[rr] + 16 + 16 * j + 2 * c + 8);
+        sp[rr][0] = __byte_perm(w0, 0u, 0x4140);
+        sp[rr][1] = __byte_perm(w1, 0u, 0x4140);
       }
-      if (lane < tn && n0 + r < N) {
-        float* dst = Cm + static_cast<long long>(t0 + lane) * ldc + n0 + r;
-        *dst = accumulate ? *dst + mine : mine;
+      float dq[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}}, dx[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {   // k-step: weights 16 h .. 16 h + 15 of the sub-block
+        const int kb = sb * 256 + 32 * j + 16 * h;
+        uint32_t bh0 = *reinterpret_cast<const uint32_t*>(xh + kb), bh1 = *reinterpret_cast<const uint32_t*>(xh + kb + 8);
+        uint32_t bl0 = *reinterpret_cast<const uint32_t*>(xl + kb), bl1 = *reinterpret_cast<const uint32_t*>(xl + kb + 8);
+        if (!tok_ok) bh0 = bh1 = bl0 = bl1 = 0u;
+#pragma unroll
+        for (int gr = 0; gr < 2; ++gr) {
+          const uint32_t a0 = q4_pair_bf16(sp[2 * gr][0], h), a1 = q4_pair_bf16(sp[2 * gr + 1][0], h);
+          const uint32_t a2 = q4_pair_bf16(sp[2 * gr][1], h), a3 = q4_pair_bf16(sp[2 * gr + 1][1], h);
+          mma_bf16_16816(dq[gr], a0, a1, a2, a3, bh0, bh1);
+          mma_bf16_16816(dq[gr], a0, a1, a2, a3, bl0, bl1);
+        }
+        mma_bf16_16816(dx, ones, ones, ones, ones, bh0, bh1);
+        mma_bf16_16816(dx, ones, ones, ones, ones, bl0, bl1);
+      }
+      // scales of sub-block j for my 4 rows, then acc += s (D - 128 X) - mn X
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const uint64_t lo = static_cast<uint64_t>(hd[rr].y) | (static_cast<uint64_t>(hd[rr].z) << 32);
+        const uint64_t hi = static_cast<uint64_t>(hd[rr].z) | (static_cast<uint64_t>(hd[rr].w) << 32);
+        const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(hd[rr].x & 0xFFFFu))) *
+                        static_cast<float>(static_cast<uint32_t>(lo >> (6 * j)) & 63u);
+        const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(hd[rr].x >> 16))) *
+                         static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * j)) & 63u);
+        const int gr = rr >> 1, i0 = 2 * (rr & 1);   // D rows g (i 0, 1) or g + 8 (i 2, 3); tokens 2c, 2c + 1
+        const float cx = -(128.f * s + mn);
+        acc[gr][i0] = fmaf(s, dq[gr][i0], fmaf(cx, dx[0], acc[gr][i0]));
+        acc[gr][i0 + 1] = fmaf(s, dq[gr][i0 + 1], fmaf(cx, dx[1], acc[gr][i0 + 1]));
       }
     }
+    __syncwarp();   // every lane is done with this slot before it is refilled
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+  if (n0 >= N) return;
+  // D layout: element i of group gr is row 16 gr + g + 8 (i >> 1), token 2c + (i & 1)
+  float* dst = out;
+  long long ld = ldo;
+  bool add = accumulate != 0;
+  if (gridDim.y > 1) {   // partial sums [split][T][N]
+    dst = out + static_cast<long long>(blockIdx.y) * T * N;
+    ld = N;
+    add = false;
+  }
+#pragma unroll
+  for (int gr = 0; gr < 2; ++gr)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int n = n0 + 16 * gr + g + 8 * (i >> 1), t = t0 + 2 * c + (i & 1);
+      if (n < N && t < T) {
+        float* p = dst + static_cast<long long>(t) * ld + n;
+        *p = add ? *p + acc[gr][i] : acc[gr][i];
+      }
+    }
+}
+
+// out[t][n] (+)= sum over splits z of ws[z][t][n], in order of z.
+__global__ void q4_split_reduce(const float* __restrict__ ws, int nz, int T, int N, float* __restrict__ out,
+                                long long ldo, int accumulate) {
+  const long long tot = static_cast<long long>(T) * N;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < tot;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float v = 0.f;
+    for (int z = 0; z < nz; ++z) v += ws[static_cast<long long>(z) * tot + i];
+    const long long t = i / N, n = i % N;
+    float* p = out + t * ldo + n;
+    *p = accumulate ? *p + v : v;
   }
 }
 
@@ -409,27 +465,24 @@ __global__ void at_prep(const float* __restrict__ z, int ldz, const int* __restr
   }
 }
 
-// x = o (* sigmoid(gate) when gate != null), as bf16 high/low parts [T][n] (and fp32 in xf).
+// x = o (* sigmoid(gate) when gate != null), as bf16 high/low parts [T][n].
 __global__ void gate_split(const float* __restrict__ o, int ldo, const float* __restrict__ gate, int ldg, int n,
-                           uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo, float* __restrict__ xf = nullptr) {
+                           uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
   const int t = blockIdx.x;
   for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < n; i += gridDim.y * blockDim.x) {
     float v = o[static_cast<long long>(t) * ldo + i];
     if (gate) v *= sigmoidf_(gate[static_cast<long long>(t) * ldg + i]);
     put_split(xhi, xlo, static_cast<long long>(t) * n + i, v);
-    if (xf) xf[static_cast<long long>(t) * n + i] = v;
   }
 }
 
-// act = SiLU(g) * u from gu[t] = [g (F) | u (F)], as bf16 high/low parts [T][F] (and fp32 in xf).
-__global__ void act_split(const float* __restrict__ gu, int F, uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo,
-                          float* __restrict__ xf = nullptr) {
+// act = SiLU(g) * u from gu[t] = [g (F) | u (F)], as bf16 high/low parts [T][F].
+__global__ void act_split(const float* __restrict__ gu, int F, uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
   const int t = blockIdx.x;
   const float* r = gu + static_cast<long long>(t) * 2 * F;
   for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < F; i += gridDim.y * blockDim.x) {
     const float v = siluf_(r[i]) * r[F + i];
     put_split(xhi, xlo, static_cast<long long>(t) * F + i, v);
-    if (xf) xf[static_cast<long long>(t) * F + i] = v;
   }
 }
 
@@ -1593,14 +1646,28 @@ __global__ void accept_prefix(const int* tokens, const unsigned long long* best,
 // Row bytes of a 4-bit matrix with K inputs (K a multiple of 256).
 inline long long q4_row_bytes(long long K) { return (K / 256) * 144; }
 
-cudaError_t launch_q4_linear(const float* X, long long ldx, const void* W, long long ldw, float* C, long long ldc,
-                             int T, int N, int K, int accumulate, cudaStream_t s) {
+// 4-bit linear layer over the T tokens' bf16 high / low activation parts [T][K].
+cudaError_t launch_q4_linear(const uint16_t* xhi, const uint16_t* xlo, const void* W, long long ldw, float* C,
+                             long long ldc, int T, int N, int K, int accumulate, float* ws, long long ws_floats,
+                             cudaStream_t s) {
   if (T <= 0 || N <= 0) return cudaSuccess;
-  const int gx = std::min((N + 8 * kQ4Rows - 1) / (8 * kQ4Rows), 1184);
-  constexpr size_t smem = 8ull * kQ4Depth * kQ4Rows * 144;
-  q4_linear_kernel<8><<<dim3(gx, (T + 7) / 8), 256, smem, s>>>(X, ldx, static_cast<const uint8_t*>(W), ldw, C, ldc, T,
-                                                                N, K, accumulate);
-  return cudaGetLastError();
+  const int tiles = (N + 127) / 128, ttiles = (T + 7) / 8, nsb = K / 256;
+  int nz = std::min(nsb, std::max(1, (4 * 148 + tiles * ttiles - 1) / (tiles * ttiles)));
+  if (static_cast<long long>(nz) * T * N > ws_floats) nz = 1;
+  int per = (nsb + nz - 1) / nz;
+  nz = (nsb + per - 1) / per;
+  if (nz <= 1) per = nsb;
+  constexpr size_t smem = 4ull * kQ4Depth * 32 * 144;
+  q4_linear_mma<<<dim3(tiles, nz, ttiles), 128, smem, s>>>(xhi, xlo, K, static_cast<const uint8_t*>(W), ldw,
+                                                            nz > 1 ? ws : C, ldc, T, N, K, per, accumulate);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && nz > 1) {
+    const long long tot = static_cast<long long>(T) * N;
+    q4_split_reduce<<<static_cast<int>(std::min<long long>((tot + 255) / 256, 1184)), 256, 0, s>>>(ws, nz, T, N, C, ldc,
+                                                                                               accumulate);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaStream_t s,
@@ -1616,13 +1683,13 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
     if (e == cudaSuccess) e = cudaGetLastError();
     ++m->launches;
   };
-  const bool q4 = b.q4 != 0;   // 4-bit weights: linear layers on the CUDA cores from fp32 inputs (pf.xf)
-  float* xf = q4 ? pf.xf : nullptr;
+  const bool q4 = b.q4 != 0;   // 4-bit weights: their own linear layer (mma.sync over <= 8-token tiles)
   // ldw is the bf16 row stride; 4-bit rows take (K / 256) * 144 bytes plus the same tail
   auto linear = [&](const void* w, long long ldw, int N, int K, float* out, long long ldc, int acc) {
     if (e != cudaSuccess) return;
     if (q4) {
-      e = launch_q4_linear(pf.xf, K, w, q4_row_bytes(K) + (ldw - 2LL * K), out, ldc, T, N, K, acc, s);
+      e = launch_q4_linear(pf.xhi, pf.xlo, w, q4_row_bytes(K) + (ldw - 2LL * K), out, ldc, T, N, K, acc, pf.splitk,
+                           kSplitKFloats, s);
     } else {
       LinearArgs a{pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, b.err, pf.splitk, kSplitKFloats};
       e = launch_linear(a, s);
@@ -1638,7 +1705,7 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     const LayerW& L = m->layers_host[l];
     const mk_prefill_layer& PL = m->pf_layers[l];
-    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm1, b.eps, pf.xhi, pf.xlo, xf);
+    rms_split<<<T, rms_threads(T), 0, s>>>(pf.h, H, L.norm1, b.eps, pf.xhi, pf.xlo);
     chk();
     if (L.kind == kDeltaNet) {
       const int rows = C + 2 * Hd;
@@ -1699,8 +1766,7 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         wy_state<<<dim3(Hd, dv / kRowGroup), 256, wy_state_smem(dk), s>>>(wy, S);
       }
       chk();
-      gate_split<<<dim3(T, (Hd * dv + 1023) / 1024), kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo,
-                                                                   xf);
+      gate_split<<<dim3(T, (Hd * dv + 1023) / 1024), kPT, 0, s>>>(pf.o, Hd * dv, nullptr, 0, Hd * dv, pf.xhi, pf.xlo);
       chk();
       linear(q4 ? L.w_out_q4 : PL.w_out, 2LL * Hd * dv, H, Hd * dv, pf.h, H, 1);
     } else {
@@ -1754,16 +1820,16 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         }
       }
       gate_split<<<dim3(T, (qd + 1023) / 1024), kPT, 0, s>>>(pf.o, qd, c.at_out_gate ? pf.z + qd : nullptr, rows, qd,
-                                                             pf.xhi, pf.xlo, xf);
+                                                             pf.xhi, pf.xlo);
       chk();
       linear(q4 ? L.w_out_q4 : PL.w_out, 2LL * qd, H, qd, pf.h, H, 1);
     }
     if (e != cudaSuccess) break;
-    rms_split<<<T, kPT, 0, s>>>(pf.h, H, L.norm2, b.eps, pf.xhi, pf.xlo, xf);
+    rms_split<<<T, rms_threads(T), 0, s>>>(pf.h, H, L.norm2, b.eps, pf.xhi, pf.xlo);
     chk();
     linear(L.w_gate, 2LL * H, F, H, pf.z, 2LL * F, 0);
     linear(L.w_up, 2LL * H, F, H, pf.z + F, 2LL * F, 0);
-    act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo, xf);
+    act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
     chk();
     linear(q4 ? L.w_down_q4 : PL.w_down, 2LL * F, H, F, pf.h, H, 1);
   }
@@ -1783,6 +1849,9 @@ cudaError_t set_prefill_smem_limits() {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(q4_linear_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(4 * kQ4Depth * 32 * 144));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(wy_state_tc<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(wy_tc_smem<128>()));
@@ -1847,12 +1916,12 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
   // 2. final norm, LM head on the tensor cores for all K + 1 positions, greedy tokens
   float* logits = d_logits ? d_logits : vs.logits;
   if (e == cudaSuccess) {
-    mk::rms_split<<<T, mk::kPT, 0, s>>>(m->pf.h, c.hidden, b.norm_f, b.eps, m->pf.xhi, m->pf.xlo,
-                                         b.q4 ? m->pf.xf : nullptr);
+    mk::rms_split<<<T, mk::rms_threads(T), 0, s>>>(m->pf.h, c.hidden, b.norm_f, b.eps, m->pf.xhi, m->pf.xlo);
     chk();
   }
   if (e == cudaSuccess && b.q4) {   // 4-bit tied LM head
-    e = mk::launch_q4_linear(m->pf.xf, c.hidden, b.embed, b.row_bytes, logits, c.vocab, T, c.vocab, c.hidden, 0, s);
+    e = mk::launch_q4_linear(m->pf.xhi, m->pf.xlo, b.embed, b.row_bytes, logits, c.vocab, T, c.vocab, c.hidden, 0,
+                             m->pf.splitk, mk::kSplitKFloats, s);
     ++m->launches;
   } else if (e == cudaSuccess) {
     mk::LinearArgs a{m->pf.xhi, m->pf.xlo, b.embed, 2LL * c.hidden, logits, c.vocab, T, c.vocab, c.hidden, 0, b.err};
