@@ -46,6 +46,21 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return warp_sum(t);
 }
 
+// Four consecutive values (i a multiple of 4) as bf16 high / low parts, 8-byte stores.
+__device__ __forceinline__ void put_split4(uint16_t* hi, uint16_t* lo, long long i, float4 v) {
+  const float a[4] = {v.x, v.y, v.z, v.w};
+  uint16_t h[4], l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    h[q] = f_to_bf16(a[q]);
+    l[q] = f_to_bf16(a[q] - bf16_to_f(h[q]));
+  }
+  *reinterpret_cast<uint2*>(hi + i) = make_uint2(h[0] | (static_cast<uint32_t>(h[1]) << 16),
+                                                 h[2] | (static_cast<uint32_t>(h[3]) << 16));
+  *reinterpret_cast<uint2*>(lo + i) = make_uint2(l[0] | (static_cast<uint32_t>(l[1]) << 16),
+                                                 l[2] | (static_cast<uint32_t>(l[3]) << 16));
+}
+
 __device__ __forceinline__ void put_split(uint16_t* hi, uint16_t* lo, long long i, float v) {
   const uint16_t h = f_to_bf16(v);
   hi[i] = h;
@@ -70,13 +85,19 @@ __global__ void rms_split(const float* __restrict__ h, int H, const uint16_t* __
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* row = h + static_cast<long long>(t) * H;
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < H; i += blockDim.x) ss += row[i] * row[i];
+  float ss = 0.f;   // H is a multiple of 4: float4 rows
+  for (int i = 4 * threadIdx.x; i < H; i += 4 * blockDim.x) {
+    const float4 v = *reinterpret_cast<const float4*>(row + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
   ss = block_sum(ss, red);
   const float inv = 1.0f / sqrtf(ss / static_cast<float>(H) + eps);
-  for (int i = threadIdx.x; i < H; i += blockDim.x) {
-    const float v = row[i] * inv * bf16_to_f(gamma[i]);
-    put_split(xhi, xlo, static_cast<long long>(t) * H + i, v);
+  for (int i = 4 * threadIdx.x; i < H; i += 4 * blockDim.x) {
+    const float4 v = *reinterpret_cast<const float4*>(row + i);
+    const uint2 gw = *reinterpret_cast<const uint2*>(gamma + i);
+    put_split4(xhi, xlo, static_cast<long long>(t) * H + i,
+               make_float4(v.x * inv * bf16lo(gw.x), v.y * inv * bf16hi(gw.x), v.z * inv * bf16lo(gw.y),
+                           v.w * inv * bf16hi(gw.y)));
   }
 }
 
@@ -316,62 +337,83 @@ __global__ void dn_prep(const float* __restrict__ z, int ldz, const int* __restr
   }
 }
 
-// The same with one warp per (token, 128-channel block) and four channels per lane
-// (float4 loads of z, the ring and the outputs; C a multiple of 128, dk 64 or 128, row
-// strides multiples of 4 floats). The q / k norms reduce over the dk / 4 lanes of a head
-// with shuffles. CTA = 8 consecutive tokens of one block, so the W overlapping z rows a
-// token reads are mostly L1 hits; block C / 128 holds the gates.
+// The same with one warp per (8 consecutive tokens, 128-channel block) and four channels
+// per lane (float4 loads of z, the ring and the outputs; C a multiple of 128, dk 64 or 128,
+// row strides multiples of 4 floats). The lane keeps the conv window of its channels in
+// registers and slides it over the warp's tokens (one new z row per token); the q / k norms
+// reduce over the dk / 4 lanes of a head with shuffles. Block C / 128 holds the gates.
+constexpr int kPrepTokensPerWarp = 8;
 __global__ void __launch_bounds__(256) dn_prep_v4(const float* __restrict__ z, int ldz, int T,
                                                   const int* __restrict__ posp, int off, const float* __restrict__ ring,
                                                   int W, int C, int Hd, int dk, const uint16_t* __restrict__ taps,
                                                   float* __restrict__ y, int ldy) {
+  constexpr int TPW = kPrepTokensPerWarp;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  const float* zt = z + static_cast<long long>(t) * ldz;
-  float* yr = y + static_cast<long long>(t) * ldy;
+  const int tb = (blockIdx.x * 8 + warp) * TPW;
+  if (tb >= T) return;
+  const int te = min(T, tb + TPW);
   if (static_cast<int>(blockIdx.y) * 128 >= C) {   // gates
-    for (int hh = lane; hh < Hd; hh += 32) {
-      const float al = zt[C + hh], be = zt[C + Hd + hh];
-      yr[C + hh] = -(fmaxf(al, 0.f) + log1pf(expf(-fabsf(al))));
-      yr[C + Hd + hh] = sigmoidf_(be);
+    for (int t = tb; t < te; ++t) {
+      const float* zt = z + static_cast<long long>(t) * ldz;
+      float* yr = y + static_cast<long long>(t) * ldy;
+      for (int hh = lane; hh < Hd; hh += 32) {
+        const float al = zt[C + hh], be = zt[C + Hd + hh];
+        yr[C + hh] = -(fmaxf(al, 0.f) + log1pf(expf(-fabsf(al))));
+        yr[C + Hd + hh] = sigmoidf_(be);
+      }
     }
     return;
   }
   const int pos0 = *posp + off;
   const int c0 = blockIdx.y * 128 + 4 * lane;
-  float x[kPrepMaxConv][4];
+  const bool qk = c0 < 2 * Hd * dk;   // warp-uniform: blocks are all q / k or all v channels
+  // window of the last kPrepMaxConv input rows; tap j of a width-W conv sits at slot j + (4 - W)
+  constexpr int MW = kPrepMaxConv;
+  float tw[4][MW];
 #pragma unroll
-  for (int j = 0; j < kPrepMaxConv; ++j) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (j < W) {
-      const int s = t - (W - 1) + j;
-      if (s >= 0) {
-        v = *reinterpret_cast<const float4*>(z + static_cast<long long>(s) * ldz + c0);
-      } else {
-        const int p = pos0 + s;
-        if (p >= 0) v = *reinterpret_cast<const float4*>(ring + static_cast<long long>(p % W) * C + c0);
-      }
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int j = 0; j < MW; ++j) {
+      const int jj = j - (MW - W);
+      tw[u][j] = jj >= 0 ? bf16_to_f(taps[static_cast<long long>(c0 + u) * W + jj]) : 0.f;
     }
-    x[j][0] = v.x; x[j][1] = v.y; x[j][2] = v.z; x[j][3] = v.w;
-  }
-  float o[4];
+  auto load = [&](int s) {   // input row s of the pass (negative: conv history)
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (s >= 0) {
+      v = *reinterpret_cast<const float4*>(z + static_cast<long long>(s) * ldz + c0);
+    } else {
+      const int p = pos0 + s;
+      if (p >= 0) v = *reinterpret_cast<const float4*>(ring + static_cast<long long>(p % W) * C + c0);
+    }
+    return v;
+  };
+  float4 win[MW];   // win[j] = input row t - (MW - 1) + j
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    float acc = 0.f;
+  for (int j = 0; j < MW - 1; ++j) win[j] = j >= MW - W ? load(tb - (MW - 1) + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int t = tb; t < te; ++t) {
+    win[MW - 1] = load(t);
+    float o[4];
 #pragma unroll
-    for (int j = 0; j < kPrepMaxConv; ++j)
-      if (j < W) acc = fmaf(bf16_to_f(taps[static_cast<long long>(c0 + u) * W + j]), x[j][u], acc);
-    o[u] = siluf_(acc);
-  }
-  if (c0 < 2 * Hd * dk) {   // q or k channel: L2 norm over the head (dk / 4 lanes, aligned)
-    float ss = o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3];
-    for (int m = dk / 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-    const float nr = 1.0f / sqrtf(ss + 1e-6f);
+    for (int u = 0; u < 4; ++u) {
+      float acc = 0.f;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) o[u] *= nr;
+      for (int j = 0; j < MW; ++j) {
+        const float xv = u == 0 ? win[j].x : (u == 1 ? win[j].y : (u == 2 ? win[j].z : win[j].w));
+        acc = fmaf(tw[u][j], xv, acc);
+      }
+      o[u] = siluf_(acc);
+    }
+    if (qk) {   // L2 norm over the head (dk / 4 lanes, aligned)
+      float ss = o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3];
+      for (int m = dk / 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      const float nr = 1.0f / sqrtf(ss + 1e-6f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) o[u] *= nr;
+    }
+    *reinterpret_cast<float4*>(y + static_cast<long long>(t) * ldy + c0) = make_float4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int j = 0; j + 1 < MW; ++j) win[j] = win[j + 1];
   }
-  *reinterpret_cast<float4*>(yr + c0) = make_float4(o[0], o[1], o[2], o[3]);
 }
 
 // The same on a (token, vector) grid: vector v < 2 Hd is one q or k head (conv + SiLU +
@@ -468,21 +510,26 @@ __global__ void at_prep(const float* __restrict__ z, int ldz, const int* __restr
 // x = o (* sigmoid(gate) when gate != null), as bf16 high/low parts [T][n].
 __global__ void gate_split(const float* __restrict__ o, int ldo, const float* __restrict__ gate, int ldg, int n,
                            uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
-  const int t = blockIdx.x;
-  for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < n; i += gridDim.y * blockDim.x) {
-    float v = o[static_cast<long long>(t) * ldo + i];
-    if (gate) v *= sigmoidf_(gate[static_cast<long long>(t) * ldg + i]);
-    put_split(xhi, xlo, static_cast<long long>(t) * n + i, v);
+  const int t = blockIdx.x;   // n, ldo, ldg multiples of 4: float4 rows
+  for (int i = 4 * (blockIdx.y * blockDim.x + threadIdx.x); i < n; i += 4 * gridDim.y * blockDim.x) {
+    float4 v = *reinterpret_cast<const float4*>(o + static_cast<long long>(t) * ldo + i);
+    if (gate) {
+      const float4 g = *reinterpret_cast<const float4*>(gate + static_cast<long long>(t) * ldg + i);
+      v.x *= sigmoidf_(g.x); v.y *= sigmoidf_(g.y); v.z *= sigmoidf_(g.z); v.w *= sigmoidf_(g.w);
+    }
+    put_split4(xhi, xlo, static_cast<long long>(t) * n + i, v);
   }
 }
 
 // act = SiLU(g) * u from gu[t] = [g (F) | u (F)], as bf16 high/low parts [T][F].
 __global__ void act_split(const float* __restrict__ gu, int F, uint16_t* __restrict__ xhi, uint16_t* __restrict__ xlo) {
-  const int t = blockIdx.x;
+  const int t = blockIdx.x;   // F a multiple of 4: float4 rows
   const float* r = gu + static_cast<long long>(t) * 2 * F;
-  for (int i = blockIdx.y * blockDim.x + threadIdx.x; i < F; i += gridDim.y * blockDim.x) {
-    const float v = siluf_(r[i]) * r[F + i];
-    put_split(xhi, xlo, static_cast<long long>(t) * F + i, v);
+  for (int i = 4 * (blockIdx.y * blockDim.x + threadIdx.x); i < F; i += 4 * gridDim.y * blockDim.x) {
+    const float4 g = *reinterpret_cast<const float4*>(r + i);
+    const float4 u = *reinterpret_cast<const float4*>(r + F + i);
+    put_split4(xhi, xlo, static_cast<long long>(t) * F + i,
+               make_float4(siluf_(g.x) * u.x, siluf_(g.y) * u.y, siluf_(g.z) * u.z, siluf_(g.w) * u.w));
   }
 }
 
@@ -1714,8 +1761,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       ++di;
       linear(L.w_in, 2LL * H + 16, rows, H, pf.z, rows, 0);
       if (C % 128 == 0 && (dk == 64 || dk == 128) && rows % 4 == 0 && Wc <= kPrepMaxConv) {
-        dn_prep_v4<<<dim3((T + 7) / 8, C / 128 + 1), 256, 0, s>>>(pf.z, rows, T, b.pos, off, ring, Wc, C, Hd, dk, L.conv,
-                                                                   pf.y, rows);
+        dn_prep_v4<<<dim3((T + 8 * kPrepTokensPerWarp - 1) / (8 * kPrepTokensPerWarp), C / 128 + 1), 256, 0, s>>>(
+            pf.z, rows, T, b.pos, off, ring, Wc, C, Hd, dk, L.conv, pf.y, rows);
       } else if (T <= 64) {   // few tokens: a (token, vector) grid keeps the GPU busy
         dn_prep_wide<<<dim3(T, 2 * Hd + (Hd * dv + 127) / 128 + 1), 128, 0, s>>>(pf.z, rows, b.pos, off, ring, Wc, C,
                                                                                 Hd, dk, dv, L.conv, pf.y, rows);
