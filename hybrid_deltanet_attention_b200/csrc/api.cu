@@ -197,7 +197,7 @@ int decode_xcap(const mk_config& c) {
 }
 
 int check_budget(const mk_config& c, int grid) {
-  const long S = static_cast<long>(mk::decode_scratch_floats(c.hidden, is_q4(c), decode_xcap(c)));
+  const long S = static_cast<long>(mk::decode_scratch_floats(c.hidden, is_q4(c), decode_xcap(c), c.n_layers));
   if (S < 256) return fail(MK_ERR_ARG, "shared-memory budget exceeded (hidden too large)");
   auto ceil_div = [](long a, long b) { return (a + b - 1) / b; };
   if (n_kind(c, 'D')) {

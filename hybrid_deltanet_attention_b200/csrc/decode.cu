@@ -61,6 +61,13 @@ struct __align__(16) Shared {
   Ranges rg;
 };
 
+// Bytes of the shared-memory copy of the layer table (16-byte multiple).
+__host__ __device__ constexpr size_t layer_table_bytes(int n_layers) {
+  return (static_cast<size_t>(n_layers) * sizeof(LayerW) + 15) / 16 * 16;
+}
+static_assert(sizeof(LayerW) % 4 == 0, "the layer table is copied in 32-bit words");
+static_assert(sizeof(Shared) % 16 == 0, "the layer table and xs follow Shared 16-byte aligned");
+
 __device__ __forceinline__ void split_range(int n, int c, int G, int& b, int& e) {
   b = static_cast<int>((static_cast<long long>(n) * c) / G);
   e = static_cast<int>((static_cast<long long>(n) * (c + 1)) / G);
@@ -509,7 +516,14 @@ __device__ __forceinline__ void rmsnorm(const DecodeParams& p, int H, int j, con
     const int g = tid + k * kConsumerThreads;
     if (g < ng) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
   }
-  ss = cons_sum(ss, sh, warp, lane);
+  // the sum of squares: warp sums meet in shared memory behind one named barrier, and every
+  // thread adds the kConsumerWarps partials itself
+  ss = warp_sum(ss);
+  if (lane == 0) sh->red[warp] = ss;
+  cons_sync(kConsumerThreads);
+  ss = 0.f;
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) ss += sh->red[w];
   const float inv = 1.0f / sqrtf(ss / static_cast<float>(H) + p.eps);
 #pragma unroll
   for (int k = 0; k < MG; ++k) {
@@ -926,7 +940,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   Shared* sh = reinterpret_cast<Shared*>(smem + static_cast<size_t>(NS) * kSlotBytes);
-  float* xs = reinterpret_cast<float*>(sh + 1);      // [xcap] normed input / staged projection input
+  LayerW* ltab = reinterpret_cast<LayerW*>(sh + 1);   // [n_layers] copy of p.layers (layers 1..)
+  float* xs = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ltab) + layer_table_bytes(p.n_layers));
   float* xsum = xs + p.xcap;                          // Q4: [xcap / 8] per-lane x sums
   float* qpart = xsum + (Q4 ? p.xcap / 8 : 0);        // Q4: [kQ4PartFloats] row partial sums
   float* fs = Q4 ? qpart + kQ4PartFloats : xs + p.H;  // scratch
@@ -981,9 +996,16 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   const int ng = H / 4;
   uint32_t n = 0;               // next chunk index
   unsigned nbar = 0;
+  {   // the layer table into shared memory; read from layer 1 on (the named barriers of
+      // layer 0's first RMSNorm publish it), so no layer starts with a global load
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(p.layers);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(ltab);
+    const int nw = p.n_layers * static_cast<int>(sizeof(LayerW) / 4);
+    for (int i = tid; i < nw; i += kConsumerThreads) dst[i] = __ldg(src + i);
+  }
 
   for (int l = 0; l < p.n_layers; ++l) {
-    const LayerW L = p.layers[l];
+    const LayerW L = l == 0 ? p.layers[0] : ltab[l];
     // ---- phase 1: pre-mixer RMSNorm + input projection (+ DeltaNet conv epilogue) ----
     if (l > 0 && !grid_barrier(p, sh, ++nbar, tid)) return;
     {
@@ -1564,24 +1586,25 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
 
 constexpr size_t kSmemLimit = 232448;
 
-// Shared memory before the scratch: the ring, Shared, the staged input vector and, with
-// Q4 weights (2 ring slots), its per-lane sums and the row partial sums.
-static size_t decode_fixed_bytes(int H, bool q4, int xcap) {
-  if (!q4) return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + static_cast<size_t>(H) * 4;
-  return 2 * static_cast<size_t>(kSlotBytes) + sizeof(Shared) + static_cast<size_t>(xcap) * 4 +
+// Shared memory before the scratch: the ring, Shared, the layer table, the staged input
+// vector and, with Q4 weights (2 ring slots), its per-lane sums and the row partial sums.
+static size_t decode_fixed_bytes(int H, bool q4, int xcap, int n_layers) {
+  const size_t lt = layer_table_bytes(n_layers);
+  if (!q4) return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + lt + static_cast<size_t>(H) * 4;
+  return 2 * static_cast<size_t>(kSlotBytes) + sizeof(Shared) + lt + static_cast<size_t>(xcap) * 4 +
          static_cast<size_t>(xcap / 8) * 4 + static_cast<size_t>(kQ4PartFloats) * 4;
 }
 
-size_t decode_scratch_floats(int H, bool q4, int xcap) {
-  const size_t fixed = decode_fixed_bytes(H, q4, xcap);
+size_t decode_scratch_floats(int H, bool q4, int xcap, int n_layers) {
+  const size_t fixed = decode_fixed_bytes(H, q4, xcap, n_layers);
   if (fixed >= kSmemLimit) return 0;
   size_t f = (kSmemLimit - fixed) / 4;
   f &= ~static_cast<size_t>(3);
   return f > 8192 ? 8192 : f;
 }
 
-size_t decode_smem_bytes(int H, bool q4, int xcap) {
-  return decode_fixed_bytes(H, q4, xcap) + decode_scratch_floats(H, q4, xcap) * 4;
+size_t decode_smem_bytes(int H, bool q4, int xcap, int n_layers) {
+  return decode_fixed_bytes(H, q4, xcap, n_layers) + decode_scratch_floats(H, q4, xcap, n_layers) * 4;
 }
 
 int decode_max_splits(int grid, int hkv) {
@@ -1601,7 +1624,7 @@ cudaError_t launch_hk(const DecodeParams& p, int grid, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, Q4, p.xcap);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, Q4, p.xcap, p.n_layers);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;

@@ -88,8 +88,8 @@ struct DecodeParams {
   float* abuf;                        // [F] SwiGLU activation (Q4)
 };
 
-size_t decode_smem_bytes(int H, bool q4 = false, int xcap = 0);
-size_t decode_scratch_floats(int H, bool q4 = false, int xcap = 0);   // fp32 scratch per CTA left after the ring, xs (and the Q4 tables)
+size_t decode_smem_bytes(int H, bool q4, int xcap, int n_layers);
+size_t decode_scratch_floats(int H, bool q4, int xcap, int n_layers);   // fp32 scratch per CTA left after the ring, the layer table, xs (and the Q4 tables)
 constexpr int kQ4Block = 144;          // bytes per 256-weight super-block
 constexpr int kQ4PartFloats = 512;     // shared-memory partial sums of the Q4 row products
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s);
