@@ -196,32 +196,48 @@ int decode_xcap(const mk_config& c) {
   return std::max({c.hidden, c.dn_heads * c.dn_dv, qd, c.ffn});
 }
 
-int check_budget(const mk_config& c, int grid) {
-  const long S = static_cast<long>(mk::decode_scratch_floats(c.hidden, is_q4(c), decode_xcap(c), c.n_layers));
-  if (S < 256) return fail(MK_ERR_ARG, "shared-memory budget exceeded (hidden too large)");
+// Whether the decode kernel's shared-memory scratch covers every phase when it keeps
+// ltab_entries layer-table entries in shared memory (why: the first shortfall).
+bool budget_ok(const mk_config& c, int grid, int ltab_entries, const char** why) {
+  auto fail_ = [&](const char* w) {
+    *why = w;
+    return false;
+  };
+  const long S = static_cast<long>(mk::decode_scratch_floats(c.hidden, is_q4(c), decode_xcap(c), ltab_entries));
+  if (S < 256) return fail_("shared-memory budget exceeded (hidden too large)");
   auto ceil_div = [](long a, long b) { return (a + b - 1) / b; };
   if (n_kind(c, 'D')) {
     const long rows = ceil_div(static_cast<long>(c.dn_heads) * c.dn_dv, grid);
     const long nh = ceil_div(rows, c.dn_dv) + 1;
-    if (nh * (2 * c.dn_dk + 2) + 2 * rows > S) return fail(MK_ERR_ARG, "DeltaNet rows per CTA exceed the scratch budget");
+    if (nh * (2 * c.dn_dk + 2) + 2 * rows > S) return fail_("DeltaNet rows per CTA exceed the scratch budget");
     if (2 * nh * c.dn_dk + rows + nh > 3L * mk::kConsumerThreads)
-      return fail(MK_ERR_ARG, "DeltaNet channels per CTA exceed the prologue budget");
+      return fail_("DeltaNet channels per CTA exceed the prologue budget");
     const long inrows = ceil_div(static_cast<long>(c.dn_heads) * (2 * c.dn_dk + c.dn_dv) + 2 * c.dn_heads, grid);
     if (inrows > mk::kConsumerThreads || 7 * inrows > S)
-      return fail(MK_ERR_ARG, "DeltaNet in-projection rows per CTA exceed the conv budget");
-    if (4L * c.dn_heads * 4 + 512 > 4096) return fail(MK_ERR_ARG, "too many DeltaNet heads for the norm buffer");
+      return fail_("DeltaNet in-projection rows per CTA exceed the conv budget");
+    if (4L * c.dn_heads * 4 + 512 > 4096) return fail_("too many DeltaNet heads for the norm buffer");
   }
   if (n_kind(c, 'A')) {
     const long grp = c.at_q_heads / c.at_kv_heads;
     if (2 * grp * c.at_head_dim + grp * mk::kAttnSub + 3 * grp + 2 * c.at_head_dim > S)
-      return fail(MK_ERR_ARG, "attention scratch budget exceeded");
+      return fail_("attention scratch budget exceeded");
     const long cols = ceil_div(static_cast<long>(c.at_q_heads) * c.at_head_dim, grid);
     const long nhd = ceil_div(cols, c.at_head_dim) + 1;
     if (nhd * mk::decode_max_splits(grid, c.at_kv_heads) + 2 * cols > S)
-      return fail(MK_ERR_ARG, "attention columns per CTA exceed the scratch budget");
+      return fail_("attention columns per CTA exceed the scratch budget");
   }
-  if (2 * ceil_div(c.ffn, grid) > S) return fail(MK_ERR_ARG, "MLP rows per CTA exceed the scratch budget");
-  return MK_OK;
+  if (2 * ceil_div(c.ffn, grid) > S) return fail_("MLP rows per CTA exceed the scratch budget");
+  return true;
+}
+
+// Valid with the smaller (two-slot) layer table; the whole table is used when it fits too.
+int check_budget(const mk_config& c, int grid) {
+  const char* why = nullptr;
+  return budget_ok(c, grid, 2, &why) ? MK_OK : fail(MK_ERR_ARG, why);
+}
+bool layer_table_fits(const mk_config& c, int grid) {
+  const char* why = nullptr;
+  return budget_ok(c, grid, c.n_layers, &why);
 }
 
 constexpr int kBatchedPrefillMin = 16;   // shorter prompts run as decode launches
@@ -680,6 +696,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   b.max_ctx = c.max_ctx;
   b.row_bytes = static_cast<int>(is_q4(c) ? q4_rb(H) : rb);
   b.q4 = is_q4(c) ? 1 : 0;
+  b.ltab_full = layer_table_fits(c, grid) ? 1 : 0;
   b.rb_dn_out = static_cast<int>(q4_rb(static_cast<size_t>(c.dn_heads) * c.dn_dv));
   b.rb_at_out = static_cast<int>(q4_rb(static_cast<size_t>(c.at_q_heads) * c.at_head_dim));
   b.rb_ffn = static_cast<int>(q4_rb(c.ffn));

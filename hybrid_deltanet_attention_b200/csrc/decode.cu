@@ -61,11 +61,13 @@ struct __align__(16) Shared {
   Ranges rg;
 };
 
-// Bytes of the shared-memory copy of the layer table (16-byte multiple).
-__host__ __device__ constexpr size_t layer_table_bytes(int n_layers) {
-  return (static_cast<size_t>(n_layers) * sizeof(LayerW) + 15) / 16 * 16;
+// Shared-memory copy of the layer table (16-byte multiple): every layer's entry, copied at
+// launch start, when the budget allows (p.ltab_full); otherwise two slots, layer l + 1's
+// entry fetched into slot (l + 1) & 1 while layer l runs.
+__host__ __device__ constexpr size_t layer_table_bytes(int entries) {
+  return (static_cast<size_t>(entries) * sizeof(LayerW) + 15) / 16 * 16;
 }
-static_assert(sizeof(LayerW) % 4 == 0, "the layer table is copied in 32-bit words");
+static_assert(sizeof(LayerW) % 4 == 0, "layer entries are copied in 32-bit words");
 static_assert(sizeof(Shared) % 16 == 0, "the layer table and xs follow Shared 16-byte aligned");
 
 __device__ __forceinline__ void split_range(int n, int c, int G, int& b, int& e) {
@@ -940,8 +942,9 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* ring = smem;
   Shared* sh = reinterpret_cast<Shared*>(smem + static_cast<size_t>(NS) * kSlotBytes);
-  LayerW* ltab = reinterpret_cast<LayerW*>(sh + 1);   // [n_layers] copy of p.layers (layers 1..)
-  float* xs = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ltab) + layer_table_bytes(p.n_layers));
+  LayerW* ltab = reinterpret_cast<LayerW*>(sh + 1);   // [n_layers] or [2] entries of p.layers
+  float* xs = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ltab) +
+                                       layer_table_bytes(p.ltab_full ? p.n_layers : 2));
   float* xsum = xs + p.xcap;                          // Q4: [xcap / 8] per-lane x sums
   float* qpart = xsum + (Q4 ? p.xcap / 8 : 0);        // Q4: [kQ4PartFloats] row partial sums
   float* fs = Q4 ? qpart + kQ4PartFloats : xs + p.H;  // scratch
@@ -996,16 +999,20 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   const int ng = H / 4;
   uint32_t n = 0;               // next chunk index
   unsigned nbar = 0;
-  {   // the layer table into shared memory; read from layer 1 on (the named barriers of
-      // layer 0's first RMSNorm publish it), so no layer starts with a global load
+  constexpr int kLayerWords = static_cast<int>(sizeof(LayerW) / 4);
+  if (p.ltab_full) {   // the whole table, read from layer 1 on (published by layer 0's named barriers)
     const uint32_t* src = reinterpret_cast<const uint32_t*>(p.layers);
     uint32_t* dst = reinterpret_cast<uint32_t*>(ltab);
-    const int nw = p.n_layers * static_cast<int>(sizeof(LayerW) / 4);
-    for (int i = tid; i < nw; i += kConsumerThreads) dst[i] = __ldg(src + i);
+    for (int i = tid; i < p.n_layers * kLayerWords; i += kConsumerThreads) dst[i] = __ldg(src + i);
   }
 
   for (int l = 0; l < p.n_layers; ++l) {
-    const LayerW L = l == 0 ? p.layers[0] : ltab[l];
+    const LayerW L = l == 0 ? p.layers[0] : ltab[p.ltab_full ? l : (l & 1)];
+    // two slots: the next layer's entry is loaded now and stored into the other slot after
+    // this layer's first barrier (the named barriers later in the layer publish it; that
+    // slot was last read at the start of layer l - 1)
+    const bool lw_mine = !p.ltab_full && l + 1 < p.n_layers && tid < kLayerWords;
+    const uint32_t lw_next = lw_mine ? __ldg(reinterpret_cast<const uint32_t*>(p.layers + l + 1) + tid) : 0u;
     // ---- phase 1: pre-mixer RMSNorm + input projection (+ DeltaNet conv epilogue) ----
     if (l > 0 && !grid_barrier(p, sh, ++nbar, tid)) return;
     {
@@ -1081,6 +1088,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
       }
     }
     if (!grid_barrier(p, sh, ++nbar, tid)) return;
+    if (lw_mine) reinterpret_cast<uint32_t*>(ltab + ((l + 1) & 1))[tid] = lw_next;
 
     if (L.kind == kDeltaNet) {
       // ---- phase 2 (DeltaNet): conv + SiLU + L2 norm + gates, delta rule on this CTA's rows of S, out-proj split-K ----
@@ -1588,23 +1596,23 @@ constexpr size_t kSmemLimit = 232448;
 
 // Shared memory before the scratch: the ring, Shared, the layer table, the staged input
 // vector and, with Q4 weights (2 ring slots), its per-lane sums and the row partial sums.
-static size_t decode_fixed_bytes(int H, bool q4, int xcap, int n_layers) {
-  const size_t lt = layer_table_bytes(n_layers);
+static size_t decode_fixed_bytes(int H, bool q4, int xcap, int ltab_entries) {
+  const size_t lt = layer_table_bytes(ltab_entries);
   if (!q4) return static_cast<size_t>(kSlots) * kSlotBytes + sizeof(Shared) + lt + static_cast<size_t>(H) * 4;
   return 2 * static_cast<size_t>(kSlotBytes) + sizeof(Shared) + lt + static_cast<size_t>(xcap) * 4 +
          static_cast<size_t>(xcap / 8) * 4 + static_cast<size_t>(kQ4PartFloats) * 4;
 }
 
-size_t decode_scratch_floats(int H, bool q4, int xcap, int n_layers) {
-  const size_t fixed = decode_fixed_bytes(H, q4, xcap, n_layers);
+size_t decode_scratch_floats(int H, bool q4, int xcap, int ltab_entries) {
+  const size_t fixed = decode_fixed_bytes(H, q4, xcap, ltab_entries);
   if (fixed >= kSmemLimit) return 0;
   size_t f = (kSmemLimit - fixed) / 4;
   f &= ~static_cast<size_t>(3);
   return f > 8192 ? 8192 : f;
 }
 
-size_t decode_smem_bytes(int H, bool q4, int xcap, int n_layers) {
-  return decode_fixed_bytes(H, q4, xcap, n_layers) + decode_scratch_floats(H, q4, xcap, n_layers) * 4;
+size_t decode_smem_bytes(int H, bool q4, int xcap, int ltab_entries) {
+  return decode_fixed_bytes(H, q4, xcap, ltab_entries) + decode_scratch_floats(H, q4, xcap, ltab_entries) * 4;
 }
 
 int decode_max_splits(int grid, int hkv) {
@@ -1624,7 +1632,7 @@ cudaError_t launch_hk(const DecodeParams& p, int grid, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, Q4, p.xcap, p.n_layers);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.H, Q4, p.xcap, p.ltab_full ? p.n_layers : 2);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;

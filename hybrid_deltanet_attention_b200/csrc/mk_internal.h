@@ -86,10 +86,12 @@ struct DecodeParams {
   int xcap;                           // floats of the staged input vector in shared memory
   float* obuf;                        // [max(Hd dv, Hq D)] mixer output (Q4)
   float* abuf;                        // [F] SwiGLU activation (Q4)
+  int ltab_full;                      // 1: the whole layer table in shared memory, 0: two slots
 };
 
-size_t decode_smem_bytes(int H, bool q4, int xcap, int n_layers);
-size_t decode_scratch_floats(int H, bool q4, int xcap, int n_layers);   // fp32 scratch per CTA left after the ring, the layer table, xs (and the Q4 tables)
+// ltab_entries: layers whose table entries the kernel keeps in shared memory (n_layers, or 2)
+size_t decode_smem_bytes(int H, bool q4, int xcap, int ltab_entries);
+size_t decode_scratch_floats(int H, bool q4, int xcap, int ltab_entries);   // fp32 scratch per CTA left after the ring, the layer table, xs (and the Q4 tables)
 constexpr int kQ4Block = 144;          // bytes per 256-weight super-block
 constexpr int kQ4PartFloats = 512;     // shared-memory partial sums of the Q4 row products
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t s);

@@ -140,7 +140,7 @@ __global__ void embed_rows_q4(const int32_t* __restrict__ tok, int T, const uint
 // the rows alone leave the GPU idle; partial sums go to a workspace and are reduced in a
 // fixed order); its rows stream through a private cp.async ring of 3 super-blocks.
 // Token tile: grid.z (8 tokens each).
-constexpr int kQ4Depth = 3;
+constexpr int kQ4Depth = 2;
 __device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -155,7 +155,7 @@ __device__ __forceinline__ uint32_t q4_pair_bf16(uint32_t spread, int hi4) {
   return ((hi4 ? (spread >> 4) : spread) & 0x000F000Fu) | 0x43004300u;
 }
 
-__global__ void __launch_bounds__(128) q4_linear_mma(const uint16_t* __restrict__ xhi, const uint16_t* __restrict__ xlo,
+__global__ void __launch_bounds__(128, 5) q4_linear_mma(const uint16_t* __restrict__ xhi, const uint16_t* __restrict__ xlo,
                                                      int ldx, const uint8_t* __restrict__ W, long long ldw,
                                                      float* __restrict__ out, long long ldo, int T, int N, int K,
                                                      int sb_per_split, int accumulate) {
@@ -224,9 +224,11 @@ __global__ void __launch_bounds__(128) q4_linear_mma(const uint16_t* __restrict_
 #pragma unroll
       for (int h = 0; h < 2; ++h) {   // k-step: weights 16 h .. 16 h + 15 of the sub-block
         const int kb = sb * 256 + 32 * j + 16 * h;
-        uint32_t bh0 = *reinterpret_cast<const uint32_t*>(xh + kb), bh1 = *reinterpret_cast<const uint32_t*>(xh + kb + 8);
-        uint32_t bl0 = *reinterpret_cast<const uint32_t*>(xl + kb), bl1 = *reinterpret_cast<const uint32_t*>(xl + kb + 8);
-        if (!tok_ok) bh0 = bh1 = bl0 = bl1 = 0u;
+        uint32_t bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;
+        if (tok_ok) {
+          bh0 = *reinterpret_cast<const uint32_t*>(xh + kb); bh1 = *reinterpret_cast<const uint32_t*>(xh + kb + 8);
+          bl0 = *reinterpret_cast<const uint32_t*>(xl + kb); bl1 = *reinterpret_cast<const uint32_t*>(xl + kb + 8);
+        }
 #pragma unroll
         for (int gr = 0; gr < 2; ++gr) {
           const uint32_t a0 = q4_pair_bf16(sp[2 * gr][0], h), a1 = q4_pair_bf16(sp[2 * gr + 1][0], h);
