@@ -305,6 +305,7 @@ size_t layer_block_bytes(const mk_config& c, char kind) {
     b += 2 * align256(qd * rb);                               // w_outT, w_out (K-major, prefill)
   }
   b += 4 * align256(static_cast<size_t>(c.ffn) * rb);     // gate, up, downT, down (K-major, prefill)
+  b += align256(2 * static_cast<size_t>(c.ffn) * rb);     // gate / up interleaved by 64 rows (prefill)
   return b;
 }
 
@@ -662,6 +663,16 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     off += align256(static_cast<size_t>(c.ffn) * rb);
     pl.w_down = P + off;
     if (e == cudaSuccess) e = copy(p + "mlp.w_down", off);
+    off += align256(static_cast<size_t>(c.ffn) * rb);
+    pl.w_gu = P + off;   // rows 128 b .. + 63: gate rows 64 b ..; rows 128 b + 64 .. + 127: up rows 64 b ..
+    if (e == cudaSuccess && c.ffn % 64 == 0) {
+      const size_t blk = 64 * rb;
+      e = cudaMemcpy2DAsync(P + off, 2 * blk, got[p + "mlp.w_gate"]->data, blk, blk, c.ffn / 64,
+                            cudaMemcpyDeviceToDevice, s);
+      if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(P + off + blk, 2 * blk, got[p + "mlp.w_up"]->data, blk, blk, c.ffn / 64,
+                              cudaMemcpyDeviceToDevice, s);
+    }
     m->layers_host.push_back(lw);
     m->pf_layers.push_back(pl);
   }

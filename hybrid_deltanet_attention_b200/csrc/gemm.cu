@@ -66,7 +66,8 @@ template <int BN>
 __global__ void __launch_bounds__(192, 1)
     linear_kernel(const __grid_constant__ CUtensorMap ta_hi, const __grid_constant__ CUtensorMap ta_lo,
                   const __grid_constant__ CUtensorMap tb, float* __restrict__ C, long long ldc, int M, int N, int K,
-                  int accumulate, int* err, float* __restrict__ ws, int nz) {
+                  int accumulate, int* err, float* __restrict__ ws, int nz, uint16_t* __restrict__ act_hi,
+                  uint16_t* __restrict__ act_lo) {
   using S = GemmShape<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -197,6 +198,38 @@ __global__ void __launch_bounds__(192, 1)
         accz = 0;
       }
       const int m = m0 + row;
+      if (act_hi) {   // SwiGLU epilogue: gate columns pair with the up columns 64 to their right
+        const uint32_t tbase = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          if (((n0 + c0) & 127) >= 64) continue;
+          float gv[16], uv[16];
+          tc::tmem_ld16(tbase + c0, gv);
+          tc::tmem_ld16(tbase + c0 + 64, uv);
+          if (m < M && n0 + c0 + 64 < N) {
+            const long long f = static_cast<long long>(m) * (N / 2) + ((n0 + c0) >> 7) * 64 + ((n0 + c0) & 63);
+            uint32_t h[8], l[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float a0 = siluf_(gv[2 * j]) * uv[2 * j];
+              const float a1 = siluf_(gv[2 * j + 1]) * uv[2 * j + 1];
+              const uint16_t h0 = f_to_bf16(a0), h1 = f_to_bf16(a1);
+              h[j] = h0 | (static_cast<uint32_t>(h1) << 16);
+              l[j] = f_to_bf16(a0 - bf16_to_f(h0)) | (static_cast<uint32_t>(f_to_bf16(a1 - bf16_to_f(h1))) << 16);
+            }
+            uint4* dh = reinterpret_cast<uint4*>(act_hi + f);
+            uint4* dl = reinterpret_cast<uint4*>(act_lo + f);
+            dh[0] = make_uint4(h[0], h[1], h[2], h[3]);
+            dh[1] = make_uint4(h[4], h[5], h[6], h[7]);
+            dl[0] = make_uint4(l[0], l[1], l[2], l[3]);
+            dl[1] = make_uint4(l[4], l[5], l[6], l[7]);
+          }
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&gb->acc_empty[buf]);
+        continue;
+      }
       float* crow = Cz + static_cast<long long>(m) * ldz + n0;
       const bool vec = (ldz % 4 == 0) && ((reinterpret_cast<uintptr_t>(Cz) & 15) == 0);
 #pragma unroll 1
@@ -340,7 +373,7 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
   // split K when the tile grid leaves most SMs idle (few tokens) and the workspace holds it
   const int tiles = static_cast<int>(grid.x * grid.y), nk = a.K / kBK;
   int nz = 1;
-  if (a.ws && grid.y == 1 && tiles < 148 && nk >= 6) {   // few tokens (one M tile) and few N tiles
+  if (a.ws && !a.act_hi && grid.y == 1 && tiles < 148 && nk >= 6) {   // few tokens (one M tile) and few N tiles
     nz = std::min({(148 + tiles - 1) / tiles, nk / 3, 16});   // about one wave, >= 3 K blocks per CTA
     const long long need = static_cast<long long>(a.M) * a.N;
     while (nz > 1 && need * nz > a.ws_floats) --nz;
@@ -348,7 +381,7 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
   const int items = tiles * nz;
   const int nctas = std::min(items, 148);
   linear_kernel<BN><<<nctas, 192, S::kSmemBytes, s>>>(ma_hi, ma_lo, mb, a.c, a.ldc, a.M, a.N, a.K, a.accumulate,
-                                                      a.err, a.ws, nz);
+                                                      a.err, a.ws, nz, a.act_hi, a.act_lo);
   cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess && nz > 1) {
     const long long total = static_cast<long long>(a.M) * a.N;
@@ -375,6 +408,9 @@ cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s) {
   if (a.K <= 0 || a.K % kBK != 0 || a.ldw_bytes % 16 != 0 || a.ldw_bytes < 2LL * a.K ||
       (reinterpret_cast<uintptr_t>(a.x_hi) & 15) || (reinterpret_cast<uintptr_t>(a.x_lo) & 15) ||
       (reinterpret_cast<uintptr_t>(a.w) & 15))
+    return cudaErrorInvalidValue;
+  if (a.act_hi && (a.N % 128 != 0 || !a.act_lo || (reinterpret_cast<uintptr_t>(a.act_hi) & 15) ||
+                   (reinterpret_cast<uintptr_t>(a.act_lo) & 15)))
     return cudaErrorInvalidValue;
   // 256-wide tiles for many tokens and wide outputs; 128-wide for few tokens (more CTAs to split over)
   return (a.N >= 2048 && a.M > kBM) ? launch_bn<256>(a, s) : launch_bn<128>(a, s);

@@ -115,6 +115,11 @@ struct LinearArgs {
   int* err;
   float* ws = nullptr;      // optional split-K partials (when the tile grid is smaller than the GPU)
   long long ws_floats = 0;
+  // SwiGLU epilogue: when set, W's rows interleave gate and up in blocks of 64 (rows 128p .. +63
+  // gate features 64p .., rows 128p + 64 .. up features 64p ..), N is a multiple of 128, and
+  // instead of C the kernel writes act = SiLU(gate) * up as bf16 high / low parts [M][N / 2]
+  uint16_t* act_hi = nullptr;
+  uint16_t* act_lo = nullptr;
 };
 cudaError_t launch_split_bf16(const float* x, long long ldx, uint16_t* hi, uint16_t* lo, int M, int K, cudaStream_t s);
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s);

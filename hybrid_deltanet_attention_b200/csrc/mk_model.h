@@ -41,6 +41,7 @@ struct mk_prefill_ws {
 struct mk_prefill_layer {   // K-major copies of the projections the decode kernel keeps transposed
   const uint8_t* w_out;      // [H][K_mix] bf16
   const uint8_t* w_down;     // [H][F] bf16
+  const uint8_t* w_gu;       // [2F][H] bf16: gate and up rows interleaved in blocks of 64 (SwiGLU epilogue)
 };
 
 // What a verify pass keeps so that the recurrent state can be committed to any accepted

@@ -1876,11 +1876,30 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
     if (e != cudaSuccess) break;
     rms_split<<<T, rms_threads(T), 0, s>>>(pf.h, H, L.norm2, b.eps, pf.xhi, pf.xlo);
     chk();
-    linear(L.w_gate, 2LL * H, F, H, pf.z, 2LL * F, 0);
-    linear(L.w_up, 2LL * H, F, H, pf.z + F, 2LL * F, 0);
-    act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
-    chk();
-    linear(q4 ? L.w_down_q4 : PL.w_down, 2LL * F, H, F, pf.h, H, 1);
+    if (!q4 && PL.w_gu && T > 128 && F % 64 == 0) {
+      // gate and up in one GEMM whose epilogue writes SiLU(gate) * up as bf16 high / low parts
+      // (into the projection buffer, which holds 2 T F floats); the down-projection reads them
+      uint16_t* ahi = reinterpret_cast<uint16_t*>(pf.z);
+      uint16_t* alo = ahi + static_cast<size_t>(T) * F;
+      if (e == cudaSuccess) {
+        LinearArgs a{pf.xhi, pf.xlo, PL.w_gu, 2LL * H, pf.z, 2LL * F, T, 2 * F, H, 0, b.err};
+        a.act_hi = ahi;
+        a.act_lo = alo;
+        e = launch_linear(a, s);
+        ++m->launches;
+      }
+      if (e == cudaSuccess) {
+        LinearArgs a{ahi, alo, PL.w_down, 2LL * F, pf.h, H, T, H, F, 1, b.err, pf.splitk, kSplitKFloats};
+        e = launch_linear(a, s);
+        ++m->launches;
+      }
+    } else {
+      linear(L.w_gate, 2LL * H, F, H, pf.z, 2LL * F, 0);
+      linear(L.w_up, 2LL * H, F, H, pf.z + F, 2LL * F, 0);
+      act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
+      chk();
+      linear(q4 ? L.w_down_q4 : PL.w_down, 2LL * F, H, F, pf.h, H, 1);
+    }
   }
   return e;
 }
