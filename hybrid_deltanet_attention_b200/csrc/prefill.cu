@@ -1421,21 +1421,43 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return warp_max(t);
 }
 
-__global__ void attn_softmax_split(const float* __restrict__ S, int nk, const int* __restrict__ posp, int off,
-                                   uint16_t* __restrict__ phi, uint16_t* __restrict__ plo) {
+__global__ void __launch_bounds__(256) attn_softmax_split(const float* __restrict__ S, int nk,
+                                                          const int* __restrict__ posp, int off,
+                                                          uint16_t* __restrict__ phi, uint16_t* __restrict__ plo) {
+  extern __shared__ float4 srow4[];   // [nk / 4] the row's scores, then e^{s - max}
   __shared__ float red[32];
   const int t = blockIdx.x;
   const int last = min(*posp + off + t, nk - 1);   // keys 0 .. last
-  const float* r = S + static_cast<long long>(t) * nk;
+  const int n4 = (last + 4) >> 2;                  // float4 groups holding keys 0 .. last
+  const float4* r4 = reinterpret_cast<const float4*>(S + static_cast<long long>(t) * nk);   // nk % 4 == 0
   float mx = -INFINITY;
-  for (int j = threadIdx.x; j <= last; j += blockDim.x) mx = fmaxf(mx, r[j]);
-  mx = block_max(mx, red);
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {   // one read of the row
+    float4 v = r4[i];
+    const int j = 4 * i;
+    if (j + 1 > last) v.y = -INFINITY;
+    if (j + 2 > last) v.z = -INFINITY;
+    if (j + 3 > last) v.w = -INFINITY;
+    srow4[i] = v;
+    mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
+  }
+  mx = block_max(mx, red);   // its barriers also publish srow
   float sum = 0.f;
-  for (int j = threadIdx.x; j <= last; j += blockDim.x) sum += expf(r[j] - mx);
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    float4 v = srow4[i];
+    v = make_float4(expf(v.x - mx), expf(v.y - mx), expf(v.z - mx), expf(v.w - mx));
+    srow4[i] = v;   // each thread rewrites only its own groups
+    sum += (v.x + v.y) + (v.z + v.w);
+  }
   sum = block_sum(sum, red);
   const float inv = 1.0f / sum;
-  for (int j = threadIdx.x; j < nk; j += blockDim.x)
-    put_split(phi, plo, static_cast<long long>(t) * nk + j, j <= last ? expf(r[j] - mx) * inv : 0.f);
+  for (int i = threadIdx.x; i < nk / 4; i += blockDim.x) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < n4) {
+      v = srow4[i];
+      v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
+    }
+    put_split4(phi, plo, static_cast<long long>(t) * nk + 4 * i, v);
+  }
 }
 
 // VT[d][j] = V[j][d] for the keys up to the pass's last position, zero past it.
@@ -1846,7 +1868,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
               ++m->launches;
             }
             if (e != cudaSuccess) break;
-            attn_softmax_split<<<T, kPT, 0, s>>>(pf.sbuf, nk, b.pos, off, pf.phi, pf.plo);
+            attn_softmax_split<<<T, kPT, static_cast<size_t>(nk) * sizeof(float), s>>>(pf.sbuf, nk, b.pos, off,
+                                                                                       pf.phi, pf.plo);
             chk();
             if (e == cudaSuccess) {   // O = P V
               LinearArgs a{pf.phi, pf.plo, pf.vt, 2LL * nk, pf.o + static_cast<size_t>(hq) * D, qd, T, D, nk, 0, b.err,
