@@ -373,8 +373,10 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
   // split K when the tile grid leaves most SMs idle (few tokens) and the workspace holds it
   const int tiles = static_cast<int>(grid.x * grid.y), nk = a.K / kBK;
   int nz = 1;
-  if (a.ws && !a.act_hi && grid.y == 1 && tiles < 148 && nk >= 6) {   // few tokens (one M tile) and few N tiles
-    nz = std::min({(148 + tiles - 1) / tiles, nk / 3, 16});   // about one wave, >= 3 K blocks per CTA
+  // few tokens (one M tile) and few N tiles: about one wave, >= 3 K blocks per CTA; a short
+  // prompt (up to 8 M tiles) whose tile grid fills at most half the GPU: 2-4 splits of >= 8 K blocks
+  if (a.ws && !a.act_hi && ((grid.y == 1 && tiles < 148 && nk >= 6) || (grid.y <= 8 && tiles <= 74 && nk >= 16))) {
+    nz = grid.y == 1 ? std::min({(148 + tiles - 1) / tiles, nk / 3, 16}) : std::min({(148 + tiles - 1) / tiles, nk / 8, 4});
     const long long need = static_cast<long long>(a.M) * a.N;
     while (nz > 1 && need * nz > a.ws_floats) --nz;
   }
