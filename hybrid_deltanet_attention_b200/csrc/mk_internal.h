@@ -13,7 +13,7 @@ constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = kConsumerThreads + 32;
 constexpr int kSlotBytes = 65536;
 constexpr int kSlots = 3;
-constexpr int kAttnSub = 64;          // positions per online-softmax sub-block
+constexpr int kAttnSub = 128;         // positions per online-softmax sub-block (one 64 KB ring slot of D = 256 keys)
 constexpr int kResCopies = 2;          // copies of each residual delta (CTA c adds into copy c % 2)
 constexpr int kAttnMinChunk = 16;     // smallest split-K chunk of the KV cache
 
