@@ -280,6 +280,110 @@ __global__ void __launch_bounds__(128, 5) q4_linear_mma(const uint16_t* __restri
     }
 }
 
+// C[t][n] (+)= sum_k X[t][k] W[n][k] for bf16 rows W and up to 8 tokens per CTA (few-token
+// passes: verify, short tails), on mma.sync m16n8k16: W tiles as the A operand (ldmatrix from
+// a per-warp cp.async ring of 64-wide K blocks, 16-byte pieces XOR-swizzled by row so the
+// matrix loads are conflict-free), the tokens' bf16 high / low activation parts as B, fp32
+// accumulation in registers. A warp owns 32 rows and a slice of K blocks (grid.y splits K;
+// partials reduced by q4_split_reduce); grid.z walks 8-token tiles.
+constexpr int kBfDepth = 4;
+__global__ void __launch_bounds__(128, 3) bf16_linear_mma(const uint16_t* __restrict__ xhi,
+                                                          const uint16_t* __restrict__ xlo, int ldx,
+                                                          const uint8_t* __restrict__ W, long long ldw,
+                                                          float* __restrict__ out, long long ldo, int T, int N, int K,
+                                                          int kb_per_split, int accumulate) {
+  constexpr int DEP = kBfDepth, RPW = 32, KB = 64;   // K block: 64 bf16 = 128 bytes per row
+  extern __shared__ __align__(16) uint8_t bfm[];     // per warp: [DEP][32 rows][128 B]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  uint8_t* ring = bfm + warp * DEP * RPW * 128;
+  const int n0 = blockIdx.x * 128 + warp * RPW;
+  const int nkb = K / KB;
+  const int kbA = blockIdx.y * kb_per_split, kbB = min(nkb, kbA + kb_per_split);
+  const int t0 = blockIdx.z * 8;
+  const bool tok_ok = t0 + g < T;
+  const uint16_t* xh = xhi + static_cast<long long>(tok_ok ? t0 + g : 0) * ldx + 2 * c;
+  const uint16_t* xl = xlo + static_cast<long long>(tok_ok ? t0 + g : 0) * ldx + 2 * c;
+  // copies: 32 rows x 8 pieces of 16 bytes per K block, 8 per lane; piece p of row r lands at
+  // r * 128 + 16 (p ^ (r & 7))
+  const uint8_t* src[8];
+  int dsto[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int i = lane + 32 * m, r = i >> 3, pc = i & 7;
+    src[m] = W + static_cast<long long>(min(n0 + r, N - 1)) * ldw + pc * 16;
+    dsto[m] = r * 128 + 16 * (pc ^ (r & 7));
+  }
+  auto issue = [&](int kb) {
+    if (kb < kbB) {
+      uint8_t* slot = ring + ((kb - kbA) % DEP) * RPW * 128;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) cp_async16(slot + dsto[m], src[m] + static_cast<long long>(kb) * 128, 16u);
+    }
+    cp_async_commit();
+  };
+  if (n0 < N) {
+#pragma unroll
+    for (int p = 0; p < DEP - 1; ++p) issue(kbA + p);
+  }
+  float acc[2][4];
+#pragma unroll
+  for (int gr = 0; gr < 2; ++gr)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[gr][i] = 0.f;
+  // ldmatrix.x4 addresses: lanes 0-15 rows 0..15 at k 0..7, lanes 16-31 rows 0..15 at k 8..15
+  const int lr = lane & 15, lk = lane >> 4;
+  for (int kb = kbA; kb < kbB && n0 < N; ++kb) {
+    issue(kb + DEP - 1);
+    cp_async_wait<DEP - 1>();
+    __syncwarp();
+    const uint8_t* slot = ring + ((kb - kbA) % DEP) * RPW * 128;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {   // 16-wide k steps
+      const int kglob = kb * KB + 16 * ks;
+      uint32_t bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;   // padding tokens stay zero
+      if (tok_ok) {
+        bh0 = *reinterpret_cast<const uint32_t*>(xh + kglob);
+        bh1 = *reinterpret_cast<const uint32_t*>(xh + kglob + 8);
+        bl0 = *reinterpret_cast<const uint32_t*>(xl + kglob);
+        bl1 = *reinterpret_cast<const uint32_t*>(xl + kglob + 8);
+      }
+#pragma unroll
+      for (int gr = 0; gr < 2; ++gr) {
+        const int r = 16 * gr + lr, pc = 2 * ks + lk;
+        const uint32_t addr = smem_u32(slot + r * 128 + 16 * (pc ^ (r & 7)));
+        uint32_t a0, a1, a2, a3;
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                     : "r"(addr));
+        mma_bf16_16816(acc[gr], a0, a1, a2, a3, bh0, bh1);
+        mma_bf16_16816(acc[gr], a0, a1, a2, a3, bl0, bl1);
+      }
+    }
+    __syncwarp();   // every lane is done with this slot before it is refilled
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+  if (n0 >= N) return;
+  float* dst = out;
+  long long ld = ldo;
+  bool add = accumulate != 0;
+  if (gridDim.y > 1) {   // partial sums [split][T][N]
+    dst = out + static_cast<long long>(blockIdx.y) * T * N;
+    ld = N;
+    add = false;
+  }
+#pragma unroll
+  for (int gr = 0; gr < 2; ++gr)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int n = n0 + 16 * gr + g + 8 * (i >> 1), t = t0 + 2 * c + (i & 1);
+      if (n < N && t < T) {
+        float* p = dst + static_cast<long long>(t) * ld + n;
+        *p = add ? *p + acc[gr][i] : acc[gr][i];
+      }
+    }
+}
+
 // out[t][n] (+)= sum over splits z of ws[z][t][n], in order of z.
 __global__ void q4_split_reduce(const float* __restrict__ ws, int nz, int T, int N, float* __restrict__ out,
                                 long long ldo, int accumulate) {
@@ -1741,6 +1845,30 @@ cudaError_t launch_q4_linear(const uint16_t* xhi, const uint16_t* xlo, const voi
   return e;
 }
 
+// bf16 linear layer for few-token passes (T <= 8 per tile) over the tokens' bf16 high / low parts.
+cudaError_t launch_bf16_linear(const uint16_t* xhi, const uint16_t* xlo, const void* W, long long ldw, float* C,
+                               long long ldc, int T, int N, int K, int accumulate, float* ws, long long ws_floats,
+                               cudaStream_t s) {
+  if (T <= 0 || N <= 0) return cudaSuccess;
+  const int tiles = (N + 127) / 128, ttiles = (T + 7) / 8, nkb = K / 64;
+  int nz = std::min(nkb, std::max(1, (3 * 148 + tiles * ttiles - 1) / (tiles * ttiles)));
+  if (static_cast<long long>(nz) * T * N > ws_floats) nz = 1;
+  int per = (nkb + nz - 1) / nz;
+  nz = (nkb + per - 1) / per;
+  if (nz <= 1) per = nkb;
+  constexpr size_t smem = 4ull * kBfDepth * 32 * 128;
+  bf16_linear_mma<<<dim3(tiles, nz, ttiles), 128, smem, s>>>(xhi, xlo, K, static_cast<const uint8_t*>(W), ldw,
+                                                              nz > 1 ? ws : C, ldc, T, N, K, per, accumulate);
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess && nz > 1) {
+    const long long tot = static_cast<long long>(T) * N;
+    q4_split_reduce<<<static_cast<int>(std::min<long long>((tot + 255) / 256, 1184)), 256, 0, s>>>(ws, nz, T, N, C, ldc,
+                                                                                               accumulate);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
 cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaStream_t s,
                          const mk_verify_ws* vs = nullptr) {
   const mk_config& c = m->cfg;
@@ -1761,6 +1889,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
     if (q4) {
       e = launch_q4_linear(pf.xhi, pf.xlo, w, q4_row_bytes(K) + (ldw - 2LL * K), out, ldc, T, N, K, acc, pf.splitk,
                            kSplitKFloats, s);
+    } else if (T <= 8) {
+      e = launch_bf16_linear(pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, pf.splitk, kSplitKFloats, s);
     } else {
       LinearArgs a{pf.xhi, pf.xlo, w, ldw, out, ldc, T, N, K, acc, b.err, pf.splitk, kSplitKFloats};
       e = launch_linear(a, s);
@@ -1941,6 +2071,9 @@ cudaError_t set_prefill_smem_limits() {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(bf16_linear_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(4 * kBfDepth * 32 * 128));
+  if (e == cudaSuccess)
     e = cudaFuncSetAttribute(q4_linear_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(4 * kQ4Depth * 32 * 144));
   if (e == cudaSuccess)
@@ -2013,6 +2146,10 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
   if (e == cudaSuccess && b.q4) {   // 4-bit tied LM head
     e = mk::launch_q4_linear(m->pf.xhi, m->pf.xlo, b.embed, b.row_bytes, logits, c.vocab, T, c.vocab, c.hidden, 0,
                              m->pf.splitk, mk::kSplitKFloats, s);
+    ++m->launches;
+  } else if (e == cudaSuccess && T <= 8) {   // bf16 tied LM head, few tokens
+    e = mk::launch_bf16_linear(m->pf.xhi, m->pf.xlo, b.embed, 2LL * c.hidden, logits, c.vocab, T, c.vocab, c.hidden, 0,
+                               m->pf.splitk, mk::kSplitKFloats, s);
     ++m->launches;
   } else if (e == cudaSuccess) {
     mk::LinearArgs a{m->pf.xhi, m->pf.xlo, b.embed, 2LL * c.hidden, logits, c.vocab, T, c.vocab, c.hidden, 0, b.err};
