@@ -179,13 +179,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest x over the ranks (a time: the slowest replica defines the job's time)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput of `world` independent replicas that each processed
+    `units_per_rank` units, timed by the slowest one (weak scaling)."""
+    return world * units_per_rank / seconds
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
@@ -320,7 +328,7 @@ def run_mk(args):
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
     decode_ms = sum(a.elapsed_time(b) for a, b in evs)
     decode_ms = max_over_ranks(decode_ms, world)
-    value = world * args.steps * TG / (total_ms / 1000.0)
+    value = replica_throughput(args.steps * TG, world, total_ms / 1000.0)
 
     # roofline of the decode kernel: algorithmic bytes per launch / average launch duration
     per = [bytes_per_token(cfg, P0 + i) for i in range(TG)]
@@ -354,7 +362,7 @@ def run_mk(args):
         for _ in range(e2e_steps):
             e2e_step()
         dt = max_over_ranks(time.perf_counter() - t0, world)
-        e2e = world * e2e_steps * TG / dt
+        e2e = replica_throughput(e2e_steps * TG, world, dt)
         e2e_io = (4, (TG + 1) * 4, "first token pinned host -> device, 128 decode launches over the seeded "
                                    "32K context, tokens device -> pinned host")
     else:
@@ -372,7 +380,7 @@ def run_mk(args):
             m.reset()
             m.generate(pinned_in.numpy(), TG, out=pinned_out.numpy())
         dt = max_over_ranks(time.perf_counter() - t0, world)
-        e2e = world * e2e_steps * TG / dt
+        e2e = replica_throughput(e2e_steps * TG, world, dt)
         e2e_io = (PROMPT * 4, TG * 4, "mk_generate: pinned host prompt (128) -> prefill -> 128 greedy tokens -> pinned host")
     if rank != 0:
         return 0
@@ -459,7 +467,7 @@ def run_prefill(args):
         barrier(world)
     assert m.sync() == 0
     ms = max_over_ranks(a.elapsed_time(b), world) / args.steps
-    value = world * T / (ms / 1000.0)
+    value = replica_throughput(T, world, ms / 1000.0)
     # end to end: pinned host prompt -> prefill -> next token to pinned host
     h_in = torch.from_numpy(prompt_np).pin_memory()
     h_out = torch.empty(1, dtype=torch.int32).pin_memory()
@@ -474,7 +482,7 @@ def run_prefill(args):
     t0 = time.perf_counter()
     for _ in range(args.steps):
         e2e_step()
-    e2e = world * args.steps * T / max_over_ranks(time.perf_counter() - t0, world)
+    e2e = replica_throughput(args.steps * T, world, max_over_ranks(time.perf_counter() - t0, world))
     if rank != 0:
         return 0
     macs = linear_macs_per_token(cfg) * (T - 1)          # the last token runs through the decode kernel
