@@ -602,9 +602,10 @@ def run_27b(args):
                    "tokens_per_pass": committed_total / n_pass,
                    "pass_ms": verify_ms / n_pass,
                    "tok_s_at_expected_acceptance": 3.689 / (verify_ms / n_pass / 1000.0),
-                   "verify_path": "one pass over the weights (batched layers, tcgen05 LM head, commit of the accepted prefix)"
-                   if small else "one pass over the 4-bit weights (batched layers, 4-bit linear layers on the CUDA "
-                                 "cores over the K+1 tokens, commit of the accepted prefix)"},
+                   "verify_path": "one pass over the weights (batched layers; linear layers and the LM head on "
+                                  "mma.sync bf16 tensor-core tiles over the K+1 tokens; commit of the accepted prefix)"
+                   if small else "one pass over the 4-bit weights (batched layers; 4-bit codes fed as exact bf16 to "
+                                 "mma.sync tensor-core tiles over the K+1 tokens; commit of the accepted prefix)"},
         "plain_decode": {"tok_s": 1000.0 / plain_ms, "ms_per_token": plain_ms,
                          "hbm_frac_of_measured": (bytes_w / (plain_ms / 1000.0) / 1e9) / measured_peaks()[0]},
         "clocks": clk.summary(),

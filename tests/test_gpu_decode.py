@@ -173,6 +173,44 @@ def test_device_error_word_on_bad_token(tiny):
     assert m.sync() == 0
 
 
+def test_grid_barrier_wait_gives_up(tiny):
+    """A grid-barrier wait that can never complete ends after its bounded limit (about a
+    second) with the timeout bit in the device error word, not with a hang or a fault.
+
+    The arrival counter the barrier polls is the first 32-bit word of the workspace; it is
+    set so far ahead of every CTA's target (in wrap-around order) that no arrival reaches
+    it: a flag that nothing sets. The producer lane, waiting meanwhile for a free ring
+    slot, runs into its own limit at about the same time, so either timeout bit may be the
+    one recorded; the other CTAs see the error word and stop. The reset that follows zeroes
+    the counter and the error word, and the next step is correct again.
+    """
+    cfg, m, W = tiny
+    dev = torch.device("cuda")
+    tok = torch.tensor([3], dtype=torch.int32, device=dev)
+    ref = torch.empty(1, dtype=torch.int32, device=dev)
+    m.reset()
+    m.decode(tok, ref)
+    assert m.sync() == 0
+    m.reset()
+    m.workspace[:4].view(torch.int32).fill_(-0x40000000)   # 0xC0000000 as an unsigned counter
+    out = torch.empty(1, dtype=torch.int32, device=dev)
+    import time
+    import hybrid_deltanet_attention_b200 as hda
+    t0 = time.monotonic()
+    m.decode(tok, out)
+    with pytest.raises(hda.MkError):
+        m.sync()
+    assert time.monotonic() - t0 < 30.0
+    err = m.device_error()
+    assert err & (hda.MK_DEVERR_BARRIER_TIMEOUT | hda.MK_DEVERR_PIPE_TIMEOUT), hex(err)
+    assert not err & ~(hda.MK_DEVERR_BARRIER_TIMEOUT | hda.MK_DEVERR_PIPE_TIMEOUT), hex(err)
+    m.reset()
+    assert m.sync() == 0
+    m.decode(tok, out)
+    assert m.sync() == 0
+    assert int(out.item()) == int(ref.item())
+
+
 @pytest.fixture(scope="module")
 def m08():
     cfg = synth.QWEN_08B
