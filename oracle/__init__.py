@@ -19,3 +19,4 @@ weights and activations" taken literally -- for diagnostics.
 from .model import *          # noqa: F401,F403
 from .chunked import *        # noqa: F401,F403
 from .q4k import *            # noqa: F401,F403
+from .sampling import *       # noqa: F401,F403
