@@ -25,6 +25,7 @@ import subprocess
 import sys
 import tempfile
 import time
+from typing import Optional
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
@@ -157,6 +158,76 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sms)}
+
+
+class EnergyMeter:
+    """Energy this GPU drew over the timed region, from NVML's total-energy counter
+    (millijoules since the driver loaded). Read only: nothing is set or reset. The GPU
+    is found by its PCI bus id (the CUDA index can differ from NVML's), else by index.
+    The counter advances in steps of tens of milliseconds and the board is shared with
+    other jobs' idle draw, so the figure is advisory. `nvml` may be a stand-in module."""
+
+    def __init__(self, cuda_index: int, pci_bus_id: Optional[str] = None, nvml=None):
+        self.index, self.bus, self.nv = cuda_index, pci_bus_id, nvml
+        self.h = None
+        self.e0 = self.e1 = None
+        self.t0 = self.t1 = None
+
+    def __enter__(self):
+        try:
+            if self.nv is None:
+                import pynvml
+                self.nv = pynvml
+            self.nv.nvmlInit()
+            h = None
+            if self.bus:
+                try:
+                    h = self.nv.nvmlDeviceGetHandleByPciBusId(self.bus)
+                except Exception:
+                    h = None
+            self.h = h if h is not None else self.nv.nvmlDeviceGetHandleByIndex(self.index)
+        except Exception:
+            self.h = None
+        return self
+
+    def _read(self):
+        try:
+            return float(self.nv.nvmlDeviceGetTotalEnergyConsumption(self.h))
+        except Exception:
+            return None
+
+    def start(self):
+        if self.h is not None:
+            self.e0, self.t0 = self._read(), time.perf_counter()
+
+    def stop(self):
+        if self.h is not None:
+            self.e1, self.t1 = self._read(), time.perf_counter()
+
+    def __exit__(self, *a):
+        if self.h is not None:
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
+
+    def summary(self, tokens: int):
+        if self.e0 is None or self.e1 is None or self.e1 < self.e0 or tokens <= 0:
+            return None
+        j = (self.e1 - self.e0) / 1000.0
+        sec = max(self.t1 - self.t0, 1e-9)
+        return {"joules": j, "seconds": sec, "avg_w": j / sec, "j_per_token": j / tokens,
+                "tokens_per_j": tokens / j if j > 0 else None,
+                "source": "NVML total-energy counter of this GPU before and after the timed region (read only; "
+                          "advisory: counter granularity, shared board)"}
+
+
+def cuda_pci_bus_id(torch, index: int) -> Optional[str]:
+    try:
+        p = torch.cuda.get_device_properties(index)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
 
 
 def dist_setup(n_gpus: int):
@@ -312,14 +383,17 @@ def run_mk(args):
     launches0 = m.launches
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    cur = torch.cuda.current_device()
+    with ClockSampler(cur) as clk, EnergyMeter(cur, cuda_pci_bus_id(torch, cur)) as energy:
         barrier(world)
         torch.cuda.synchronize()
+        energy.start()
         t_start.record(stream)
         for k in range(args.steps):
             one_step(evs[k])
         t_end.record(stream)
         torch.cuda.synchronize()
+        energy.stop()
         barrier(world)
     dev_err = m.sync()
     if dev_err:
@@ -407,6 +481,7 @@ def run_mk(args):
                 "what": e2e_io[2]},
         "gpu_launches": launches,
         "clocks": clocks,
+        "energy": energy.summary(args.steps * TG),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -584,6 +659,38 @@ def run_27b(args):
             committed_total += n + 1
             verify_ms += a.elapsed_time(b)
     assert m.sync() == 0
+    # sampling-mode verify passes at temperature 1 (same draft recipe; the uniforms are
+    # seeded inputs drawn on the host before the pass)
+    m.state.copy_(snap)
+    m.set_position(CTX - 1)
+    last = int(ctx[-1].item())
+    samp_total, samp_ms = 0, 0.0
+    urng = np.random.default_rng(4)
+    uni = torch.empty(2 * (K + 1), dtype=torch.float32, device=dev)
+    for ps in range(args.warmup + n_pass):
+        pos = int(m.pos_tensor.item())
+        keep = m.state.clone()
+        g_t[0] = last
+        for i in range(K):
+            m.decode(g_t[i:i + 1], g_t[i + 1:i + 2])
+        greedy = g_t[1:].cpu().numpy()
+        m.state.copy_(keep)
+        m.set_position(pos)
+        use, ids = synth.draft_choices(4, ps, K, cfg.vocab)
+        drafts = synth.compose_drafts(greedy, use, ids, cfg.vocab)
+        tin = torch.from_numpy(np.concatenate([[last], drafts]).astype(np.int32)).to(dev)
+        uni.copy_(torch.from_numpy(urng.random(2 * (K + 1)).astype(np.float32)))
+        torch.cuda.synchronize()
+        a.record(stream)
+        m.verify_sampled(tin, 1.0, uni, n_acc, out)
+        b.record(stream)
+        torch.cuda.synchronize()
+        n = int(n_acc.item())
+        last = int(out[n].item())
+        if ps >= args.warmup:
+            samp_total += n + 1
+            samp_ms += a.elapsed_time(b)
+    assert m.sync() == 0
     if rank != 0:
         return 0
     eff = committed_total / (verify_ms / 1000.0)
@@ -606,6 +713,10 @@ def run_27b(args):
                                   "mma.sync bf16 tensor-core tiles over the K+1 tokens; commit of the accepted prefix)"
                    if small else "one pass over the 4-bit weights (batched layers; 4-bit codes fed as exact bf16 to "
                                  "mma.sync tensor-core tiles over the K+1 tokens; commit of the accepted prefix)"},
+        "sampled_verify": {"temperature": 1.0, "pass_ms": samp_ms / n_pass, "tokens_per_pass": samp_total / n_pass,
+                           "acceptance_cost_ms": (samp_ms - verify_ms) / n_pass,
+                           "note": "random-init weights give a near-uniform distribution at temperature 1, so "
+                                   "drafts are rarely kept; the pass time is the figure"},
         "plain_decode": {"tok_s": 1000.0 / plain_ms, "ms_per_token": plain_ms,
                          "hbm_frac_of_measured": (bytes_w / (plain_ms / 1000.0) / 1e9) / measured_peaks()[0]},
         "clocks": clk.summary(),

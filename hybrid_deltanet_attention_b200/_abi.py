@@ -34,7 +34,7 @@ MK_MAX_LAYERS = 128
 # every symbol include/mk.h declares
 EXPORTS = [
     "mk_query_sizes", "mk_load_weights", "mk_reset_state", "mk_set_position", "mk_prefill",
-    "mk_decode_step", "mk_decode_step_noalloc", "mk_verify_drafts", "mk_generate", "mk_sync_status", "mk_phase_trace", "mk_launch_count",
+    "mk_decode_step", "mk_decode_step_noalloc", "mk_verify_drafts", "mk_verify_drafts_sampled", "mk_generate", "mk_sync_status", "mk_phase_trace", "mk_launch_count",
     "mk_linear", "mk_last_error", "mk_free",
 ]
 
@@ -114,6 +114,7 @@ def load_library(path: str = LIB_PATH) -> C.CDLL:
         "mk_decode_step": (C.c_int, [vp, vp, vp, vp, vp]),
         "mk_decode_step_noalloc": (C.c_int, [vp, vp, vp, vp, vp]),
         "mk_verify_drafts": (C.c_int, [vp, vp, i32, vp, vp, vp, vp]),
+        "mk_verify_drafts_sampled": (C.c_int, [vp, vp, i32, C.c_float, vp, vp, vp, vp, vp]),
         "mk_generate": (C.c_int, [vp, vp, i32, vp, i32, vp]),
         "mk_sync_status": (C.c_int, [vp, vp, p_i32]),
         "mk_phase_trace": (C.c_int, [vp, vp, i32]),

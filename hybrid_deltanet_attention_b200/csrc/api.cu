@@ -258,7 +258,7 @@ struct Layout {
   long long pf_nk;
   // batched verify saves
   int vf_rows;
-  size_t vf_delta, vf_k, vf_g, vf_raw, vf_logits, vf_greedy;
+  size_t vf_delta, vf_k, vf_g, vf_raw, vf_logits, vf_greedy, vf_stats;
 };
 
 // Tokens per batched prefill pass: the whole context up to 4096 (64 with 4-bit weights,
@@ -407,6 +407,7 @@ Layout make_layout(const mk_config& c, int grid) {
     L.vf_raw = off; off = align256(off + R * C * 4);
     L.vf_logits = off; off = align256(off + static_cast<size_t>(L.vf_rows) * c.vocab * 4);
     L.vf_greedy = off; off = align256(off + static_cast<size_t>(L.vf_rows) * 4);
+    L.vf_stats = off; off = align256(off + static_cast<size_t>(L.vf_rows) * 16);   // sampled verify: max, sum
   }
   L.sz.workspace_bytes = off;
   L.sz.grid_ctas = grid;
@@ -772,6 +773,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     m->vf.raw = reinterpret_cast<float*>(W + L.vf_raw);
     m->vf.logits = reinterpret_cast<float*>(W + L.vf_logits);
     m->vf.greedy = reinterpret_cast<int32_t*>(W + L.vf_greedy);
+    m->vf.stats = reinterpret_cast<double*>(W + L.vf_stats);
   }
   *out = m;
   return MK_OK;
@@ -879,6 +881,21 @@ int mk_verify_drafts(mk_model* m, const int32_t* d_tokens, int32_t K, int32_t* d
   m->pos_hint = pos0 + 1;   // at least one position is always committed; the exact count is on the device
   m->pos_max = pos0 + K + 1;
   return MK_OK;
+}
+
+int mk_verify_drafts_sampled(mk_model* m, const int32_t* d_tokens, int32_t K, float temperature,
+                             const float* d_uniforms, int32_t* d_n_accepted, int32_t* d_out_tokens, float* d_logits,
+                             void* stream) {
+  if (!m) return fail(MK_ERR_ARG, "model is NULL");
+  if (!d_tokens || !d_uniforms || !d_n_accepted || !d_out_tokens) return fail(MK_ERR_ARG, "pointer is NULL");
+  if (K < 1 || K > m->cfg.max_draft) return fail(MK_ERR_ARG, "K outside [1, max_draft]");
+  if (!(temperature > 0.0f) || !std::isfinite(temperature))
+    return fail(MK_ERR_ARG, "temperature must be positive and finite");
+  if (m->pos_hint + K + 1 > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "drafts exceed the context capacity");
+  if (m->vf.rows < K + 1)
+    return fail(MK_ERR_CAPACITY, "sampled verify needs the batched verify workspace (max_draft + 1 <= 64)");
+  return mk_verify_batched(m, d_tokens, K, d_n_accepted, d_out_tokens, d_logits, static_cast<cudaStream_t>(stream),
+                           temperature, d_uniforms);
 }
 
 int mk_generate(mk_model* m, const int32_t* h_prompt, int32_t n_prompt, int32_t* h_out, int32_t n_new, void* stream) {

@@ -54,14 +54,17 @@ struct mk_verify_ws {
   float* raw = nullptr;      // [n_dn][rows][C] conv inputs
   float* logits = nullptr;   // [rows][V]
   int32_t* greedy = nullptr; // [rows]
+  double* stats = nullptr;   // [rows][2]: row maximum and sum of weights (sampled verify)
 };
 
 // Batched prefill of n tokens at the device position: every layer, no logits.
 int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t s);
 // Verify pass of K+1 tokens in one pass over the weights, acceptance, and commit of the
 // accepted prefix (DeltaNet state and conv history rebuilt from the saved updates).
+// Greedy acceptance when d_uniforms is NULL, else sampled acceptance at `temperature`
+// with the 2(K+1) uniforms of d_uniforms.
 int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
-                      float* d_logits, cudaStream_t s);
+                      float* d_logits, cudaStream_t s, float temperature = 1.0f, const float* d_uniforms = nullptr);
 
 struct mk_model {
   mk_config cfg;

@@ -1815,6 +1815,150 @@ __global__ void accept_prefix(const int* tokens, const unsigned long long* best,
   *n_acc = n;
 }
 
+// ---------------------------------------------------------------- sampled acceptance
+// Sampling-mode speculative verify (standard speculative sampling with each draft a
+// point mass): draft d at position i is kept iff u[2i] < p_i(d), p_i = softmax(z_i / tau);
+// at the first rejection the output token is drawn from p_i with d removed, else after
+// K kept drafts from p_K, by the inverse of the cumulative distribution with u[2i + 1]
+// (the smallest token index whose running weight exceeds u * total). This keeps the law
+// of the emitted tokens equal to sampling from the model without drafts.
+// The weights, sums and thresholds are float64: with V ~ 1.5e5 tokens the cumulative
+// boundaries lie ~1e-5 apart, well inside float32's summation error, and the decision
+// should depend on the logits and the uniforms only.
+
+// Weight of a token relative to its row's maximum m; the maximum itself weighs exactly 1.
+__device__ __forceinline__ double samp_weight(float z, double m, double inv_tau) {
+  return exp((static_cast<double>(z) - m) * inv_tau);
+}
+
+constexpr int kSampThreads = 1024;
+
+template <bool kMax, typename F>
+__device__ __forceinline__ F block_reduce(F v, F* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int o = 16; o > 0; o >>= 1) {
+    const F x = __shfl_xor_sync(0xffffffffu, v, o);
+    v = kMax ? (x > v ? x : v) : v + x;
+  }
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < static_cast<int>(blockDim.x >> 5) ? red[lane] : (kMax ? static_cast<F>(-INFINITY) : F(0));
+    for (int o = 16; o > 0; o >>= 1) {
+      const F x = __shfl_xor_sync(0xffffffffu, v, o);
+      v = kMax ? (x > v ? x : v) : v + x;
+    }
+    if (lane == 0) red[32] = v;
+  }
+  __syncthreads();
+  v = red[32];
+  __syncthreads();
+  return v;
+}
+
+// stats[2t] = max of logits row t, stats[2t + 1] = sum of its weights (>= 1). One CTA per row.
+__global__ void __launch_bounds__(kSampThreads) row_softmax_stats(const float* __restrict__ logits, int V,
+                                                                  double inv_tau, double* __restrict__ stats) {
+  __shared__ float redf[33];
+  __shared__ double redd[33];
+  const float* r = logits + static_cast<long long>(blockIdx.x) * V;
+  float mf = -INFINITY;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) mf = fmaxf(mf, r[i]);
+  const double m = block_reduce<true>(mf, redf);
+  double s = 0.0;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) s += samp_weight(r[i], m, inv_tau);
+  s = block_reduce<false>(s, redd);
+  if (threadIdx.x == 0) {
+    stats[2 * blockIdx.x] = m;
+    stats[2 * blockIdx.x + 1] = s;
+  }
+}
+
+// One CTA: thread 0 tests the drafts in order; then every thread sums the weights of its
+// contiguous slice of the stopping row (the rejected draft left out), thread 0 walks the
+// slice sums in index order (each partial sum is >= the one before: every term is >= 0)
+// to the slice where the running weight first exceeds u * total, and scans that slice.
+__global__ void __launch_bounds__(kSampThreads) accept_sampled(const int* __restrict__ tokens, int K,
+                                                               const float* __restrict__ logits, int V,
+                                                               double inv_tau, const double* __restrict__ stats,
+                                                               const float* __restrict__ uni, int* n_out, int* n_acc,
+                                                               int* out) {
+  __shared__ double csum[kSampThreads];
+  __shared__ int sh_n, sh_excl;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    while (n < K) {
+      const int d = tokens[1 + n];
+      double pd = 0.0;
+      if (d >= 0 && d < V)
+        pd = samp_weight(logits[static_cast<long long>(n) * V + d], stats[2 * n], inv_tau) / stats[2 * n + 1];
+      if (static_cast<double>(uni[2 * n]) < pd) ++n;
+      else break;
+    }
+    sh_n = n;
+    sh_excl = n < K ? tokens[1 + n] : -1;
+  }
+  __syncthreads();
+  const int n = sh_n, excl = sh_excl;
+  const float* r = logits + static_cast<long long>(n) * V;
+  const double m = stats[2 * n];
+  const int per = (V + kSampThreads - 1) / kSampThreads;
+  {
+    const int j0 = threadIdx.x * per, j1 = min(V, j0 + per);
+    double s = 0.0;
+    for (int j = j0; j < j1; ++j)
+      if (j != excl) s += samp_weight(r[j], m, inv_tau);
+    csum[threadIdx.x] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  double total = 0.0;
+  int last_c = -1;
+  for (int c = 0; c < kSampThreads; ++c) {
+    total += csum[c];
+    if (csum[c] > 0.0) last_c = c;
+  }
+  const double target = static_cast<double>(uni[2 * n + 1]) * total;
+  int c = -1;
+  double before = 0.0, run = 0.0;
+  for (int i = 0; i < kSampThreads; ++i) {   // the same additions, in the same order, as total
+    const double nxt = run + csum[i];
+    if (nxt > target) {
+      c = i;
+      before = run;
+      break;
+    }
+    run = nxt;
+  }
+  if (c < 0 && last_c >= 0) {   // u * total rounded up to total (u within an ulp of 1)
+    c = last_c;
+    before = 0.0;
+    for (int i = 0; i < c; ++i) before += csum[i];
+  }
+  int tok = excl;               // no other token has weight (only if u[2n] >= 1)
+  if (c >= 0) {
+    const double rem = target - before;   // >= 0
+    double acc = 0.0;
+    int lastpos = -1;
+    tok = -1;
+    for (int j = c * per; j < min(V, c * per + per); ++j) {
+      if (j == excl) continue;
+      const double w = samp_weight(r[j], m, inv_tau);
+      if (w > 0.0) lastpos = j;
+      acc += w;
+      if (acc > rem) {
+        tok = j;
+        break;
+      }
+    }
+    if (tok < 0) tok = lastpos;   // rounding left the running weight just short of the target
+  }
+  for (int i = 0; i < n; ++i) out[i] = tokens[1 + i];
+  out[n] = tok;
+  *n_out = n;
+  *n_acc = n;
+}
+
 // One pass of every layer over T tokens at device position *pos + off. With vs (a verify
 // pass, T <= 64) the DeltaNet layers keep their state and conv history untouched and
 // save what the commit of an accepted prefix needs.
@@ -2121,7 +2265,7 @@ int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t
 }
 
 int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
-                      float* d_logits, cudaStream_t s) {
+                      float* d_logits, cudaStream_t s, float temperature, const float* d_uniforms) {
   const mk::DecodeParams& b = m->base;
   const mk_config& c = m->cfg;
   const int T = K + 1;
@@ -2156,15 +2300,31 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
     e = mk::launch_linear(a, s);
     ++m->launches;
   }
-  if (e == cudaSuccess) e = cudaMemsetAsync(m->pf.best, 0, sizeof(unsigned long long) * T, s);
-  if (e == cudaSuccess) {
-    mk::row_argmax<<<dim3(T, 64), 256, 0, s>>>(logits, c.vocab, m->pf.best);
-    chk();
-  }
-  // 3. longest matching prefix plus the bonus token
-  if (e == cudaSuccess) {
-    mk::accept_prefix<<<1, 32, 0, s>>>(d_tokens, m->pf.best, K, m->ws_n, d_n_accepted, d_out_tokens, vs.greedy);
-    chk();
+  if (d_uniforms) {
+    // 3'. sampled acceptance: row statistics of softmax(z / T), then the draft tests and
+    // the draw
+    double* stats = vs.stats;
+    const double inv_tau = 1.0 / static_cast<double>(temperature);
+    if (e == cudaSuccess) {
+      mk::row_softmax_stats<<<T, mk::kSampThreads, 0, s>>>(logits, c.vocab, inv_tau, stats);
+      chk();
+    }
+    if (e == cudaSuccess) {
+      mk::accept_sampled<<<1, mk::kSampThreads, 0, s>>>(d_tokens, K, logits, c.vocab, inv_tau, stats, d_uniforms,
+                                                        m->ws_n, d_n_accepted, d_out_tokens);
+      chk();
+    }
+  } else {
+    if (e == cudaSuccess) e = cudaMemsetAsync(m->pf.best, 0, sizeof(unsigned long long) * T, s);
+    if (e == cudaSuccess) {
+      mk::row_argmax<<<dim3(T, 64), 256, 0, s>>>(logits, c.vocab, m->pf.best);
+      chk();
+    }
+    // 3. longest matching prefix plus the bonus token
+    if (e == cudaSuccess) {
+      mk::accept_prefix<<<1, 32, 0, s>>>(d_tokens, m->pf.best, K, m->ws_n, d_n_accepted, d_out_tokens, vs.greedy);
+      chk();
+    }
   }
   // 4. commit: DeltaNet states and conv histories of the accepted prefix, then the position
   int di = 0;

@@ -162,6 +162,16 @@ class Model:
         check(self.lib.mk_verify_drafts(self.h, tokens.data_ptr(), K, n_accepted.data_ptr(), out_tokens.data_ptr(),
                                         _ptr(logits), _stream_ptr(stream)))
 
+    def verify_sampled(self, tokens: torch.Tensor, temperature: float, uniforms: torch.Tensor,
+                       n_accepted: torch.Tensor, out_tokens: torch.Tensor, logits: Optional[torch.Tensor] = None,
+                       stream=None):
+        """Sampling-mode verify; uniforms: float32 CUDA tensor of 2 * tokens.numel() values in [0, 1)."""
+        K = tokens.numel() - 1
+        assert uniforms.dtype == torch.float32 and uniforms.is_cuda and uniforms.numel() >= 2 * (K + 1)
+        check(self.lib.mk_verify_drafts_sampled(self.h, tokens.data_ptr(), K, float(temperature),
+                                                uniforms.data_ptr(), n_accepted.data_ptr(), out_tokens.data_ptr(),
+                                                _ptr(logits), _stream_ptr(stream)))
+
     def generate(self, prompt, n_new: int, stream=None, out: Optional[np.ndarray] = None) -> np.ndarray:
         """Host prompt in, host tokens out (pinned or pageable numpy int32 arrays)."""
         p = np.ascontiguousarray(prompt, dtype=np.int32)

@@ -211,6 +211,26 @@ int mk_decode_step_noalloc(mk_model* m, const int32_t* d_in_token, int32_t* d_ou
 int mk_verify_drafts(mk_model* m, const int32_t* d_tokens, int32_t K, int32_t* d_n_accepted,
                      int32_t* d_out_tokens, float* d_logits, void* stream);
 
+/* Speculative verify in sampling mode (the open-jet follow-up's speed section: with
+ * sampling, speculation keeps the distribution the model has without drafts). Standard
+ * speculative sampling with each draft a point mass: with p_i = softmax(z_i / temperature)
+ * the model's distribution after input i of [last, d_1 .. d_K],
+ *   - d_{i+1} is kept iff d_uniforms[2i] < p_i(d_{i+1}), for i = 0, 1, ... until the first
+ *     rejection or until all K are kept (n = the number kept);
+ *   - the token after them is drawn from p_n with d_{n+1} removed and the rest
+ *     renormalised (n < K), or from p_K (n = K): the smallest token index whose running
+ *     weight exceeds d_uniforms[2n + 1] times the total.
+ * d_uniforms: device float[2(K+1)], each in [0, 1), caller-drawn (the library draws no
+ * random numbers); other values give a valid token id but no distribution guarantee.
+ * temperature: > 0 and finite (MK_ERR_ARG otherwise). The weights, sums and comparisons
+ * are float64, from the float32 logits.
+ * Outputs, commit of the accepted prefix and the state afterwards as mk_verify_drafts.
+ * Needs the batched verify workspace (max_draft + 1 <= 64 and a prefill workspace),
+ * MK_ERR_CAPACITY otherwise. */
+int mk_verify_drafts_sampled(mk_model* m, const int32_t* d_tokens, int32_t K, float temperature,
+                             const float* d_uniforms, int32_t* d_n_accepted, int32_t* d_out_tokens,
+                             float* d_logits, void* stream);
+
 /* Convenience end-to-end call with HOST buffers: copy h_prompt[n_prompt] to the
  * device, prefill it, greedily generate n_new tokens, copy them to h_out[n_new].
  * Synchronises `stream` before returning. Uses the workspace; no allocation. */

@@ -75,6 +75,7 @@ def test_null_arguments_rejected(lib):
     assert lib.mk_decode_step(None, None, None, None, None) == _abi.MK_ERR_ARG
     assert lib.mk_prefill(None, None, 0, None, None, None) == _abi.MK_ERR_ARG
     assert lib.mk_verify_drafts(None, None, 1, None, None, None, None) == _abi.MK_ERR_ARG
+    assert lib.mk_verify_drafts_sampled(None, None, 1, 1.0, None, None, None, None, None) == _abi.MK_ERR_ARG
     assert lib.mk_generate(None, None, 0, None, 0, None) == _abi.MK_ERR_ARG
     assert lib.mk_launch_count(None) == 0
     lib.mk_free(None)
