@@ -407,7 +407,7 @@ Layout make_layout(const mk_config& c, int grid) {
     L.vf_raw = off; off = align256(off + R * C * 4);
     L.vf_logits = off; off = align256(off + static_cast<size_t>(L.vf_rows) * c.vocab * 4);
     L.vf_greedy = off; off = align256(off + static_cast<size_t>(L.vf_rows) * 4);
-    L.vf_stats = off; off = align256(off + static_cast<size_t>(L.vf_rows) * 16);   // sampled verify: max, sum
+    L.vf_stats = off; off = align256(off + samp_scratch_bytes(L.vf_rows));   // sampled verify
   }
   L.sz.workspace_bytes = off;
   L.sz.grid_ctas = grid;

@@ -46,6 +46,21 @@ struct mk_prefill_layer {   // K-major copies of the projections the decode kern
 
 // What a verify pass keeps so that the recurrent state can be committed to any accepted
 // prefix afterwards (per DeltaNet layer, per token of the pass).
+// Sampled verify scratch (double stats of mk_verify_ws): per-slice row statistics, the
+// decision, and the chunk sums of the stopping row.
+constexpr int kSampSlices = 24;      // CTAs per logits row for the row statistics
+constexpr int kDrawChunks = 4096;    // slices of the stopping row for the draw
+constexpr int kDrawGroup = 64;       // chunks per group of the draw's walk
+struct SampDecision {
+  double M;                          // maximum of the stopping row
+  int n;                             // drafts kept
+  int excl;                          // the rejected draft (-1: none)
+};
+inline size_t samp_scratch_bytes(int rows) {
+  return static_cast<size_t>(rows) * kSampSlices * 2 * sizeof(double) + sizeof(SampDecision) +
+         static_cast<size_t>(kDrawChunks) * sizeof(double);
+}
+
 struct mk_verify_ws {
   int rows = 0;              // tokens per pass it holds (max_draft + 1); 0: no batched verify
   float* delta = nullptr;    // [n_dn][rows][Hd dv] delta-rule updates
@@ -54,7 +69,7 @@ struct mk_verify_ws {
   float* raw = nullptr;      // [n_dn][rows][C] conv inputs
   float* logits = nullptr;   // [rows][V]
   int32_t* greedy = nullptr; // [rows]
-  double* stats = nullptr;   // [rows][2]: row maximum and sum of weights (sampled verify)
+  double* stats = nullptr;   // samp_scratch_bytes(rows): sampled verify scratch
 };
 
 // Batched prefill of n tokens at the device position: every layer, no logits.

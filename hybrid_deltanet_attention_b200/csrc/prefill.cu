@@ -1831,8 +1831,6 @@ __device__ __forceinline__ double samp_weight(float z, double m, double inv_tau)
   return exp((static_cast<double>(z) - m) * inv_tau);
 }
 
-constexpr int kSampThreads = 1024;
-
 template <bool kMax, typename F>
 __device__ __forceinline__ F block_reduce(F v, F* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1856,102 +1854,163 @@ __device__ __forceinline__ F block_reduce(F v, F* red) {
   return v;
 }
 
-// stats[2t] = max of logits row t, stats[2t + 1] = sum of its weights (>= 1). One CTA per row.
-__global__ void __launch_bounds__(kSampThreads) row_softmax_stats(const float* __restrict__ logits, int V,
-                                                                  double inv_tau, double* __restrict__ stats) {
+constexpr int kSampThreads = 256;
+
+// Slice sl of logits row t (kSampSlices slices per row): part[(t * kSampSlices + sl) * 2] = the
+// slice maximum m_s, [+1] = sum of exp((z - m_s) / tau) over the slice (an empty slice: -inf, 0).
+__global__ void __launch_bounds__(kSampThreads) row_softmax_partials(const float* __restrict__ logits, int V,
+                                                                     double inv_tau, double* __restrict__ part) {
   __shared__ float redf[33];
   __shared__ double redd[33];
-  const float* r = logits + static_cast<long long>(blockIdx.x) * V;
+  const int t = blockIdx.x, sl = blockIdx.y;
+  const int L = (V + kSampSlices - 1) / kSampSlices;
+  const int j0 = sl * L, j1 = min(V, j0 + L);
+  const float* r = logits + static_cast<long long>(t) * V;
   float mf = -INFINITY;
-  for (int i = threadIdx.x; i < V; i += blockDim.x) mf = fmaxf(mf, r[i]);
+  for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) mf = fmaxf(mf, r[j]);
   const double m = block_reduce<true>(mf, redf);
   double s = 0.0;
-  for (int i = threadIdx.x; i < V; i += blockDim.x) s += samp_weight(r[i], m, inv_tau);
+  for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) s += samp_weight(r[j], m, inv_tau);
   s = block_reduce<false>(s, redd);
   if (threadIdx.x == 0) {
-    stats[2 * blockIdx.x] = m;
-    stats[2 * blockIdx.x + 1] = s;
+    part[(t * kSampSlices + sl) * 2] = m;
+    part[(t * kSampSlices + sl) * 2 + 1] = s;
   }
 }
 
-// One CTA: thread 0 tests the drafts in order; then every thread sums the weights of its
-// contiguous slice of the stopping row (the rejected draft left out), thread 0 walks the
-// slice sums in index order (each partial sum is >= the one before: every term is >= 0)
-// to the slice where the running weight first exceeds u * total, and scans that slice.
-__global__ void __launch_bounds__(kSampThreads) accept_sampled(const int* __restrict__ tokens, int K,
-                                                               const float* __restrict__ logits, int V,
-                                                               double inv_tau, const double* __restrict__ stats,
-                                                               const float* __restrict__ uni, int* n_out, int* n_acc,
-                                                               int* out) {
-  __shared__ double csum[kSampThreads];
-  __shared__ int sh_n, sh_excl;
-  if (threadIdx.x == 0) {
-    int n = 0;
-    while (n < K) {
-      const int d = tokens[1 + n];
-      double pd = 0.0;
-      if (d >= 0 && d < V)
-        pd = samp_weight(logits[static_cast<long long>(n) * V + d], stats[2 * n], inv_tau) / stats[2 * n + 1];
-      if (static_cast<double>(uni[2 * n]) < pd) ++n;
-      else break;
+// One warp: row statistics (maximum M, Z = sum over slices of sum_s exp((m_s - M) / tau)) and
+// the draft tests in order. Every lane computes the same values (the butterfly sums are
+// order-symmetric), so the loop runs in lockstep; lane 0 writes the decision.
+__global__ void samp_decide(const int* __restrict__ tokens, int K, const float* __restrict__ logits, int V,
+                            double inv_tau, const double* __restrict__ part, const float* __restrict__ uni,
+                            SampDecision* __restrict__ dec) {
+  const int lane = threadIdx.x;
+  int n = 0;
+  double M = 0.0;
+  for (;;) {
+    double ms = -INFINITY, ss = 0.0;
+    if (lane < kSampSlices) {
+      ms = part[(n * kSampSlices + lane) * 2];
+      ss = part[(n * kSampSlices + lane) * 2 + 1];
     }
-    sh_n = n;
-    sh_excl = n < K ? tokens[1 + n] : -1;
+    double mx = ms;
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    double z = ss > 0.0 ? ss * exp((ms - mx) * inv_tau) : 0.0;
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    M = mx;
+    if (n >= K) break;
+    const int d = tokens[1 + n];
+    double pd = 0.0;
+    if (d >= 0 && d < V) pd = samp_weight(logits[static_cast<long long>(n) * V + d], M, inv_tau) / z;
+    if (static_cast<double>(uni[2 * n]) < pd) ++n;
+    else break;
   }
-  __syncthreads();
-  const int n = sh_n, excl = sh_excl;
+  if (lane == 0) {
+    dec->M = M;
+    dec->n = n;
+    dec->excl = n < K ? tokens[1 + n] : -1;
+  }
+}
+
+// Chunk c (kDrawChunks contiguous chunks) of the stopping row: the sum of its weights
+// exp((z - M) / tau), the rejected draft left out.
+__global__ void __launch_bounds__(kSampThreads) samp_chunk_sums(const float* __restrict__ logits, int V,
+                                                                double inv_tau, const SampDecision* __restrict__ dec,
+                                                                double* __restrict__ csum) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= kDrawChunks) return;
+  const int n = dec->n, excl = dec->excl;
+  const double M = dec->M;
   const float* r = logits + static_cast<long long>(n) * V;
-  const double m = stats[2 * n];
-  const int per = (V + kSampThreads - 1) / kSampThreads;
-  {
-    const int j0 = threadIdx.x * per, j1 = min(V, j0 + per);
+  const int per = (V + kDrawChunks - 1) / kDrawChunks;
+  const int j0 = c * per, j1 = min(V, j0 + per);
+  double s = 0.0;
+  for (int j = j0; j < j1; ++j)
+    if (j != excl) s += samp_weight(r[j], M, inv_tau);
+  csum[c] = s;
+}
+
+// One warp: the draw by the inverse CDF, walked in index order at three levels (groups of
+// kDrawGroup chunks, chunks, tokens). Each level's running sum adds the same terms in the
+// same order as the sum it is compared with, so it only grows and its last value equals that
+// sum; rounding between levels is caught by taking the last token with weight.
+__global__ void samp_select(const int* __restrict__ tokens, const float* __restrict__ logits, int V, double inv_tau,
+                            const SampDecision* __restrict__ dec, const double* __restrict__ csum,
+                            const float* __restrict__ uni, int* n_out, int* n_acc, int* out) {
+  constexpr int kGroups = kDrawChunks / kDrawGroup;
+  __shared__ double gsum[kGroups];
+  const int lane = threadIdx.x;
+  for (int g = lane; g < kGroups; g += 32) {
     double s = 0.0;
-    for (int j = j0; j < j1; ++j)
-      if (j != excl) s += samp_weight(r[j], m, inv_tau);
-    csum[threadIdx.x] = s;
+    for (int i = 0; i < kDrawGroup; ++i) s += csum[g * kDrawGroup + i];
+    gsum[g] = s;
   }
-  __syncthreads();
-  if (threadIdx.x != 0) return;
+  __syncwarp();
+  if (lane != 0) return;
+  const int n = dec->n, excl = dec->excl;
+  const double M = dec->M;
   double total = 0.0;
-  int last_c = -1;
-  for (int c = 0; c < kSampThreads; ++c) {
-    total += csum[c];
-    if (csum[c] > 0.0) last_c = c;
+  int last_g = -1;
+  for (int g = 0; g < kGroups; ++g) {
+    total += gsum[g];
+    if (gsum[g] > 0.0) last_g = g;
   }
   const double target = static_cast<double>(uni[2 * n + 1]) * total;
-  int c = -1;
+  int g = -1;
   double before = 0.0, run = 0.0;
-  for (int i = 0; i < kSampThreads; ++i) {   // the same additions, in the same order, as total
-    const double nxt = run + csum[i];
+  for (int i = 0; i < kGroups; ++i) {
+    const double nxt = run + gsum[i];
     if (nxt > target) {
-      c = i;
+      g = i;
       before = run;
       break;
     }
     run = nxt;
   }
-  if (c < 0 && last_c >= 0) {   // u * total rounded up to total (u within an ulp of 1)
-    c = last_c;
+  if (g < 0 && last_g >= 0) {   // u * total rounded up to total
+    g = last_g;
     before = 0.0;
-    for (int i = 0; i < c; ++i) before += csum[i];
+    for (int i = 0; i < g; ++i) before += gsum[i];
   }
   int tok = excl;               // no other token has weight (only if u[2n] >= 1)
-  if (c >= 0) {
-    const double rem = target - before;   // >= 0
+  if (g >= 0) {
+    const double* cs = csum + g * kDrawGroup;
+    const double rem = target - before;
+    int c = -1, last_c = -1;
+    double before2 = 0.0, run2 = 0.0;
+    for (int i = 0; i < kDrawGroup; ++i) {
+      if (cs[i] > 0.0) last_c = i;
+      const double nxt = run2 + cs[i];
+      if (c < 0 && nxt > rem) {
+        c = i;
+        before2 = run2;
+      }
+      run2 = nxt;
+    }
+    if (c < 0) {
+      c = last_c;
+      before2 = 0.0;
+      for (int i = 0; i < c; ++i) before2 += cs[i];
+    }
+    if (c < 0) c = 0;             // not reached: a group with weight has a chunk with weight
+    const double rem2 = rem - before2;
+    const float* r = logits + static_cast<long long>(n) * V;
+    const int per = (V + kDrawChunks - 1) / kDrawChunks;
+    const int j0 = (g * kDrawGroup + c) * per, j1 = min(V, j0 + per);
     double acc = 0.0;
     int lastpos = -1;
     tok = -1;
-    for (int j = c * per; j < min(V, c * per + per); ++j) {
+    for (int j = j0; j < j1; ++j) {
       if (j == excl) continue;
-      const double w = samp_weight(r[j], m, inv_tau);
+      const double w = samp_weight(r[j], M, inv_tau);
       if (w > 0.0) lastpos = j;
       acc += w;
-      if (acc > rem) {
+      if (acc > rem2) {
         tok = j;
         break;
       }
     }
-    if (tok < 0) tok = lastpos;   // rounding left the running weight just short of the target
+    if (tok < 0) tok = lastpos;
   }
   for (int i = 0; i < n; ++i) out[i] = tokens[1 + i];
   out[n] = tok;
@@ -2301,17 +2360,28 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
     ++m->launches;
   }
   if (d_uniforms) {
-    // 3'. sampled acceptance: row statistics of softmax(z / T), then the draft tests and
-    // the draw
-    double* stats = vs.stats;
+    // 3'. sampled acceptance: per-slice row statistics, the draft tests, the chunk sums of
+    // the stopping row, the draw
+    double* part = vs.stats;
+    SampDecision* dec = reinterpret_cast<SampDecision*>(part + static_cast<size_t>(vs.rows) * kSampSlices * 2);
+    double* csum = reinterpret_cast<double*>(dec + 1);
     const double inv_tau = 1.0 / static_cast<double>(temperature);
     if (e == cudaSuccess) {
-      mk::row_softmax_stats<<<T, mk::kSampThreads, 0, s>>>(logits, c.vocab, inv_tau, stats);
+      mk::row_softmax_partials<<<dim3(T, kSampSlices), mk::kSampThreads, 0, s>>>(logits, c.vocab, inv_tau, part);
       chk();
     }
     if (e == cudaSuccess) {
-      mk::accept_sampled<<<1, mk::kSampThreads, 0, s>>>(d_tokens, K, logits, c.vocab, inv_tau, stats, d_uniforms,
-                                                        m->ws_n, d_n_accepted, d_out_tokens);
+      mk::samp_decide<<<1, 32, 0, s>>>(d_tokens, K, logits, c.vocab, inv_tau, part, d_uniforms, dec);
+      chk();
+    }
+    if (e == cudaSuccess) {
+      mk::samp_chunk_sums<<<kDrawChunks / mk::kSampThreads, mk::kSampThreads, 0, s>>>(logits, c.vocab, inv_tau, dec,
+                                                                                      csum);
+      chk();
+    }
+    if (e == cudaSuccess) {
+      mk::samp_select<<<1, 32, 0, s>>>(d_tokens, logits, c.vocab, inv_tau, dec, csum, d_uniforms, m->ws_n,
+                                       d_n_accepted, d_out_tokens);
       chk();
     }
   } else {

@@ -65,6 +65,7 @@ def test_sampled_verify_matches_oracle_tiny(tiny, tau):
     cfg, m, W = tiny
     dev = torch.device("cuda")
     rng = np.random.default_rng(int(tau * 1000))
+    tau = float(np.float32(tau))       # the library takes the temperature as float32
     K = 4
     m.reset()
     st = oracle.new_state(cfg, 128)
@@ -175,7 +176,7 @@ def test_sampled_verify_full_vocab_08b():
             u[0, 0], u[0, 1] = 0.999, 0.0                  # reject d_1, then the first token with weight
         if it == 1:
             u[0, 0], u[0, 1] = 0.999, np.nextafter(np.float32(1), np.float32(0))   # ... the last one
-        tau = 1.0 if it < 2 or it % 2 == 0 else 0.3
+        tau = 1.0 if it < 2 or it % 2 == 0 else float(np.float32(0.3))   # as the library receives it
         n, committed, lg, u = _run_pass(m, [last] + drafts, tau, u, cfg.vocab)
         _valid(n, committed, drafts, lg, tau)
         n_k, c_k, margin_k = oracle.accept_sampled(lg, drafts, tau, u)
