@@ -20,3 +20,4 @@ from .model import *          # noqa: F401,F403
 from .chunked import *        # noqa: F401,F403
 from .q4k import *            # noqa: F401,F403
 from .sampling import *       # noqa: F401,F403
+from .kvq8 import *           # noqa: F401,F403

@@ -22,6 +22,8 @@ from typing import Dict, List, Optional
 
 import numpy as np
 
+from .kvq8 import q8_roundtrip
+
 __all__ = [
     "round_bf16", "decode_bf16_bits", "rmsnorm", "silu", "sigmoid", "softplus", "l2norm",
     "conv_silu", "delta_rule_step", "rope", "attention_decode", "swiglu",
@@ -162,21 +164,22 @@ def prepare_weights(cfg, raw: Dict[str, np.ndarray]) -> Dict[str, np.ndarray]:
 class OracleState:
     S: List[np.ndarray]        # per DeltaNet layer [Hd, dv, dk]
     conv: List[np.ndarray]     # per DeltaNet layer [W-1, C] previous raw conv inputs, oldest first
-    K: List[np.ndarray]        # per attention layer [Hkv, max_ctx, D] (bf16-valued)
+    K: List[np.ndarray]        # per attention layer [Hkv, max_ctx, D] (bf16-valued, or q8 read-back values)
     V: List[np.ndarray]
     pos: int = 0
+    kv_q8: bool = False        # 8-bit block entries (oracle/kvq8.py) instead of bf16
 
     def copy(self) -> "OracleState":
         return copy.deepcopy(self)
 
 
-def new_state(cfg, max_ctx: int) -> OracleState:
+def new_state(cfg, max_ctx: int, kv_q8: bool = False) -> OracleState:
     S = [np.zeros((cfg.dn_heads, cfg.dn_dv, cfg.dn_dk)) for _ in range(cfg.n_dn)]
     conv = [np.zeros((cfg.conv_width - 1, cfg.dn_conv_channels)) for _ in range(cfg.n_dn)]
     shp = (cfg.at_kv_heads, max_ctx, cfg.at_head_dim)
     K = [np.zeros(shp) for _ in range(cfg.n_at)]
     V = [np.zeros(shp) for _ in range(cfg.n_at)]
-    return OracleState(S, conv, K, V, 0)
+    return OracleState(S, conv, K, V, 0, kv_q8)
 
 
 # ------------------------------------------------------------------ the forward step
@@ -210,8 +213,12 @@ def _attention_mixer(cfg, W, p, st: OracleState, li: int, x: np.ndarray) -> np.n
     pos = st.pos
     q = rope(q, pos, cfg.rope_theta)
     k = rope(k, pos, cfg.rope_theta)
-    st.K[li][:, pos] = round_bf16(k)          # the KV cache is stored in bf16
-    st.V[li][:, pos] = round_bf16(v)
+    if st.kv_q8:                              # 8-bit blocks of 32 with an fp16 scale
+        st.K[li][:, pos] = q8_roundtrip(k)
+        st.V[li][:, pos] = q8_roundtrip(v)
+    else:                                     # the KV cache is stored in bf16
+        st.K[li][:, pos] = round_bf16(k)
+        st.V[li][:, pos] = round_bf16(v)
     o = attention_decode(q, st.K[li][:, :pos + 1], st.V[li][:, :pos + 1]).reshape(-1)
     if cfg.at_out_gate:
         o = o * sigmoid(g)
