@@ -1,0 +1,29 @@
+"""The roofline numerator: algorithmic bytes one decode step reads, pinned by a count made
+by hand from the 0.8B-shaped architecture and by the loader's own tensor list."""
+import numpy as np
+
+import bench
+import synth
+
+
+def test_weights_equal_the_tensor_list():
+    for cfg in (synth.TINY, synth.MINI, synth.QWEN_08B):
+        specs = synth.tensor_specs(cfg)
+        assert bench.bytes_per_token(cfg, 0)["weights"] == sum(int(np.prod(s)) for _, s, _ in specs) * 2
+
+
+def test_08b_bytes_by_hand():
+    cfg = synth.QWEN_08B
+    H, V, F = 1024, 151936, 3584
+    per_mlp = 2 * H + 3 * F * H                                    # two gains, gate, up, down
+    per_dn = (3 * 16 * 128 + 2 * 16) * H + 3 * 16 * 128 * 4 + H * 16 * 128   # in-proj, conv taps, out-proj
+    per_at = (8 * 256 + 8 * 256 + 2 * 256 + 2 * 256) * H + H * 8 * 256       # q, gate, k, v; out-proj
+    weights = 2 * (V * H + H + 24 * per_mlp + 18 * per_dn + 6 * per_at)     # tied head + final gain
+    b = bench.bytes_per_token(cfg, 191)
+    assert b["weights"] == weights == 1_231_882_240
+    assert b["state"] == 18 * 16 * 128 * 128 * 4                 # fp32 S of every DeltaNet layer
+    assert b["kv"] == 6 * 2 * 256 * 2 * 2 * 192                  # bf16 K and V, positions 0..191
+    assert b["kv"] == 12_288 * 192
+    assert b["read"] == b["weights"] + b["state"] + b["conv"] + b["kv"]
+    # about 1.255 GB a token at the tg128 positions: 192 us at the measured copy bandwidth
+    assert 1.2548e9 < b["read"] < 1.2550e9
