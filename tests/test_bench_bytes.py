@@ -27,3 +27,9 @@ def test_08b_bytes_by_hand():
     assert b["read"] == b["weights"] + b["state"] + b["conv"] + b["kv"]
     # about 1.255 GB a token at the tg128 positions: 192 us at the measured copy bandwidth
     assert 1.2548e9 < b["read"] < 1.2550e9
+
+
+def test_08b_prefill_linear_macs_by_hand():
+    H, F = 1024, 3584
+    macs = 24 * 3 * F * H + 18 * (6176 * H + H * 2048) + 6 * (5120 * H + H * 2048)
+    assert bench.linear_macs_per_token(synth.QWEN_08B) == macs == 459_866_112   # 0.92 GFLOP a token
