@@ -8,19 +8,22 @@
  * one kernel launch per forward pass, BF16 weights and activations with FP32
  * accumulation, cooperative grid synchronisation instead of kernel boundaries) and
  * in the open-jet Qwen3.8-27B megakernel follow-up (speculative verify of several
- * drafted tokens per pass, exact greedy acceptance, type-checked tensor loading).
+ * drafted tokens per pass, exact greedy acceptance or sampling that keeps the model's
+ * distribution, type-checked tensor loading).
  *
- * Per token (pre-norm residual blocks, no biases):
+ * Per token (pre-norm residual blocks, no biases; weights bf16 or 4-bit blocks, every
+ * activation fp32 -- the batched passes' tensor-core products take each fp32 input as a
+ * bf16 high + low pair, about 16 mantissa bits -- and the KV cache entries stored in bf16):
  *   h = E[tok]
- *   per layer:  x = bf16(RMSNorm(h) * g1)
+ *   per layer:  x = RMSNorm(h) * g1
  *     DeltaNet: [q;k;v;alpha;beta] = W_in x; q,k,v = SiLU(causal depthwise conv_W);
  *               q,k L2-normalised per head; a = exp(-softplus(alpha)); b = sigmoid(beta);
- *               S = a S (I - b k k^T) + b v k^T;  o = S q;     h += W_out bf16(o)
+ *               S = a S (I - b k k^T) + b v k^T;  o = S q;     h += W_out o
  *     attention:[q;gate;k;v] = W_in x; RoPE(q,k) (half split, theta); append bf16 k,v;
  *               o = softmax(q K^T / sqrt(D)) V per query head (GQA);
- *               o *= sigmoid(gate) (if gated);                  h += W_out bf16(o)
- *     MLP:      x = bf16(RMSNorm(h) * g2);  h += W_down bf16(SiLU(W_gate x) * (W_up x))
- *   logits = E bf16(RMSNorm(h) * g_f)  (tied embedding);  next = argmax, lowest index on ties
+ *               o *= sigmoid(gate) (if gated);                  h += W_out o
+ *     MLP:      x = RMSNorm(h) * g2;  h += W_down (SiLU(W_gate x) * (W_up x))
+ *   logits = E (RMSNorm(h) * g_f)  (tied embedding);  next = argmax, lowest index on ties
  *
  * Memory ownership: the caller allocates ALL device memory (packed weights, state,
  * workspace) and passes raw device pointers; the library never allocates device
