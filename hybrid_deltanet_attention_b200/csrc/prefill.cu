@@ -1816,12 +1816,13 @@ __global__ void accept_prefix(const int* tokens, const unsigned long long* best,
 }
 
 // ---------------------------------------------------------------- sampled acceptance
-// Sampling-mode speculative verify (standard speculative sampling with each draft a
-// point mass): draft d at position i is kept iff u[2i] < p_i(d), p_i = softmax(z_i / tau);
-// at the first rejection the output token is drawn from p_i with d removed, else after
-// K kept drafts from p_K, by the inverse of the cumulative distribution with u[2i + 1]
-// (the smallest token index whose running weight exceeds u * total). This keeps the law
-// of the emitted tokens equal to sampling from the model without drafts.
+// Sampling-mode speculative verify. The open-jet Qwen3.8-27B megakernel follow-up (speed
+// section) states that with sampling, speculation keeps the distribution the model has
+// without drafts; the rule is standard speculative sampling (Leviathan et al. 2023, Chen et
+// al. 2023) with each draft a point mass: draft d at position i is kept iff u[2i] < p_i(d),
+// p_i = softmax(z_i / tau); at the first rejection the output token is drawn from p_i with d
+// removed, else after K kept drafts from p_K, by the inverse of the cumulative distribution
+// with u[2i + 1] (the smallest token index whose running weight exceeds u * total).
 // The weights, sums and thresholds are float64: with V ~ 1.5e5 tokens the cumulative
 // boundaries lie ~1e-5 apart, well inside float32's summation error, and the decision
 // should depend on the logits and the uniforms only.
