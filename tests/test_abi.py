@@ -90,3 +90,30 @@ def test_no_cpu_fallback_when_library_missing(tmp_path):
             _abi.load_library(str(tmp_path / "libmk.so"))
     finally:
         _abi._lib = saved
+
+
+def test_linear_rejects_unaligned_shapes_before_any_launch(lib):
+    """The tensor-core linear layer stages K-blocks of 64 with TMA, whose copies need 16-byte
+    aligned starts; shapes and pointers that break that are refused on the host (no device
+    call is made, so fake addresses are safe here)."""
+    from hybrid_deltanet_attention_b200 import _abi
+    a, odd = 0x100000, 0x100008                      # 16-byte aligned / only 8-byte aligned
+    err = a
+    big = 1 << 30
+    ok = dict(x=a, ldx=128, M=4, K=128, w=a, ldw=256, N=64, c=a, ldc=64, acc=0, scr=a, scr_bytes=big)
+
+    def call(**kw):
+        v = dict(ok, **kw)
+        return lib.mk_linear(v["x"], v["ldx"], v["M"], v["K"], v["w"], v["ldw"], v["N"], v["c"], v["ldc"],
+                             v["acc"], v["scr"], v["scr_bytes"], err, None)
+
+    assert call(K=96, ldx=96, ldw=192) == _abi.MK_ERR_ARG            # K not a multiple of 64
+    assert call(ldw=264) == _abi.MK_ERR_ARG                          # row pitch not a multiple of 16 bytes
+    assert call(ldw=128) == _abi.MK_ERR_ARG                          # row pitch shorter than a row
+    assert call(ldx=64) == _abi.MK_ERR_ARG                           # input pitch shorter than K
+    assert call(scr_bytes=4 * 4 * 128 - 1) == _abi.MK_ERR_ARG        # scratch below 4*M*K bytes
+    assert call(w=odd) == _abi.MK_ERR_ARG                            # weights not 16-byte aligned
+    assert call(scr=odd) == _abi.MK_ERR_ARG                          # scratch not 16-byte aligned
+    assert call(x=0) == _abi.MK_ERR_ARG                              # NULL input
+    assert call(w=odd) == _abi.MK_ERR_ARG and "16-byte" in lib.mk_last_error().decode()
+    assert call(M=0) == _abi.MK_OK                                   # nothing to do, nothing launched
