@@ -491,14 +491,9 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   *out = nullptr;
   if (!tensors || n_tensors <= 0) return fail(MK_ERR_ARG, "no tensors given");
   if (!d_packed || !d_state || !d_workspace) return fail(MK_ERR_ARG, "device buffer pointer is NULL");
-  int grid = 0, dev = 0;
-  rc = device_grid(&grid, &dev);
-  if (rc) return rc;
-  rc = check_budget(*cfg, grid);
-  if (rc) return rc;
   const mk_config& c = *cfg;
 
-  // ---- type-check every tensor ----
+  // ---- type-check every tensor (host only: nothing here touches the device) ----
   std::map<std::string, Expect> ex;
   expected_tensors(c, ex);
   std::map<std::string, const mk_tensor*> got;
@@ -523,6 +518,12 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   }
   for (auto& kv : ex)
     if (!got.count(kv.first)) return fail(MK_ERR_TENSOR, "missing tensor '" + kv.first + "'");
+
+  int grid = 0, dev = 0;
+  rc = device_grid(&grid, &dev);
+  if (rc) return rc;
+  rc = check_budget(*cfg, grid);
+  if (rc) return rc;
 
   // ---- layout, repack ----
   Layout L = make_layout(c, grid);

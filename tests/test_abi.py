@@ -4,6 +4,7 @@ import ctypes as C
 import os
 import re
 
+import numpy as np
 import pytest
 
 import synth
@@ -117,3 +118,61 @@ def test_linear_rejects_unaligned_shapes_before_any_launch(lib):
     assert call(x=0) == _abi.MK_ERR_ARG                              # NULL input
     assert call(w=odd) == _abi.MK_ERR_ARG and "16-byte" in lib.mk_last_error().decode()
     assert call(M=0) == _abi.MK_OK                                   # nothing to do, nothing launched
+
+
+# ------------------------------------------------------------------ the loader's type checks
+def _tiny_tensor_list():
+    """The tiny model's tensors as the binding marshals them, with fake 16-byte aligned
+    device addresses (the type checks read only the descriptors)."""
+    from hybrid_deltanet_attention_b200 import _abi
+    specs = synth.tensor_specs(synth.TINY)
+    names = [n.encode() for n, _, _ in specs]
+    arr = (_abi.MkTensor * len(specs))()
+    for i, (n, shape, _) in enumerate(specs):
+        arr[i].name = names[i]
+        arr[i].dtype = _abi.MK_DT_BF16
+        arr[i].ndim = len(shape)
+        for d, v in enumerate(shape):
+            arr[i].shape[d] = v
+        arr[i].data = 0x10000000 + i * 0x100000
+        arr[i].bytes = 2 * int(np.prod(shape))
+    return arr, names
+
+
+def _load(lib, arr, n=None):
+    import hybrid_deltanet_attention_b200 as hda
+    from hybrid_deltanet_attention_b200 import _abi
+    cfg = hda.make_config(synth.TINY, 64, 0)
+    h = C.c_void_p()
+    buf = 0x40000000
+    rc = lib.mk_load_weights(C.byref(cfg), arr, len(arr) if n is None else n, buf, buf, buf, None, C.byref(h))
+    return rc, lib.mk_last_error().decode(), _abi
+
+
+def test_loader_checks_every_tensor_before_touching_the_device(lib):
+    """The open-jet follow-up's loader "checks every tensor's type": name, dtype, rank, shape,
+    byte size, address alignment, none missing, none unknown, none twice."""
+    arr, _ = _tiny_tensor_list()
+    cases = []
+
+    def case(mutate, frag):
+        a, _ = _tiny_tensor_list()
+        n = mutate(a)
+        rc, msg, _abi = _load(lib, a, n)
+        cases.append((rc, msg, frag, _abi.MK_ERR_TENSOR))
+
+    case(lambda a: setattr(a[3], "dtype", 2), "wrong dtype")
+    case(lambda a: setattr(a[3], "ndim", 3), "wrong rank")
+    case(lambda a: a[2].shape.__setitem__(0, a[2].shape[0] + 1), "shape")
+    case(lambda a: setattr(a[4], "bytes", a[4].bytes - 2), "wrong byte size")
+    case(lambda a: setattr(a[5], "data", 0x10000008), "16-byte aligned")
+    case(lambda a: setattr(a[5], "data", None), "data is NULL")
+    case(lambda a: setattr(a[6], "name", b"layers.0.not_a_weight"), "unknown tensor")
+    case(lambda a: setattr(a[7], "name", a[1].name), "given twice")
+    case(lambda a: len(a) - 1, "missing tensor")
+    for rc, msg, frag, want in cases:
+        assert rc == want and frag in msg, (rc, msg, frag)
+    # the intact list passes every check; what fails next is the device query (no GPU here)
+    rc, msg, _abi = _load(lib, arr)
+    if rc != _abi.MK_OK:
+        assert rc != _abi.MK_ERR_TENSOR, msg
