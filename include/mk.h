@@ -2,11 +2,11 @@
  * mk.h -- C ABI of the hybrid Gated-DeltaNet + attention megakernel library (libmk.so).
  *
  * What it computes: batch-1 autoregressive inference of a hybrid language model
- * whose layers are either Gated DeltaNet mixers ("linear attention with a learned
- * recurrence") or full softmax attention, each followed by a SwiGLU MLP, as in the
- * Hacker News post on the fused 24-layer Qwen3.5-0.8B megakernel (design bullets:
- * one kernel launch per forward pass, BF16 weights and activations with FP32
- * accumulation, cooperative grid synchronisation instead of kernel boundaries) and
+ * whose layers are either Gated DeltaNet mixers (linear attention whose state
+ * evolves by a learned recurrence) or full softmax attention, each followed by a
+ * SwiGLU MLP, as in the Hacker News post on the fused 24-layer Qwen3.5-0.8B
+ * megakernel (design bullets: a single launch per forward pass, bf16 storage with
+ * fp32 sums, cooperative grid syncs in place of kernel boundaries) and
  * in the open-jet Qwen3.8-27B megakernel follow-up (speculative verify of several
  * drafted tokens per pass, exact greedy acceptance or sampling that keeps the model's
  * distribution, type-checked tensor loading).
@@ -156,8 +156,8 @@ typedef struct mk_model mk_model;   /* opaque host-side handle */
 int mk_query_sizes(const mk_config* cfg, mk_sizes* out);
 
 /* Check every tensor (name, dtype, shape, byte size, alignment; none missing, none
- * unknown, none twice) -- the open-jet follow-up's "loader checks every tensor's type" --
- * then repack them into d_packed (asynchronously on `stream`), zero the state and the
+ * unknown, none twice; the open-jet follow-up reports that its loader type-checks every
+ * tensor), then repack them into d_packed (asynchronously on `stream`), zero the state and the
  * workspace, and return a handle in *out. The input tensors may be freed once the
  * stream has passed this call. */
 int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_tensors,

@@ -13,8 +13,8 @@ Rounding contract: weights are bf16 and the KV cache entries are stored in bf16;
 every other quantity stays in full precision (float64 here, float32 on the GPU,
 where activations live in registers and shared memory and never leave the chip).
 ``act_bf16=True`` additionally rounds every projection input (normalised hidden
-state, mixer output, SwiGLU activation) to bf16 -- the megakernel post's "BF16
-weights and activations" taken literally -- for diagnostics.
+state, mixer output, SwiGLU activation) to bf16 -- the megakernel post's bf16
+activations taken literally -- for diagnostics.
 """
 from .model import *          # noqa: F401,F403
 from .chunked import *        # noqa: F401,F403

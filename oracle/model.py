@@ -4,9 +4,10 @@ Test infrastructure only (see the package docstring).
 
 Sources for what is computed:
   * Hacker News post on the fused 24-layer Qwen3.5-0.8B megakernel, design
-    bullets: hybrid of 18 DeltaNet layers ("linear attention with a learned
-    recurrence") and 6 full-attention layers; BF16 weights and activations with
-    FP32 accumulation; attention = QKV, RoPE, causal softmax, output projection.
+    bullets: 18 of the 24 layers are DeltaNet mixers (linear attention whose
+    state evolves by a learned recurrence), 6 are full attention; weights and
+    activations are kept in bf16 and sums in fp32; attention = QKV, RoPE,
+    causal softmax, output projection.
   * Gated DeltaNet (Yang, Kautz and Hatamizadeh, "Gated Delta Networks", 2024):
     S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T, o_t = S_t q_t,
     with a_t = exp(-softplus(.)), b_t = sigmoid(.), L2-normalised q, k and a

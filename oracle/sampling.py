@@ -2,10 +2,10 @@
 
 Test infrastructure only (see the package docstring).
 
-Source: the open-jet Qwen3.8-27B megakernel follow-up post (speed section) states
-that speculative decoding is exact in both modes: greedy output equals the main
-model's greedy choice, and sampling keeps the distribution the model has without
-drafts. The post gives no rule; the one written here is standard speculative
+Source: the open-jet Qwen3.8-27B megakernel follow-up post (speed section) says that
+speculation changes no output: in greedy mode the tokens are those the model alone
+would pick, and in sampling mode the tokens follow the model's own distribution.
+The post gives no rule; the one written here is standard speculative
 sampling (Leviathan, Kalman and Matias, "Fast Inference from Transformers via
 Speculative Decoding", 2023; Chen et al., "Accelerating Large Language Model
 Decoding with Speculative Sampling", 2023): a drafted token x drawn from q is kept

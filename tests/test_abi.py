@@ -150,7 +150,7 @@ def _load(lib, arr, n=None):
 
 
 def test_loader_checks_every_tensor_before_touching_the_device(lib):
-    """The open-jet follow-up's loader "checks every tensor's type": name, dtype, rank, shape,
+    """The open-jet follow-up reports that its loader type-checks every tensor: name, dtype, rank, shape,
     byte size, address alignment, none missing, none unknown, none twice."""
     arr, _ = _tiny_tensor_list()
     cases = []
