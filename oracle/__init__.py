@@ -21,3 +21,4 @@ from .chunked import *        # noqa: F401,F403
 from .q4k import *            # noqa: F401,F403
 from .sampling import *       # noqa: F401,F403
 from .kvq8 import *           # noqa: F401,F403
+from .sequence import *       # noqa: F401,F403
