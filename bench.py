@@ -44,6 +44,9 @@ WORKLOAD = ("0.8B-shaped hybrid Gated-DeltaNet + attention (24 layers [D,D,D,A]x
 LONG_WORKLOAD = ("0.8B-shaped hybrid (as tg128), long context: seeded bf16 KV cache of 32768 positions per "
                  "attention layer (N(0,1), RoPE applied, seed 3), DeltaNet states N(0,0.1), then 128 greedy "
                  "decode steps at batch 1 from position 32768")
+LONG_Q8_WORKLOAD = ("0.8B-shaped hybrid (as tg128), long context with the 8-bit KV cache (blocks of 32, fp16 "
+                    "scales): a 32768-token random prompt prefilled through the library, then 128 greedy decode "
+                    "steps at batch 1 from position 32768")
 KERNEL_SOURCES = ["hybrid_deltanet_attention_b200/csrc/decode.cu", "hybrid_deltanet_attention_b200/csrc/dev.cuh",
                   "hybrid_deltanet_attention_b200/csrc/mk_internal.h"]
 
@@ -56,8 +59,9 @@ def kernel_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def bytes_per_token(cfg, pos: int) -> dict:
-    """Algorithmic bytes one decode step at position `pos` reads (and writes)."""
+def bytes_per_token(cfg, pos: int, kv_row_bytes: int = 0) -> dict:
+    """Algorithmic bytes one decode step at position `pos` reads (and writes); kv_row_bytes:
+    bytes of one cache row (0: bf16, 2 * D)."""
     H, V, F = cfg.hidden, cfg.vocab, cfg.ffn
     w = V * H * 2 + H * 2                                  # tied LM head + final gain
     for kind in cfg.pattern:
@@ -69,7 +73,7 @@ def bytes_per_token(cfg, pos: int) -> dict:
             w += cfg.at_in_rows * H * 2 + H * cfg.at_q_heads * cfg.at_head_dim * 2
     s = cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
     conv = cfg.n_dn * cfg.conv_width * cfg.dn_conv_channels * 4
-    kv = cfg.n_at * cfg.at_kv_heads * (pos + 1) * cfg.at_head_dim * 2 * 2
+    kv = cfg.n_at * cfg.at_kv_heads * (pos + 1) * (kv_row_bytes or 2 * cfg.at_head_dim) * 2
     return {"weights": w, "state": s, "conv": conv, "kv": kv, "read": w + s + conv + kv,
             "write": s + cfg.n_dn * cfg.dn_conv_channels * 4 + cfg.n_at * cfg.at_kv_heads * cfg.at_head_dim * 4}
 
@@ -345,17 +349,23 @@ def run_mk(args):
     rank, world, local = dist_setup(args.gpus)
     cfg = synth.QWEN_08B
     dev = torch.device("cuda", local)
-    long_ctx = args.workload == "long"
+    long_ctx = args.workload in ("long", "long_q8")
+    kv_q8 = args.workload == "long_q8"
     P0 = LONG_POS if long_ctx else PROMPT
     raw = synth.make_weights(cfg)
-    m = hda.Model(cfg, hda.weights_to_device(raw, dev), max_ctx=(LONG_POS + TG + 16) if long_ctx else MAX_CTX)
+    m = hda.Model(cfg, hda.weights_to_device(raw, dev), max_ctx=(LONG_POS + TG + 16) if long_ctx else MAX_CTX,
+                  kv_format=hda._abi.MK_KV_Q8 if kv_q8 else hda._abi.MK_KV_BF16)
     del raw
     prompt_np = synth.make_prompt(cfg, PROMPT)
     prompt = torch.from_numpy(prompt_np).to(dev)
 
     # context after the prompt (or the seeded long context), snapshotted once; every step restores it
     first = torch.empty(1, dtype=torch.int32, device=dev)
-    if long_ctx:
+    if kv_q8:   # the 8-bit rows are written by the library itself: prefill a random long prompt
+        m.reset()
+        ctx = torch.from_numpy(synth.make_prompt(cfg, LONG_POS, tag="long.ctx")).to(dev)
+        m.prefill(ctx, next_token=first)
+    elif long_ctx:
         first.fill_(seed_long_context(m, cfg, LONG_POS, dev))
     else:
         m.reset()
@@ -405,7 +415,7 @@ def run_mk(args):
     value = replica_throughput(args.steps * TG, world, total_ms / 1000.0)
 
     # roofline of the decode kernel: algorithmic bytes per launch / average launch duration
-    per = [bytes_per_token(cfg, P0 + i) for i in range(TG)]
+    per = [bytes_per_token(cfg, P0 + i, int(m.sizes.kv_row_bytes)) for i in range(TG)]
     read_avg = float(np.mean([b["read"] for b in per]))
     write_avg = float(np.mean([b["write"] for b in per]))
     t_launch = decode_ms / 1000.0 / (args.steps * TG)
@@ -469,7 +479,8 @@ def run_mk(args):
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": LONG_WORKLOAD if long_ctx else WORKLOAD, "tokens_per_step": TG,
+        "config": {"workload": (LONG_Q8_WORKLOAD if kv_q8 else LONG_WORKLOAD) if long_ctx else WORKLOAD,
+                   "tokens_per_step": TG,
                    "context_at_start": P0,
                    "l2": "inputs larger than L2: every step streams 1.23 GB of weights (L2 is 126 MB)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
@@ -732,7 +743,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="tg128", choices=["tg128", "long", "pp520", "pp4096", "27b", "verify08"])
+    ap.add_argument("--workload", default="tg128",
+                    choices=["tg128", "long", "long_q8", "pp520", "pp4096", "27b", "verify08"])
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -29,6 +29,8 @@ MK_DT_F32 = 2
 MK_DT_Q4K = 3
 MK_W_BF16 = 0
 MK_W_Q4K = 1
+MK_KV_BF16 = 0
+MK_KV_Q8 = 1
 MK_MAX_LAYERS = 128
 
 # every symbol include/mk.h declares
@@ -59,6 +61,7 @@ class MkConfig(C.Structure):
         ("weight_format", C.c_int32),
         ("max_ctx", C.c_int32),
         ("max_draft", C.c_int32),
+        ("kv_format", C.c_int32),
     ]
 
 
@@ -85,7 +88,7 @@ class MkSizes(C.Structure):
         ("off_pos", C.c_uint64),
         ("off_err", C.c_uint64),
         ("grid_ctas", C.c_int32),
-        ("reserved", C.c_int32),
+        ("kv_row_bytes", C.c_int32),
     ]
 
 

@@ -136,6 +136,13 @@ __global__ void accept_kernel(const int* tokens, const int* g, int K, int* n_out
 
 namespace {
 
+// Bytes per (layer, kv head, position) row of the KV cache.
+size_t kv_row_bytes(const mk_config& c) {
+  const size_t D = static_cast<size_t>(c.at_head_dim);
+  if (c.kv_format == MK_KV_Q8) return (D + D / 16 + 15) / 16 * 16;   // codes, fp16 scales, padding
+  return 2 * D;
+}
+
 int check_config(const mk_config* c) {
   if (!c) return fail(MK_ERR_ARG, "config is NULL");
   if (c->n_layers < 1 || c->n_layers > MK_MAX_LAYERS) return fail(MK_ERR_ARG, "n_layers out of range");
@@ -150,6 +157,7 @@ int check_config(const mk_config* c) {
   if (c->max_ctx <= 0) return fail(MK_ERR_ARG, "max_ctx must be positive");
   if (c->max_draft < 0 || c->max_draft > 16) return fail(MK_ERR_ARG, "max_draft must be in [0, 16]");
   if (c->weight_format != MK_W_BF16 && c->weight_format != MK_W_Q4K) return fail(MK_ERR_ARG, "unknown weight_format");
+  if (c->kv_format != MK_KV_BF16 && c->kv_format != MK_KV_Q8) return fail(MK_ERR_ARG, "unknown kv_format");
   if (c->weight_format == MK_W_Q4K) {
     const long qd = static_cast<long>(c->at_q_heads) * c->at_head_dim;
     if (c->hidden % 256 || c->ffn % 256 || (static_cast<long>(c->dn_heads) * c->dn_dv) % 256 || qd % 256)
@@ -254,6 +262,7 @@ struct Layout {
   // batched prefill workspace
   int pf_rows;
   size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec, pf_apart, pf_splitk, pf_best;
+  size_t pf_kvd = 0;
   size_t pf_sbuf, pf_phi, pf_plo, pf_vt, pf_img = 0;
   long long pf_nk;
   // batched verify saves
@@ -328,7 +337,8 @@ Layout make_layout(const mk_config& c, int grid) {
   off = 0;
   L.sz.off_S = off; off = align256(off + static_cast<size_t>(nd) * c.dn_heads * c.dn_dv * c.dn_dk * 4);
   L.sz.off_conv = off; off = align256(off + static_cast<size_t>(nd) * c.conv_width * C * 4);
-  const size_t kv = static_cast<size_t>(na) * c.at_kv_heads * c.max_ctx * c.at_head_dim * 2;
+  const size_t kv = static_cast<size_t>(na) * c.at_kv_heads * c.max_ctx * kv_row_bytes(c);
+  L.sz.kv_row_bytes = static_cast<int32_t>(kv_row_bytes(c));
   L.sz.off_k = off; off = align256(off + kv);
   L.sz.off_v = off; off = align256(off + kv);
   L.sz.off_pos = off; off = align256(off + 4);
@@ -396,6 +406,10 @@ Layout make_layout(const mk_config& c, int grid) {
       L.pf_phi = off; off = align256(off + T * nk * 2);
       L.pf_plo = off; off = align256(off + T * nk * 2);
       L.pf_vt = off; off = align256(off + static_cast<size_t>(c.at_head_dim) * nk * 2);
+    }
+    if (na && c.kv_format == MK_KV_Q8) {   // one layer's K and V read back as bf16 for the attention kernels
+      L.pf_kvd = off;
+      off = align256(off + 2ull * c.at_kv_heads * c.max_ctx * c.at_head_dim * 2);
     }
   }
   L.vf_rows = (L.pf_rows > 0 && c.max_draft > 0 && c.max_draft + 1 <= std::min(64, L.pf_rows)) ? c.max_draft + 1 : 0;
@@ -721,6 +735,8 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   b.conv_ring = reinterpret_cast<float*>(St + L.sz.off_conv);
   b.kc = reinterpret_cast<uint16_t*>(St + L.sz.off_k);
   b.vc = reinterpret_cast<uint16_t*>(St + L.sz.off_v);
+  b.kv_q8 = c.kv_format == MK_KV_Q8 ? 1 : 0;
+  b.kv_rb = static_cast<int>(kv_row_bytes(c));
   b.pos = reinterpret_cast<int*>(St + L.sz.off_pos);
   b.err = reinterpret_cast<int*>(St + L.sz.off_err);
   b.hbuf = reinterpret_cast<float*>(W + L.w_h);
@@ -758,6 +774,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     m->pf.splitk = reinterpret_cast<float*>(W + L.pf_splitk);
     m->pf.best = reinterpret_cast<unsigned long long*>(W + L.pf_best);
     m->pf.nk_max = L.pf_nk;
+    m->pf.kvd = L.pf_kvd ? reinterpret_cast<uint16_t*>(W + L.pf_kvd) : nullptr;
     if (L.pf_img) m->pf.img = W + L.pf_img;
     if (L.pf_nk > 0) {
       m->pf.sbuf = reinterpret_cast<float*>(W + L.pf_sbuf);

@@ -162,11 +162,10 @@ __device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Range
         rb = p.dk * 4;
       } else {
         const int sb = r.au_p0 + (s >> 1) * kAttnSub;
-        const uint16_t* base = ((s & 1) ? p.vc : p.kc) +
-                               (static_cast<size_t>(L.idx) * p.Hkv + r.au_g) * p.max_ctx * p.D + static_cast<size_t>(sb) * p.D;
-        src = reinterpret_cast<const uint8_t*>(base);
+        src = reinterpret_cast<const uint8_t*>((s & 1) ? p.vc : p.kc) +
+              ((static_cast<size_t>(L.idx) * p.Hkv + r.au_g) * p.max_ctx + sb) * p.kv_rb;
         rows = min(kAttnSub, r.au_q1 - sb);
-        rb = p.D * 2;
+        rb = p.kv_rb;
       }
       return true;
     }
@@ -227,12 +226,10 @@ __device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Range
   } else {
     if (s < nkv) {
       const int sb = r.au_p0 + (s >> 1) * kAttnSub;
-      const uint16_t* base = ((s & 1) ? p.vc : p.kc) +
-                             (static_cast<size_t>(L.idx) * p.Hkv + r.au_g) * p.max_ctx * p.D +
-                             static_cast<size_t>(sb) * p.D;
-      src = reinterpret_cast<const uint8_t*>(base);
+      src = reinterpret_cast<const uint8_t*>((s & 1) ? p.vc : p.kc) +
+            ((static_cast<size_t>(L.idx) * p.Hkv + r.au_g) * p.max_ctx + sb) * p.kv_rb;
       rows = min(kAttnSub, r.au_q1 - sb);
-      rb = p.D * 2;
+      rb = p.kv_rb;
       return true;
     }
     s -= nkv;
@@ -1227,20 +1224,47 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
             const float x1 = __ldcg(p.z + hq * D + i), x2 = __ldcg(p.z + hq * D + i + half);
             qs[t * D + i] = (x1 * cs - x2 * sn) * scale;
             qs[t * D + i + half] = (x1 * sn + x2 * cs) * scale;
-          } else {   // current key: rotate, round to bf16, append to the cache
+          } else {   // current key: rotate, then append it to the cache (bf16 here, 8-bit below)
             const float x1 = __ldcg(p.z + koff + ug * D + i), x2 = __ldcg(p.z + koff + ug * D + i + half);
-            const uint16_t k1 = f_to_bf16(x1 * cs - x2 * sn), k2 = f_to_bf16(x1 * sn + x2 * cs);
-            p.kc[cache_g + static_cast<size_t>(pos) * D + i] = k1;
-            p.kc[cache_g + static_cast<size_t>(pos) * D + i + half] = k2;
-            kcur[i] = bf16_to_f(k1);
-            kcur[i + half] = bf16_to_f(k2);
+            if (p.kv_q8) {   // 8-bit rows: quantised below, once the whole vector is here
+              kcur[i] = x1 * cs - x2 * sn;
+              kcur[i + half] = x1 * sn + x2 * cs;
+            } else {
+              const uint16_t k1 = f_to_bf16(x1 * cs - x2 * sn), k2 = f_to_bf16(x1 * sn + x2 * cs);
+              p.kc[cache_g + static_cast<size_t>(pos) * D + i] = k1;
+              p.kc[cache_g + static_cast<size_t>(pos) * D + i + half] = k2;
+              kcur[i] = bf16_to_f(k1);
+              kcur[i + half] = bf16_to_f(k2);
+            }
           }
         }
         if (has_cur) {
           for (int d = tid; d < D; d += kConsumerThreads) {
-            const uint16_t vb = f_to_bf16(__ldcg(p.z + voff + ug * D + d));
-            p.vc[cache_g + static_cast<size_t>(pos) * D + d] = vb;
-            vcur[d] = bf16_to_f(vb);
+            const float vx = __ldcg(p.z + voff + ug * D + d);
+            if (p.kv_q8) {
+              vcur[d] = vx;
+            } else {
+              const uint16_t vb = f_to_bf16(vx);
+              p.vc[cache_g + static_cast<size_t>(pos) * D + d] = vb;
+              vcur[d] = bf16_to_f(vb);
+            }
+          }
+          if (p.kv_q8) {   // blocks of 32 of the key, then of the value, one warp per block
+            cons_sync(kConsumerThreads);
+            const int nb = D / 32;
+            const size_t row = ((static_cast<size_t>(L.idx) * p.Hkv + ug) * p.max_ctx + pos) * p.kv_rb;
+            for (int blk = warp; blk < 2 * nb; blk += kConsumerWarps) {
+              const bool isv = blk >= nb;
+              const int j = (blk - (isv ? nb : 0)) * 32 + lane;
+              float* cur = isv ? vcur : kcur;
+              uint8_t* dst = reinterpret_cast<uint8_t*>(isv ? p.vc : p.kc) + row;
+              unsigned short sbits;
+              float back;
+              const int q = q8_block_lane(cur[j], sbits, back);
+              dst[j] = static_cast<uint8_t>(static_cast<int8_t>(q));
+              if (lane == 0) reinterpret_cast<unsigned short*>(dst + D)[j >> 5] = sbits;
+              cur[j] = back;   // the current position attends to what the cache holds
+            }
           }
         }
         if (tid < grp) {
@@ -1256,11 +1280,19 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
         for (int sb = p0; sb < q1; sb += kAttnSub) {
           const int np = min(kAttnSub, q1 - sb);
           {   // scores q_t . K[pp] from the K rows in shared memory, one warp per row
-            const uint16_t* kch = reinterpret_cast<const uint16_t*>(acquire<NS>(p, sh, ring, n, tid, lane));
+            const uint8_t* kb8 = acquire<NS>(p, sh, ring, n, tid, lane);
+            const uint16_t* kch = reinterpret_cast<const uint16_t*>(kb8);
             for (int pp = warp; pp < np; pp += kConsumerWarps) {
               const uint16_t* krow = kch + static_cast<size_t>(pp) * D + lane * dpl;
               float kf[8];
-              if (dpl == 8) {
+              if (p.kv_q8) {   // lane's dpl codes lie in one block of 32: one scale
+                const uint8_t* kr8 = kb8 + static_cast<size_t>(pp) * p.kv_rb;
+                const float ks = __half2float(__ushort_as_half(
+                    reinterpret_cast<const unsigned short*>(kr8 + D)[(lane * dpl) >> 5]));
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                  kf[q] = (q < dpl) ? ks * static_cast<float>(static_cast<int8_t>(kr8[lane * dpl + q])) : 0.f;
+              } else if (dpl == 8) {
                 const uint4 kw = *reinterpret_cast<const uint4*>(krow);
                 kf[0] = bf16lo(kw.x); kf[1] = bf16hi(kw.x); kf[2] = bf16lo(kw.y); kf[3] = bf16hi(kw.y);
                 kf[4] = bf16lo(kw.z); kf[5] = bf16hi(kw.z); kf[6] = bf16lo(kw.w); kf[7] = bf16hi(kw.w);
@@ -1301,8 +1333,24 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
           softmax_block(sc, mlc, grp, np, warp, lane);
           cons_sync(kConsumerThreads);
           {   // values: thread d accumulates sum_pp p[pp] V[pp][d]
-            const uint16_t* vch = reinterpret_cast<const uint16_t*>(acquire<NS>(p, sh, ring, n, tid, lane));
-            if (tid < D) {
+            const uint8_t* vb8 = acquire<NS>(p, sh, ring, n, tid, lane);
+            const uint16_t* vch = reinterpret_cast<const uint16_t*>(vb8);
+            if (tid < D && p.kv_q8) {   // 8-bit rows: code tid and the scale of its block
+              float vsum[8];
+#pragma unroll
+              for (int t = 0; t < 8; ++t) vsum[t] = 0.f;
+              for (int pp = 0; pp < np; ++pp) {
+                const uint8_t* vr = vb8 + static_cast<size_t>(pp) * p.kv_rb;
+                const float vvv = __half2float(__ushort_as_half(reinterpret_cast<const unsigned short*>(vr + D)[tid >> 5])) *
+                                  static_cast<float>(static_cast<int8_t>(vr[tid]));
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                  if (t < grp) vsum[t] = fmaf(sc[t * kAttnSub + pp], vvv, vsum[t]);
+              }
+#pragma unroll
+              for (int t = 0; t < 8; ++t)
+                if (t < grp) oacc[t] = oacc[t] * mlc[3 * t + 2] + vsum[t];
+            } else if (tid < D) {
               float vsum[8];
 #pragma unroll
               for (int t = 0; t < 8; ++t) vsum[t] = 0.f;

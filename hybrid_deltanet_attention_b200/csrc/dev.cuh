@@ -2,6 +2,7 @@
 // with a time limit, and small numeric helpers.
 #pragma once
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace mk {
@@ -165,6 +166,21 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
+}
+
+// One block of 32 entries of the 8-bit KV-cache format, one entry per lane of a full warp:
+// scale = max|x| / 127 (float32 division), code = x / scale rounded to nearest, ties to even,
+// clamped to +-127 (0 for an all-zero block). Returns the code; sets the scale as fp16 bits
+// and the value the entry reads back as (fp16 scale times code).
+__device__ __forceinline__ int q8_block_lane(float x, unsigned short& scale_bits, float& readback) {
+  const float amax = warp_max(fabsf(x));
+  const float d = amax / 127.0f;
+  int q = 0;
+  if (d > 0.f) q = max(-127, min(127, static_cast<int>(rintf(x / d))));
+  const __half h = __float2half_rn(d);
+  scale_bits = __half_as_ushort(h);
+  readback = __half2float(h) * static_cast<float>(q);
+  return q;
 }
 
 // 8 bf16 weights (one uint4) dotted with 8 bf16 activations (one uint4).

@@ -51,8 +51,10 @@ struct DecodeParams {
   // state (caller-owned)
   float* S;                 // [n_dn][Hd][dv][dk]
   float* conv_ring;         // [n_dn][W][C]
-  uint16_t* kc;             // [n_at][Hkv][max_ctx][D]
+  uint16_t* kc;             // [n_at][Hkv][max_ctx] rows of kv_rb bytes: bf16 [D], or 8-bit (kv_q8)
   uint16_t* vc;
+  int kv_q8;                // 1: a row is D int8 codes, then D/32 fp16 scales (blocks of 32)
+  int kv_rb;                // bytes per cache row (2 * D for bf16)
   int* pos;
   int* err;
   // workspace (caller-owned)

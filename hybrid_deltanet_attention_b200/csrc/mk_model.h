@@ -36,7 +36,10 @@ struct mk_prefill_ws {
   uint16_t* plo = nullptr;
   uint16_t* vt = nullptr;
   // chunked delta rule on the tensor cores: bf16 operand images [chunks][Hd][bytes per image]
-  uint8_t* img = nullptr;};
+  uint8_t* img = nullptr;
+  // 8-bit KV cache: one attention layer's K and V read back as bf16 [2][Hkv][max_ctx][D]
+  uint16_t* kvd = nullptr;
+};
 
 struct mk_prefill_layer {   // K-major copies of the projections the decode kernel keeps transposed
   const uint8_t* w_out;      // [H][K_mix] bf16

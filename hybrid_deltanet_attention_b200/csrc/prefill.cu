@@ -585,7 +585,8 @@ __global__ void conv_history_update(const float* __restrict__ z, int ldz, int T,
 // appended to the bf16 cache at position pos0 + t.
 __global__ void at_prep(const float* __restrict__ z, int ldz, const int* __restrict__ posp, int off,
                         const double* __restrict__ inv_freq, int Hq, int Hkv, int D, int gated, uint16_t* __restrict__ kc,
-                        uint16_t* __restrict__ vc, int max_ctx, float* __restrict__ q, int ldq) {
+                        uint16_t* __restrict__ vc, int max_ctx, float* __restrict__ q, int ldq, int kv_rb, int kv_q8) {
+  extern __shared__ float kvs[];   // 8-bit cache: the token's roped keys [Hkv][D], then values [Hkv][D]
   const int t = blockIdx.x, pos = *posp + off + t, half = D / 2;
   if (pos < 0 || pos >= max_ctx) return;    // capacity: latched by check_capacity
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
@@ -602,15 +603,51 @@ __global__ void at_prep(const float* __restrict__ z, int ldz, const int* __restr
     } else {
       const int g = hv - Hq;
       const float x1 = zr[koff + g * D + i], x2 = zr[koff + g * D + i + half];
-      const long long base = (static_cast<long long>(g) * max_ctx + pos) * D;
-      kc[base + i] = f_to_bf16(x1 * cs - x2 * sn);
-      kc[base + i + half] = f_to_bf16(x1 * sn + x2 * cs);
+      if (kv_q8) {
+        kvs[g * D + i] = x1 * cs - x2 * sn;
+        kvs[g * D + i + half] = x1 * sn + x2 * cs;
+      } else {
+        const long long base = (static_cast<long long>(g) * max_ctx + pos) * D;
+        kc[base + i] = f_to_bf16(x1 * cs - x2 * sn);
+        kc[base + i + half] = f_to_bf16(x1 * sn + x2 * cs);
+      }
     }
   }
   for (int idx = threadIdx.x; idx < Hkv * D; idx += blockDim.x) {
     const int g = idx / D, d = idx % D;
-    vc[(static_cast<long long>(g) * max_ctx + pos) * D + d] = f_to_bf16(zr[voff + idx]);
+    if (kv_q8) kvs[Hkv * D + idx] = zr[voff + idx];
+    else vc[(static_cast<long long>(g) * max_ctx + pos) * D + d] = f_to_bf16(zr[voff + idx]);
   }
+  if (!kv_q8) return;
+  __syncthreads();   // 8-bit rows: blocks of 32 entries, one warp per block
+  const int nb = D / 32, lane = threadIdx.x & 31;
+  for (int blk = threadIdx.x >> 5; blk < 2 * Hkv * nb; blk += blockDim.x >> 5) {
+    const bool isv = blk >= Hkv * nb;
+    const int b2 = blk - (isv ? Hkv * nb : 0), g = b2 / nb, jb = b2 % nb;
+    uint8_t* row = reinterpret_cast<uint8_t*>(isv ? vc : kc) + (static_cast<size_t>(g) * max_ctx + pos) * kv_rb;
+    unsigned short sbits;
+    float back;
+    const int qc = q8_block_lane(kvs[(isv ? Hkv * D : 0) + g * D + jb * 32 + lane], sbits, back);
+    row[jb * 32 + lane] = static_cast<uint8_t>(static_cast<int8_t>(qc));
+    if (lane == 0) reinterpret_cast<unsigned short*>(row + D)[jb] = sbits;
+  }
+}
+
+// Rows [0, nrows) of one attention layer's 8-bit K and V, read back as bf16 into
+// out [2][Hkv][max_ctx][D] for the attention kernels; rows past the pass's last key
+// (device position) are written as zeros.
+__global__ void kv_dequant_bf16(const uint8_t* __restrict__ kq, const uint8_t* __restrict__ vq, int Hkv, int D,
+                                int max_ctx, int kv_rb, const int* __restrict__ posp, int last_off,
+                                uint16_t* __restrict__ out) {
+  const int r = blockIdx.x, g = blockIdx.y, which = blockIdx.z;
+  const int last = min(*posp + last_off, max_ctx - 1);
+  uint16_t* dst = out + ((static_cast<size_t>(which) * Hkv + g) * max_ctx + r) * D;
+  const uint8_t* src = (which ? vq : kq) + (static_cast<size_t>(g) * max_ctx + r) * kv_rb;
+  const unsigned short* sc = reinterpret_cast<const unsigned short*>(src + D);
+  for (int d = threadIdx.x; d < D; d += blockDim.x)
+    dst[d] = r <= last ? f_to_bf16(__half2float(__ushort_as_half(sc[d >> 5])) *
+                                   static_cast<float>(static_cast<int8_t>(src[d])))
+                       : static_cast<uint16_t>(0);
 }
 
 // x = o (* sigmoid(gate) when gate != null), as bf16 high/low parts [T][n].
@@ -2176,14 +2213,25 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       linear(q4 ? L.w_out_q4 : PL.w_out, 2LL * Hd * dv, H, Hd * dv, pf.h, H, 1);
     } else {
       const int rows = b.at_in_rows;
-      uint16_t* kc = b.kc + static_cast<size_t>(ai) * Hkv * c.max_ctx * D;
-      uint16_t* vc = b.vc + static_cast<size_t>(ai) * Hkv * c.max_ctx * D;
+      uint16_t* kc = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(b.kc) +
+                                                 static_cast<size_t>(ai) * Hkv * c.max_ctx * b.kv_rb);
+      uint16_t* vc = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(b.vc) +
+                                                 static_cast<size_t>(ai) * Hkv * c.max_ctx * b.kv_rb);
       ++ai;
       linear(L.w_in, 2LL * H, rows, H, pf.z, rows, 0);
-      at_prep<<<T, kPT, 0, s>>>(pf.z, rows, b.pos, off, b.inv_freq, Hq, Hkv, D, c.at_out_gate, kc, vc, c.max_ctx,
-                                 pf.y, qd);
+      at_prep<<<T, kPT, b.kv_q8 ? 2 * static_cast<size_t>(Hkv) * D * sizeof(float) : 0, s>>>(
+          pf.z, rows, b.pos, off, b.inv_freq, Hq, Hkv, D, c.at_out_gate, kc, vc, c.max_ctx, pf.y, qd, b.kv_rb, b.kv_q8);
       chk();
       const long long nk_gemm = (m->pos_max + off + T + 63) / 64 * 64;   // covers every key of the pass
+      if (b.kv_q8 && e == cudaSuccess) {   // the attention kernels below read bf16 rows
+        const int nrows = static_cast<int>(std::min<long long>(nk_gemm, c.max_ctx));
+        kv_dequant_bf16<<<dim3(nrows, Hkv, 2), 64, 0, s>>>(reinterpret_cast<const uint8_t*>(kc),
+                                                           reinterpret_cast<const uint8_t*>(vc), Hkv, D, c.max_ctx,
+                                                           b.kv_rb, b.pos, off + T - 1, pf.kvd);
+        chk();
+        kc = pf.kvd;
+        vc = pf.kvd + static_cast<size_t>(Hkv) * c.max_ctx * D;
+      }
       if (T >= kGemmAttnMinRows && pf.sbuf && nk_gemm <= pf.nk_max) {
         const int nk = static_cast<int>(nk_gemm);
         const int grp = Hq / Hkv;

@@ -16,7 +16,7 @@ from . import _abi
 from ._abi import MkConfig, MkSizes, MkTensor, check
 
 
-def make_config(cfg, max_ctx: int, max_draft: int = 0) -> MkConfig:
+def make_config(cfg, max_ctx: int, max_draft: int = 0, kv_format: int = 0) -> MkConfig:
     """Build the C config from any object with the model-shape attributes
     (n_layers, pattern, hidden, vocab, rms_eps, dn_heads, dn_dk, dn_dv, conv_width,
     at_q_heads, at_kv_heads, at_head_dim, rope_theta, at_out_gate, ffn, weight_format)."""
@@ -39,6 +39,7 @@ def make_config(cfg, max_ctx: int, max_draft: int = 0) -> MkConfig:
     c.weight_format = cfg.weight_format
     c.max_ctx = max_ctx
     c.max_draft = max_draft
+    c.kv_format = kv_format
     return c
 
 
@@ -60,10 +61,11 @@ class Model:
     """
 
     def __init__(self, cfg, weights: Dict[str, torch.Tensor], max_ctx: int, max_draft: int = 0,
-                 stream: Optional[torch.cuda.Stream] = None):
+                 stream: Optional[torch.cuda.Stream] = None, kv_format: int = 0):
         self.lib = _abi.load_library()
         self.shape = cfg
-        self.cfg = make_config(cfg, max_ctx, max_draft)
+        self.kv_format = int(kv_format)
+        self.cfg = make_config(cfg, max_ctx, max_draft, self.kv_format)
         self.sizes = MkSizes()
         check(self.lib.mk_query_sizes(C.byref(self.cfg), C.byref(self.sizes)))
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -124,15 +126,28 @@ class Model:
         c = self.shape
         return self._view(self.sizes.off_conv, torch.float32, (c.n_dn, c.conv_width, c.dn_conv_channels))
 
+    def _kv_view(self, off: int) -> torch.Tensor:
+        c = self.shape
+        if self.kv_format == _abi.MK_KV_Q8:      # raw rows: D int8 codes, D/32 fp16 scales, padding
+            return self._view(off, torch.uint8, (c.n_at, c.at_kv_heads, self.cfg.max_ctx, int(self.sizes.kv_row_bytes)))
+        return self._view(off, torch.bfloat16, (c.n_at, c.at_kv_heads, self.cfg.max_ctx, c.at_head_dim))
+
     @property
     def k_cache(self) -> torch.Tensor:
-        c = self.shape
-        return self._view(self.sizes.off_k, torch.bfloat16, (c.n_at, c.at_kv_heads, self.cfg.max_ctx, c.at_head_dim))
+        return self._kv_view(self.sizes.off_k)
 
     @property
     def v_cache(self) -> torch.Tensor:
-        c = self.shape
-        return self._view(self.sizes.off_v, torch.bfloat16, (c.n_at, c.at_kv_heads, self.cfg.max_ctx, c.at_head_dim))
+        return self._kv_view(self.sizes.off_v)
+
+    def kv_q8_rows(self, which: str):
+        """8-bit cache rows split into (codes int8 [n_at, Hkv, max_ctx, D], scales float16
+        [n_at, Hkv, max_ctx, D/32]), on the host."""
+        D = self.shape.at_head_dim
+        raw = (self.k_cache if which == "k" else self.v_cache).cpu()
+        codes = raw[..., :D].contiguous().view(torch.int8)
+        scales = raw[..., D:D + D // 16].contiguous().view(torch.float16)
+        return codes.numpy(), scales.numpy()
 
     @property
     def pos_tensor(self) -> torch.Tensor:

@@ -74,6 +74,14 @@ extern "C" {
 #define MK_W_BF16   0     /* every tensor bf16 */
 #define MK_W_Q4K    1     /* 2-D projections (incl. the tied embedding) as MK_DT_Q4K; conv taps, gains bf16 */
 
+/* ---- KV-cache entry formats ---- */
+#define MK_KV_BF16  0     /* one bf16 per entry */
+#define MK_KV_Q8    1     /* per (layer, kv head, position) row: D int8 codes, then D/32 fp16 scales,
+                             the row padded to a multiple of 16 bytes; entry j reads back as
+                             scale[j / 32] * code[j]; blocks of 32 with scale = max|x| / 127 and
+                             code = round(x / scale) (float32, ties to even); the 8-bit cache the
+                             open-jet follow-up's limits section uses for long contexts */
+
 #define MK_MAX_LAYERS 128
 
 /* Model shape. Plain data; copied at load. */
@@ -96,6 +104,7 @@ typedef struct mk_config {
   int32_t weight_format;   /* MK_W_BF16 or MK_W_Q4K */
   int32_t max_ctx;         /* KV-cache capacity in positions */
   int32_t max_draft;       /* largest K accepted by mk_verify_drafts */
+  int32_t kv_format;       /* MK_KV_BF16 or MK_KV_Q8 */
 } mk_config;
 
 /* One input weight tensor (device memory, caller-owned, read during mk_load_weights only).
@@ -136,8 +145,9 @@ typedef struct mk_tensor {
  * State buffer (all offsets in bytes, 256-byte aligned):
  *   off_S    fp32 [n_dn][Hd][dv][dk]     DeltaNet states S (row i of head h = value dim i)
  *   off_conv fp32 [n_dn][W][Hd*(2dk+dv)] raw conv inputs; slot (p mod W) holds position p
- *   off_k    bf16 [n_at][Hkv][max_ctx][D] key cache (RoPE applied)
- *   off_v    bf16 [n_at][Hkv][max_ctx][D] value cache
+ *   off_k    [n_at][Hkv][max_ctx] rows of the key cache (RoPE applied): bf16 [D], or with
+ *            MK_KV_Q8 the 8-bit row format above (kv_row_bytes in mk_sizes)
+ *   off_v    the value cache, same layout
  *   off_pos  int32   number of positions consumed so far
  *   off_err  int32   device error word (MK_DEVERR_* bits)
  */
@@ -147,7 +157,7 @@ typedef struct mk_sizes {
   uint64_t workspace_bytes;
   uint64_t off_S, off_conv, off_k, off_v, off_pos, off_err;
   int32_t  grid_ctas;      /* persistent CTAs the decode kernel will use on the current device */
-  int32_t  reserved;
+  int32_t  kv_row_bytes;   /* bytes per (layer, kv head, position) row of the KV cache */
 } mk_sizes;
 
 typedef struct mk_model mk_model;   /* opaque host-side handle */
