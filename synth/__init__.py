@@ -129,7 +129,11 @@ MID_Q4 = _preset("mid-q4", n_layers=8, pattern="DDDA" * 2, hidden=1024, vocab=32
 # (about 1.4 GB of 4-bit weights), for profiling.
 QWEN_27B_4L = dataclasses.replace(QWEN_27B, name="27b-4l", n_layers=4, pattern="DDDA")
 
-CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI, TINY_Q4, MID_Q4, QWEN_27B_4L)}
+# The same four 27B-shaped layers with a 32K vocabulary: small enough for the float64 oracle
+# (1.7 B weights), and it runs the hidden-5120 decode instance the 27B model runs.
+QWEN_27B_4L_32K = dataclasses.replace(QWEN_27B, name="27b-4l-32k", n_layers=4, pattern="DDDA", vocab=32768)
+
+CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI, TINY_Q4, MID_Q4, QWEN_27B_4L, QWEN_27B_4L_32K)}
 
 
 def with_changes(cfg: ModelConfig, **kw) -> ModelConfig:

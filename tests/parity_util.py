@@ -40,3 +40,34 @@ def conv_history_as_window(ring, pos, width):
         p = pos - m
         rows.append(ring[p % width] if p >= 0 else np.zeros_like(ring[0]))
     return np.stack(rows)
+
+
+def assert_bf16_cache_close(got, want, rel_rms=5e-3, max_changed=0.15):
+    """bf16 cache entries: both sides round a float value to bf16, so an entry may differ
+    by one bf16 step when the two unrounded values straddle a rounding midpoint, and the
+    unrounded values themselves differ by the path's activation error, which scales with
+    the slice, not with a small entry. Bound per entry: one bf16 step at the larger of the
+    two magnitudes plus rel_rms times the root mean square of its (layer, kv head) slice.
+    At most max_changed of the entries may differ at all. A RoPE, ordering or position
+    slip moves entries by about the slice's scale and fails the bound by orders of
+    magnitude. On failure the message lists the worst entries (index, oracle, GPU) and the
+    largest excess beyond one bf16 step, in units of the slice's RMS."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape
+    lead = got.shape[:-2]
+    g = got.reshape(-1, *got.shape[-2:])
+    w = want.reshape(-1, *want.shape[-2:])
+    for i in range(g.shape[0]):
+        rms = float(np.sqrt(np.mean(w[i] ** 2))) if w[i].size else 0.0
+        mag = np.maximum(np.abs(w[i]), np.abs(g[i]))
+        ulp = np.where(mag > 0, 2.0 ** (np.floor(np.log2(np.maximum(mag, 1e-38))) - 7), 0.0)
+        d = np.abs(g[i] - w[i])
+        excess = np.maximum(d - ulp, 0.0) / max(rms, 1e-30)
+        bad = excess > rel_rms
+        if bad.any():
+            order = np.argsort(excess, axis=None)[::-1][:5]
+            worst = [(np.unravel_index(k, excess.shape), float(w[i].flat[k]), float(g[i].flat[k])) for k in order]
+            raise AssertionError(f"slice {np.unravel_index(i, lead) if lead else i}: max excess "
+                                 f"{float(excess.max()):.3g} x rms (rms {rms:.3g}); worst {worst}")
+        assert (d > 0).mean() <= max_changed, float((d > 0).mean())

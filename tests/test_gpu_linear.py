@@ -75,3 +75,12 @@ def test_linear_rejects_bad_sizes():
     assert lib.mk_linear(p, 96, 4, 96, p, 192, 4, p, 4, 0, p, buf.numel(), err.data_ptr(), None) == -1
     # scratch too small
     assert lib.mk_linear(p, 64, 64, 64, p, 128, 4, p, 4, 0, p, 100, err.data_ptr(), None) == -1
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(4096, 6176, 1024, 7), (2048, 7168, 1024, 8), (4096, 1024, 3584, 9)])
+def test_linear_many_tiles_per_cta(M, N, K, seed):
+    """Hundreds of output tiles (800, 448 and 128-plus-K-split work items at the prefill's
+    in-projection, gate/up and down shapes): each persistent CTA walks several tiles and
+    alternates its two TMEM accumulators, so one tile's epilogue overlaps the next tile's
+    MMAs. Every element is checked against the float64 product."""
+    _run(M, N, K, row_pad_bytes=16 if N == 6176 else 0, seed=seed)

@@ -141,3 +141,53 @@ def test_mid_q4_verify_one_pass():
         assert max(rel_frob(S[li], st.S[li]) for li in range(cfg.n_dn)) <= STATE_REL_FROB
         assert int(m.pos_tensor.item()) == st.pos
         last = int(committed[-1])
+
+
+@pytest.fixture(scope="module")
+def q27():
+    """Four layers of the 27B shape (hidden 5120, 48 DeltaNet heads, 24/4 attention heads,
+    FFN 17408, seed-4 4-bit weights) with a 32K vocabulary."""
+    cfg = synth.QWEN_27B_4L_32K
+    m, W = _setup(cfg, 96, max_draft=5)
+    return cfg, m, W
+
+
+def test_27b_shape_q4_decode_parity(q27):
+    """The hidden-5120 decode instance the 27B model runs (prompt through decode launches,
+    then teacher-forced steps), against the oracle."""
+    cfg, m, W = q27
+    _teacher_forced(cfg, m, W, 8, 6, 96)
+
+
+def test_27b_shape_q4_batched_prefill_and_verify(q27):
+    """A 40-token prompt through the batched 4-bit prefill, then two verify passes of five
+    drafts (all right, then the seeded mix), against the oracle."""
+    cfg, m, W = q27
+    dev = torch.device("cuda")
+    K = 5
+    prompt = synth.make_prompt(cfg, 41, tag="q27v")
+    m.reset()
+    st = oracle.new_state(cfg, 96)
+    oracle.prefill(cfg, W, st, prompt[:-1])
+    m.prefill(torch.from_numpy(prompt[:-1]).to(dev))
+    last = int(prompt[-1])
+    for ps in range(2):
+        greedy, _ = oracle.greedy_generate(cfg, W, st.copy(), last, K)
+        use, ids = synth.draft_choices(4, ps, K, cfg.vocab)
+        if ps == 0:
+            use[:] = True
+        drafts = synth.compose_drafts(greedy, use, ids, cfg.vocab)
+        n_or, committed, z_or = oracle.verify_drafts(cfg, W, st, last, drafts)
+        toks = torch.from_numpy(np.concatenate([[last], drafts]).astype(np.int32)).to(dev)
+        n_acc = torch.zeros(1, dtype=torch.int32, device=dev)
+        out = torch.full((K + 1,), -1, dtype=torch.int32, device=dev)
+        logits = torch.empty((K + 1, cfg.vocab), dtype=torch.float32, device=dev)
+        m.verify(toks, n_acc, out, logits)
+        assert m.sync() == 0
+        assert int(n_acc.item()) == n_or
+        assert list(out.cpu().numpy()[:n_or + 1]) == list(committed)
+        assert np.abs(logits.cpu().numpy() - z_or).max() <= LOGIT_MAX_ABS
+        S = m.S.cpu().numpy()
+        assert max(rel_frob(S[li], st.S[li]) for li in range(cfg.n_dn)) <= STATE_REL_FROB
+        assert int(m.pos_tensor.item()) == st.pos
+        last = int(committed[-1])
