@@ -1,14 +1,17 @@
 // A decode step whose scratch memory lives in a fixed device array of this library, for
 // callers that cannot allocate device memory at the point where they step the model:
-// code running in a CUDA host callback or a stream-ordered host function (where CUDA
-// calls that allocate are not allowed), hard real-time loops that must not hit the
-// implicit synchronisation of cudaMalloc/cudaFree, and hosts that own a fixed memory
-// budget and hand this library only the model's own buffers.
+// hard real-time loops that must not hit the implicit synchronisation of cudaMalloc /
+// cudaFree, and hosts that own a fixed device-memory budget and hand this library only
+// the model's own buffers. It is called from ordinary host code like every other entry
+// point (not from a CUDA host callback or a stream-ordered host function: CUDA allows no
+// CUDA call at all there, and this function makes several).
 //
-// The scratch array below is reserved on every GPU that loads libmk.so, for as long as
-// the process lives. Every call shares it and it keeps the last call's contents, so
-// calls whose kernels overlap on the GPU (on different streams, or from different
-// threads) race on it; the call clears, on its stream, the part that must start at zero.
+// CUDA loads this library's device code lazily by default (since CUDA 12.2), so the
+// scratch array is loaded and reserved on a device at the first call there (the address
+// lookup below), and kept until the process exits. Every call shares it and it keeps the
+// last call's contents, so calls whose kernels overlap on the GPU (on different streams,
+// or from different threads) race on it; the call clears, on its stream, the part that
+// must start at zero.
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -19,7 +22,9 @@
 
 namespace {
 
-// 4 MiB: the 0.8B-shaped model's per-step scratch at a 32K-position context is about 0.7 MB.
+// 4 MiB. The per-step scratch does not depend on the context length (the attention
+// partials are sized by the grid and the KV heads): about 0.7 MB for the 0.8B-shaped model
+// and 1.3 MB for the 27B-shaped one.
 constexpr size_t kStaticScratchBytes = 4u << 20;
 constexpr size_t kZeroHeadBytes = 4096;   // barrier/arrival/argmax words and per-head sums of squares
 constexpr int kMaxDevices = 64;
