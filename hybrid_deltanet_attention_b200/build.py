@@ -45,15 +45,35 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
-    cmd = [nvcc(), *ARCH, *FLAGS]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES] + ["-o", LIB + ".tmp"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
-    if verbose:
-        sys.stderr.write(r.stdout + r.stderr)
+    # one nvcc per source file in parallel (relocatable device code is not needed: the
+    # files share host-side declarations only), then one link step
+    import concurrent.futures as cf
+    import tempfile
+    tmp = tempfile.mkdtemp(prefix="mk_build_")
+    compile_flags = [f for f in FLAGS if f != "-shared"]
+
+    def one(src):
+        obj = os.path.join(tmp, os.path.splitext(src)[0] + ".o")
+        cmd = [nvcc(), *ARCH, *compile_flags, "-c", os.path.join(CSRC, src), "-o", obj]
+        if verbose:
+            cmd += ["-Xptxas", "-v"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, cmd, r
+
+    try:
+        with cf.ThreadPoolExecutor(len(SOURCES)) as ex:
+            results = list(ex.map(one, SOURCES))
+        for src, obj, cmd, r in results:
+            if r.returncode != 0:
+                raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+            if verbose:
+                sys.stderr.write(r.stdout + r.stderr)
+        link = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", *[o for _, o, _, _ in results], "-o", LIB + ".tmp"]
+        r = subprocess.run(link, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError("nvcc link failed:\n" + " ".join(link) + "\n" + r.stdout + r.stderr)
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

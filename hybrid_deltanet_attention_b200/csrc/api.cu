@@ -231,7 +231,8 @@ bool budget_ok(const mk_config& c, int grid, int ltab_entries, const char** why)
       return fail_("attention scratch budget exceeded");
     const long cols = ceil_div(static_cast<long>(c.at_q_heads) * c.at_head_dim, grid);
     const long nhd = ceil_div(cols, c.at_head_dim) + 1;
-    if (nhd * mk::decode_max_splits(grid, c.at_kv_heads) + 2 * cols > S)
+    const long ms = mk::decode_max_splits(grid, c.at_kv_heads);
+    if (2 * nhd * ms + cols * ms + 2 * cols > S)   // m, l per head and split; the columns' split accumulators
       return fail_("attention columns per CTA exceed the scratch budget");
   }
   if (2 * ceil_div(c.ffn, grid) > S) return fail_("MLP rows per CTA exceed the scratch budget");
@@ -748,8 +749,6 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
   b.ssq = reinterpret_cast<float*>(W + L.w_sync + 512);
   b.ybuf = reinterpret_cast<float*>(W + L.w_y);
   b.max_splits = L.max_splits;
-  b.prefetch_bytes = 0;   // L2 prefetch ahead of the ring: measured slower on B200, off by default
-  if (const char* env = getenv("MK_PREFETCH_KB")) b.prefetch_bytes = atoi(env) * 1024;
   m->ws_tok = reinterpret_cast<int32_t*>(W + L.w_tok);
   m->ws_g = reinterpret_cast<int32_t*>(W + L.w_g);
   m->ws_n = reinterpret_cast<int32_t*>(W + L.w_n);
@@ -834,7 +833,7 @@ int mk_prefill(mk_model* m, const int32_t* d_tokens, int32_t n, float* d_last_lo
   if (m->pos_hint + n > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "prompt exceeds the context capacity");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* sink = m->ws_tok + m->cfg.max_ctx + 4;
-  if (m->pf.rows > 0 && n > kBatchedPrefillMin && !getenv("MK_PREFILL_BY_DECODE")) {
+  if (m->pf.rows > 0 && n > kBatchedPrefillMin) {
     // all but the last token through the batched layers, the last one through the
     // decode kernel (its logits and the next token)
     int rc = mk_prefill_batched(m, d_tokens, n - 1, s);
@@ -856,7 +855,7 @@ int mk_verify_drafts(mk_model* m, const int32_t* d_tokens, int32_t K, int32_t* d
   if (K < 1 || K > m->cfg.max_draft) return fail(MK_ERR_ARG, "K outside [1, max_draft]");
   if (m->pos_hint + K + 1 > m->cfg.max_ctx) return fail(MK_ERR_CAPACITY, "drafts exceed the context capacity");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (m->vf.rows >= K + 1 && !getenv("MK_VERIFY_BY_DECODE"))
+  if (m->vf.rows >= K + 1)
     return mk_verify_batched(m, d_tokens, K, d_n_accepted, d_out_tokens, d_logits, s);
   const mk::DecodeParams& b = m->base;
   uint8_t* snapS = m->ws_snap;

@@ -251,58 +251,23 @@ __device__ __forceinline__ bool layer_segment(const DecodeParams& p, const Range
   return false;
 }
 
-// A second walk over the same chunk sequence, used to issue L2 prefetches ahead of the
-// shared-memory fill. next() yields the chunks in stream order; false at the end.
-template <bool Q4>
-struct PrefetchCursor {
-  int l = 0, s = -1, r0 = 0, rows = 0, rb = 1;
-  const uint8_t* src = nullptr;
-  LayerW L;
-
-  __device__ bool next(const DecodeParams& p, const Ranges& r, const uint8_t*& ptr, uint32_t& bytes) {
-    for (;;) {
-      if (l > p.n_layers) return false;
-      if (r0 < rows) {
-        const int rpc = kSlotBytes / rb;
-        ptr = src + static_cast<size_t>(r0) * rb;
-        bytes = static_cast<uint32_t>(min(rpc, rows - r0)) * rb;
-        r0 += rpc;
-        return true;
-      }
-      if (s < 0) L = p.layers[l < p.n_layers ? l : p.n_layers - 1];
-      ++s;
-      r0 = 0;
-      rows = 0;
-      if (!layer_segment<Q4>(p, r, L, l, s, src, rows, rb)) {
-        ++l;
-        s = -1;
-        rows = 0;
-      }
-    }
-  }
-};
-
-// One lane streams the CTA's chunks into the shared-memory ring. With a nonzero
-// p.prefetch_bytes it also keeps L2 prefetches of the chunks that follow running that
-// many bytes ahead, so HBM keeps streaming while the ring is full and the consumers
-// wait at a grid barrier.
-template <int NS, bool Q4>
-__device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) {
+// One lane streams the CTA's chunks into the shared-memory ring: every segment that
+// seg(p, r, L, l, s, src, rows, rb) yields for layers l = 0 .. n_layers (the last one the LM
+// head), in chunks of whole rows of up to kSlotBytes. Consumers take the chunks in the same
+// order. The layer table entry of layer l + 1 is loaded while layer l streams.
+template <int NS, typename Seg>
+__device__ void producer_walk(const DecodeParams& p, Shared* sh, uint8_t* ring, Seg&& seg) {
   const uint64_t pol = policy_evict_first();
   const Ranges r = sh->rg;
   volatile int* abort = &sh->abort_flag;
   uint32_t n = 0;
   bool ok = true;
-  PrefetchCursor<Q4> pf;
-  const uint64_t pf_dist = p.prefetch_bytes > 0 ? static_cast<uint64_t>(p.prefetch_bytes) : 0;
-  uint64_t filled = 0, prefetched = 0;
-  bool pf_live = pf_dist > 0;
   LayerW L = p.layers[0];
   for (int l = 0; l <= p.n_layers && ok; ++l) {
     const LayerW Lnext = (l + 1 < p.n_layers) ? p.layers[l + 1] : L;   // load ahead of use
     const uint8_t* src;
     int rows, rb;
-    for (int s = 0; ok && layer_segment<Q4>(p, r, L, l, s, src, rows, rb); ++s) {
+    for (int s = 0; ok && seg(p, r, L, l, s, src, rows, rb); ++s) {
       const int rpc = kSlotBytes / rb;
       for (int r0 = 0; r0 < rows; r0 += rpc) {
         const uint32_t bytes = static_cast<uint32_t>(min(rpc, rows - r0)) * rb;
@@ -320,17 +285,6 @@ __device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) 
                  &sh->full[slot], pol);
         trace_at(p, kTraceChunks + 4 * static_cast<int>(n));
         ++n;
-        filled += bytes;
-        while (pf_live && prefetched < filled + pf_dist) {
-          const uint8_t* pp;
-          uint32_t pb;
-          if (!pf.next(p, r, pp, pb)) {
-            pf_live = false;
-            break;
-          }
-          if (prefetched + pb > filled) prefetch_l2(pp, pb);   // chunks already in the ring need none
-          prefetched += pb;
-        }
       }
     }
     L = Lnext;
@@ -340,6 +294,13 @@ __device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) 
   int never = 0;
   for (uint32_t m = (n > static_cast<uint32_t>(NS) ? n - NS : 0); m < n; ++m)
     mbar_wait(&sh->full[m % NS], (m / NS) & 1, &never, kDrainLimitNs);
+}
+
+template <int NS, bool Q4>
+__device__ void producer_loop(const DecodeParams& p, Shared* sh, uint8_t* ring) {
+  producer_walk<NS>(p, sh, ring,
+                    [](const DecodeParams& pp, const Ranges& r, const LayerW& L, int l, int s, const uint8_t*& src,
+                       int& rows, int& rb) { return layer_segment<Q4>(pp, r, L, l, s, src, rows, rb); });
 }
 
 // ------------------------------------------------------------------ consumer helpers
@@ -1142,42 +1103,57 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
           for (int i = tid; i < 2 * p.Hd; i += kConsumerThreads) nz[i] = 0.f;
         }
         cons_sync(kConsumerThreads);
-        // S rows: S = a S; u = S k; S += b (v - u) k^T; o = S q
+        // S rows: s = a S; u = s k; S' = s + b (v - u) k^T; o = S' q = s q + b (v - u) (k q).
+        // One pass over a row gives s k, s q and k q (three interleaved warp sums), so the
+        // readout needs no second reduction; each warp takes two rows at a time.
         const int srb = p.dk * 4, srpc = kSlotBytes / srb, vpl = p.dk / 32;
         for (int r0 = 0; r0 < nrows; r0 += srpc) {
           const float* ch = reinterpret_cast<const float*>(acquire<NS>(p, sh, ring, n, tid, lane));
           const int nr = min(srpc, nrows - r0);
-          for (int r = warp; r < nr; r += kConsumerWarps) {
-            const int lr = r0 + r;
-            const int g = g0 + lr;
-            const int hl = g / p.dv - h0;
-            const float a = ab[2 * hl], bb = ab[2 * hl + 1];
-            const float* qv = qk + (2 * hl) * p.dk;
-            const float* kv = qk + (2 * hl + 1) * p.dk;
-            const float* srow = ch + static_cast<size_t>(r) * p.dk;
-            float s[8];
-            float ukk = 0.f;
+          for (int r = warp; r < nr; r += 2 * kConsumerWarps) {
+            const int rr[2] = {r, r + kConsumerWarps};
+            float sv[2][8], red[2][3];
+            int hl[2];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (q < vpl) {
-                s[q] = a * srow[lane + 32 * q];
-                ukk = fmaf(s[q], kv[lane + 32 * q], ukk);
+            for (int u = 0; u < 2; ++u) {
+              const int rw = rr[u] < nr ? rr[u] : r;
+              hl[u] = (g0 + r0 + rw) / p.dv - h0;
+              const float a = ab[2 * hl[u]];
+              const float* qv = qk + (2 * hl[u]) * p.dk;
+              const float* kv = qk + (2 * hl[u] + 1) * p.dk;
+              const float* srow = ch + static_cast<size_t>(rw) * p.dk;
+              red[u][0] = red[u][1] = red[u][2] = 0.f;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                if (q < vpl) {
+                  const float kk = kv[lane + 32 * q], qq = qv[lane + 32 * q];
+                  sv[u][q] = a * srow[lane + 32 * q];
+                  red[u][0] = fmaf(sv[u][q], kk, red[u][0]);
+                  red[u][1] = fmaf(sv[u][q], qq, red[u][1]);
+                  red[u][2] = fmaf(kk, qq, red[u][2]);
+                }
               }
             }
-            ukk = warp_sum(ukk);
-            const float coef = bb * (vv[lr] - ukk);
-            float o = 0.f;
-            float* sg_out = p.S + (static_cast<size_t>(L.idx) * p.Hd * p.dv + g) * p.dk;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (q < vpl) {
-                s[q] = fmaf(coef, kv[lane + 32 * q], s[q]);
-                o = fmaf(s[q], qv[lane + 32 * q], o);
-                __stcg(sg_out + lane + 32 * q, s[q]);
-              }
+            for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int c = 0; c < 3; ++c) red[u][c] += __shfl_xor_sync(0xFFFFFFFFu, red[u][c], o);
             }
-            o = warp_sum(o);
-            if (lane == 0) oc[lr] = o;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              if (rr[u] >= nr) continue;
+              const int lr = r0 + rr[u];
+              const int g = g0 + lr;
+              const float coef = ab[2 * hl[u] + 1] * (vv[lr] - red[u][0]);
+              const float* kv = qk + (2 * hl[u] + 1) * p.dk;
+              float* sg_out = p.S + (static_cast<size_t>(L.idx) * p.Hd * p.dv + g) * p.dk;
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                if (q < vpl) __stcg(sg_out + lane + 32 * q, fmaf(coef, kv[lane + 32 * q], sv[u][q]));
+              if (lane == 0) oc[lr] = fmaf(coef, red[u][2], red[u][1]);
+            }
           }
           release<NS>(p, sh, n, lane);
         }
@@ -1427,43 +1403,59 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
       if (ncol > 0) {
         const int hA = c0 / p.D, hB = (c1 - 1) / p.D;
         const int nhd = hB - hA + 1;
-        // scratch: wts[nhd][nsplit] (m_j, then e^{m_j - M} / L) | gte[ncol] | oc[ncol]
-        float* wts = fs;
-        float* gte = wts + nhd * nsplit;
-        float* oc = gte + ncol;
-        for (int i = tid; i < nhd * nsplit + ncol; i += kConsumerThreads) {
-          if (i < nhd * nsplit) {
-            const int hq = hA + i / nsplit, j = i % nsplit;
-            wts[i] = __ldcg(p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (p.D + 2) + p.D);
-          } else {
-            const int cc = i - nhd * nsplit;
-            gte[cc] = p.gated ? sigmoidf_(__ldcg(p.z + p.Hq * p.D + c0 + cc)) : 1.0f;
+        // scratch: mv[nhd][nsplit] (m_j, then the weight e^{m_j - M} / L) | lv[nhd][nsplit] (l_j) |
+        // gte[ncol] | pv[ncol][nsplit] (the splits' accumulators of this CTA's columns) | oc[ncol]
+        float* mv = fs;
+        float* lv = mv + nhd * nsplit;
+        float* gte = lv + nhd * nsplit;
+        float* pv = gte + ncol;
+        float* oc = pv + ncol * nsplit;
+        // everything the combine reads from the other CTAs, in one batch of loads
+        const int n_ml = nhd * nsplit, n_pv = ncol * nsplit, total = 2 * n_ml + ncol + n_pv;
+        for (int base = 0; base < total; base += 8 * kConsumerThreads) {
+          float v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int i = base + tid + k * kConsumerThreads;
+            v[k] = 0.f;
+            if (i < 2 * n_ml) {
+              const int i2 = i < n_ml ? i : i - n_ml;
+              const int hq = hA + i2 / nsplit, j = i2 % nsplit;
+              v[k] = __ldcg(p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (p.D + 2) + p.D + (i < n_ml ? 0 : 1));
+            } else if (i < 2 * n_ml + ncol) {
+              v[k] = p.gated ? __ldcg(p.z + p.Hq * p.D + c0 + (i - 2 * n_ml)) : 0.f;
+            } else if (i < total) {
+              const int i3 = i - 2 * n_ml - ncol, cc = i3 / nsplit, j = i3 % nsplit;
+              const int col = c0 + cc;
+              v[k] = __ldcg(p.part + (static_cast<size_t>(col / p.D) * p.max_splits + j) * (p.D + 2) + col % p.D);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int i = base + tid + k * kConsumerThreads;
+            if (i < 2 * n_ml) mv[i] = v[k];   // mv and lv are contiguous
+            else if (i < 2 * n_ml + ncol) gte[i - 2 * n_ml] = p.gated ? sigmoidf_(v[k]) : 1.0f;
+            else if (i < total) pv[i - 2 * n_ml - ncol] = v[k];
           }
         }
         cons_sync(kConsumerThreads);
-        for (int hh = warp; hh < nhd; hh += kConsumerWarps) {
-          const int hq = hA + hh;
+        for (int hh = warp; hh < nhd; hh += kConsumerWarps) {   // split weights e^{m_j - M} / L per head
           float M = -INFINITY;
-          for (int j = lane; j < nsplit; j += 32) M = fmaxf(M, wts[hh * nsplit + j]);
+          for (int j = lane; j < nsplit; j += 32) M = fmaxf(M, mv[hh * nsplit + j]);
           M = warp_max(M);
           float Ls = 0.f;
-          for (int j = lane; j < nsplit; j += 32)
-            Ls = fmaf(__ldcg(p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (p.D + 2) + p.D + 1),
-                      expf(wts[hh * nsplit + j] - M), Ls);
+          for (int j = lane; j < nsplit; j += 32) Ls = fmaf(lv[hh * nsplit + j], expf(mv[hh * nsplit + j] - M), Ls);
           Ls = warp_sum(Ls);
           __syncwarp();
-          for (int j = lane; j < nsplit; j += 32) wts[hh * nsplit + j] = expf(wts[hh * nsplit + j] - M) / Ls;
+          for (int j = lane; j < nsplit; j += 32) mv[hh * nsplit + j] = expf(mv[hh * nsplit + j] - M) / Ls;
         }
         cons_sync(kConsumerThreads);
-        for (int cc = warp; cc < ncol; cc += kConsumerWarps) {   // warp per column, lanes over splits
-          const int col = c0 + cc;
-          const int hq = col / p.D, d = col % p.D;
-          const float* wrow = wts + (hq - hA) * nsplit;
+        for (int cc = tid; cc < ncol; cc += kConsumerThreads) {   // thread per column
+          const float* wrow = mv + ((c0 + cc) / p.D - hA) * nsplit;
+          const float* prow = pv + cc * nsplit;
           float o = 0.f;
-          for (int j = lane; j < nsplit; j += 32)
-            o = fmaf(__ldcg(p.part + (static_cast<size_t>(hq) * p.max_splits + j) * (p.D + 2) + d), wrow[j], o);
-          o = warp_sum(o);
-          if (lane == 0) oc[cc] = o * gte[cc];
+          for (int j = 0; j < nsplit; ++j) o = fmaf(prow[j], wrow[j], o);
+          oc[cc] = o * gte[cc];
         }
         cons_sync(kConsumerThreads);
         if constexpr (Q4) {
@@ -1670,13 +1662,12 @@ int decode_max_splits(int grid, int hkv) {
 
 template <int HK, bool Q4>
 cudaError_t launch_hk(const DecodeParams& p, int grid, cudaStream_t s) {
-  static bool attr_set = false;   // per process; the attribute is the same on every device
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(mk_decode_kernel<HK, Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemLimit));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};   // per device
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(mk_decode_kernel<HK, Q4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kSmemLimit));
+  });
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);

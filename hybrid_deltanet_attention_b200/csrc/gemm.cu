@@ -362,13 +362,11 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
       !cached_map(&ma_lo, a.x_lo, a.M, a.K, static_cast<long long>(a.K) * 2, kBM) ||
       !cached_map(&mb, a.w, a.N, a.K, a.ldw_bytes, BN))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;   // per process; the attribute is the same on every device
-  if (!attr_set) {
-    const cudaError_t attr =
-        cudaFuncSetAttribute(linear_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
-    if (attr != cudaSuccess) return attr;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};   // per device
+  const cudaError_t attr = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(linear_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmemBytes);
+  });
+  if (attr != cudaSuccess) return attr;
   dim3 grid((a.N + BN - 1) / BN, (a.M + kBM - 1) / kBM);
   // split K when the tile grid leaves most SMs idle (few tokens) and the workspace holds it
   const int tiles = static_cast<int>(grid.x * grid.y), nk = a.K / kBK;

@@ -1,9 +1,27 @@
 // Internal definitions shared by the C-ABI layer (api.cu) and the kernels.
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 namespace mk {
+
+// One-time setup per device (kernel attributes such as the dynamic shared-memory limit
+// are set per device): runs setup() on the current device unless it already succeeded
+// there. done holds one bit per device index below 64 (higher indices run setup every
+// time). Safe to call from several threads: setup may then run twice, which is harmless
+// for idempotent attribute settings.
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<uint64_t>& done, F&& setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = setup();
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // Persistent decode kernel geometry: 8 consumer warps do the math, one producer
 // warp streams this CTA's weights through a ring of shared-memory slots with bulk
@@ -79,8 +97,6 @@ struct DecodeParams {
   // barrier arrival and exit, and at the end: trace[0], trace[2k-1], trace[2k], ...
   unsigned long long* trace;
   int trace_cap;
-  // how far (bytes per CTA) the L2 prefetch cursor runs ahead of the shared-memory fill
-  int prefetch_bytes;
   // Q4_K-style weights: row_bytes is then (H / 256) * 144, and the out- and down-projections
   // are split over output rows (their inputs staged from obuf / abuf)
   int q4;

@@ -93,6 +93,7 @@ int mk_decode_step_noalloc(mk_model* m, const int32_t* d_in_token, int32_t* d_ou
   p.part = rebase(p.part);
   p.obuf = rebase(p.obuf);
   p.abuf = rebase(p.abuf);
+
   p.in_token = d_in_token;
   p.out_token = d_out_token;
   p.logits = d_logits;

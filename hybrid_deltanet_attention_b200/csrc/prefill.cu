@@ -69,14 +69,14 @@ __device__ __forceinline__ void put_split(uint16_t* hi, uint16_t* lo, long long 
 
 // h[t] = E[tok[t]] (bf16 -> fp32). An out-of-range id latches MK_DEVERR_BAD_TOKEN and
 // gives a zero row.
-__global__ void embed_rows(const int32_t* __restrict__ tok, int T, const uint16_t* __restrict__ embed, int H, int V,
-                           float* __restrict__ h, int* err) {
+__global__ void embed_rows(const int32_t* __restrict__ tok, int T, const uint16_t* __restrict__ embed, int lde, int H,
+                           int V, float* __restrict__ h, int* err) {
   const int t = blockIdx.x;
   const int id = tok[t];
   const bool ok = id >= 0 && id < V;
   if (!ok && threadIdx.x == 0) atomicOr(err, MK_DEVERR_BAD_TOKEN);
   for (int i = threadIdx.x; i < H; i += blockDim.x)
-    h[static_cast<long long>(t) * H + i] = ok ? bf16_to_f(embed[static_cast<long long>(id) * H + i]) : 0.f;
+    h[static_cast<long long>(t) * H + i] = ok ? bf16_to_f(embed[static_cast<long long>(id) * lde + i]) : 0.f;
 }
 
 // x[t] = h[t] / sqrt(mean(h[t]^2) + eps) * gamma, written as bf16 high/low parts.
@@ -2124,6 +2124,9 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
     ++m->launches;
   };
   const bool q4 = b.q4 != 0;   // 4-bit weights: their own linear layer (mma.sync over <= 8-token tiles)
+  // bf16 row stride of the decode kernel's [out][H] matrices (rows padded to 2H + 16 bytes);
+  // with 4-bit weights the lambda below turns 2H into the super-block row bytes
+  const long long ldw_dec = q4 ? 2LL * H : static_cast<long long>(b.row_bytes);
   // ldw is the bf16 row stride; 4-bit rows take (K / 256) * 144 bytes plus the same tail
   auto linear = [&](const void* w, long long ldw, int N, int K, float* out, long long ldc, int acc) {
     if (e != cudaSuccess) return;
@@ -2141,7 +2144,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
   if (q4)
     embed_rows_q4<<<T, kPT, 0, s>>>(tok, T, b.embed, b.row_bytes, H, c.vocab, pf.h, b.err);
   else
-    embed_rows<<<T, kPT, 0, s>>>(tok, T, reinterpret_cast<const uint16_t*>(b.embed), H, c.vocab, pf.h, b.err);
+    embed_rows<<<T, kPT, 0, s>>>(tok, T, reinterpret_cast<const uint16_t*>(b.embed), b.row_bytes / 2, H, c.vocab,
+                                  pf.h, b.err);
   chk();
   int di = 0, ai = 0;
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
@@ -2218,7 +2222,7 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
       uint16_t* vc = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(b.vc) +
                                                  static_cast<size_t>(ai) * Hkv * c.max_ctx * b.kv_rb);
       ++ai;
-      linear(L.w_in, 2LL * H, rows, H, pf.z, rows, 0);
+      linear(L.w_in, ldw_dec, rows, H, pf.z, rows, 0);
       at_prep<<<T, kPT, b.kv_q8 ? 2 * static_cast<size_t>(Hkv) * D * sizeof(float) : 0, s>>>(
           pf.z, rows, b.pos, off, b.inv_freq, Hq, Hkv, D, c.at_out_gate, kc, vc, c.max_ctx, pf.y, qd, b.kv_rb, b.kv_q8);
       chk();
@@ -2299,8 +2303,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         ++m->launches;
       }
     } else {
-      linear(L.w_gate, 2LL * H, F, H, pf.z, 2LL * F, 0);
-      linear(L.w_up, 2LL * H, F, H, pf.z + F, 2LL * F, 0);
+      linear(L.w_gate, ldw_dec, F, H, pf.z, 2LL * F, 0);
+      linear(L.w_up, ldw_dec, F, H, pf.z + F, 2LL * F, 0);
       act_split<<<dim3(T, (F + 1023) / 1024), kPT, 0, s>>>(pf.z, F, pf.xhi, pf.xlo);
       chk();
       linear(q4 ? L.w_down_q4 : PL.w_down, 2LL * F, H, F, pf.h, H, 1);
@@ -2312,30 +2316,30 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
 }  // namespace
 
 cudaError_t set_prefill_smem_limits() {
-  static bool done = false;   // per process; the attributes are the same on every device
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(wy_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(dn_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(bf16_linear_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(4 * kBfDepth * 32 * 128));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(q4_linear_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(4 * kQ4Depth * 32 * 144));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(wy_state_tc<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(wy_tc_smem<128>()));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(wy_state_tc<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(wy_tc_smem<64>()));
-  if (e == cudaSuccess) done = true;
-  return e;
+  static std::atomic<uint64_t> done{0};   // per device
+  return once_per_device(done, [] {
+    cudaError_t e = cudaFuncSetAttribute(wy_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(dn_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_prep_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(wy_state_fast<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bf16_linear_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(4 * kBfDepth * 32 * 128));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(q4_linear_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(4 * kQ4Depth * 32 * 144));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wy_state_tc<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(wy_tc_smem<128>()));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wy_state_tc<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(wy_tc_smem<64>()));
+    return e;
+  });
 }
 
 size_t prefill_smem_need(int dk, int dv, int grp, int D, int C) {
@@ -2400,11 +2404,11 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
                              m->pf.splitk, mk::kSplitKFloats, s);
     ++m->launches;
   } else if (e == cudaSuccess && T <= 8) {   // bf16 tied LM head, few tokens
-    e = mk::launch_bf16_linear(m->pf.xhi, m->pf.xlo, b.embed, 2LL * c.hidden, logits, c.vocab, T, c.vocab, c.hidden, 0,
+    e = mk::launch_bf16_linear(m->pf.xhi, m->pf.xlo, b.embed, b.row_bytes, logits, c.vocab, T, c.vocab, c.hidden, 0,
                                m->pf.splitk, mk::kSplitKFloats, s);
     ++m->launches;
   } else if (e == cudaSuccess) {
-    mk::LinearArgs a{m->pf.xhi, m->pf.xlo, b.embed, 2LL * c.hidden, logits, c.vocab, T, c.vocab, c.hidden, 0, b.err};
+    mk::LinearArgs a{m->pf.xhi, m->pf.xlo, b.embed, b.row_bytes, logits, c.vocab, T, c.vocab, c.hidden, 0, b.err};
     e = mk::launch_linear(a, s);
     ++m->launches;
   }
