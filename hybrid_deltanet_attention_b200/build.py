@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["api.cu", "decode.cu", "noalloc.cu", "gemm.cu", "prefill.cu"]
+SOURCES = ["api.cu", "decode.cu", "noalloc.cu", "gemm.cu", "prefill.cu", "attn.cu"]
 HEADERS = ["mk_internal.h", "mk_model.h", "dev.cuh", "tc.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

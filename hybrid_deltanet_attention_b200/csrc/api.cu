@@ -264,7 +264,7 @@ struct Layout {
   int pf_rows;
   size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec, pf_apart, pf_splitk, pf_best;
   size_t pf_kvd = 0;
-  size_t pf_sbuf, pf_phi, pf_plo, pf_vt, pf_img = 0;
+  size_t pf_vt = 0, pf_img = 0;
   long long pf_nk;
   // batched verify saves
   int vf_rows;
@@ -400,13 +400,11 @@ Layout make_layout(const mk_config& c, int grid) {
       const size_t img = 2ull * (c.dn_dk / 64) * 16384 + 16384 + 32768;     // operand images per (chunk, head)
       L.pf_img = off; off = align256(off + nch * c.dn_heads * img);
     }
-    L.pf_nk = na ? std::min<long long>(8192, (static_cast<long long>(c.max_ctx) + 63) / 64 * 64) : 0;
+    // V^T of every kv head of one attention layer for the flash attention: [Hkv][D][nk]
+    L.pf_nk = (na && mk::attn_flash_supported(c.at_head_dim)) ? (static_cast<long long>(c.max_ctx) + 63) / 64 * 64 : 0;
     if (L.pf_nk > 0) {
-      const size_t nk = static_cast<size_t>(L.pf_nk);
-      L.pf_sbuf = off; off = align256(off + T * nk * 4);
-      L.pf_phi = off; off = align256(off + T * nk * 2);
-      L.pf_plo = off; off = align256(off + T * nk * 2);
-      L.pf_vt = off; off = align256(off + static_cast<size_t>(c.at_head_dim) * nk * 2);
+      L.pf_vt = off;
+      off = align256(off + static_cast<size_t>(c.at_kv_heads) * c.at_head_dim * static_cast<size_t>(L.pf_nk) * 2);
     }
     if (na && c.kv_format == MK_KV_Q8) {   // one layer's K and V read back as bf16 for the attention kernels
       L.pf_kvd = off;
@@ -776,9 +774,6 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     m->pf.kvd = L.pf_kvd ? reinterpret_cast<uint16_t*>(W + L.pf_kvd) : nullptr;
     if (L.pf_img) m->pf.img = W + L.pf_img;
     if (L.pf_nk > 0) {
-      m->pf.sbuf = reinterpret_cast<float*>(W + L.pf_sbuf);
-      m->pf.phi = reinterpret_cast<uint16_t*>(W + L.pf_phi);
-      m->pf.plo = reinterpret_cast<uint16_t*>(W + L.pf_plo);
       m->pf.vt = reinterpret_cast<uint16_t*>(W + L.pf_vt);
     }
   }

@@ -394,6 +394,11 @@ cudaError_t launch_bn(const LinearArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+bool tensor_map_bf16(CUtensorMap* map, const void* base, long long rows, long long cols, long long stride_bytes,
+                     int box_rows) {
+  return cached_map(map, base, rows, cols, stride_bytes, box_rows);
+}
+
 cudaError_t launch_split_bf16(const float* x, long long ldx, uint16_t* hi, uint16_t* lo, int M, int K,
                               cudaStream_t s) {
   const long long total = static_cast<long long>(M) * K;

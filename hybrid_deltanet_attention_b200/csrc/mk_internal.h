@@ -2,6 +2,7 @@
 #pragma once
 #include <atomic>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace mk {
@@ -140,6 +141,15 @@ struct LinearArgs {
   uint16_t* act_lo = nullptr;
 };
 cudaError_t launch_split_bf16(const float* x, long long ldx, uint16_t* hi, uint16_t* lo, int M, int K, cudaStream_t s);
+// 2-D tensor map of a bf16 row-major [rows][cols] matrix (row stride stride_bytes), box of 64
+// columns x box_rows rows, 128-byte swizzle; cached per (base, shape, box).
+bool tensor_map_bf16(CUtensorMap* map, const void* base, long long rows, long long cols, long long stride_bytes,
+                     int box_rows);
+// flash-style causal prefill attention on the tensor cores (attn.cu)
+bool attn_flash_supported(int D);
+cudaError_t launch_attn_flash(const uint16_t* q_hi, const uint16_t* q_lo, const uint16_t* k, const uint16_t* vt,
+                              const int* posp, int off, int T, int Hq, int Hkv, int D, int max_ctx, long long nk,
+                              float* out, long long ldo, int* err, cudaStream_t s);
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s);
 
 // repack helpers (api.cu launches them)

@@ -28,12 +28,9 @@ struct mk_prefill_ws {
   float* apart = nullptr;    // [min(rows, kAttnSplitRows)][Hq][kAttnMaxSplit][D + 2] attention key-split partials
   float* splitk = nullptr;   // [kSplitKFloats] split-K partials of the linear layers
   unsigned long long* best = nullptr;   // [rows] packed (value, index) row maxima of the verify logits
-  // attention as two GEMMs: scores [rows][nk_max] fp32, probabilities as bf16 high/low
-  // parts [rows][nk_max], V^T [D][nk_max]
+  // flash attention on the tensor cores: V^T of one layer's kv heads [Hkv][D][nk_max]
+  // (nk_max = max_ctx rounded up to 64; 0 when the head dim has no flash kernel)
   long long nk_max = 0;
-  float* sbuf = nullptr;
-  uint16_t* phi = nullptr;
-  uint16_t* plo = nullptr;
   uint16_t* vt = nullptr;
   // chunked delta rule on the tensor cores: bf16 operand images [chunks][Hd][bytes per image]
   uint8_t* img = nullptr;

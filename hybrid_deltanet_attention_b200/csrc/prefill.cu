@@ -1562,45 +1562,6 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return warp_max(t);
 }
 
-__global__ void __launch_bounds__(256) attn_softmax_split(const float* __restrict__ S, int nk,
-                                                          const int* __restrict__ posp, int off,
-                                                          uint16_t* __restrict__ phi, uint16_t* __restrict__ plo) {
-  extern __shared__ float4 srow4[];   // [nk / 4] the row's scores, then e^{s - max}
-  __shared__ float red[32];
-  const int t = blockIdx.x;
-  const int last = min(*posp + off + t, nk - 1);   // keys 0 .. last
-  const int n4 = (last + 4) >> 2;                  // float4 groups holding keys 0 .. last
-  const float4* r4 = reinterpret_cast<const float4*>(S + static_cast<long long>(t) * nk);   // nk % 4 == 0
-  float mx = -INFINITY;
-  for (int i = threadIdx.x; i < n4; i += blockDim.x) {   // one read of the row
-    float4 v = r4[i];
-    const int j = 4 * i;
-    if (j + 1 > last) v.y = -INFINITY;
-    if (j + 2 > last) v.z = -INFINITY;
-    if (j + 3 > last) v.w = -INFINITY;
-    srow4[i] = v;
-    mx = fmaxf(fmaxf(mx, fmaxf(v.x, v.y)), fmaxf(v.z, v.w));
-  }
-  mx = block_max(mx, red);   // its barriers also publish srow
-  float sum = 0.f;
-  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-    float4 v = srow4[i];
-    v = make_float4(expf(v.x - mx), expf(v.y - mx), expf(v.z - mx), expf(v.w - mx));
-    srow4[i] = v;   // each thread rewrites only its own groups
-    sum += (v.x + v.y) + (v.z + v.w);
-  }
-  sum = block_sum(sum, red);
-  const float inv = 1.0f / sum;
-  for (int i = threadIdx.x; i < nk / 4; i += blockDim.x) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < n4) {
-      v = srow4[i];
-      v.x *= inv; v.y *= inv; v.z *= inv; v.w *= inv;
-    }
-    put_split4(phi, plo, static_cast<long long>(t) * nk + 4 * i, v);
-  }
-}
-
 // VT[d][j] = V[j][d] for the keys up to the pass's last position, zero past it.
 __global__ void v_transpose(const uint16_t* __restrict__ vg, int D, int nk, const int* __restrict__ posp, int last_off,
                             int max_ctx, uint16_t* __restrict__ vt) {
@@ -1623,7 +1584,7 @@ __global__ void v_transpose(const uint16_t* __restrict__ vg, int D, int nk, cons
 // cached positions 0 .. pos0+t in blocks of 64 keys with an online softmax.
 constexpr int kKeyBlock = 64;
 constexpr int kMaxDraftRows = 17;   // max_draft <= 16
-constexpr int kGemmAttnMinRows = 64;   // prompts from this many tokens run attention as two GEMMs
+constexpr int kFlashAttnMinRows = 64;   // prompts from this many tokens run the flash attention
 
 // With nsplit > 1 (few tokens: T * Hkv CTAs would leave most SMs idle) CTA z takes the
 // z-th of nsplit equal ranges of the token's keys and writes its unnormalised partial
@@ -2236,34 +2197,23 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         kc = pf.kvd;
         vc = pf.kvd + static_cast<size_t>(Hkv) * c.max_ctx * D;
       }
-      if (T >= kGemmAttnMinRows && pf.sbuf && nk_gemm <= pf.nk_max) {
+      if (T >= kFlashAttnMinRows && pf.vt && nk_gemm <= pf.nk_max) {
+        // flash attention on the tensor cores: V^T of every kv head, the queries of every
+        // head as bf16 high / low parts, then one launch over (query tile, head)
         const int nk = static_cast<int>(nk_gemm);
-        const int grp = Hq / Hkv;
         for (int g = 0; g < Hkv && e == cudaSuccess; ++g) {
           v_transpose<<<dim3(nk / 32, (D + 31) / 32), dim3(32, 8), 0, s>>>(
-              vc + static_cast<size_t>(g) * c.max_ctx * D, D, nk, b.pos, off + T - 1, c.max_ctx, pf.vt);
+              vc + static_cast<size_t>(g) * c.max_ctx * D, D, nk, b.pos, off + T - 1, c.max_ctx,
+              pf.vt + static_cast<size_t>(g) * D * nk);
           chk();
-          for (int u = 0; u < grp && e == cudaSuccess; ++u) {
-            const int hq = g * grp + u;
-            e = launch_split_bf16(pf.y + static_cast<size_t>(hq) * D, qd, pf.xhi, pf.xlo, T, D, s);
-            ++m->launches;
-            if (e == cudaSuccess) {   // S = Q K^T over the cached keys (rows past max_ctx read as zero)
-              LinearArgs a{pf.xhi, pf.xlo, kc + static_cast<size_t>(g) * c.max_ctx * D, 2LL * D, pf.sbuf, nk, T,
-                           std::min(nk, c.max_ctx), D, 0, b.err, pf.splitk, kSplitKFloats};
-              e = launch_linear(a, s);
-              ++m->launches;
-            }
-            if (e != cudaSuccess) break;
-            attn_softmax_split<<<T, kPT, static_cast<size_t>(nk) * sizeof(float), s>>>(pf.sbuf, nk, b.pos, off,
-                                                                                       pf.phi, pf.plo);
-            chk();
-            if (e == cudaSuccess) {   // O = P V
-              LinearArgs a{pf.phi, pf.plo, pf.vt, 2LL * nk, pf.o + static_cast<size_t>(hq) * D, qd, T, D, nk, 0, b.err,
-                           pf.splitk, kSplitKFloats};
-              e = launch_linear(a, s);
-              ++m->launches;
-            }
-          }
+        }
+        if (e == cudaSuccess) {
+          e = launch_split_bf16(pf.y, qd, pf.xhi, pf.xlo, T, qd, s);
+          ++m->launches;
+        }
+        if (e == cudaSuccess) {
+          e = launch_attn_flash(pf.xhi, pf.xlo, kc, pf.vt, b.pos, off, T, Hq, Hkv, D, c.max_ctx, nk, pf.o, qd, b.err, s);
+          ++m->launches;
         }
       } else {
         // key splits when T * Hkv CTAs would leave most of the GPU idle (verify passes, short prompts)
