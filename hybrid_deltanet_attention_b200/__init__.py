@@ -5,4 +5,4 @@ Python binding. There is no CPU fallback.
 """
 from ._abi import (MK_DEVERR_BAD_TOKEN, MK_DEVERR_BARRIER_TIMEOUT, MK_DEVERR_CAPACITY,  # noqa: F401
                    MK_DEVERR_PIPE_TIMEOUT, MkError, load_library)
-from .model import Model, make_config, weights_to_device  # noqa: F401
+from .model import Model, make_config, query_sizes, weights_to_device  # noqa: F401

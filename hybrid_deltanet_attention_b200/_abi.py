@@ -89,6 +89,7 @@ class MkSizes(C.Structure):
         ("off_err", C.c_uint64),
         ("grid_ctas", C.c_int32),
         ("kv_row_bytes", C.c_int32),
+        ("layer_table_entries", C.c_int32),
     ]
 
 

@@ -424,6 +424,7 @@ Layout make_layout(const mk_config& c, int grid) {
   }
   L.sz.workspace_bytes = off;
   L.sz.grid_ctas = grid;
+  L.sz.layer_table_entries = layer_table_fits(c, grid) ? c.n_layers : 2;
   return L;
 }
 

@@ -43,6 +43,15 @@ def make_config(cfg, max_ctx: int, max_draft: int = 0, kv_format: int = 0) -> Mk
     return c
 
 
+def query_sizes(cfg, max_ctx: int, max_draft: int = 0, kv_format: int = 0) -> MkSizes:
+    """mk_query_sizes for a model shape on the current CUDA device: buffer sizes, state
+    offsets, the decode grid and the decode kernel's layer-table form."""
+    sizes = MkSizes()
+    check(_abi.load_library().mk_query_sizes(C.byref(make_config(cfg, max_ctx, max_draft, kv_format)),
+                                             C.byref(sizes)))
+    return sizes
+
+
 def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream

@@ -158,6 +158,9 @@ typedef struct mk_sizes {
   uint64_t off_S, off_conv, off_k, off_v, off_pos, off_err;
   int32_t  grid_ctas;      /* persistent CTAs the decode kernel will use on the current device */
   int32_t  kv_row_bytes;   /* bytes per (layer, kv head, position) row of the KV cache */
+  int32_t  layer_table_entries;  /* layer-table entries the decode kernel keeps in shared memory:
+                                    n_layers when the whole table fits beside its scratch, else 2
+                                    (each layer's entry is then fetched during the layer before) */
 } mk_sizes;
 
 typedef struct mk_model mk_model;   /* opaque host-side handle */

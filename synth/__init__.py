@@ -133,7 +133,22 @@ QWEN_27B_4L = dataclasses.replace(QWEN_27B, name="27b-4l", n_layers=4, pattern="
 # (1.7 B weights), and it runs the hidden-5120 decode instance the 27B model runs.
 QWEN_27B_4L_32K = dataclasses.replace(QWEN_27B, name="27b-4l-32k", n_layers=4, pattern="DDDA", vocab=32768)
 
-CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI, TINY_Q4, MID_Q4, QWEN_27B_4L, QWEN_27B_4L_32K)}
+# Two models whose decode scratch leaves no room for the whole layer table, so the decode
+# kernel keeps two table slots and fetches each layer's entry during the layer before (as
+# the 64-layer 27B model does): eight query heads of 256 per KV head need 5656 floats of
+# attention scratch per CTA, and the bf16 hidden size of 2880, or the 4-bit FFN of 16640
+# (staged whole by the down-projection), takes the room that eight table entries would need.
+WIDE_GQA8 = _preset("wide-gqa8", n_layers=8, pattern="DDDA" * 2, hidden=2880, vocab=4096, rms_eps=1e-6,
+                    dn_heads=4, dn_dk=128, dn_dv=128, conv_width=4,
+                    at_q_heads=8, at_kv_heads=1, at_head_dim=256, rope_theta=1e7, at_out_gate=1,
+                    ffn=1024, seed=12)
+WIDE_GQA8_Q4 = _preset("wide-gqa8-q4", n_layers=8, pattern="DDDA" * 2, hidden=256, vocab=4096, rms_eps=1e-6,
+                       dn_heads=4, dn_dk=128, dn_dv=128, conv_width=4,
+                       at_q_heads=8, at_kv_heads=1, at_head_dim=256, rope_theta=1e7, at_out_gate=1,
+                       ffn=16640, weight_format=W_Q4K, seed=13)
+
+CONFIGS = {c.name: c for c in (TINY, QWEN_08B, QWEN_27B, MINI, TINY_Q4, MID_Q4, QWEN_27B_4L, QWEN_27B_4L_32K,
+                               WIDE_GQA8, WIDE_GQA8_Q4)}
 
 
 def with_changes(cfg: ModelConfig, **kw) -> ModelConfig:
