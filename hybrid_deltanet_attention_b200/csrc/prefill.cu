@@ -204,10 +204,13 @@ __global__ void __launch_bounds__(128, 5) q4_linear_mma(const uint16_t* __restri
     // my rows: rr = 0..3 -> row 16 (rr >> 1) + 8 (rr & 1) + g of the warp's 32
     const uint8_t* rb[4];
     uint4 hd[4];
+    float dsc[4], dmn[4];   // the super-block's fp16 d and dmin of my 4 rows, once per super-block
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr) {
       rb[rr] = slot + ((rr >> 1) * 16 + (rr & 1) * 8 + g) * 144;
       hd[rr] = *reinterpret_cast<const uint4*>(rb[rr]);
+      dsc[rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd[rr].x & 0xFFFFu)));
+      dmn[rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd[rr].x >> 16)));
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -239,15 +242,16 @@ __global__ void __launch_bounds__(128, 5) q4_linear_mma(const uint16_t* __restri
         mma_bf16_16816(dx, ones, ones, ones, ones, bh0, bh1);
         mma_bf16_16816(dx, ones, ones, ones, ones, bl0, bl1);
       }
-      // scales of sub-block j for my 4 rows, then acc += s (D - 128 X) - mn X
+      // scales of sub-block j for my 4 rows, then acc += s (D - 128 X) - mn X; the 6-bit
+      // fields become floats through the exponent field (2^23 + v is exact), not a conversion
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
         const uint64_t lo = static_cast<uint64_t>(hd[rr].y) | (static_cast<uint64_t>(hd[rr].z) << 32);
         const uint64_t hi = static_cast<uint64_t>(hd[rr].z) | (static_cast<uint64_t>(hd[rr].w) << 32);
-        const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(hd[rr].x & 0xFFFFu))) *
-                        static_cast<float>(static_cast<uint32_t>(lo >> (6 * j)) & 63u);
-        const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(hd[rr].x >> 16))) *
-                         static_cast<float>(static_cast<uint32_t>(hi >> (16 + 6 * j)) & 63u);
+        const uint32_t scb = static_cast<uint32_t>(lo >> (6 * j)) & 63u;
+        const uint32_t mmb = static_cast<uint32_t>(hi >> (16 + 6 * j)) & 63u;
+        const float s = dsc[rr] * (__uint_as_float(0x4B000000u | scb) - 8388608.0f);
+        const float mn = dmn[rr] * (__uint_as_float(0x4B000000u | mmb) - 8388608.0f);
         const int gr = rr >> 1, i0 = 2 * (rr & 1);   // D rows g (i 0, 1) or g + 8 (i 2, 3); tokens 2c, 2c + 1
         const float cx = -(128.f * s + mn);
         acc[gr][i0] = fmaf(s, dq[gr][i0], fmaf(cx, dx[0], acc[gr][i0]));
@@ -1289,6 +1293,386 @@ struct WyTcBars {
 };
 constexpr uint64_t kWyWaitNs = 1000000000ull;
 
+// Chunk-local part of the chunked delta rule with its three contractions on the tensor cores
+// (one CTA of 128 threads per (chunk, head); writes what wy_prep_fast writes for the
+// tensor-core state pass: U, gamma, the decay factors and the operand images A1, P, K^T).
+//   (1) [K; Q] K^T  (M = 128 rows: the chunk's keys, then its queries; N = 64 keys; K = dk)
+//       gives k_r.k_s and q_r.k_s in TMEM; A = strictly-lower(b_r e^{g_r-g_s} k_r.k_s) and
+//       P = lower(e^{g_r-g_s} q_r.k_s) are formed from them in registers.
+//   (2) T = (I + A)^-1 by forward substitution on the CUDA cores (one column per thread, 64
+//       columns: a quarter of the work of substituting all dv + dk right-hand sides).
+//   (3) U^T = (diag(b) V)^T T^T and W^T = (diag(b gamma) K)^T T^T (M = 128 feature rows, N = 64
+//       tokens, K = 64 tokens), i.e. [U | W] = T [diag(b) V | diag(b gamma) K].
+// Every product takes bf16 high and low parts (hi.hi + hi.lo + lo.hi, fp32 accumulation),
+// which keeps about 16 bits of each operand. Shared memory (~98 KB, two CTAs per SM): the
+// [K; Q] image (64 KB; once (1) has consumed it, it holds the columns of T, then the V and K
+// images of step 3, then the W rows of the A1 image on their way out) and a
+// 33 KB region that first stages the fp32 key rows, then the query rows (one bulk round trip
+// each), and then holds the T image and A.
+struct WyPrepTcLayout {
+  static constexpr uint32_t kImg = 0;                    // [K;Q] image | later V and K images, 64 KB
+  static constexpr uint32_t kStage = 65536;              // fp32 rows [64][128] | later T image + A
+  static constexpr uint32_t kT = kStage;                 // T image: [hi, lo][64 rows][128 B]
+  static constexpr uint32_t kA = kStage + 16384;         // fp32 A [64][68]
+  static constexpr uint32_t kG = kA + 64 * 68 * 4;       // g, b, gamma = e^g, b gamma: [64] each
+  static constexpr uint32_t kBar = kG + 4 * 64 * 4;      // mbarrier, TMEM base, abort flag
+  static constexpr uint32_t kBytes = kBar + 32;
+};
+static_assert(WyPrepTcLayout::kG - WyPrepTcLayout::kStage >= 64 * 128 * 4, "the staging region holds 64 fp32 rows");
+constexpr size_t kWyPrepTcSmem = WyPrepTcLayout::kBytes + 1024;   // + alignment slack
+
+// bf16 high / low parts of v, written at (row, k) of a K-major 128-byte-swizzled tile pair
+// (the low part tile `lo_off` bytes after the high part).
+__device__ __forceinline__ void put_bf16_pair(uint8_t* tile, uint32_t lo_off, uint32_t row, uint32_t k, float v) {
+  const uint16_t hi = f_to_bf16(v);
+  const uint32_t off = tc::sw128_offset(row, k);
+  *reinterpret_cast<uint16_t*>(tile + off) = hi;
+  *reinterpret_cast<uint16_t*>(tile + lo_off + off) = f_to_bf16(v - bf16_to_f(hi));
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(128, 2) wy_prep_tc(WyBufs b) {
+  static_assert(DK == DV && (DK == 64 || DK == 128), "dk = dv = 64 or 128");
+  using Lyt = WyPrepTcLayout;
+  using I = WyImg<DK>;
+  constexpr int KB = DK / 64, AP = kChunk + 4;
+  extern __shared__ uint8_t wyp_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(wyp_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* KQ = sm + Lyt::kImg;     // [hi: KB blocks][lo: KB blocks] of 128 rows x 128 B
+  uint8_t* VI = sm + Lyt::kImg;     // step 3: diag(b) V image [hi][lo] of 128 rows x 128 B (K = tokens)
+  uint8_t* KI = VI + 32768;         //         diag(b gamma) K image, same shape
+  float* stg = reinterpret_cast<float*>(sm + Lyt::kStage);   // [64][DK] fp32 rows
+  uint8_t* TI = sm + Lyt::kT;       // T image [hi][lo] of 64 rows x 128 B (K = tokens)
+  float* A = reinterpret_cast<float*>(sm + Lyt::kA);
+  float* g = reinterpret_cast<float*>(sm + Lyt::kG);
+  float* bb = g + kChunk;
+  float* gm = bb + kChunk;    // gamma_r = e^{g_r}
+  float* bgm = gm + kChunk;   // b_r gamma_r
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + Lyt::kBar);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Lyt::kBar + 8);
+  volatile int* abort = reinterpret_cast<volatile int*>(sm + Lyt::kBar + 12);
+  const int Hd = b.Hd, tid = threadIdx.x, warp = tid >> 5;
+  const int ch = blockIdx.x, h = blockIdx.y;
+  const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
+  const int qo = h * DK, ko = Hd * DK + h * DK, vo = 2 * Hd * DK + h * DV;
+  const int C = 2 * Hd * DK + Hd * DV;
+  uint8_t* img = b.img + (static_cast<size_t>(ch) * Hd + h) * I::kBytes;
+  uint8_t* a1 = img;
+  uint8_t* pimg = img + I::kA1;
+  uint8_t* kt = pimg + I::kP;
+  // fp32 rows [64][DK] of the chunk at column offset `col` of y into the staging region (rows
+  // past the prompt read as zero)
+  auto stage_rows = [&](int col) {
+    for (int idx = tid; idx < kChunk * DK / 4; idx += 128) {
+      const int r = idx / (DK / 4), j4 = idx % (DK / 4);
+      const float* yr = b.y + static_cast<long long>(t0 + min(r, n - 1)) * b.ldy + col + 4 * j4;
+      cp_async16(stg + r * DK + 4 * j4, yr, r < n ? 16u : 0u);
+    }
+  };
+
+  stage_rows(ko);
+  {   // gates of the chunk
+    const int r = tid & (kChunk - 1);
+    const float* yr = b.y + static_cast<long long>(t0 + min(r, n - 1)) * b.ldy;
+    if (tid < kChunk) cp_async4(g + r, yr + C + h, r < n ? 4u : 0u);
+    else cp_async4(bb + r, yr + C + Hd + h, r < n ? 4u : 0u);
+  }
+  cp_async_commit();
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(tslot, 256);
+    tc::tmem_relinquish();
+  }
+  cp_async_wait<0>();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tslot;
+  const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+  if (tid < 32) {   // inclusive prefix sum of log a over the chunk (two values per lane)
+    float v0 = g[2 * tid], v1 = g[2 * tid + 1];
+    v1 += v0;
+    float run = v1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float x = __shfl_up_sync(0xffffffffu, run, o);
+      if (tid >= o) run += x;
+    }
+    const float before = run - v1;
+    g[2 * tid] = before + v0;
+    g[2 * tid + 1] = run;
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = 2 * tid + u;
+      gm[r] = expf(g[r]);
+      bgm[r] = bb[r] * gm[r];
+    }
+  }
+  // ---- key rows: rows 0..63 of the [K; Q] image, and the K^T image (row j: k_r[j] over the
+  // chunk's r; rows j >= dk zero, global)
+  for (int idx = tid; idx < kChunk * (DK / 8); idx += 128) {
+    const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
+    uint4 hv, lv;
+    split8_bf16(stg + r * DK + 8 * c8, hv, lv);
+    const uint32_t off = static_cast<uint32_t>(r) * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4);
+    *reinterpret_cast<uint4*>(KQ + kb * 16384 + off) = hv;
+    *reinterpret_cast<uint4*>(KQ + (KB + kb) * 16384 + off) = lv;
+  }
+  {
+    const int j = tid;
+#pragma unroll 2
+    for (int c = 0; c < 8; ++c) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = j < DK ? stg[(8 * c + u) * DK + j] : 0.f;
+      uint4 hv, lv;
+      split8_bf16(v, hv, lv);
+      const uint32_t off = static_cast<uint32_t>(j) * 128u + ((static_cast<uint32_t>(c) ^ (j & 7u)) << 4);
+      *reinterpret_cast<uint4*>(kt + off) = hv;
+      *reinterpret_cast<uint4*>(kt + 16384 + off) = lv;
+    }
+  }
+  __syncthreads();   // the staging region is free; gamma is published
+  // ---- query rows: rows 64..127 of the [K; Q] image and the gamma Q rows of the A1 image
+  stage_rows(qo);
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  for (int idx = tid; idx < kChunk * (DK / 8); idx += 128) {
+    const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
+    const int row = kChunk + r;
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = stg[r * DK + 8 * c8 + u];
+    uint4 hv, lv;
+    split8_bf16(v, hv, lv);
+    const uint32_t off = static_cast<uint32_t>(row) * 128u + ((static_cast<uint32_t>(c) ^ (row & 7u)) << 4);
+    *reinterpret_cast<uint4*>(KQ + kb * 16384 + off) = hv;
+    *reinterpret_cast<uint4*>(KQ + (KB + kb) * 16384 + off) = lv;
+    const float gr = gm[r];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] *= gr;
+    split8_bf16(v, hv, lv);
+    const uint32_t offq = static_cast<uint32_t>(r) * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4);
+    *reinterpret_cast<uint4*>(a1 + kb * 16384 + offq) = hv;
+    *reinterpret_cast<uint4*>(a1 + (KB + kb) * 16384 + offq) = lv;
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  // ---- (1) D_A = [K; Q] K^T  (TMEM columns 0..63)
+  if (tid == 0) {
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(128, 64);
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t dh = tc::desc_kmajor_sw128(KQ + kb * 16384 + kk * 32);
+        const uint64_t dl = tc::desc_kmajor_sw128(KQ + (KB + kb) * 16384 + kk * 32);
+        tc::mma_bf16(tbase, dh, dh, idesc, (kb | kk) ? 1u : 0u);
+        tc::mma_bf16(tbase, dh, dl, idesc, 1u);
+        tc::mma_bf16(tbase, dl, dh, idesc, 1u);
+      }
+    tc::mma_commit(bar);
+  }
+  if (tid < n) {
+    b.gam[static_cast<long long>(t0 + tid) * Hd + h] = gm[tid];
+    b.dec[static_cast<long long>(t0 + tid) * Hd + h] = expf(g[n - 1] - g[tid]);
+  }
+  if (!mbar_wait(bar, 0, abort, kWyWaitNs)) {
+    if (!*abort) atomicOr(b.err, MK_DEVERR_PIPE_TIMEOUT);
+    *abort = 1;
+  }
+  tc::fence_after_sync();
+  // ---- A (lanes 0..63) into shared memory, P (lanes 64..127) as the P image (global)
+  {
+    const int r = tid & (kChunk - 1);
+    const bool isq = tid >= kChunk;
+    const float gr = g[r], br = bb[r];
+    const bool live = r < n;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float d[16];
+      tc::tmem_ld16(tbase + lane_off + 16 * q, d);
+      if (!isq) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int s = 16 * q + u;
+          A[r * AP + s] = (s < r && live) ? br * expf(gr - g[s]) * d[u] : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int s = 16 * q + u;
+          d[u] = (s <= r && live) ? expf(gr - g[s]) * d[u] : 0.f;
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint4 hv, lv;
+          split8_bf16(d + 8 * hh, hv, lv);
+          const uint32_t c = 2 * q + hh;
+          const uint32_t off = static_cast<uint32_t>(r) * 128u + ((c ^ (r & 7u)) << 4);
+          *reinterpret_cast<uint4*>(pimg + off) = hv;
+          *reinterpret_cast<uint4*>(pimg + 8192 + off) = lv;
+        }
+      }
+    }
+  }
+  __syncthreads();   // A complete; the [K; Q] image has been consumed
+  if (*abort) {
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, 256);
+    return;
+  }
+  // ---- (2) T = (I + A)^-1, one column per thread (threads 0..63), by blocks of 16 rows:
+  // x_B = (e_j)_B - sum_{C < B} A_{BC} x_C, then the unit-lower 16 x 16 diagonal block. The
+  // columns are kept in shared memory (the [K; Q] image is consumed), so the loop over the
+  // earlier blocks stays a loop and the code stays small.
+  float* X = reinterpret_cast<float*>(sm + Lyt::kImg);   // [64 rows][64 columns] fp32
+  if (tid < kChunk) {
+    const int j = tid;
+#pragma unroll 1
+    for (int bk = 0; bk < kChunk / 16; ++bk) {
+      float xb[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xb[i] = (16 * bk + i == j) ? 1.f : 0.f;
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4 * bk; ++c4) {   // columns s = 4 c4 .. 4 c4 + 3 of the earlier blocks
+        const float x0 = X[(4 * c4 + 0) * kChunk + j], x1 = X[(4 * c4 + 1) * kChunk + j];
+        const float x2 = X[(4 * c4 + 2) * kChunk + j], x3 = X[(4 * c4 + 3) * kChunk + j];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 a4 = *reinterpret_cast<const float4*>(A + (16 * bk + i) * AP + 4 * c4);
+          xb[i] = fmaf(-a4.x, x0, xb[i]);
+          xb[i] = fmaf(-a4.y, x1, xb[i]);
+          xb[i] = fmaf(-a4.z, x2, xb[i]);
+          xb[i] = fmaf(-a4.w, x3, xb[i]);
+        }
+      }
+      const float* Ad = A + (16 * bk) * AP + 16 * bk;
+#pragma unroll
+      for (int i = 1; i < 16; ++i)
+#pragma unroll
+        for (int s2 = 0; s2 < i; ++s2) xb[i] = fmaf(-Ad[i * AP + s2], xb[s2], xb[i]);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) X[(16 * bk + i) * kChunk + j] = xb[i];
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < kChunk * 8; idx += 128) {   // T image (row r, K = column) from X
+    const int r = idx >> 3, c = idx & 7;
+    uint4 hv, lv;
+    split8_bf16(X + r * kChunk + 8 * c, hv, lv);
+    const uint32_t off = static_cast<uint32_t>(r) * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4);
+    *reinterpret_cast<uint4*>(TI + off) = hv;
+    *reinterpret_cast<uint4*>(TI + 8192 + off) = lv;
+  }
+  __syncthreads();   // X is consumed: the V and K images take its place
+  {   // the diag(b) V and diag(b gamma) K images (row = feature, K = token): thread = feature row
+    const int f = tid;
+#pragma unroll 1
+    for (int part = 0; part < 2; ++part) {
+      const bool isk = part == 1;
+      uint8_t* dst = isk ? KI : VI;
+      const float* scale = isk ? bgm : bb;
+      const bool rowlive = f < DK;
+      float v[kChunk];   // the whole row in flight at once
+#pragma unroll
+      for (int r = 0; r < kChunk; ++r)
+        v[r] = (rowlive && r < n) ? b.y[static_cast<long long>(t0 + r) * b.ldy + (isk ? ko : vo) + f] : 0.f;
+#pragma unroll
+      for (int r = 0; r < kChunk; ++r) v[r] *= scale[r];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 hv, lv;
+        split8_bf16(v + 8 * c, hv, lv);
+        const uint32_t off = static_cast<uint32_t>(f) * 128u + ((static_cast<uint32_t>(c) ^ (f & 7u)) << 4);
+        *reinterpret_cast<uint4*>(dst + off) = hv;
+        *reinterpret_cast<uint4*>(dst + 16384 + off) = lv;
+      }
+    }
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  // ---- (3) D_U = (diag(b) V)^T T^T (columns 64..127), D_W = (diag(b gamma) K)^T T^T (128..191)
+  if (tid == 0) {
+    constexpr uint32_t idesc = tc::idesc_bf16_f32(128, 64);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t th = tc::desc_kmajor_sw128(TI + kk * 32), tl = tc::desc_kmajor_sw128(TI + 8192 + kk * 32);
+      const uint64_t vh = tc::desc_kmajor_sw128(VI + kk * 32), vl = tc::desc_kmajor_sw128(VI + 16384 + kk * 32);
+      const uint64_t kh = tc::desc_kmajor_sw128(KI + kk * 32), kl = tc::desc_kmajor_sw128(KI + 16384 + kk * 32);
+      tc::mma_bf16(tbase + 64, vh, th, idesc, kk ? 1u : 0u);
+      tc::mma_bf16(tbase + 64, vh, tl, idesc, 1u);
+      tc::mma_bf16(tbase + 64, vl, th, idesc, 1u);
+      tc::mma_bf16(tbase + 128, kh, th, idesc, kk ? 1u : 0u);
+      tc::mma_bf16(tbase + 128, kh, tl, idesc, 1u);
+      tc::mma_bf16(tbase + 128, kl, th, idesc, 1u);
+    }
+    tc::mma_commit(bar);
+  }
+  if (!mbar_wait(bar, 1, abort, kWyWaitNs)) {
+    if (!*abort) atomicOr(b.err, MK_DEVERR_PIPE_TIMEOUT);
+    *abort = 1;
+  }
+  tc::fence_after_sync();
+  // ---- epilogue: lane i holds U[r][i] and W[r][i] over the chunk's r
+  if (!*abort) {
+    const int f = tid;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float d[16];
+      tc::tmem_ld16(tbase + lane_off + 64 + 16 * q, d);
+      if (f < DV) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r = 16 * q + u;
+          if (r < n) b.u[static_cast<long long>(t0 + r) * Hd * DV + h * DV + f] = d[u];
+        }
+      }
+    }
+    // W rows (rows 64 + r of A1, K = feature; rows past the prompt zero): staged as the
+    // image's 64 rows in shared memory (the V / K images are consumed), then copied out in
+    // 16-byte pieces
+    uint8_t* ws = sm + Lyt::kImg;   // [hi: KB blocks][lo: KB blocks] of 64 rows x 128 B
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float d[16];
+      tc::tmem_ld16(tbase + lane_off + 128 + 16 * q, d);
+      if (f < DK) {
+        const int kb = f >> 6, kf = f & 63;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r = 16 * q + u;
+          put_bf16_pair(ws + kb * 8192, KB * 8192, r, kf, r < n ? d[u] : 0.f);
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tbase, 256);
+  if (*abort) return;
+  {   // row r of the staged tile is row 64 + r of A1: the same swizzle phase (64 = 0 mod 8)
+    const uint8_t* ws = sm + Lyt::kImg;
+    for (int idx = tid; idx < 2 * KB * 64 * 8; idx += 128) {
+      const int blk = idx >> 9, rem = idx & 511;   // blk: part * KB + kb; rem: row * 8 + chunk
+      *reinterpret_cast<uint4*>(a1 + blk * 16384 + 64 * 128 + rem * 16) =
+          *reinterpret_cast<const uint4*>(ws + blk * 8192 + rem * 16);
+    }
+  }
+}
+
+
 template <int DK>
 constexpr size_t wy_tc_smem() {
   return WyImg<DK>::kA1 + 2ull * (WyImg<DK>::kP + WyImg<DK>::kKT) + 2ull * (DK / 64) * 2048 + 2 * 4096 +
@@ -2151,11 +2535,11 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
         wy.img = pf.img;
         wy.err = b.err;
         if (dk == 128) {
-          wy_prep_fast<128, 128><<<dim3(nch, Hd), 256, wy_fast_smem<128, 128>(false), s>>>(wy);
+          wy_prep_tc<128, 128><<<dim3(nch, Hd), 128, kWyPrepTcSmem, s>>>(wy);
           chk();
           wy_state_tc<128, 128><<<dim3(Hd, dv / kRowGroup), 128, wy_tc_smem<128>(), s>>>(wy, S);
         } else {
-          wy_prep_fast<64, 64><<<dim3(nch, Hd), 256, wy_fast_smem<64, 64>(false), s>>>(wy);
+          wy_prep_tc<64, 64><<<dim3(nch, Hd), 128, kWyPrepTcSmem, s>>>(wy);
           chk();
           wy_state_tc<64, 64><<<dim3(Hd, dv / kRowGroup), 128, wy_tc_smem<64>(), s>>>(wy, S);
         }
@@ -2288,6 +2672,12 @@ cudaError_t set_prefill_smem_limits() {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(wy_state_tc<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(wy_tc_smem<64>()));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wy_prep_tc<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kWyPrepTcSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(wy_prep_tc<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kWyPrepTcSmem));
     return e;
   });
 }
