@@ -341,20 +341,20 @@ def seed_long_context(m, cfg, n_pos, dev):
     return int(synth.stream(3, "long.first_token").integers(0, cfg.vocab))
 
 
-EXTRA_WORKLOADS = ("pp520", "pp4096", "long", "long_q8")
+EXTRA_WORKLOADS = ("pp520", "pp4096", "long", "long_q8", "27b")
 
 
 def extra_workloads(args) -> dict:
     """The other measured configurations, each in its own process (so every one starts from a
     clean device), summarised for the headline line: prefill pp520 / pp4096, long-context
-    decode with the bf16 and the 8-bit KV cache. Each runs 3 timed steps after 2 warm-up steps.
-    (The 27B-shaped 4-bit model runs on its own: --workload 27b.)"""
+    decode with the bf16 and the 8-bit KV cache, the 27B-shaped 4-bit model (plain decode and
+    K = 5 verify). Each runs 3 timed steps after 2 warm-up steps."""
     out = {}
     for w in EXTRA_WORKLOADS:
         cmd = [sys.executable, os.path.abspath(__file__), "--workload", w, "--steps", "3", "--warmup", "2",
                "--no-cpu-baseline"]
         try:
-            r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+            r = subprocess.run(cmd, capture_output=True, text=True, timeout=600)
             lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
             if r.returncode != 0 or not lines:
                 out[w] = {"error": (r.stderr or r.stdout).strip().splitlines()[-1:] or ["exit %d" % r.returncode]}

@@ -231,18 +231,24 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tc::fence_after_sync();
       if (j == 0) {
         m_used = mx;   // key 0 is visible to every query, so mx is finite
-      } else if (mx > m_used + kRescaleAt) {   // raise the running maximum: rescale O and l
-        const float f = __expf(m_used - mx);
-        l *= f;
+      } else {
+        // raise the running maximum of the rows whose tile maximum passed it by more than
+        // kRescaleAt: rescale their O and l. The TMEM loads and stores are warp-collective,
+        // so the whole warp walks O whenever one of its rows needs it (factor 1 elsewhere).
+        const bool raise = mx > m_used + kRescaleAt;
+        if (__any_sync(0xffffffffu, raise)) {
+          const float f = raise ? __expf(m_used - mx) : 1.0f;
+          l *= f;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 16) {
-          float o[16];
-          tc::tmem_ld16(tmem + lane_base + kColO + c, o);
+          for (int c = 0; c < D; c += 16) {
+            float o[16];
+            tc::tmem_ld16(tmem + lane_base + kColO + c, o);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] *= f;
-          tc::tmem_st16(tmem + lane_base + kColO + c, o);
+            for (int i = 0; i < 16; ++i) o[i] *= f;
+            tc::tmem_st16(tmem + lane_base + kColO + c, o);
+          }
+          if (raise) m_used = mx;
         }
-        m_used = mx;
       }
       // P = exp(S - m) as bf16 high and low parts, K-major 128-byte-swizzled rows
       uint8_t* rh = phi + r * 128;

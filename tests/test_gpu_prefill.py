@@ -150,3 +150,34 @@ def test_08b_verify_one_pass():
             assert rel_frob(conv_history_as_window(ring[li], st.pos, cfg.conv_width), st.conv[li]) <= STATE_REL_FROB
         assert int(m.pos_tensor.item()) == st.pos
         last = int(committed[-1])
+
+
+def test_flash_attention_sharp_scores_and_continued_prompts():
+    """The tiny model with its query and key projections scaled by 16 (exact in bf16), so the
+    attention scores span hundreds of units: within a query row a later key tile often beats
+    the running maximum by far more than the flash kernel's rescale threshold, and rows of the
+    same warp take different branches. A 199-token batched pass (two query tiles), then
+    continued prompts of 71 and 65 tokens whose queries sit past earlier positions (up to six
+    key tiles per row), against the oracle."""
+    import hybrid_deltanet_attention_b200 as hda
+    cfg = synth.TINY
+    raw = synth.make_weights(cfg)
+    for li, kind in enumerate(cfg.pattern):
+        if kind != "A":
+            continue
+        name = f"layers.{li}.attn.w_in"
+        w = raw[name].copy()
+        qk = cfg.at_q_heads * cfg.at_head_dim * (2 if cfg.at_out_gate else 1) + cfg.at_kv_heads * cfg.at_head_dim
+        vals = (w[:qk].astype(np.uint32) << 16).view(np.float32) * np.float32(16.0)
+        w[:qk] = synth.f32_to_bf16_bits(vals)
+        raw[name] = w
+    m = hda.Model(cfg, hda.weights_to_device(raw), max_ctx=512)
+    W = oracle.prepare_weights(cfg, raw)
+    st = oracle.new_state(cfg, 512)
+    m.reset()
+    prompt = synth.make_prompt(cfg, 200 + 72 + 66, tag="sharp")
+    o = 0
+    for n in (200, 72, 66):   # batched passes of 199, 71 and 65 tokens, each ending in a decode launch
+        zo, zg, tg = _prefill_both(cfg, m, st, W, prompt[o:o + n])
+        _check(cfg, m, st, zo, zg, tg)
+        o += n
