@@ -1278,16 +1278,19 @@ __global__ void __launch_bounds__(256) wy_state_fast(WyBufs b, float* __restrict
 // N = 16, K = 16):
 //   A: D1 = [gamma Q; W] S0^T                   (lanes 0..63: gamma Q S0^T, 64..127: W S0^T)
 //   Delta = U - W S0^T (lanes 64..127), written as bf16 tiles Delta^T, (dec Delta)^T
+//   C: D3 = gamma_last S0^T + K^T (dec Delta)   (S^T accumulates in TMEM across chunks;
+//                                                committed on its own barrier)
 //   B: D1[0..63] += P Delta                     (o; the P tile's M = 128 operand spans the
 //                                                next 64 rows of the image, whose products
 //                                                land in lanes 64..127, which are not read)
-//   C: D3 = gamma_last S0^T + K^T (dec Delta)   (S^T accumulates in TMEM across chunks)
 // then S1 = D3 is copied to the S0 operand tile and pre-scaled by the next chunk's
-// gamma_last. Operand images arrive by bulk copies: A1 of the next chunk as soon as phase
-// A has consumed it, P and K^T two chunks ahead (double buffer); U and the decay factors
-// by cp.async. Every wait has a time limit; on expiry the CTA latches an error and stops.
+// gamma_last. Only A, Delta and C lie on the chain from one chunk's state to the next: D1 is
+// double-buffered, so B and the store of o run while the next chunk's A is under way.
+// Operand images arrive by bulk copies: A1 of the next chunk as soon as phase A has consumed
+// it, P and K^T two chunks ahead (double buffer); U and the decay factors by cp.async. Every
+// wait has a time limit; on expiry the CTA latches an error and stops.
 struct WyTcBars {
-  uint64_t a1, pk[2], mma;
+  uint64_t a1, pk[2], mma, mmas;
   uint32_t tmem;
   int abort;
 };
@@ -1415,6 +1418,7 @@ __global__ void __launch_bounds__(128, 2) wy_prep_tc(WyBufs b) {
   }
   // ---- key rows: rows 0..63 of the [K; Q] image, and the K^T image (row j: k_r[j] over the
   // chunk's r; rows j >= dk zero, global)
+#pragma unroll 1
   for (int idx = tid; idx < kChunk * (DK / 8); idx += 128) {
     const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
     uint4 hv, lv;
@@ -1443,6 +1447,7 @@ __global__ void __launch_bounds__(128, 2) wy_prep_tc(WyBufs b) {
   cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
+#pragma unroll 1
   for (int idx = tid; idx < kChunk * (DK / 8); idx += 128) {
     const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
     const int row = kChunk + r;
@@ -1496,7 +1501,8 @@ __global__ void __launch_bounds__(128, 2) wy_prep_tc(WyBufs b) {
     const bool isq = tid >= kChunk;
     const float gr = g[r], br = bb[r];
     const bool live = r < n;
-#pragma unroll
+    // decay factors e^{g_r - g_s} <= 1 (s <= r) by the fast exponential: relative error ~2^-21
+#pragma unroll 1
     for (int q = 0; q < 4; ++q) {
       float d[16];
       tc::tmem_ld16(tbase + lane_off + 16 * q, d);
@@ -1504,13 +1510,13 @@ __global__ void __launch_bounds__(128, 2) wy_prep_tc(WyBufs b) {
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int s = 16 * q + u;
-          A[r * AP + s] = (s < r && live) ? br * expf(gr - g[s]) * d[u] : 0.f;
+          A[r * AP + s] = (s < r && live) ? br * __expf(gr - g[s]) * d[u] : 0.f;
         }
       } else {
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int s = 16 * q + u;
-          d[u] = (s <= r && live) ? expf(gr - g[s]) * d[u] : 0.f;
+          d[u] = (s <= r && live) ? __expf(gr - g[s]) * d[u] : 0.f;
         }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -1707,18 +1713,22 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
     mbar_init(&bars->pk[0], 1);
     mbar_init(&bars->pk[1], 1);
     mbar_init(&bars->mma, 1);
+    mbar_init(&bars->mmas, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
   if (warp == 0) {
-    tc::tmem_alloc(&bars->tmem, 32);
+    tc::tmem_alloc(&bars->tmem, 64);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
-  const uint32_t d1 = bars->tmem + lane_off, d3 = bars->tmem + 16 + lane_off;
+  // D1 of chunk c in columns 16 (c & 1) .. + 15 (o of chunk c is read during chunk c + 1),
+  // D3 (S^T) in columns 32 .. 47
+  auto d1_of = [&](int c) { return bars->tmem + 16u * static_cast<uint32_t>(c & 1) + lane_off; };
+  const uint32_t d3 = bars->tmem + 32 + lane_off;
 
   int n_a1 = 0, n_pk[2] = {0, 0};   // bulk copies issued per barrier (thread 0)
   if (tid == 0) {
@@ -1763,6 +1773,17 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
       }
     }
   };
+  // o of chunk c (lanes 0..63 of its D1) to global; warps 0 and 1, every lane takes part
+  auto store_o = [&](int c) {
+    const int t0 = c * kChunk, n = min(kChunk, b.T - t0);
+    float o[RG];
+    tc::tmem_ld16(d1_of(c), o);
+    if (tid < n) {
+      float4* dst = reinterpret_cast<float4*>(b.o + static_cast<long long>(t0 + tid) * Hd * DV + h * DV + i0);
+#pragma unroll
+      for (int q = 0; q < RG / 4; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+  };
   float sv[RG];
 #pragma unroll
   for (int i = 0; i < RG; ++i)
@@ -1780,16 +1801,16 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
   __syncthreads();
   tc::fence_after_sync();
 
-  uint32_t mph = 0;
+  uint32_t mph = 0, sph = 0;
   for (int ch = 0; ch < nch; ++ch) {
-    const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
-    // ---- A: D1 = [gamma Q; W] S0^T
+    // ---- A: D1(ch) = [gamma Q; W] S0^T
     if (tid == 0) {
       if (!mbar_wait(&bars->a1, ch & 1, abort, kWyWaitNs)) {
         if (!*abort) atomicOr(b.err, MK_DEVERR_PIPE_TIMEOUT);
         *abort = 1;
       } else {
         tc::fence_after_sync();
+        const uint32_t d1 = d1_of(ch) - lane_off;
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
@@ -1798,31 +1819,42 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
             const uint64_t al = tc::desc_kmajor_sw128(A1 + (KB + kb) * 16384 + kk * 32);
             const uint64_t bh = tc::desc_kmajor_sw128(B1 + kb * 2048 + kk * 32);
             const uint64_t bl = tc::desc_kmajor_sw128(B1 + (KB + kb) * 2048 + kk * 32);
-            tc::mma_bf16(d1 - lane_off, ah, bh, idesc, (kb | kk) ? 1u : 0u);
-            tc::mma_bf16(d1 - lane_off, ah, bl, idesc, 1u);
-            tc::mma_bf16(d1 - lane_off, al, bh, idesc, 1u);
+            tc::mma_bf16(d1, ah, bh, idesc, (kb | kk) ? 1u : 0u);
+            tc::mma_bf16(d1, ah, bl, idesc, 1u);
+            tc::mma_bf16(d1, al, bh, idesc, 1u);
           }
         tc::mma_commit(&bars->mma);
       }
     }
+    // (MMAs complete in issue order: this wait also covers B of the previous chunk)
     if (!mbar_wait(&bars->mma, mph, abort, kWyWaitNs)) *abort = 1;
     mph ^= 1u;
     tc::fence_after_sync();
-    if (tid == 0 && ch + 1 < nch && !*abort) {   // A1 is consumed: stage the next chunk's
-      mbar_arrive_expect_tx(&bars->a1, I::kA1);
-      tc::bulk_load(A1, img_at(ch + 1), I::kA1, &bars->a1);
-      ++n_a1;
+    if (tid == 0 && !*abort) {
+      if (ch + 1 < nch) {   // A1 is consumed: stage the next chunk's
+        mbar_arrive_expect_tx(&bars->a1, I::kA1);
+        tc::bulk_load(A1, img_at(ch + 1), I::kA1, &bars->a1);
+        ++n_a1;
+      }
+      if (ch >= 1 && ch + 1 < nch) {   // P / K^T of chunk ch - 1 are consumed: stage chunk ch + 1's
+        const int bf = (ch + 1) & 1;
+        mbar_arrive_expect_tx(&bars->pk[bf], kPK);
+        tc::bulk_load(PK0 + bf * kPK, img_at(ch + 1) + I::kA1, kPK, &bars->pk[bf]);
+        ++n_pk[bf];
+      }
     }
     if (ch + 1 < nch) fetch_ud(ch + 1);
     cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();   // U and the decay factors of this chunk
     if (*abort) break;
-    // ---- Delta = U - W S0^T; the tiles Delta^T and (dec Delta)^T (row i, K = token r)
-    if (warp >= 2) {
+    if (warp < 2) {
+      if (ch > 0) store_o(ch - 1);   // o of the previous chunk, off the state's critical path
+    } else {
+      // ---- Delta = U - W S0^T; the tiles Delta^T and (dec Delta)^T (row i, K = token r)
       const int r = tid - 64;
       float ws[RG];
-      tc::tmem_ld16(d1, ws);
+      tc::tmem_ld16(d1_of(ch), ws);
       const float* U = Ub + (ch & 1) * kChunk * RG;
       const float dr = dcb[(ch & 1) * kChunk + r];
 #pragma unroll
@@ -1840,7 +1872,7 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncthreads();
-    // ---- B: D1[0..63] += P Delta;  C: D3 += K^T (dec Delta)
+    // ---- C: D3 += K^T (dec Delta) (the state: committed on its own), then B: D1(ch)[0..63] += P Delta
     if (tid == 0) {
       if (!mbar_wait(&bars->pk[ch & 1], (ch >> 1) & 1, abort, kWyWaitNs)) {
         if (!*abort) atomicOr(b.err, MK_DEVERR_PIPE_TIMEOUT);
@@ -1850,13 +1882,6 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
         const uint8_t* PK = PK0 + (ch & 1) * kPK;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ph = tc::desc_kmajor_sw128(PK + kk * 32);
-          const uint64_t pl = tc::desc_kmajor_sw128(PK + 8192 + kk * 32);
-          const uint64_t dh = tc::desc_kmajor_sw128(B2 + kk * 32);
-          const uint64_t dl = tc::desc_kmajor_sw128(B2 + 2048 + kk * 32);
-          tc::mma_bf16(d1 - lane_off, ph, dh, idesc, 1u);
-          tc::mma_bf16(d1 - lane_off, ph, dl, idesc, 1u);
-          tc::mma_bf16(d1 - lane_off, pl, dh, idesc, 1u);
           const uint64_t kh = tc::desc_kmajor_sw128(PK + I::kP + kk * 32);
           const uint64_t kl = tc::desc_kmajor_sw128(PK + I::kP + 16384 + kk * 32);
           const uint64_t eh = tc::desc_kmajor_sw128(B3 + kk * 32);
@@ -1865,29 +1890,25 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
           tc::mma_bf16(d3 - lane_off, kh, el, idesc, 1u);
           tc::mma_bf16(d3 - lane_off, kl, eh, idesc, 1u);
         }
-        tc::mma_commit(&bars->mma);
-      }
-    }
-    if (!mbar_wait(&bars->mma, mph, abort, kWyWaitNs)) *abort = 1;
-    mph ^= 1u;
-    tc::fence_after_sync();
-    if (tid == 0 && ch + 2 < nch && !*abort) {   // this P / K^T buffer is consumed
-      mbar_arrive_expect_tx(&bars->pk[ch & 1], kPK);
-      tc::bulk_load(PK0 + (ch & 1) * kPK, img_at(ch + 2) + I::kA1, kPK, &bars->pk[ch & 1]);
-      ++n_pk[ch & 1];
-    }
-    __syncthreads();
-    if (*abort) break;
-    // ---- outputs of this chunk (lanes 0..63) and the state after it
-    if (warp < 2) {   // every lane of the warp takes part in the load
-      float o[RG];
-      tc::tmem_ld16(d1, o);
-      if (tid < n) {
-        float4* dst = reinterpret_cast<float4*>(b.o + static_cast<long long>(t0 + tid) * Hd * DV + h * DV + i0);
+        tc::mma_commit(&bars->mmas);
+        const uint32_t d1 = d1_of(ch) - lane_off;
 #pragma unroll
-        for (int q = 0; q < RG / 4; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ph = tc::desc_kmajor_sw128(PK + kk * 32);
+          const uint64_t pl = tc::desc_kmajor_sw128(PK + 8192 + kk * 32);
+          const uint64_t dh = tc::desc_kmajor_sw128(B2 + kk * 32);
+          const uint64_t dl = tc::desc_kmajor_sw128(B2 + 2048 + kk * 32);
+          tc::mma_bf16(d1, ph, dh, idesc, 1u);
+          tc::mma_bf16(d1, ph, dl, idesc, 1u);
+          tc::mma_bf16(d1, pl, dh, idesc, 1u);
+        }
       }
     }
+    if (!mbar_wait(&bars->mmas, sph, abort, kWyWaitNs)) *abort = 1;
+    sph ^= 1u;
+    tc::fence_after_sync();
+    if (*abort) break;
+    // ---- the state after this chunk
     tc::tmem_ld16(d3, sv);
     if (ch + 1 < nch) {
       put_s(sv);
@@ -1904,6 +1925,13 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
     __syncthreads();
     tc::fence_after_sync();
   }
+  // o of the last chunk once its B has completed
+  if (!*abort && nch > 0) {
+    if (tid == 0) tc::mma_commit(&bars->mma);
+    if (!mbar_wait(&bars->mma, mph, abort, kWyWaitNs)) *abort = 1;
+    tc::fence_after_sync();
+    if (!*abort && warp < 2) store_o(nch - 1);
+  }
   cp_async_wait<0>();
   if (tid == 0) {   // let issued bulk copies land before the CTA ends (bounded)
     int never = 0;
@@ -1913,7 +1941,7 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc::tmem_dealloc(bars->tmem, 32);
+  if (warp == 0) tc::tmem_dealloc(bars->tmem, 64);
 }
 
 template <int DK, int DV>
