@@ -272,13 +272,19 @@ def replica_throughput(units_per_rank: float, world: int, seconds: float) -> flo
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
+_ORACLE_W = None
+
+
 def oracle_sample(seconds_budget: float = 15.0, n_prompt: int = 16, n_decode: int = 64):
     """Time the CPU oracle on a bounded sample of the same workload: weights prepared
     untimed, a short prompt fed untimed, then n_decode greedy steps timed."""
     import oracle
     import synth
     cfg = synth.QWEN_08B
-    W = oracle.prepare_weights(cfg, synth.make_weights(cfg))
+    global _ORACLE_W
+    if _ORACLE_W is None:   # prepared once per process (untimed)
+        _ORACLE_W = oracle.prepare_weights(cfg, synth.make_weights(cfg))
+    W = _ORACLE_W
     st = oracle.new_state(cfg, n_prompt + n_decode + 1)
     z = oracle.prefill(cfg, W, st, synth.make_prompt(cfg, n_prompt))
     tok = int(np.argmax(z))
@@ -501,6 +507,13 @@ def run_mk(args):
     if world == 1 and not args.no_cpu_baseline and not long_ctx:
         v, cores, sample = oracle_sample()
         cpu = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample}
+        try:   # the same oracle on one thread (BLAS pools limited to 1), a shorter sample
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                v1, _, sample1 = oracle_sample(seconds_budget=8.0, n_prompt=8, n_decode=16)
+            cpu["one_thread"] = {"value": v1, "unit": "tok/s", "cores": 1, "sample": sample1}
+        except Exception as ex:   # the multi-threaded figure stands on its own
+            cpu["one_thread"] = {"error": repr(ex)}
 
     clocks = clk.summary()
     line = {

@@ -515,40 +515,12 @@ __device__ __forceinline__ void load_xreg(XReg<XK>& x, const float* xs, int H, i
   }
 }
 
-// Dot products of two bf16 rows with x (register or shared-memory copy).
-template <int XK>
-__device__ __forceinline__ void dot2_rows(const uint8_t* p0, const uint8_t* p1, const XReg<XK>& x, const float* xs,
-                                          int H, int lane, float& a0, float& a1) {
-  a0 = 0.f;
-  a1 = 0.f;
-  if (XK > 0) {
-    uint4 w0[XK > 0 ? XK : 1], w1[XK > 0 ? XK : 1];
-#pragma unroll
-    for (int k = 0; k < XK; ++k) {     // all shared-memory loads first, then the arithmetic
-      const int c = lane * 8 + 256 * k;
-      w0[k] = *reinterpret_cast<const uint4*>(p0 + 2 * c);
-      w1[k] = *reinterpret_cast<const uint4*>(p1 + 2 * c);
-    }
-#pragma unroll
-    for (int k = 0; k < XK; ++k) {
-      a0 = dot8_bf16_f32(w0[k], x.a[k], x.b[k], a0);
-      a1 = dot8_bf16_f32(w1[k], x.a[k], x.b[k], a1);
-    }
-  } else {
-    for (int c = lane * 8; c < H; c += 256) {
-      const float4 xa = *reinterpret_cast<const float4*>(xs + c);
-      const float4 xb = *reinterpret_cast<const float4*>(xs + c + 4);
-      a0 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p0 + 2 * c), xa, xb, a0);
-      a1 = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p1 + 2 * c), xa, xb, a1);
-    }
-  }
-}
-
-// Dot products of up to four bf16 rows with x, four independent accumulator chains.
+// Dot products of up to four bf16 rows with x, four independent accumulator chains, each
+// split into even and odd positions by the packed fp32 FMA.
 template <int XK>
 __device__ __forceinline__ void dot4_rows(const uint8_t* p0, const uint8_t* p1, const uint8_t* p2, const uint8_t* p3,
                                           const XReg<XK>& x, const float* xs, int H, int lane, float* a) {
-  a[0] = a[1] = a[2] = a[3] = 0.f;
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
   if (XK > 0) {
 #pragma unroll
     for (int k = 0; k < XK; ++k) {
@@ -557,21 +529,23 @@ __device__ __forceinline__ void dot4_rows(const uint8_t* p0, const uint8_t* p1, 
       const uint4 w1 = *reinterpret_cast<const uint4*>(p1 + 2 * c);
       const uint4 w2 = *reinterpret_cast<const uint4*>(p2 + 2 * c);
       const uint4 w3 = *reinterpret_cast<const uint4*>(p3 + 2 * c);
-      a[0] = dot8_bf16_f32(w0, x.a[k], x.b[k], a[0]);
-      a[1] = dot8_bf16_f32(w1, x.a[k], x.b[k], a[1]);
-      a[2] = dot8_bf16_f32(w2, x.a[k], x.b[k], a[2]);
-      a[3] = dot8_bf16_f32(w3, x.a[k], x.b[k], a[3]);
+      dot8_bf16_f2(w0, x.a[k], x.b[k], acc[0]);
+      dot8_bf16_f2(w1, x.a[k], x.b[k], acc[1]);
+      dot8_bf16_f2(w2, x.a[k], x.b[k], acc[2]);
+      dot8_bf16_f2(w3, x.a[k], x.b[k], acc[3]);
     }
   } else {
     for (int c = lane * 8; c < H; c += 256) {
       const float4 xa = *reinterpret_cast<const float4*>(xs + c);
       const float4 xb = *reinterpret_cast<const float4*>(xs + c + 4);
-      a[0] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p0 + 2 * c), xa, xb, a[0]);
-      a[1] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p1 + 2 * c), xa, xb, a[1]);
-      a[2] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p2 + 2 * c), xa, xb, a[2]);
-      a[3] = dot8_bf16_f32(*reinterpret_cast<const uint4*>(p3 + 2 * c), xa, xb, a[3]);
+      dot8_bf16_f2(*reinterpret_cast<const uint4*>(p0 + 2 * c), xa, xb, acc[0]);
+      dot8_bf16_f2(*reinterpret_cast<const uint4*>(p1 + 2 * c), xa, xb, acc[1]);
+      dot8_bf16_f2(*reinterpret_cast<const uint4*>(p2 + 2 * c), xa, xb, acc[2]);
+      dot8_bf16_f2(*reinterpret_cast<const uint4*>(p3 + 2 * c), xa, xb, acc[3]);
     }
   }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) a[q] = f2_sum(acc[q]);
 }
 
 // DeltaNet conv epilogue of the in-projection: for a q/k/v row g with raw value x_t,

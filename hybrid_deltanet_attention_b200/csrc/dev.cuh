@@ -205,6 +205,30 @@ __device__ __forceinline__ float dot8_bf16_f32(const uint4 w, const float4 a, co
   return acc;
 }
 
+// Two fp32 values in one 64-bit register (low word first), for the packed fp32 FMA of sm_100.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f2_sum(uint64_t v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
+// d = a * b + d in both halves (fma.rn.f32x2: two round-to-nearest fp32 FMAs)
+__device__ __forceinline__ void ffma2(uint64_t& d, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+// 8 bf16 weights w against x[0..7] = (a, b) into the two partial sums of acc (even and odd
+// positions): four packed FMAs instead of eight.
+__device__ __forceinline__ void dot8_bf16_f2(const uint4 w, const float4 a, const float4 b, uint64_t& acc) {
+  ffma2(acc, f2_pack(bf16lo(w.x), bf16hi(w.x)), f2_pack(a.x, a.y));
+  ffma2(acc, f2_pack(bf16lo(w.y), bf16hi(w.y)), f2_pack(a.z, a.w));
+  ffma2(acc, f2_pack(bf16lo(w.z), bf16hi(w.z)), f2_pack(b.x, b.y));
+  ffma2(acc, f2_pack(bf16lo(w.w), bf16hi(w.w)), f2_pack(b.z, b.w));
+}
+
 // Ordered key for a float so that unsigned comparison follows float order.
 __device__ __forceinline__ uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f);
