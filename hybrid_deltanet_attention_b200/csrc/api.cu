@@ -264,7 +264,7 @@ struct Layout {
   int pf_rows;
   size_t pf_h, pf_xhi, pf_xlo, pf_z, pf_y, pf_o, pf_u, pf_w, pf_p, pf_gam, pf_dec, pf_apart, pf_splitk, pf_best;
   size_t pf_kvd = 0;
-  size_t pf_vt = 0, pf_img = 0;
+  size_t pf_vt = 0, pf_img = 0, pf_fq = 0;
   long long pf_nk;
   // batched verify saves
   int vf_rows;
@@ -405,6 +405,8 @@ Layout make_layout(const mk_config& c, int grid) {
     if (L.pf_nk > 0) {
       L.pf_vt = off;
       off = align256(off + static_cast<size_t>(c.at_kv_heads) * c.at_head_dim * static_cast<size_t>(L.pf_nk) * 2);
+      L.pf_fq = off;   // the flash kernel's work counter
+      off = align256(off + 4);
     }
     if (na && c.kv_format == MK_KV_Q8) {   // one layer's K and V read back as bf16 for the attention kernels
       L.pf_kvd = off;
@@ -776,6 +778,7 @@ int mk_load_weights(const mk_config* cfg, const mk_tensor* tensors, int32_t n_te
     if (L.pf_img) m->pf.img = W + L.pf_img;
     if (L.pf_nk > 0) {
       m->pf.vt = reinterpret_cast<uint16_t*>(W + L.pf_vt);
+      m->pf.flash_items = reinterpret_cast<int*>(W + L.pf_fq);
     }
   }
   m->vf.rows = L.vf_rows;

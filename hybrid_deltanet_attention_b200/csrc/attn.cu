@@ -1,5 +1,5 @@
-// Causal GQA attention of a prefill pass on the sm_100a tensor cores, flash style: one CTA
-// per (128-query tile, query head) walks the cached keys in tiles of 64, keeps the scores of
+// Causal GQA attention of a prefill pass on the sm_100a tensor cores, flash style: for each
+// (128-query tile, query head) work item a CTA walks the cached keys in tiles of 64, keeps the scores of
 // the current tile in tensor memory, turns them into probabilities with an online softmax in
 // registers, and accumulates O = P V in tensor memory. No score or probability matrix
 // leaves the chip; tiles above the diagonal are never computed.
@@ -15,10 +15,14 @@
 // tile's maximum exceeds it by more than kRescaleAt; otherwise the stale maximum is kept,
 // so every probability is at most e^kRescaleAt and the result O / l is the same softmax.
 //
+// The kernel is persistent: one CTA per SM takes items from a counter, the longest key
+// ranges first (the last query tile of every head, then the one before, ...), so the causal
+// imbalance evens out across the SMs; between items the CTA drains and re-arms its barriers.
 // Roles (192 threads): warp 0 lane 0 issues the TMA loads (Q once, then K and V^T tiles),
 // warp 1 lane 0 issues the MMAs, warps 2..5 (one TMEM lane quarter each, one query row per
 // thread) run the softmax and write O / l. Every wait has a time limit; on expiry the CTA
 // latches an error bit and winds down.
+#include <algorithm>
 #include <cstdint>
 #include <cuda.h>
 
@@ -61,6 +65,7 @@ struct FlashBars {
   uint64_t s_full[2], s_empty[2];
   uint32_t tmem;
   int abort;
+  int item;   // the work item this CTA runs next
 };
 static_assert(sizeof(FlashBars) <= 256, "barriers fit their slot");
 
@@ -77,7 +82,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     attn_flash_kernel(const __grid_constant__ CUtensorMap tq_hi, const __grid_constant__ CUtensorMap tq_lo,
                       const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tvt,
                       const int* __restrict__ posp, int off, int T, int Hq, int Hkv, int max_ctx, float* __restrict__ out,
-                      long long ldo, int* err) {
+                      long long ldo, int* items, int* err) {
   using Lay = FlashLayout<D>;
   constexpr int kNB = Lay::kNB;
   constexpr int kOffQhi = Lay::kOffQhi, kOffQlo = Lay::kOffQlo, kOffK = Lay::kOffK, kOffVt = Lay::kOffVt;
@@ -88,28 +93,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
   FlashBars* fb = reinterpret_cast<FlashBars*>(smem + Lay::kOffBars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntile_q = (T + kFM - 1) / kFM;
-  const int qt = ntile_q - 1 - static_cast<int>(blockIdx.x);   // the longest key ranges first
-  const int h = blockIdx.y, g = h / (Hq / Hkv);
-  const int m0 = qt * kFM;
+  const int n_items = ntile_q * Hq;
   const int pos0 = *posp + off;
-  // keys 0 .. pos0 + (last valid query of the tile)
-  const int nkeys = pos0 + min(m0 + kFM, T);
-  const int nt = (nkeys + kFN - 1) / kFN;
 
   if (threadIdx.x == 0) {
-    mbar_init(&fb->q_full, 1);
-    mbar_init(&fb->k_full, 1);
-    mbar_init(&fb->k_empty, 1);
-    mbar_init(&fb->v_full, 1);
-    mbar_init(&fb->v_empty, 1);
-    mbar_init(&fb->p_full, 4);
-    mbar_init(&fb->p_empty, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&fb->s_full[b], 1);
-      mbar_init(&fb->s_empty[b], 4);
-    }
     fb->abort = 0;
-    fence_barrier_init();
     tc::prefetch_tensormap(&tq_hi);
     tc::prefetch_tensormap(&tq_lo);
     tc::prefetch_tensormap(&tk);
@@ -123,6 +111,32 @@ __global__ void __launch_bounds__(kFThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = fb->tmem;
+
+  for (;;) {
+  if (threadIdx.x == 0) {   // next item; the barriers start a fresh sequence (nothing is pending)
+    fb->item = fb->abort ? n_items : atomicAdd(items, 1);
+    mbar_init(&fb->q_full, 1);
+    mbar_init(&fb->k_full, 1);
+    mbar_init(&fb->k_empty, 1);
+    mbar_init(&fb->v_full, 1);
+    mbar_init(&fb->v_empty, 1);
+    mbar_init(&fb->p_full, 4);
+    mbar_init(&fb->p_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&fb->s_full[b], 1);
+      mbar_init(&fb->s_empty[b], 4);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int item = fb->item;
+  if (item >= n_items) break;
+  const int qt = ntile_q - 1 - item / Hq;   // the longest key ranges first
+  const int h = item % Hq, g = h / (Hq / Hkv);
+  const int m0 = qt * kFM;
+  // keys 0 .. pos0 + (last valid query of the tile)
+  const int nkeys = pos0 + min(m0 + kFM, T);
+  const int nt = (nkeys + kFN - 1) / kFN;
 
   if (warp == 0) {
     if (lane == 0) {   // ---- TMA producer
@@ -297,6 +311,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
     }
   }
   tc::fence_before_sync();
+  __syncthreads();   // the item is done in every role (O read out, copies landed)
+  tc::fence_after_sync();
+  }
+  tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
@@ -307,16 +325,22 @@ __global__ void __launch_bounds__(kFThreads, 1)
 template <int D>
 cudaError_t launch_flash_d(const CUtensorMap& mqh, const CUtensorMap& mql, const CUtensorMap& mk_, const CUtensorMap& mvt,
                            const int* posp, int off, int T, int Hq, int Hkv, int max_ctx, float* out, long long ldo,
-                           int* err, cudaStream_t s) {
+                           int* items, int* err, cudaStream_t s) {
   static std::atomic<uint64_t> attr_set{0};   // per device
   const cudaError_t e = once_per_device(attr_set, [] {
     return cudaFuncSetAttribute(attn_flash_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 FlashLayout<D>::kSmem);
   });
   if (e != cudaSuccess) return e;
-  dim3 grid((T + kFM - 1) / kFM, Hq);
-  attn_flash_kernel<D><<<grid, kFThreads, FlashLayout<D>::kSmem, s>>>(mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv,
-                                                                       max_ctx, out, ldo, err);
+  const int n_items = (T + kFM - 1) / kFM * Hq;
+  int dev = 0, sms = 0;
+  cudaError_t e2 = cudaGetDevice(&dev);
+  if (e2 == cudaSuccess) e2 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e2 != cudaSuccess) return e2;
+  e2 = cudaMemsetAsync(items, 0, sizeof(int), s);
+  if (e2 != cudaSuccess) return e2;
+  attn_flash_kernel<D><<<std::min(n_items, sms), kFThreads, FlashLayout<D>::kSmem, s>>>(
+      mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv, max_ctx, out, ldo, items, err);
   return cudaGetLastError();
 }
 
@@ -331,8 +355,9 @@ bool attn_flash_supported(int D) { return D == 64 || D == 128 || D == 256; }
 // on the device; the key range is bounded by the host with nk (a multiple of 64, >= pos0 + T).
 cudaError_t launch_attn_flash(const uint16_t* q_hi, const uint16_t* q_lo, const uint16_t* k, const uint16_t* vt,
                               const int* posp, int off, int T, int Hq, int Hkv, int D, int max_ctx, long long nk,
-                              float* out, long long ldo, int* err, cudaStream_t s) {
-  if (!attn_flash_supported(D) || T <= 0 || Hq % Hkv || nk % 64 || ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15))
+                              float* out, long long ldo, int* items, int* err, cudaStream_t s) {
+  if (!attn_flash_supported(D) || T <= 0 || Hq % Hkv || nk % 64 || ldo % 4 || (reinterpret_cast<uintptr_t>(out) & 15) ||
+      !items)
     return cudaErrorInvalidValue;
   CUtensorMap mqh, mql, mk_, mvt;
   const long long qd = static_cast<long long>(Hq) * D;
@@ -340,9 +365,9 @@ cudaError_t launch_attn_flash(const uint16_t* q_hi, const uint16_t* q_lo, const 
       !tensor_map_bf16(&mk_, k, static_cast<long long>(Hkv) * max_ctx, D, 2LL * D, kFN) ||
       !tensor_map_bf16(&mvt, vt, static_cast<long long>(Hkv) * D, nk, 2 * nk, D))
     return cudaErrorInvalidValue;
-  if (D == 256) return launch_flash_d<256>(mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv, max_ctx, out, ldo, err, s);
-  if (D == 128) return launch_flash_d<128>(mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv, max_ctx, out, ldo, err, s);
-  return launch_flash_d<64>(mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv, max_ctx, out, ldo, err, s);
+  if (D == 256) return launch_flash_d<256>(mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv, max_ctx, out, ldo, items, err, s);
+  if (D == 128) return launch_flash_d<128>(mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv, max_ctx, out, ldo, items, err, s);
+  return launch_flash_d<64>(mqh, mql, mk_, mvt, posp, off, T, Hq, Hkv, max_ctx, out, ldo, items, err, s);
 }
 
 }  // namespace mk

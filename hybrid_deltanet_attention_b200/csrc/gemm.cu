@@ -417,8 +417,12 @@ cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s) {
   if (a.act_hi && (a.N % 128 != 0 || !a.act_lo || (reinterpret_cast<uintptr_t>(a.act_hi) & 15) ||
                    (reinterpret_cast<uintptr_t>(a.act_lo) & 15)))
     return cudaErrorInvalidValue;
-  // 256-wide tiles for many tokens and wide outputs; 128-wide for few tokens (more CTAs to split over)
-  return (a.N >= 2048 && a.M > kBM) ? launch_bn<256>(a, s) : launch_bn<128>(a, s);
+  // 256-wide tiles for many tokens and wide outputs, or whenever they still fill about a wave
+  // (a 1024-wide output over thousands of tokens: 128 tiles of 256 in one wave rather than 256
+  // tiles of 128 in 1.7); 128-wide for few tokens (more CTAs to split over)
+  const long long tiles256 = static_cast<long long>((a.N + 255) / 256) * ((a.M + kBM - 1) / kBM);
+  const bool wide = a.M > kBM && (a.N >= 2048 || tiles256 >= 120);
+  return wide ? launch_bn<256>(a, s) : launch_bn<128>(a, s);
 }
 
 }  // namespace mk

@@ -149,7 +149,7 @@ bool tensor_map_bf16(CUtensorMap* map, const void* base, long long rows, long lo
 bool attn_flash_supported(int D);
 cudaError_t launch_attn_flash(const uint16_t* q_hi, const uint16_t* q_lo, const uint16_t* k, const uint16_t* vt,
                               const int* posp, int off, int T, int Hq, int Hkv, int D, int max_ctx, long long nk,
-                              float* out, long long ldo, int* err, cudaStream_t s);
+                              float* out, long long ldo, int* items, int* err, cudaStream_t s);
 cudaError_t launch_linear(const LinearArgs& a, cudaStream_t s);
 
 // repack helpers (api.cu launches them)

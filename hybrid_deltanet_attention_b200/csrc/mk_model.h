@@ -32,6 +32,7 @@ struct mk_prefill_ws {
   // (nk_max = max_ctx rounded up to 64; 0 when the head dim has no flash kernel)
   long long nk_max = 0;
   uint16_t* vt = nullptr;
+  int* flash_items = nullptr;   // work counter of the persistent flash kernel (reset before each launch)
   // chunked delta rule on the tensor cores: bf16 operand images [chunks][Hd][bytes per image]
   uint8_t* img = nullptr;
   // 8-bit KV cache: one attention layer's K and V read back as bf16 [2][Hkv][max_ctx][D]

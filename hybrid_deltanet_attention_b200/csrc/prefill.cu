@@ -2624,7 +2624,8 @@ cudaError_t prefill_pass(mk_model* m, const int32_t* tok, int T, int off, cudaSt
           ++m->launches;
         }
         if (e == cudaSuccess) {
-          e = launch_attn_flash(pf.xhi, pf.xlo, kc, pf.vt, b.pos, off, T, Hq, Hkv, D, c.max_ctx, nk, pf.o, qd, b.err, s);
+          e = launch_attn_flash(pf.xhi, pf.xlo, kc, pf.vt, b.pos, off, T, Hq, Hkv, D, c.max_ctx, nk, pf.o, qd,
+                                pf.flash_items, b.err, s);
           ++m->launches;
         }
       } else {
