@@ -383,7 +383,7 @@ Layout make_layout(const mk_config& c, int grid) {
     L.pf_h = off; off = align256(off + T * H * 4);
     L.pf_xhi = off; off = align256(off + T * kmax * 2);
     L.pf_xlo = off; off = align256(off + T * kmax * 2);
-    L.pf_z = off; off = align256(off + T * zmax * 4);
+    L.pf_z = off; off = align256(off + std::max(T * zmax, static_cast<size_t>(c.vocab)) * 4);   // also the prompt's last logits
     L.pf_y = off; off = align256(off + T * ymax * 4);
     L.pf_o = off; off = align256(off + T * omax * 4);
     L.pf_u = off; off = align256(off + T * kdn * 4);
@@ -833,11 +833,11 @@ int mk_prefill(mk_model* m, const int32_t* d_tokens, int32_t n, float* d_last_lo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* sink = m->ws_tok + m->cfg.max_ctx + 4;
   if (m->pf.rows > 0 && n > kBatchedPrefillMin) {
-    // all but the last token through the batched layers, the last one through the
-    // decode kernel (its logits and the next token)
-    int rc = mk_prefill_batched(m, d_tokens, n - 1, s);
+    // every token through the batched layers, then the last token's logits and greedy token
+    // from its residual row (final norm, LM head over one row, argmax)
+    int rc = mk_prefill_batched(m, d_tokens, n, s);
     if (rc) return rc;
-    return launch_step(m, d_tokens + n - 1, d_next_token ? d_next_token : sink, d_last_logits, s);
+    return mk_prefill_tail(m, n, d_last_logits, d_next_token, s);
   }
   for (int i = 0; i < n; ++i) {
     const bool last = (i == n - 1);

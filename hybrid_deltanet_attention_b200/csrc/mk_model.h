@@ -17,7 +17,7 @@ struct mk_prefill_ws {
   float* h = nullptr;        // [rows][H] residual stream
   uint16_t* xhi = nullptr;   // [rows][Kmax] bf16 high part of the current GEMM input
   uint16_t* xlo = nullptr;   // [rows][Kmax] bf16 low part
-  float* z = nullptr;        // [rows][Zmax] projection outputs
+  float* z = nullptr;        // [rows][Zmax] projection outputs (at least V floats: the prompt's last logits)
   float* y = nullptr;        // [rows][Ymax] DeltaNet q k v log-a b / roped attention queries
   float* o = nullptr;        // [rows][Omax] mixer outputs
   float* u = nullptr;        // [rows][Hd dv] chunked delta rule: U
@@ -75,6 +75,7 @@ struct mk_verify_ws {
 
 // Batched prefill of n tokens at the device position: every layer, no logits.
 int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t s);
+int mk_prefill_tail(mk_model* m, int n, float* d_logits, int32_t* d_next_token, cudaStream_t s);
 // Verify pass of K+1 tokens in one pass over the weights, acceptance, and commit of the
 // accepted prefix (DeltaNet state and conv history rebuilt from the saved updates).
 // Greedy acceptance when d_uniforms is NULL, else sampled acceptance at `temperature`

@@ -2205,6 +2205,11 @@ __global__ void commit_conv(const float* __restrict__ raw, float* __restrict__ r
     ring[static_cast<long long>(p % W) * C + c] = raw[static_cast<long long>(r) * C + c];
 }
 
+// The greedy token of a row_argmax result (lowest index among equal maxima).
+__global__ void argmax_token(const unsigned long long* best, int32_t* out) {
+  *out = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(*best & 0xFFFFFFFFull));
+}
+
 __global__ void advance_pos_accepted(int* pos, const int* n_acc, int max_ctx) {
   *pos = min(*pos + *n_acc + 1, max_ctx);
 }
@@ -2742,6 +2747,45 @@ int mk_prefill_batched(mk_model* m, const int32_t* d_tokens, int n, cudaStream_t
   }
   m->pos_hint += n;
   m->pos_max += n;
+  return MK_OK;
+}
+
+// After a batched prefill of n tokens: the final RMSNorm of the last token's residual row (row
+// (n - 1) mod rows of the last pass), the tied LM head over that one row on the tensor cores,
+// and its greedy token; logits into d_logits (or the projection scratch when it is null).
+int mk_prefill_tail(mk_model* m, int n, float* d_logits, int32_t* d_next_token, cudaStream_t s) {
+  const mk::DecodeParams& b = m->base;
+  const mk_config& c = m->cfg;
+  const int rows = m->pf.rows;
+  const int r = (n - 1) % rows;
+  float* logits = d_logits ? d_logits : m->pf.z;
+  cudaError_t e = cudaSuccess;
+  mk::rms_split<<<1, mk::rms_threads(1), 0, s>>>(m->pf.h + static_cast<size_t>(r) * c.hidden, c.hidden, b.norm_f, b.eps,
+                                                  m->pf.xhi, m->pf.xlo);
+  e = cudaGetLastError();
+  ++m->launches;
+  if (e == cudaSuccess) {
+    e = b.q4 ? mk::launch_q4_linear(m->pf.xhi, m->pf.xlo, b.embed, b.row_bytes, logits, c.vocab, 1, c.vocab, c.hidden, 0,
+                                    m->pf.splitk, mk::kSplitKFloats, s)
+             : mk::launch_bf16_linear(m->pf.xhi, m->pf.xlo, b.embed, b.row_bytes, logits, c.vocab, 1, c.vocab, c.hidden,
+                                      0, m->pf.splitk, mk::kSplitKFloats, s);
+    ++m->launches;
+  }
+  if (e == cudaSuccess) e = cudaMemsetAsync(m->pf.best, 0, sizeof(unsigned long long), s);
+  if (e == cudaSuccess) {
+    mk::row_argmax<<<dim3(1, 64), 256, 0, s>>>(logits, c.vocab, m->pf.best);
+    e = cudaGetLastError();
+    ++m->launches;
+  }
+  if (e == cudaSuccess && d_next_token) {
+    mk::argmax_token<<<1, 1, 0, s>>>(m->pf.best, d_next_token);
+    e = cudaGetLastError();
+    ++m->launches;
+  }
+  if (e != cudaSuccess) {
+    mk_set_last_error(std::string("prefill logits: ") + cudaGetErrorString(e));
+    return MK_ERR_CUDA;
+  }
   return MK_OK;
 }
 
