@@ -83,6 +83,24 @@ int mk_prefill_tail(mk_model* m, int n, float* d_logits, int32_t* d_next_token, 
 int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
                       float* d_logits, cudaStream_t s, float temperature = 1.0f, const float* d_uniforms = nullptr);
 
+// A captured verify pass (CUDA graph) and the arguments it was captured with: passes with
+// the same arguments replay it on the model's own stream, ordered after and before the
+// caller's stream by two events.
+struct mk_verify_graph {
+  cudaGraphExec_t exec = nullptr;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t ev_in = nullptr, ev_out = nullptr;
+  const int32_t* tokens = nullptr;
+  int K = -1;
+  int32_t* n_accepted = nullptr;
+  int32_t* out_tokens = nullptr;
+  float* logits = nullptr;
+  float temperature = 0.f;
+  const float* uniforms = nullptr;
+  int seen = 0;            // uncaptured passes run with these arguments
+  int64_t launches = 0;    // kernel launches in one pass
+};
+
 struct mk_model {
   mk_config cfg;
   mk_sizes sz;
@@ -106,4 +124,11 @@ struct mk_model {
   mk_prefill_ws pf;
   std::vector<mk_prefill_layer> pf_layers;
   mk_verify_ws vf;
+  mk_verify_graph vgraph;
+  ~mk_model() {
+    if (vgraph.exec) cudaGraphExecDestroy(vgraph.exec);
+    if (vgraph.ev_in) cudaEventDestroy(vgraph.ev_in);
+    if (vgraph.ev_out) cudaEventDestroy(vgraph.ev_out);
+    if (vgraph.stream) cudaStreamDestroy(vgraph.stream);
+  }
 };

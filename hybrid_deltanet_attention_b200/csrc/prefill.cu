@@ -2789,8 +2789,9 @@ int mk_prefill_tail(mk_model* m, int n, float* d_logits, int32_t* d_next_token, 
   return MK_OK;
 }
 
-int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
-                      float* d_logits, cudaStream_t s, float temperature, const float* d_uniforms) {
+// One verify pass on stream s (every launch; no host-side bookkeeping of the position).
+static int verify_pass(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
+                       float* d_logits, cudaStream_t s, float temperature, const float* d_uniforms) {
   const mk::DecodeParams& b = m->base;
   const mk_config& c = m->cfg;
   const int T = K + 1;
@@ -2886,6 +2887,80 @@ int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_
     mk_set_last_error(std::string("verify pass: ") + cudaGetErrorString(e));
     return MK_ERR_CUDA;
   }
+  return MK_OK;
+}
+
+// Verify passes with the output arguments of the previous one replay a CUDA graph of the ~10
+// launches per layer (the first pass with new arguments runs uncaptured, so every lazy setup is
+// done; the second is captured and replayed). The drafts are first copied into the model's
+// own token buffer, so every launch argument of a pass is fixed by the model, K and the output
+// arguments; the device position is read by the kernels. Models with the 8-bit KV cache size one
+// launch from the host's bound of the position, so they always run uncaptured.
+int mk_verify_batched(mk_model* m, const int32_t* d_tokens, int K, int32_t* d_n_accepted, int32_t* d_out_tokens,
+                      float* d_logits, cudaStream_t s, float temperature, const float* d_uniforms) {
+  const int T = K + 1;
+  int rc = MK_OK;
+  mk_verify_graph& g = m->vgraph;
+  // the pass reads the tokens from the model's own buffer (ws_g, max_draft + 1 entries), so a
+  // new token array does not need a new graph
+  if (cudaMemcpyAsync(m->ws_g, d_tokens, sizeof(int32_t) * T, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+    mk_set_last_error("verify pass: token copy failed");
+    return MK_ERR_CUDA;
+  }
+  d_tokens = m->ws_g;
+  const bool same = g.tokens == d_tokens && g.K == K && g.n_accepted == d_n_accepted && g.out_tokens == d_out_tokens &&
+                    g.logits == d_logits && g.temperature == temperature && g.uniforms == d_uniforms;
+  if (!same) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g.exec = nullptr;
+    g.tokens = d_tokens;
+    g.K = K;
+    g.n_accepted = d_n_accepted;
+    g.out_tokens = d_out_tokens;
+    g.logits = d_logits;
+    g.temperature = temperature;
+    g.uniforms = d_uniforms;
+    g.seen = 0;
+  }
+  const bool capturable = m->cfg.kv_format == MK_KV_BF16 && mk::set_prefill_smem_limits() == cudaSuccess;
+  if (!capturable || (!g.exec && g.seen == 0)) {
+    rc = verify_pass(m, d_tokens, K, d_n_accepted, d_out_tokens, d_logits, s, temperature, d_uniforms);
+    g.seen = 1;
+  } else {
+    cudaError_t e = cudaSuccess;
+    if (!g.stream) e = cudaStreamCreateWithFlags(&g.stream, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !g.ev_in) e = cudaEventCreateWithFlags(&g.ev_in, cudaEventDisableTiming);
+    if (e == cudaSuccess && !g.ev_out) e = cudaEventCreateWithFlags(&g.ev_out, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(g.ev_in, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(g.stream, g.ev_in, 0);
+    if (e == cudaSuccess && !g.exec) {   // capture this pass
+      e = cudaStreamBeginCapture(g.stream, cudaStreamCaptureModeThreadLocal);
+      if (e == cudaSuccess) {
+        const int64_t l0 = m->launches;
+        const int prc = verify_pass(m, d_tokens, K, d_n_accepted, d_out_tokens, d_logits, g.stream, temperature,
+                                    d_uniforms);
+        cudaGraph_t graph = nullptr;
+        e = cudaStreamEndCapture(g.stream, &graph);
+        if (prc != MK_OK) {
+          if (graph) cudaGraphDestroy(graph);
+          return prc;
+        }
+        if (e == cudaSuccess) e = cudaGraphInstantiate(&g.exec, graph, 0);
+        if (graph) cudaGraphDestroy(graph);
+        g.launches = m->launches - l0;
+        m->launches = l0;
+      }
+    }
+    if (e == cudaSuccess) e = cudaGraphLaunch(g.exec, g.stream);
+    if (e == cudaSuccess) e = cudaEventRecord(g.ev_out, g.stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, g.ev_out, 0);
+    if (e != cudaSuccess) {
+      mk_set_last_error(std::string("verify pass (graph): ") + cudaGetErrorString(e));
+      return MK_ERR_CUDA;
+    }
+    m->launches += g.launches;
+  }
+  if (rc != MK_OK) return rc;
   m->pos_hint += 1;   // at least one position is always committed; the exact count is on the device
   m->pos_max += T;
   return MK_OK;
