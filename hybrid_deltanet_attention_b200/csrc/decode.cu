@@ -749,13 +749,6 @@ __device__ __forceinline__ Q4Lane q4_lane(int lane) {
   return q;
 }
 
-// 1 + q/16 for the 4-bit field of c whose lowest bit is `bit` (exact in fp32).
-template <int BIT>
-__device__ __forceinline__ float q4_unit(uint32_t c) {
-  const uint32_t v = BIT <= 19 ? (c << (19 - BIT)) : (c >> (BIT - 19));
-  return __uint_as_float((v & 0x00780000u) | 0x3F800000u);
-}
-
 __device__ __forceinline__ float q4_part(const uint8_t* blk, const Q4Lane& ql, const float4& xl, const float4& xh,
                                          float xsv) {
   const uint32_t dd = *reinterpret_cast<const uint32_t*>(blk);
@@ -770,17 +763,21 @@ __device__ __forceinline__ float q4_part(const uint8_t* blk, const Q4Lane& ql, c
   const float mmf = __uint_as_float(0x4B000000u | mm) - 8388608.0f;
   const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu))) * scf;
   const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16))) * mmf;
-  // sum (1 + q/16) x over the lane's 8 weights (two chains); sum q x = 16 (that - sum x)
-  float u0 = q4_unit<0>(c) * xl.x;
-  float u1 = q4_unit<4>(c) * xh.x;
-  u0 = fmaf(q4_unit<8>(c), xl.y, u0);
-  u1 = fmaf(q4_unit<12>(c), xh.y, u1);
-  u0 = fmaf(q4_unit<16>(c), xl.z, u0);
-  u1 = fmaf(q4_unit<20>(c), xh.z, u1);
-  u0 = fmaf(q4_unit<24>(c), xl.w, u0);
-  u1 = fmaf(q4_unit<28>(c), xh.w, u1);
-  const float s16 = 16.0f * s;
-  return fmaf(s16, u0 + u1, -(s16 + mn) * xsv);
+  // each code q becomes the float v = 0.5 + q/256 exactly, by one byte permute of its nibble
+  // under the exponent byte of 0.5 (bits 16..19 of the mantissa); the lane's 8 weights go in
+  // four packed FMAs, and sum q x = 256 (sum v x) - 128 (sum x)
+  const uint32_t lo = c & 0x0F0F0F0Fu, hi = (c >> 4) & 0x0F0F0F0Fu;
+  constexpr uint32_t kHalfHi = 0x3F000000u;   // bytes 0..2 zero, byte 3 = 0.5's exponent byte
+  uint64_t acc = 0ull;
+  ffma2(acc, f2_pack(__uint_as_float(__byte_perm(lo, kHalfHi, 0x7044)), __uint_as_float(__byte_perm(lo, kHalfHi, 0x7144))),
+        f2_pack(xl.x, xl.y));
+  ffma2(acc, f2_pack(__uint_as_float(__byte_perm(lo, kHalfHi, 0x7244)), __uint_as_float(__byte_perm(lo, kHalfHi, 0x7344))),
+        f2_pack(xl.z, xl.w));
+  ffma2(acc, f2_pack(__uint_as_float(__byte_perm(hi, kHalfHi, 0x7044)), __uint_as_float(__byte_perm(hi, kHalfHi, 0x7144))),
+        f2_pack(xh.x, xh.y));
+  ffma2(acc, f2_pack(__uint_as_float(__byte_perm(hi, kHalfHi, 0x7244)), __uint_as_float(__byte_perm(hi, kHalfHi, 0x7344))),
+        f2_pack(xh.z, xh.w));
+  return fmaf(256.0f * s, f2_sum(acc), -fmaf(128.0f, s, mn) * xsv);
 }
 
 // xsum[sb * 32 + l] = the sum of the 8 x values lane l pairs with in super-block sb.
