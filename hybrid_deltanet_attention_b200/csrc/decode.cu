@@ -614,11 +614,36 @@ __device__ __forceinline__ void gemv_rows(const uint8_t* chunk, int nrows, int r
 }
 
 // Split-K accumulate into registers: acc[out] += sum_r row_r[out] * coef[r]. Thread tid
-// owns float4 groups tid, tid + 256, ... Rows are taken four at a time, loads first.
+// owns float4 groups tid, tid + 256, ... Rows are taken four at a time, loads first; each
+// pair of outputs takes one packed FMA per row (the same per-element order as scalar FMAs).
 template <int MG>
 __device__ __forceinline__ void splitk_rows(const uint8_t* chunk, int nrows, int rb, const float* coef, int H,
                                             float4* acc, int tid) {
   const int ng = H / 4;
+  if constexpr (MG >= 8) {   // the any-size instance: scalar FMAs (the packed pairs cost it registers)
+    for (int r = 0; r < nrows; ++r) {
+      const uint8_t* row = chunk + static_cast<size_t>(r) * rb;
+      const float cf = coef[r];
+#pragma unroll
+      for (int k = 0; k < MG; ++k) {
+        const int g = tid + k * kConsumerThreads;
+        if (g < ng) {
+          const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * g);
+          acc[k].x = fmaf(bf16lo(w.x), cf, acc[k].x);
+          acc[k].y = fmaf(bf16hi(w.x), cf, acc[k].y);
+          acc[k].z = fmaf(bf16lo(w.y), cf, acc[k].z);
+          acc[k].w = fmaf(bf16hi(w.y), cf, acc[k].w);
+        }
+      }
+    }
+    return;
+  }
+  uint64_t a2[MG][2];
+#pragma unroll
+  for (int k = 0; k < MG; ++k) {
+    a2[k][0] = f2_pack(acc[k].x, acc[k].y);
+    a2[k][1] = f2_pack(acc[k].z, acc[k].w);
+  }
   int r = 0;
   for (; r + 4 <= nrows; r += 4) {
     uint2 w[4][MG];
@@ -634,32 +659,34 @@ __device__ __forceinline__ void splitk_rows(const uint8_t* chunk, int nrows, int
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
+      const uint64_t c2 = f2_pack(cf[q], cf[q]);
 #pragma unroll
       for (int k = 0; k < MG; ++k) {
         const int g = tid + k * kConsumerThreads;
         if (g < ng) {
-          acc[k].x = fmaf(bf16lo(w[q][k].x), cf[q], acc[k].x);
-          acc[k].y = fmaf(bf16hi(w[q][k].x), cf[q], acc[k].y);
-          acc[k].z = fmaf(bf16lo(w[q][k].y), cf[q], acc[k].z);
-          acc[k].w = fmaf(bf16hi(w[q][k].y), cf[q], acc[k].w);
+          ffma2(a2[k][0], f2_pack(bf16lo(w[q][k].x), bf16hi(w[q][k].x)), c2);
+          ffma2(a2[k][1], f2_pack(bf16lo(w[q][k].y), bf16hi(w[q][k].y)), c2);
         }
       }
     }
   }
   for (; r < nrows; ++r) {
     const uint8_t* row = chunk + static_cast<size_t>(r) * rb;
-    const float cf = coef[r];
+    const uint64_t c2 = f2_pack(coef[r], coef[r]);
 #pragma unroll
     for (int k = 0; k < MG; ++k) {
       const int g = tid + k * kConsumerThreads;
       if (g < ng) {
         const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * g);
-        acc[k].x = fmaf(bf16lo(w.x), cf, acc[k].x);
-        acc[k].y = fmaf(bf16hi(w.x), cf, acc[k].y);
-        acc[k].z = fmaf(bf16lo(w.y), cf, acc[k].z);
-        acc[k].w = fmaf(bf16hi(w.y), cf, acc[k].w);
+        ffma2(a2[k][0], f2_pack(bf16lo(w.x), bf16hi(w.x)), c2);
+        ffma2(a2[k][1], f2_pack(bf16lo(w.y), bf16hi(w.y)), c2);
       }
     }
+  }
+#pragma unroll
+  for (int k = 0; k < MG; ++k) {
+    const float2 lo = f2_unpack(a2[k][0]), hi = f2_unpack(a2[k][1]);
+    acc[k] = make_float4(lo.x, lo.y, hi.x, hi.y);
   }
 }
 
