@@ -914,11 +914,10 @@ __global__ void __launch_bounds__(256) wy_state(WyBufs b, float* __restrict__ S 
 // access patterns below), 4 x 4 output tiles per thread, and the forward substitution on
 // a right-hand-side column held in registers.
 // Forward substitution (I + A) X = RHS for the first CH rows of a chunk (CH >= n), column
-// j of X held in registers; writes the U (j < DV) or W column (W into wst [64][DK + 4] in
-// shared memory when wst is set).
+// j of X held in registers; writes the U (j < DV) or W column.
 template <int CH, int DK, int DV>
 __device__ __forceinline__ void wy_fsub(const WyBufs& b, const float* K, const float* A, const float* g,
-                                        const float* bb, int t0, int n, int h, int j, int vo, float* wst) {
+                                        const float* bb, int t0, int n, int h, int j, int vo) {
   constexpr int KP = DK + 4, AP = kChunk + 4;
   const int Hd = b.Hd;
   float x[CH];
@@ -946,9 +945,7 @@ __device__ __forceinline__ void wy_fsub(const WyBufs& b, const float* K, const f
   }
 #pragma unroll
   for (int r = 0; r < CH; ++r) {
-    if (j >= DV && wst) {
-      wst[r * KP + (j - DV)] = x[r];   // rows past n are zero
-    } else if (r < n) {
+    if (r < n) {
       if (j < DV) b.u[static_cast<long long>(t0 + r) * Hd * DV + h * DV + j] = x[r];
       else b.w[static_cast<long long>(t0 + r) * Hd * DK + h * DK + (j - DV)] = x[r];
     }
@@ -965,7 +962,6 @@ __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
   float* A = Q + kChunk * KP;                 // [64][AP]
   float* g = A + kChunk * AP;                 // [64]
   float* bb = g + kChunk;                     // [64]
-  float* Ps = bb + kChunk;                    // [64][AP] P, staged for the operand images
   const int Hd = b.Hd, tid = threadIdx.x;
   const int ch = blockIdx.x, h = blockIdx.y;
   const int t0 = ch * kChunk, n = min(kChunk, b.T - t0);
@@ -1035,70 +1031,14 @@ __global__ void __launch_bounds__(256) wy_prep_fast(WyBufs b) {
         const bool live = r < n;
         const float e = (s2 <= r && live) ? expf(g[r] - g[s2]) : 0.f;
         A[r * AP + s2] = (s2 < r) ? bb[r] * e * akk[a][c] : 0.f;
-        if (b.img) Ps[r * AP + s2] = e * aqk[a][c];
-        else P[r * kChunk + s2] = e * aqk[a][c];
+        P[r * kChunk + s2] = e * aqk[a][c];
       }
   }
   __syncthreads();
-  uint8_t* img = b.img ? b.img + (static_cast<size_t>(ch) * Hd + h) * WyImg<DK>::kBytes : nullptr;
-  if (img) {   // gamma Q (A1 rows 0..63), P, K^T as bf16 high / low tiles
-    constexpr int KB = DK / 64;
-    uint8_t* a1 = img;
-    uint8_t* pi = img + WyImg<DK>::kA1;
-    uint8_t* kt = pi + WyImg<DK>::kP;
-    float v[8];
-    uint4 hv, lv;
-    for (int idx = tid; idx < kChunk * (DK / 8); idx += 256) {
-      const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
-      const float gr = expf(g[r]);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = gr * Q[r * KP + 8 * c8 + u];
-      split8_bf16(v, hv, lv);
-      const uint32_t off = r * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4);
-      *reinterpret_cast<uint4*>(a1 + kb * 16384 + off) = hv;
-      *reinterpret_cast<uint4*>(a1 + (KB + kb) * 16384 + off) = lv;
-    }
-    for (int idx = tid; idx < kChunk * 8; idx += 256) {
-      const int r = idx >> 3, c = idx & 7;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = Ps[r * AP + 8 * c + u];
-      split8_bf16(v, hv, lv);
-      const uint32_t off = r * 128u + ((static_cast<uint32_t>(c) ^ (r & 7u)) << 4);
-      *reinterpret_cast<uint4*>(pi + off) = hv;
-      *reinterpret_cast<uint4*>(pi + 8192 + off) = lv;
-    }
-    for (int idx = tid; idx < 128 * 8; idx += 256) {   // row j of K^T: k_r[j] over the chunk's r
-      const int j = idx & 127, c = idx >> 7;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = j < DK ? K[(8 * c + u) * KP + j] : 0.f;
-      split8_bf16(v, hv, lv);
-      const uint32_t off = j * 128u + ((static_cast<uint32_t>(c) ^ (j & 7u)) << 4);
-      *reinterpret_cast<uint4*>(kt + off) = hv;
-      *reinterpret_cast<uint4*>(kt + 16384 + off) = lv;
-    }
-    __syncthreads();   // Q is consumed: W is staged in its place
-  }
   // (I + A) X = [diag(b) V | diag(b gamma) K]: column j of X in registers
   if (tid < XW) {
-    float* wst = img ? Q : nullptr;
-    if (n <= 16) wy_fsub<16, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo, wst);
-    else wy_fsub<kChunk, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo, wst);
-  }
-  if (img) {   // W (A1 rows 64..127)
-    constexpr int KB = DK / 64;
-    __syncthreads();
-    float v[8];
-    uint4 hv, lv;
-    for (int idx = tid; idx < kChunk * (DK / 8); idx += 256) {
-      const int r = idx / (DK / 8), c8 = idx % (DK / 8), kb = c8 >> 3, c = c8 & 7;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = r < n ? Q[r * KP + 8 * c8 + u] : 0.f;   // rows past n: zero
-      split8_bf16(v, hv, lv);
-      const uint32_t row = 64u + r;
-      const uint32_t off = row * 128u + ((static_cast<uint32_t>(c) ^ (row & 7u)) << 4);
-      *reinterpret_cast<uint4*>(img + kb * 16384 + off) = hv;
-      *reinterpret_cast<uint4*>(img + (KB + kb) * 16384 + off) = lv;
-    }
+    if (n <= 16) wy_fsub<16, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo);
+    else wy_fsub<kChunk, DK, DV>(b, K, A, g, bb, t0, n, h, tid, vo);
   }
   if (tid < n) {
     b.gam[static_cast<long long>(t0 + tid) * Hd + h] = expf(g[tid]);
@@ -1946,7 +1886,7 @@ __global__ void __launch_bounds__(128, 1) wy_state_tc(WyBufs b, float* __restric
 
 template <int DK, int DV>
 size_t wy_fast_smem(bool state_pass) {
-  const size_t prep = sizeof(float) * (2 * kChunk * (DK + 4) + 2 * kChunk * (kChunk + 4) + 2 * kChunk);
+  const size_t prep = sizeof(float) * (2 * kChunk * (DK + 4) + kChunk * (kChunk + 4) + 2 * kChunk);
   const size_t state = sizeof(float) * (kRowGroup * (DK + 4) + 3 * kChunk * (DK + 4) + kChunk * (kChunk + 4) +
                                         kRowGroup * (kChunk + 4) + kChunk * kRowGroup + 4 * kChunk);
   return state_pass ? state : prep;
