@@ -1,19 +1,20 @@
 // Batched prefill: a prompt's tokens go through every layer together, the projections
 // as tensor-core GEMMs (gemm.cu), the DeltaNet mixer in its chunked (WY) form, the
-// attention mixer causally over the KV cache. The last prompt token then runs through
-// the decode megakernel, which produces its logits and the next token.
+// attention mixer causally over the KV cache (attn.cu for 64+ tokens). The last token's
+// logits and the next token then come from its residual row (mk_prefill_tail).
 //
 // Per layer, for T tokens at positions pos0 .. pos0+T-1 (activations fp32 in HBM; every
 // GEMM input is written as bf16 high/low parts):
 //   x = RMSNorm(h)                          rms_split
 //   DeltaNet: z = x W_in^T                  linear
-//             conv + SiLU, q/k L2 norms,    dn_prep, conv_history_update
+//             conv + SiLU, q/k L2 norms,    dn_prep_v4, conv_history_update
 //             log a = -softplus(alpha), b = sigmoid(beta)
-//             chunked delta rule            wy_prep (per chunk and head), wy_state (per head and row group)
+//             chunked delta rule            wy_prep_tc / wy_prep_fast (per chunk and head),
+//                                           wy_state_tc / wy_state_fast (per head and row group)
 //   attention: z = x W_in^T                 linear
 //             RoPE, K/V into the cache      at_prep
-//             causal softmax attention      attn_prefill
-//   h += o W_out^T                          split (with the output gate), linear (accumulate)
+//             causal softmax attention      attn_flash_kernel (64+ tokens), attn_prefill
+//   h += o W_out^T                          gate_split (with the output gate), linear (accumulate)
 //   x = RMSNorm(h); g|u = x [W_gate|W_up]^T; h += (SiLU(g) u) W_down^T
 #include <algorithm>
 #include <cmath>

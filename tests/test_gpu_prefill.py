@@ -1,8 +1,9 @@
 """Batched prefill (tensor-core projections, chunked WY delta rule, causal attention)
 through mk_prefill, against the oracle's token-by-token prefill.
 
-Prompts longer than 16 tokens take the batched path for all but the last token; the
-last token runs through the decode kernel. The lengths below cover one partial chunk,
+Prompts longer than 16 tokens take the batched path for every token; the last token's
+logits come from its residual row (final norm, one LM-head row, argmax). Shorter prompts run
+through the decode kernel token by token. The lengths below cover one partial chunk,
 exact chunks of 64, ragged tails, several chunks, and a second prefill that continues
 from a non-empty state (conv history and KV cache carried over).
 """

@@ -101,8 +101,8 @@ def test_tiny_q4_verify_matches_oracle():
 
 
 def test_mid_q4_batched_prefill_two_passes():
-    """A 70-token prompt on the mid-size 4-bit model: two batched passes (64 + 5 tokens,
-    4-bit linear layers on 8-token tiles) and the last token through the decode kernel."""
+    """A 70-token prompt on the mid-size 4-bit model: two batched passes (64 + 6 tokens,
+    4-bit linear layers on 8-token tiles), then the last token's logits from its residual row."""
     cfg = synth.MID_Q4
     m, W = _setup(cfg, 128)
     _teacher_forced(cfg, m, W, 70, 2, 128)
