@@ -229,7 +229,15 @@ int mk_decode_step_noalloc(mk_model* m, const int32_t* d_in_token, int32_t* d_ou
  * state exactly as if [last, d_1..d_n] had been decoded one by one.
  * Writes *d_n_accepted = n (device int32), d_out_tokens[0..n] = d_1..d_n, g_n
  * (device int32[K+1]; entries past n are left as is) and, if non-NULL, d_logits
- * [(K+1) x V] fp32 for every scored position. */
+ * [(K+1) x V] fp32 for every scored position.
+ * With the batched verify workspace (max_draft + 1 <= 64 and a prefill workspace) the pass
+ * runs as ~10 kernels per layer; the drafts are first copied into the model's own buffer,
+ * and from the second pass with the same K, d_n_accepted, d_out_tokens, d_logits (and, in
+ * sampling mode, temperature and d_uniforms) the pass is replayed as one CUDA graph on a
+ * stream the model owns, ordered after and before `stream` by two events (the graph, the
+ * stream and the events are released by mk_free; models with the 8-bit KV cache always
+ * launch kernel by kernel). The first such call must not be made while `stream` is being
+ * captured. */
 int mk_verify_drafts(mk_model* m, const int32_t* d_tokens, int32_t K, int32_t* d_n_accepted,
                      int32_t* d_out_tokens, float* d_logits, void* stream);
 
